@@ -1,0 +1,389 @@
+"""Pins of the fp64 oracle to things other than itself: hand-worked fixtures,
+closed forms, library routines on special cases, brute force, invariants.
+
+Each test is chosen so that a plausible slip in the oracle (a dropped term, a
+swapped operand, a transposed matrix, a wrong nibble order, a wrong group
+index, a wrong tie rule) fails it.  CPU only.
+"""
+import collections
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle
+import synth
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+def _bf16(v):
+    """float -> bf16 bit patterns via torch (library rounding)."""
+    return torch.tensor(np.asarray(v, dtype=np.float32)).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+
+
+# ----------------------------------------------------------------------------
+# number formats and packing
+# ----------------------------------------------------------------------------
+def test_bf16_patterns_hand():
+    g = _gold("dequant.json")
+    for c in g["bf16"]:
+        assert oracle.bf16_to_f64(np.array([int(c["bits_hex"], 16)]))[0] == c["value"]
+
+
+def test_bf16_rounding_half_even():
+    # 1 + 2^-8 is half-way between bf16 neighbours 1 and 1+2^-7 -> even (1.0)
+    assert oracle.f64_to_bf16_bits(np.array([1.0 + 2.0**-8]))[0] == 0x3F80
+    # 1 + 3*2^-8 is half-way between 1+2^-7 (odd) and 1+2^-6 (even) -> 1+2^-6
+    assert oracle.f64_to_bf16_bits(np.array([1.0 + 3 * 2.0**-8]))[0] == 0x3F82
+    v = np.random.default_rng(0).standard_normal(1000)
+    ref = torch.tensor(v, dtype=torch.float64).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    assert np.array_equal(oracle.f64_to_bf16_bits(v), ref)
+
+
+@pytest.mark.parametrize("case", ["int4", "int4_edges", "int8"])
+def test_unpack_hand_cases(case):
+    c = _gold("int4_pack.json")[case]
+    bits = 8 if case == "int8" else 4
+    packed = np.frombuffer(bytes.fromhex(c["bytes_hex"]), dtype=np.uint8)[None, :]
+    got = oracle.unpack_codes(packed, bits, len(c["codes"]))
+    assert got[0].tolist() == c["codes"]
+    if "u32_le" in c:
+        assert int.from_bytes(packed.tobytes(), "little") == int(c["u32_le"], 16)
+
+
+@pytest.mark.parametrize("case", ["int4", "int4_edges", "int8"])
+def test_generator_packer_matches_hand_cases(case):
+    c = _gold("int4_pack.json")[case]
+    bits = 8 if case == "int8" else 4
+    q = torch.tensor([c["codes"]], dtype=torch.uint8)
+    assert bytes(synth.pack_codes(q, bits)[0].tolist()).hex() == c["bytes_hex"]
+
+
+def test_dequant_hand_cases():
+    for c in _gold("dequant.json")["cases"]:
+        q = np.full((1, 64), c["q"], dtype=np.int64)
+        w = oracle.dequantize(q, np.array([[c["scale"]]]), np.array([[c["bias"]]]))
+        assert np.all(w == c["w"])
+
+
+def test_dequant_group_index():
+    # two groups with different scale/bias: a wrong group index mixes them
+    q = np.ones((1, 128), dtype=np.int64)
+    q[0, 64:] = 2
+    w = oracle.dequantize(q, np.array([[1.0, 2.0]]), np.array([[0.0, 10.0]]))
+    assert np.all(w[0, :64] == 1.0) and np.all(w[0, 64:] == 14.0)
+
+
+def test_blob_layout_hand():
+    for c in _gold("blob_layout.json")["cases"]:
+        offs, sizes, stride = oracle.blob_layout(c["hidden"], c["inter"], c["bits"])
+        assert offs == c["offsets"]
+        assert stride == c["stride"]
+        secs, st2 = synth.blob_sections(c["hidden"], c["inter"], c["bits"])
+        assert [o for o, _ in secs] == c["offsets"] and st2 == c["stride"]
+
+
+def test_blob_disk_size_cross_check():
+    # pages: 42 GB (80B, 48 layers x 512 experts), 18 GB (35B, 40 x 256)
+    stride = oracle.blob_layout(2048, 512, 4)[2]
+    assert abs(48 * 512 * stride / 1e9 - 43.5) < 0.1
+    assert abs(40 * 256 * stride / 1e9 - 18.1) < 0.1
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_blob_roundtrip_generator_vs_decoder(bits):
+    H, I = 192, 64
+    parts = synth.expert_parts(H, I, bits, [11, 12], "cpu")
+    stride = synth.blob_stride(H, I, bits)
+    blobs = torch.empty(2, stride, dtype=torch.uint8)
+    synth.pack_blobs(parts, H, I, bits, blobs)
+    for n in range(2):
+        wg, wu, wd = oracle.read_expert(blobs[n].numpy(), H, I, bits)
+        for w, qk, sk, bk in ((wg, "qg", "sg", "bg"), (wu, "qu", "su", "bu"), (wd, "qd", "sd", "bd")):
+            q = parts[qk][n].double()
+            s = parts[sk][n].double().repeat_interleave(64, dim=1)
+            b = parts[bk][n].double().repeat_interleave(64, dim=1)
+            assert np.array_equal(w, (q * s + b).numpy())
+
+
+# ----------------------------------------------------------------------------
+# router
+# ----------------------------------------------------------------------------
+def test_router_all_zero_weights_picks_lowest_indices():
+    T, H, E, k = 3, 128, 12, 4
+    x = _bf16(np.random.default_rng(1).standard_normal((T, H)))
+    wr = np.zeros((E, H), dtype=np.uint16)
+    idx, p = oracle.route(oracle.router_logits(x, wr), k)
+    assert idx.tolist() == [list(range(k))] * T
+    assert np.allclose(p, 1.0 / k, atol=0, rtol=1e-15)
+
+
+def test_router_one_hot_picks_column():
+    H, E = 64, 16
+    rng = np.random.default_rng(2)
+    wr = _bf16(rng.standard_normal((E, H)) * 0.02)
+    for i in (0, 17, 63):
+        x = np.zeros((1, H), dtype=np.uint16)
+        x[0, i] = 0x3F80  # 1.0
+        l = oracle.router_logits(x, wr)
+        assert np.array_equal(l[0], oracle.bf16_to_f64(wr[:, i]))
+
+
+def test_router_logit_is_exact_dot_on_small_integers():
+    # integer-valued bf16 inputs: the dot product is an exact integer
+    rng = np.random.default_rng(3)
+    xi = rng.integers(-4, 5, (2, 64))
+    wi = rng.integers(-4, 5, (8, 64))
+    l = oracle.router_logits(_bf16(xi), _bf16(wi))
+    assert np.array_equal(l, (xi @ wi.T).astype(np.float64))
+    b = np.arange(8, dtype=np.float32) * 0.5
+    assert np.array_equal(oracle.router_logits(_bf16(xi), _bf16(wi), b), (xi @ wi.T) + b[None, :])
+
+
+def test_route_k_equals_E_is_full_softmax():
+    rng = np.random.default_rng(4)
+    logits = rng.standard_normal((5, 9))
+    idx, p = oracle.route(logits, 9)
+    full = scipy.special.softmax(logits, axis=1)
+    for t in range(5):
+        assert np.allclose(p[t], full[t, idx[t]], rtol=1e-13, atol=0)
+        assert idx[t].tolist() == np.argsort(-logits[t], kind="stable").tolist()
+
+
+def test_route_brute_force_with_ties():
+    rng = np.random.default_rng(5)
+    for trial in range(50):
+        E, k = int(rng.integers(2, 20)), 0
+        k = int(rng.integers(1, E + 1))
+        logits = rng.integers(-3, 4, (3, E)).astype(np.float64)  # many ties
+        idx, p = oracle.route(logits, k)
+        for t in range(3):
+            ranked = sorted(range(E), key=lambda e: (-logits[t, e], e))[:k]
+            assert idx[t].tolist() == ranked
+            ref = scipy.special.softmax(logits[t, ranked])
+            assert np.allclose(p[t], ref, rtol=1e-13)
+            assert abs(p[t].sum() - 1.0) < 1e-14
+
+
+def test_route_bias_shift_invariance_and_forcing():
+    rng = np.random.default_rng(6)
+    l = rng.standard_normal((4, 10))
+    i1, p1 = oracle.route(l, 3)
+    i2, p2 = oracle.route(l + 7.0, 3)
+    assert np.array_equal(i1, i2) and np.allclose(p1, p2, rtol=1e-13)
+    l2 = l.copy()
+    l2[:, 9] += 100.0
+    i3, _ = oracle.route(l2, 3)
+    assert np.all(i3[:, 0] == 9)
+
+
+# ----------------------------------------------------------------------------
+# experts and the layer
+# ----------------------------------------------------------------------------
+def _onehot_parts(H, I, bits, pg, pu, pd):
+    """An expert whose dequantised matrices are 0/1 selection matrices.
+
+    Wg[r, pg[r]] = 1, Wu[r, pu[r]] = 1, Wd[j, pd[j]] = 1 (scale 1, bias 0).
+    """
+    one = torch.tensor(1.0).to(torch.bfloat16)
+    zero = torch.tensor(0.0).to(torch.bfloat16)
+    qg = torch.zeros(1, I, H, dtype=torch.uint8)
+    qu = torch.zeros(1, I, H, dtype=torch.uint8)
+    qd = torch.zeros(1, H, I, dtype=torch.uint8)
+    qg[0, torch.arange(I), torch.tensor(pg)] = 1
+    qu[0, torch.arange(I), torch.tensor(pu)] = 1
+    qd[0, torch.arange(H), torch.tensor(pd)] = 1
+    return dict(qg=qg, qu=qu, qd=qd,
+                sg=one.expand(1, I, H // 64).clone(), bg=zero.expand(1, I, H // 64).clone(),
+                su=one.expand(1, I, H // 64).clone(), bu=zero.expand(1, I, H // 64).clone(),
+                sd=one.expand(1, H, I // 64).clone(), bd=zero.expand(1, H, I // 64).clone())
+
+
+def _pack(parts, H, I, bits):
+    n = parts["qg"].shape[0]
+    out = torch.empty(n, synth.blob_stride(H, I, bits), dtype=torch.uint8)
+    synth.pack_blobs(parts, H, I, bits, out)
+    return out.numpy()
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_expert_selection_matrices_closed_form(bits):
+    H, I = 128, 64
+    rng = np.random.default_rng(7)
+    pg = rng.permutation(H)[:I]
+    pu = rng.permutation(H)[:I]
+    pd = rng.integers(0, I, H)
+    blob = _pack(_onehot_parts(H, I, bits, pg, pu, pd), H, I, bits)[0]
+    x = rng.standard_normal(H)
+    y = oracle.expert_forward(oracle.read_expert(blob, H, I, bits), x)
+    a = x[pg]
+    u = x[pu]
+    h = [a[r] / (1.0 + math.exp(-a[r])) * u[r] for r in range(I)]
+    ref = np.array([h[pd[j]] for j in range(H)])
+    assert np.allclose(y, ref, rtol=1e-14, atol=1e-15)
+
+
+def test_expert_zero_scale_is_bias_broadcast():
+    # scale 0 everywhere -> each row is its group biases: a_r = sum_g bias[r,g] * sum_{i in g} x_i
+    H, I = 128, 64
+    rng = np.random.default_rng(8)
+    parts = synth.expert_parts(H, I, 4, [99], "cpu")
+    for key in ("sg", "su", "sd"):
+        parts[key].zero_()
+    blob = _pack(parts, H, I, 4)[0]
+    x = rng.standard_normal(H)
+    wgts = oracle.read_expert(blob, H, I, 4)
+    bg = parts["bg"][0].double().numpy()
+    bu = parts["bu"][0].double().numpy()
+    bd = parts["bd"][0].double().numpy()
+    X = [sum(x[64 * g:64 * g + 64]) for g in range(H // 64)]
+    a = [sum(bg[r, g] * X[g] for g in range(H // 64)) for r in range(I)]
+    u = [sum(bu[r, g] * X[g] for g in range(H // 64)) for r in range(I)]
+    h = [a[r] / (1 + math.exp(-a[r])) * u[r] for r in range(I)]
+    Hs = sum(h)  # I = 64: one group along the down input
+    ref = np.array([bd[j, 0] * Hs for j in range(H)])
+    assert np.allclose(oracle.expert_forward(wgts, x), ref, rtol=1e-12, atol=1e-15)
+
+
+def test_expert_matches_library_matmul():
+    # E = 1, k = 1: the layer is a dense SwiGLU MLP; torch fp64 matmul + silu as the library check
+    H, I = 128, 64
+    parts = synth.expert_parts(H, I, 4, [5], "cpu")
+    blob = _pack(parts, H, I, 4)[0]
+    wg = (parts["qg"][0].double() * parts["sg"][0].double().repeat_interleave(64, 1) + parts["bg"][0].double().repeat_interleave(64, 1))
+    wu = (parts["qu"][0].double() * parts["su"][0].double().repeat_interleave(64, 1) + parts["bu"][0].double().repeat_interleave(64, 1))
+    wd = (parts["qd"][0].double() * parts["sd"][0].double().repeat_interleave(64, 1) + parts["bd"][0].double().repeat_interleave(64, 1))
+    x = torch.randn(3, H, dtype=torch.float64, generator=torch.Generator().manual_seed(0))
+    ref = (torch.nn.functional.silu(x @ wg.T) * (x @ wu.T)) @ wd.T
+    got = oracle.expert_forward(oracle.read_expert(blob, H, I, 4), x.numpy())
+    assert np.allclose(got, ref.numpy(), rtol=1e-12, atol=1e-14)
+
+
+def _tiny_layer(seed, E, k, H=128, I=64, Is=64, bits=4, T=3, bias=False, zero_gate=False):
+    rng = np.random.default_rng(seed)
+    blobs = _pack(synth.expert_parts(H, I, bits, list(range(seed * 100, seed * 100 + E)), "cpu"), H, I, bits)
+    shared = _pack(synth.expert_parts(H, Is, bits, [seed * 100 + 99], "cpu"), H, Is, bits)[0]
+    x = _bf16(rng.standard_normal((T, H)))
+    wr = _bf16(rng.standard_normal((E, H)) * 0.02)
+    wsg = np.zeros(H, dtype=np.uint16) if zero_gate else _bf16(rng.standard_normal(H) * 0.02)
+    b = rng.standard_normal(E).astype(np.float32) if bias else None
+    res = _bf16(rng.standard_normal((T, H)))
+    return dict(x=x, wr=wr, b=b, blobs=blobs, shared=shared, wsg=wsg, res=res, H=H, I=I, Is=Is, bits=bits, k=k)
+
+
+def _sparse(L, residual=True):
+    return oracle.layer_forward(L["x"], L["wr"], L["b"], L["k"], lambda e: L["blobs"][e], L["shared"],
+                                L["wsg"], L["H"], L["I"], L["Is"], L["bits"],
+                                residual_bits=L["res"] if residual else None)
+
+
+@pytest.mark.parametrize("seed,E,k,bias", [(1, 1, 1, False), (2, 4, 2, False), (3, 16, 2, True),
+                                           (4, 9, 9, False), (5, 13, 5, True), (6, 16, 1, False)])
+def test_layer_sparse_equals_dense_masked_bruteforce(seed, E, k, bias):
+    L = _tiny_layer(seed, E, k, bias=bias)
+    r = _sparse(L)
+    dense = oracle.layer_forward_dense_masked(L["x"], L["wr"], L["b"], k, list(L["blobs"]), L["shared"],
+                                              L["wsg"], L["H"], L["I"], L["Is"], L["bits"],
+                                              residual_bits=L["res"])
+    assert np.allclose(r["out"], dense, rtol=1e-12, atol=1e-13)
+    assert np.allclose(r["p"].sum(1), 1.0, atol=1e-15)
+
+
+def test_layer_single_expert_zero_gate_closed_form():
+    # E = 1, k = 1: p = 1; zero shared-gate weights: sigmoid(0) = 1/2
+    L = _tiny_layer(7, 1, 1, zero_gate=True)
+    r = _sparse(L, residual=False)
+    x = oracle.bf16_to_f64(L["x"])
+    y1 = oracle.expert_forward(oracle.read_expert(L["blobs"][0], 128, 64, 4), x)
+    ys = oracle.expert_forward(oracle.read_expert(L["shared"], 128, 64, 4), x)
+    assert np.all(r["gate"] == 0.5) and np.all(r["p"] == 1.0)
+    assert np.allclose(r["out"], y1 + 0.5 * ys, rtol=1e-14, atol=1e-15)
+    r2 = _sparse(L, residual=True)
+    assert np.allclose(r2["out"] - r["out"], oracle.bf16_to_f64(L["res"]), rtol=0, atol=1e-12)
+
+
+def test_layer_token_permutation_equivariance():
+    L = _tiny_layer(8, 16, 3, T=5, bias=True)
+    r = _sparse(L)
+    perm = np.array([3, 0, 4, 2, 1])
+    L2 = dict(L, x=L["x"][perm], res=L["res"][perm])
+    r2 = _sparse(L2)
+    assert np.allclose(r2["out"], r["out"][perm], rtol=1e-13, atol=1e-14)
+    assert np.array_equal(r2["idx"], r["idx"][perm])
+
+
+def test_layer_expert_relabelling_invariance():
+    L = _tiny_layer(9, 12, 3, T=4, bias=True)
+    r = _sparse(L)
+    perm = np.random.default_rng(9).permutation(12)  # new expert n = old perm[n]
+    L2 = dict(L, wr=L["wr"][perm], b=L["b"][perm], blobs=L["blobs"][perm])
+    r2 = _sparse(L2)
+    assert np.allclose(r2["out"], r["out"], rtol=1e-13, atol=1e-14)
+    inv = np.argsort(perm)
+    # same experts picked, as a set, per token (order may differ only on exact ties)
+    for t in range(4):
+        assert sorted(perm[r2["idx"][t]].tolist()) == sorted(r["idx"][t].tolist())
+        assert sorted(inv[r["idx"][t]].tolist()) == sorted(r2["idx"][t].tolist())
+
+
+def test_silu_sigmoid_special_values():
+    assert oracle.silu(0.0) == 0.0 and oracle.sigmoid(0.0) == 0.5
+    assert abs(oracle.silu(40.0) - 40.0) < 1e-15 * 40
+    assert abs(oracle.silu(-40.0)) < 1e-15
+    assert abs(oracle.sigmoid(1.0) - 1 / (1 + math.e ** -1)) < 1e-16
+
+
+# ----------------------------------------------------------------------------
+# prefill grouping
+# ----------------------------------------------------------------------------
+def test_group_pairs_is_stable_sort():
+    rng = np.random.default_rng(10)
+    for E, T, k in ((16, 7, 2), (512, 300, 10), (5, 1, 5)):
+        idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+        counts, offsets, order = oracle.group_pairs(idx, E)
+        flat = idx.reshape(-1)
+        assert order.tolist() == np.argsort(flat, kind="stable").tolist()
+        c = collections.Counter(flat.tolist())
+        assert counts.tolist() == [c.get(e, 0) for e in range(E)]
+        assert offsets[0] == 0 and offsets[-1] == T * k
+
+
+# ----------------------------------------------------------------------------
+# bounded slot pool
+# ----------------------------------------------------------------------------
+def test_slot_cache_hand_traces():
+    for tr in _gold("slot_cache_traces.json")["traces"]:
+        c = oracle.SlotCache(tr["n_experts"], tr["n_slots"])
+        for step, want in zip(tr["steps"], tr["loads"]):
+            assert [list(l) for l in c.step(step)] == want
+        assert c.slot_of.tolist() == tr["final_slot_of"]
+        assert (c.lookups, c.hits, c.misses, c.evictions) == (tr["lookups"], tr["hits"], tr["misses"], tr["evictions"])
+        with pytest.raises(OverflowError):
+            c.step(tr["capacity_error_next"])
+
+
+def test_slot_cache_invariants_random():
+    rng = np.random.default_rng(11)
+    E, S, k = 64, 16, 6
+    c = oracle.SlotCache(E, S)
+    for s in range(300):
+        need = rng.choice(E, size=k, replace=False, p=None)
+        c.step(need)
+        for e in need:
+            assert c.slot_of[e] >= 0
+        res = np.nonzero(c.slot_of >= 0)[0]
+        assert len(res) <= S
+        for e in res:
+            assert c.expert_in[c.slot_of[e]] == e
+        assert c.hits + c.misses == c.lookups
+    assert c.misses - c.evictions == S  # every miss after the pool fills evicts exactly one
