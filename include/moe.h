@@ -1,0 +1,235 @@
+/*
+ * moe.h -- C ABI of the routed Mixture-of-Experts layer forward for NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes (Swiftlet pages: «Paquets Swiftlet 80B Qwen dans Mac…»,
+ * xix.ai, paragraphs 5 and 9; «Swiftlet: 在 Mac 和 iPhone 上執行 80B 與 35B Qwen 模型»,
+ * agentlenshq.com, section 記憶體管理與權重串流; «Swiftlet — это Swift + Metal
+ * рантайм…», news.bugfactory.tech, paragraph 3):
+ *
+ *   router   l[t,e] = sum_i x[t,i] * Wr[e,i] (+ b[e]); the k experts with the largest
+ *            logits (ties: lower index first) are selected and weighted by a softmax
+ *            over the k selected logits (weights sum to 1);
+ *   experts  each selected expert is a SwiGLU MLP y = Wd (silu(Wg x) * (Wu x)) whose
+ *            weights are MLX-style affine group-quantised codes (int4 or int8, group
+ *            64 along the input dimension, bf16 scale and bias per group):
+ *            w = scale * q + bias;
+ *   shared   an always-on shared expert with the same blob format, scaled by
+ *            sigmoid(w_sg . x);
+ *   combine  out[t] = sum_k p[t,k] y_k + sigmoid(w_sg . x[t]) y_shared (+ residual[t]).
+ *
+ * Expert storage.  Every expert is one fixed-stride blob ("one read = one fetch"):
+ * nine sections, each starting on a 256-byte boundary, in the order
+ *   Wg.q [I, H*b/8], Wu.q [I, H*b/8], Wd.q [H, I*b/8]              (u8 codes)
+ *   Wg.s, Wg.bias, Wu.s, Wu.bias [I, H/64], Wd.s, Wd.bias [H, I/64]  (bf16)
+ * Codes are packed little-endian as MLX does: for int4, byte n of a row holds element
+ * 2n in its low nibble and element 2n+1 in its high nibble; for int8 byte n is element
+ * n.  A pool is n_slots blobs back to back; slot s starts at byte s * stride (64-bit
+ * offsets).  slot_table[e] names the slot that holds expert e.
+ *
+ * Conventions for every call:
+ *   - Pointers marked (dev) are device pointers, (host) are host pointers.  All device
+ *     memory is owned by the caller; the library keeps no pointer after a call returns
+ *     (except the pool object, which keeps the ones given to moe_pool_create).
+ *   - bf16 tensors are passed as raw 16-bit patterns; all tensors are dense row-major.
+ *   - Device pointers must be 16-byte aligned; the pool and blob pointers 256-byte
+ *     aligned.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and
+ *     is asynchronous, except where a call says it synchronises.
+ *   - Arguments are validated before anything is enqueued; a bad argument returns
+ *     MOE_ERR_INVALID (or MOE_ERR_UNSUPPORTED for a valid shape this build has no
+ *     kernel for) and enqueues nothing.  Nothing aborts or throws across this ABI.
+ *     moe_last_error() gives a message for the calling thread's last failure.
+ *   - Errors detected on the device (an expert id outside [0, E), a slot outside
+ *     [0, n_slots), non-finite router logits) set bits in the workspace's error word
+ *     and the offending term is skipped; read them with moe_ws_check().
+ *   - The workspace must be zero-filled once before its first use; every call leaves
+ *     its internal counters at zero again.  Calls that share a workspace must not run
+ *     concurrently.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID = -1,      /* bad argument (null pointer, bad size, misalignment) */
+  MOE_ERR_CUDA = -2,         /* a CUDA runtime call failed; see moe_last_error() */
+  MOE_ERR_CAPACITY = -3,     /* a pool step needs more distinct experts than slots */
+  MOE_ERR_NOT_RESIDENT = -4, /* reserved: an expert the call needs has no slot */
+  MOE_ERR_UNSUPPORTED = -5,  /* valid request with no kernel in this build */
+  MOE_ERR_TIMEOUT = -6,      /* a bounded device-side wait gave up */
+  MOE_ERR_DEVICE = -7        /* the device set an error bit (moe_ws_check) */
+} moe_status;
+
+/* Device error-word bits (moe_ws_check). */
+#define MOE_DEVERR_BAD_EXPERT 0x1u   /* a top-k expert id outside [0, E) was skipped   */
+#define MOE_DEVERR_BAD_SLOT 0x2u     /* slot_table gave a slot outside [0, n_slots)     */
+#define MOE_DEVERR_NONFINITE 0x4u    /* a router logit was NaN/Inf; top-k may be short  */
+#define MOE_DEVERR_TIMEOUT 0x8u      /* a bounded device wait gave up                   */
+
+typedef struct {
+  int32_t hidden;       /* H: model width (multiple of 64)                                 */
+  int32_t inter;        /* I: routed-expert intermediate width (multiple of 64)            */
+  int32_t shared_inter; /* I_s: shared-expert intermediate width (this build: I_s == I)    */
+  int32_t n_experts;    /* E: routed experts per layer (1..1024)                           */
+  int32_t top_k;        /* k: experts per token (1..min(E, 32))                            */
+  int32_t bits;         /* 4 or 8                                                          */
+  int32_t group;        /* quantisation group along the input dimension: must be 64        */
+} moe_shape;
+
+/*
+ * moe_blob_layout -- byte offsets of the nine sections of one expert blob and its stride.
+ * Defines the fixed-stride blob ("one contiguous read per expert", «Swiftlet: 在 Mac 和
+ * iPhone 上執行…», 記憶體管理與權重串流).  hidden/inter must be multiples of 64, bits 4 or
+ * 8, group 64.  offsets (host, 9 entries) and stride (host) are written on success.
+ */
+MOE_API moe_status moe_blob_layout(int32_t hidden, int32_t inter, int32_t bits, int32_t group,
+                           int64_t offsets[9], int64_t* stride);
+
+/*
+ * moe_workspace_size -- bytes of device workspace that moe_router_topk / moe_layer_forward
+ * need for T tokens of this shape.  *bytes (host) is written on success.
+ */
+MOE_API moe_status moe_workspace_size(const moe_shape* shape, int32_t T, size_t* bytes);
+
+/*
+ * moe_router_topk -- router GEMV + softmax top-k (the per-layer router: «Paquets Swiftlet…»
+ * paragraph 5, 10 of 512 / 8 of 256 experts per token).
+ *   x           (dev) bf16 [T, H] activations
+ *   w_router    (dev) bf16 [E, H]
+ *   router_bias (dev) fp32 [E] or NULL: added to the logits before selection and softmax
+ *   topk_idx    (dev) int32 [T, k] out: expert ids, logit descending, ties lower id first
+ *   topk_w      (dev) fp32  [T, k] out: softmax over the k selected logits
+ *   ws          (dev) workspace of ws_bytes >= moe_workspace_size(shape, T)
+ * Logits are accumulated in fp64 from exact bf16*bf16 products, so the selection is the
+ * exact-arithmetic selection except for logits that tie to within fp64 rounding.
+ * T: 1..8 on the decode path.
+ */
+MOE_API moe_status moe_router_topk(const moe_shape* shape, const void* x, int32_t T, const void* w_router,
+                           const float* router_bias, int32_t* topk_idx, float* topk_w, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/*
+ * moe_layer_forward -- the routed-MoE layer forward for T tokens.
+ *   x            (dev) bf16 [T, H]
+ *   w_router     (dev) bf16 [E, H]      (unused when topk_idx_in != NULL)
+ *   router_bias  (dev) fp32 [E] or NULL
+ *   topk_idx_in  (dev) int32 [T, k] or NULL: precomputed routing (e.g. from moe_router_topk
+ *                before moe_expert_pool_load); NULL routes inside this call
+ *   topk_w_in    (dev) fp32 [T, k]: weights for topk_idx_in (required with it)
+ *   pool         (dev) u8 [n_slots * stride] expert blobs; stride from moe_blob_layout
+ *   slot_table   (dev) int32 [E]: slot of each expert; entries of experts that a call
+ *                selects must be in [0, n_slots)
+ *   n_slots      number of blobs in pool (bounds-checks slot_table on the device)
+ *   shared_blob  (dev) u8 blob of the shared expert (layout with inter = I_s)
+ *   w_shared_gate(dev) bf16 [H]: shared-expert gate, scale = sigmoid(w . x[t])
+ *   residual     (dev) bf16 [T, H] or NULL: added to the output
+ *   out          (dev) bf16 [T, H] out (round-to-nearest-even of the fp32 sum)
+ *   topk_idx_out, topk_w_out (dev) [T, k] or NULL: the routing used (when routed inside)
+ *   ws, ws_bytes workspace (see moe_workspace_size)
+ * T: 1..8 (decode path).  Deterministic: the same inputs give the same bits, whichever
+ * slots the experts sit in.
+ */
+MOE_API moe_status moe_layer_forward(const moe_shape* shape, const void* x, int32_t T, const void* w_router,
+                             const float* router_bias, const int32_t* topk_idx_in,
+                             const float* topk_w_in, const uint8_t* pool, const int32_t* slot_table,
+                             int64_t n_slots, const uint8_t* shared_blob, const void* w_shared_gate,
+                             const void* residual, void* out, int32_t* topk_idx_out,
+                             float* topk_w_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_ws_check -- synchronise `stream`, read and clear the workspace's device error word.
+ *   *flags (host) receives the MOE_DEVERR_* bits.  Returns MOE_ERR_DEVICE if any bit was
+ *   set, MOE_OK otherwise.
+ */
+MOE_API moe_status moe_ws_check(void* ws, void* stream, uint32_t* flags);
+
+/* ------------------------------------------------------------------------------------ */
+/* Bounded slot pool with LFU + recency eviction («Paquets Swiftlet…» paragraph 5;       */
+/* «Swiftlet: 在 Mac 和 iPhone 上執行…», 記憶體管理與權重串流).  Misses are copied from   */
+/* pinned host blobs with cudaMemcpyAsync on the pool's own side stream.                 */
+/* ------------------------------------------------------------------------------------ */
+typedef struct moe_pool moe_pool;
+
+typedef struct {
+  int64_t steps;      /* moe_expert_pool_load calls that succeeded                          */
+  int64_t lookups;    /* distinct (step, expert) lookups                                    */
+  int64_t hits;       /* lookups whose expert was resident                                  */
+  int64_t misses;     /* lookups that loaded a blob                                         */
+  int64_t evictions;  /* loads that replaced a resident expert                              */
+  int64_t h2d_bytes;  /* bytes copied host -> device for misses                             */
+} moe_pool_stats_t;
+
+/*
+ * moe_pool_create -- a pool of n_slots slots over caller memory.
+ *   host_blobs (host, pinned) u8 [E * stride]: expert e's blob at byte e * stride
+ *   dev_pool   (dev) u8 [n_slots * stride];  dev_slot_table (dev) int32 [E]
+ * The slot table is initialised to -1 (no expert resident); the pool starts empty.
+ * *out receives the handle (owned by the caller; free with moe_pool_destroy).
+ * Creates one non-blocking side stream and two events.
+ */
+MOE_API moe_status moe_pool_create(const moe_shape* shape, int32_t n_slots, const uint8_t* host_blobs,
+                           uint8_t* dev_pool, int32_t* dev_slot_table, moe_pool** out);
+
+/*
+ * moe_expert_pool_load -- make every expert named in topk_idx (dev int32 [T, k]) resident.
+ * SYNCHRONISES `stream` (the ids are needed on the host): copies the ids back, looks them
+ * up (distinct ids in first-appearance order; hits refresh use count and last use), loads
+ * each miss into the lowest empty slot, else evicts the slot with the smallest
+ * (use count, last use step, slot index) among slots this step does not need, copies the
+ * missed blobs and the updated slot table on the side stream, and makes `stream` wait for
+ * them.  MOE_ERR_CAPACITY (nothing changed) if a step needs more distinct experts than
+ * slots; MOE_ERR_INVALID for an id outside [0, E).  If a copy fails the slot is left
+ * empty, the table stays consistent, and MOE_ERR_CUDA is returned.
+ */
+MOE_API moe_status moe_expert_pool_load(moe_pool* pool, const int32_t* topk_idx, int32_t T, void* stream);
+
+/* moe_pool_stats -- counters since creation (host struct). */
+MOE_API moe_status moe_pool_stats(const moe_pool* pool, moe_pool_stats_t* stats);
+
+/*
+ * moe_pool_slot_table -- copy of the host mirror of the slot table (host int32 [E]) and of
+ * the slot -> expert map (host int32 [n_slots]; either pointer may be NULL).
+ */
+MOE_API moe_status moe_pool_slot_table(const moe_pool* pool, int32_t* slot_of_expert, int32_t* expert_in_slot);
+
+/*
+ * moe_pool_inject_copy_failure -- test hook: the n-th blob copy from now (0 = the next one)
+ * reports failure without being issued; -1 disarms.  Host-side only.
+ */
+MOE_API moe_status moe_pool_inject_copy_failure(moe_pool* pool, int64_t nth);
+
+/* moe_pool_destroy -- waits for the side stream, releases the handle. NULL is a no-op. */
+MOE_API void moe_pool_destroy(moe_pool* pool);
+
+/*
+ * moe_profile_events -- measurement hook.  While set (events != NULL), each
+ * moe_layer_forward / moe_router_topk call on this thread records events[2*i] on its stream
+ * just before its i-th kernel launch and events[2*i+1] just after it, for i < n
+ * (i = 0: router or grouping, 1: gate/up + SwiGLU, 2: down + combine).  events are
+ * cudaEvent_t handles owned by the caller.  Thread-local; NULL disables.
+ */
+MOE_API moe_status moe_profile_events(void* const* events, int32_t n);
+
+/* Message of the calling thread's last failed call ("" if none). */
+MOE_API const char* moe_last_error(void);
+
+/* Library version string. */
+MOE_API const char* moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

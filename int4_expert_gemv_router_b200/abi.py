@@ -1,0 +1,207 @@
+"""Thin ctypes binding of libmoe.so (include/moe.h): same names, argument marshalling only.
+
+Every function takes torch tensors (or None for optional pointers) and passes
+their data pointers; `stream` defaults to torch's current CUDA stream.  A
+non-OK status raises MoeError with the library's message.  Nothing here
+computes any part of the layer: there is no fallback if the library is
+missing; loading fails loudly instead.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_OK = 0
+STATUS = {0: "MOE_OK", -1: "MOE_ERR_INVALID", -2: "MOE_ERR_CUDA", -3: "MOE_ERR_CAPACITY",
+          -4: "MOE_ERR_NOT_RESIDENT", -5: "MOE_ERR_UNSUPPORTED", -6: "MOE_ERR_TIMEOUT",
+          -7: "MOE_ERR_DEVICE"}
+DEVERR_BAD_EXPERT, DEVERR_BAD_SLOT, DEVERR_NONFINITE, DEVERR_TIMEOUT = 1, 2, 4, 8
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class moe_shape(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("inter", ctypes.c_int32), ("shared_inter", ctypes.c_int32),
+                ("n_experts", ctypes.c_int32), ("top_k", ctypes.c_int32), ("bits", ctypes.c_int32),
+                ("group", ctypes.c_int32)]
+
+
+class moe_pool_stats_t(ctypes.Structure):
+    _fields_ = [("steps", ctypes.c_int64), ("lookups", ctypes.c_int64), ("hits", ctypes.c_int64),
+                ("misses", ctypes.c_int64), ("evictions", ctypes.c_int64), ("h2d_bytes", ctypes.c_int64)]
+
+    def as_dict(self):
+        return {k: int(getattr(self, k)) for k, _ in self._fields_}
+
+
+_P = ctypes.c_void_p
+_I32, _I64, _SZ = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+_SIGS = {
+    "moe_blob_layout": (ctypes.c_int, [_I32, _I32, _I32, _I32, ctypes.POINTER(_I64), ctypes.POINTER(_I64)]),
+    "moe_workspace_size": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, ctypes.POINTER(_SZ)]),
+    "moe_router_topk": (ctypes.c_int, [ctypes.POINTER(moe_shape), _P, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_layer_forward": (ctypes.c_int, [ctypes.POINTER(moe_shape), _P, _I32, _P, _P, _P, _P, _P, _P, _I64,
+                                         _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_ws_check": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
+    "moe_pool_create": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, _P, _P, _P, ctypes.POINTER(_P)]),
+    "moe_expert_pool_load": (ctypes.c_int, [_P, _P, _I32, _P]),
+    "moe_pool_stats": (ctypes.c_int, [_P, ctypes.POINTER(moe_pool_stats_t)]),
+    "moe_pool_slot_table": (ctypes.c_int, [_P, _P, _P]),
+    "moe_pool_inject_copy_failure": (ctypes.c_int, [_P, _I64]),
+    "moe_pool_destroy": (None, [_P]),
+    "moe_profile_events": (ctypes.c_int, [_P, _I32]),
+    "moe_last_error": (ctypes.c_char_p, []),
+    "moe_version": (ctypes.c_char_p, []),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m int4_expert_gemv_router_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def exported_symbols():
+    return list(_SIGS)
+
+
+def _check(st: int):
+    if st != MOE_OK:
+        raise MoeError(st, lib().moe_last_error().decode())
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if isinstance(t, torch.Tensor):
+        if not t.is_contiguous():
+            raise ValueError("tensor must be contiguous")
+        return t.data_ptr()
+    raise TypeError(f"expected a tensor, an int address or None, got {type(t)}")
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def make_shape(hidden, inter, shared_inter, n_experts, top_k, bits, group=64) -> moe_shape:
+    return moe_shape(hidden, inter, shared_inter, n_experts, top_k, bits, group)
+
+
+def shape_of(w) -> moe_shape:
+    """moe_shape from any object with hidden/inter/shared_inter/n_experts/top_k/bits attributes."""
+    return make_shape(w.hidden, w.inter, w.shared_inter, w.n_experts, w.top_k, w.bits)
+
+
+def moe_version() -> str:
+    return lib().moe_version().decode()
+
+
+def moe_blob_layout(hidden: int, inter: int, bits: int, group: int = 64):
+    offs = (_I64 * 9)()
+    stride = _I64()
+    _check(lib().moe_blob_layout(hidden, inter, bits, group, offs, ctypes.byref(stride)))
+    return list(offs), int(stride.value)
+
+
+def moe_workspace_size(shape: moe_shape, T: int) -> int:
+    n = _SZ()
+    _check(lib().moe_workspace_size(ctypes.byref(shape), T, ctypes.byref(n)))
+    return int(n.value)
+
+
+def moe_router_topk(shape, x, T, w_router, router_bias, topk_idx, topk_w, ws, stream=None):
+    _check(lib().moe_router_topk(ctypes.byref(shape), _ptr(x), T, _ptr(w_router), _ptr(router_bias),
+                                 _ptr(topk_idx), _ptr(topk_w), _ptr(ws), ws.numel() * ws.element_size(),
+                                 _stream(stream)))
+
+
+def moe_layer_forward(shape, x, T, w_router, router_bias, topk_idx_in, topk_w_in, pool, slot_table, n_slots,
+                      shared_blob, w_shared_gate, residual, out, topk_idx_out, topk_w_out, ws, stream=None):
+    _check(lib().moe_layer_forward(ctypes.byref(shape), _ptr(x), T, _ptr(w_router), _ptr(router_bias),
+                                   _ptr(topk_idx_in), _ptr(topk_w_in), _ptr(pool), _ptr(slot_table), n_slots,
+                                   _ptr(shared_blob), _ptr(w_shared_gate), _ptr(residual), _ptr(out),
+                                   _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_ws_check(ws, stream=None, raise_on_error: bool = False) -> int:
+    flags = ctypes.c_uint32()
+    st = lib().moe_ws_check(_ptr(ws), _stream(stream), ctypes.byref(flags))
+    if st not in (MOE_OK, -7) or (raise_on_error and st != MOE_OK):
+        _check(st)
+    return int(flags.value)
+
+
+def moe_pool_create(shape, n_slots, host_blobs, dev_pool, dev_slot_table) -> int:
+    h = _P()
+    _check(lib().moe_pool_create(ctypes.byref(shape), n_slots, _ptr(host_blobs), _ptr(dev_pool),
+                                 _ptr(dev_slot_table), ctypes.byref(h)))
+    return h.value
+
+
+def moe_expert_pool_load(pool: int, topk_idx, T: int, stream=None):
+    _check(lib().moe_expert_pool_load(pool, _ptr(topk_idx), T, _stream(stream)))
+
+
+def moe_pool_stats(pool: int) -> dict:
+    s = moe_pool_stats_t()
+    _check(lib().moe_pool_stats(pool, ctypes.byref(s)))
+    return s.as_dict()
+
+
+def moe_pool_slot_table(pool: int, n_experts: int, n_slots: int):
+    a = (ctypes.c_int32 * n_experts)()
+    b = (ctypes.c_int32 * n_slots)()
+    _check(lib().moe_pool_slot_table(pool, a, b))
+    return list(a), list(b)
+
+
+def moe_pool_inject_copy_failure(pool: int, nth: int):
+    _check(lib().moe_pool_inject_copy_failure(pool, nth))
+
+
+def moe_pool_destroy(pool: int):
+    lib().moe_pool_destroy(pool)
+
+
+_prof_keep = None
+
+
+def moe_profile_events(events, n: int = 0):
+    """events: a list of torch.cuda.Event (2 per kernel) or None to disable."""
+    global _prof_keep
+    if events is None:
+        _prof_keep = None
+        _check(lib().moe_profile_events(None, 0))
+        return
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    _prof_keep = arr
+    _check(lib().moe_profile_events(arr, n or len(events) // 2))

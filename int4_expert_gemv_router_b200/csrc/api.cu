@@ -1,0 +1,237 @@
+// C-ABI entry points (include/moe.h): argument validation, workspace carving and the launch
+// sequence of each call.  No kernel arithmetic lives here.
+#include "../../include/moe.h"
+#include "common.cuh"
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+namespace moe {
+
+static thread_local std::string g_last_error;
+static thread_local void* const* g_prof_events = nullptr;
+static thread_local int g_prof_n = 0;
+
+// Records the profiling event of kernel i (begin or end) if the hook is armed.
+static void prof_mark(int i, bool end, cudaStream_t s) {
+  if (g_prof_events && i < g_prof_n) cudaEventRecord(static_cast<cudaEvent_t>(g_prof_events[2 * i + (end ? 1 : 0)]), s);
+}
+
+moe_status set_error(moe_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+moe_status cuda_fail(cudaError_t e, const char* what) {
+  return set_error(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+static bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+moe_status check_shape(const moe_shape* s) {
+  if (!s) return set_error(MOE_ERR_INVALID, "shape is NULL");
+  if (s->group != kGroup) return set_error(MOE_ERR_INVALID, "group must be 64 (got %d)", s->group);
+  if (s->bits != 4 && s->bits != 8) return set_error(MOE_ERR_INVALID, "bits must be 4 or 8 (got %d)", s->bits);
+  if (s->hidden <= 0 || s->hidden % kGroup)
+    return set_error(MOE_ERR_INVALID, "hidden must be a positive multiple of 64 (got %d)", s->hidden);
+  if (s->inter <= 0 || s->inter % kGroup)
+    return set_error(MOE_ERR_INVALID, "inter must be a positive multiple of 64 (got %d)", s->inter);
+  if (s->shared_inter <= 0 || s->shared_inter % kGroup)
+    return set_error(MOE_ERR_INVALID, "shared_inter must be a positive multiple of 64 (got %d)", s->shared_inter);
+  if (s->n_experts < 1 || s->n_experts > kMaxExperts)
+    return set_error(MOE_ERR_INVALID, "n_experts must be in [1, %d] (got %d)", kMaxExperts, s->n_experts);
+  if (s->top_k < 1 || s->top_k > s->n_experts || s->top_k > kMaxTopK)
+    return set_error(MOE_ERR_INVALID, "top_k must be in [1, min(E, %d)] (got %d)", kMaxTopK, s->top_k);
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+const char* moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
+
+moe_status moe_blob_layout(int32_t hidden, int32_t inter, int32_t bits, int32_t group, int64_t offsets[9],
+                           int64_t* stride) {
+  if (!offsets || !stride) return set_error(MOE_ERR_INVALID, "offsets/stride is NULL");
+  if (group != kGroup) return set_error(MOE_ERR_INVALID, "group must be 64 (got %d)", group);
+  if (bits != 4 && bits != 8) return set_error(MOE_ERR_INVALID, "bits must be 4 or 8 (got %d)", bits);
+  if (hidden <= 0 || hidden % kGroup || inter <= 0 || inter % kGroup)
+    return set_error(MOE_ERR_INVALID, "hidden and inter must be positive multiples of 64");
+  const BlobLayout L = make_blob_layout(hidden, inter, bits);
+  for (int i = 0; i < 9; ++i) offsets[i] = L.off[i];
+  *stride = L.stride;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_size(const moe_shape* shape, int32_t T, size_t* bytes) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!bytes) return set_error(MOE_ERR_INVALID, "bytes is NULL");
+  if (T < 1) return set_error(MOE_ERR_INVALID, "T must be >= 1 (got %d)", T);
+  *bytes = make_ws_layout(T, shape->n_experts, shape->top_k, shape->inter, shape->shared_inter).total;
+  return MOE_OK;
+}
+
+static moe_status fill_decode_args(const moe_shape* shape, int32_t T, void* ws, size_t ws_bytes, DecodeArgs* a) {
+  memset(a, 0, sizeof *a);
+  if (T < 1 || T > kMaxDecodeT)
+    return set_error(MOE_ERR_UNSUPPORTED, "T must be in [1, %d] on the decode path (got %d)", kMaxDecodeT, T);
+  if (!ws || !aligned(ws, kAlign)) return set_error(MOE_ERR_INVALID, "ws must be non-NULL and 256-byte aligned");
+  const WsLayout W = make_ws_layout(T, shape->n_experts, shape->top_k, shape->inter, shape->shared_inter);
+  if (ws_bytes < W.total)
+    return set_error(MOE_ERR_INVALID, "ws_bytes %zu < required %zu", ws_bytes, W.total);
+  char* b = static_cast<char*>(ws);
+  a->H = shape->hidden;
+  a->I = shape->inter;
+  a->Is = shape->shared_inter;
+  a->E = shape->n_experts;
+  a->k = shape->top_k;
+  a->T = T;
+  a->L = make_blob_layout(shape->hidden, shape->inter, shape->bits);
+  a->Ls = make_blob_layout(shape->hidden, shape->shared_inter, shape->bits);
+  a->ctrl = reinterpret_cast<Ctrl*>(b + W.ctrl);
+  a->logits = reinterpret_cast<double*>(b + W.logits);
+  a->topk_idx = reinterpret_cast<int32_t*>(b + W.topk_idx);
+  a->topk_w = reinterpret_cast<float*>(b + W.topk_w);
+  a->gate = reinterpret_cast<float*>(b + W.gate);
+  a->order = reinterpret_cast<int32_t*>(b + W.order);
+  a->act_e = reinterpret_cast<int32_t*>(b + W.act_e);
+  a->act_begin = reinterpret_cast<int32_t*>(b + W.act_begin);
+  a->h = reinterpret_cast<float*>(b + W.h);
+  a->hs = reinterpret_cast<float*>(b + W.hs);
+  return MOE_OK;
+}
+
+moe_status moe_router_topk(const moe_shape* shape, const void* x, int32_t T, const void* w_router,
+                           const float* router_bias, int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                           void* stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!x || !w_router || !topk_idx || !topk_w)
+    return set_error(MOE_ERR_INVALID, "x, w_router, topk_idx and topk_w must be non-NULL");
+  if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) ||
+      (router_bias && !aligned(router_bias, 4)))
+    return set_error(MOE_ERR_INVALID, "x and w_router must be 16-byte aligned");
+  DecodeArgs a;
+  if ((st = fill_decode_args(shape, T, ws, ws_bytes, &a)) != MOE_OK) return st;
+  a.x = static_cast<const uint16_t*>(x);
+  a.wr = static_cast<const uint16_t*>(w_router);
+  a.rbias = router_bias;
+  // The shared-gate row is not needed here; point it at the first router row (its logit
+  // lands in the workspace and is ignored).
+  a.wsg = a.wr;
+  a.topk_idx = topk_idx;
+  a.topk_w = topk_w;
+  prof_mark(0, false, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_router_decode(a, false, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "router launch");
+  prof_mark(0, true, static_cast<cudaStream_t>(stream));
+  return MOE_OK;
+}
+
+moe_status moe_layer_forward(const moe_shape* shape, const void* x, int32_t T, const void* w_router,
+                             const float* router_bias, const int32_t* topk_idx_in, const float* topk_w_in,
+                             const uint8_t* pool, const int32_t* slot_table, int64_t n_slots,
+                             const uint8_t* shared_blob, const void* w_shared_gate, const void* residual, void* out,
+                             int32_t* topk_idx_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->shared_inter != shape->inter)
+    return set_error(MOE_ERR_UNSUPPORTED, "this build needs shared_inter == inter (%d vs %d)", shape->shared_inter,
+                     shape->inter);
+  if (!decode_shape_supported(shape->hidden, shape->inter, shape->bits))
+    return set_error(MOE_ERR_UNSUPPORTED,
+                     "no decode kernel for hidden=%d inter=%d bits=%d (hidden: power of two in [256, 4096], "
+                     "inter: power of two in [64, 1024])",
+                     shape->hidden, shape->inter, shape->bits);
+  if (!x || !pool || !slot_table || !shared_blob || !w_shared_gate || !out)
+    return set_error(MOE_ERR_INVALID, "x, pool, slot_table, shared_blob, w_shared_gate and out must be non-NULL");
+  if (!topk_idx_in && !w_router) return set_error(MOE_ERR_INVALID, "w_router is NULL and no topk_idx_in given");
+  if (topk_idx_in && !topk_w_in) return set_error(MOE_ERR_INVALID, "topk_idx_in given without topk_w_in");
+  if ((topk_idx_out == nullptr) != (topk_w_out == nullptr))
+    return set_error(MOE_ERR_INVALID, "topk_idx_out and topk_w_out must both be given or both be NULL");
+  if (n_slots < 1) return set_error(MOE_ERR_INVALID, "n_slots must be >= 1");
+  if (!aligned(x, 16) || !aligned(out, 16) || (w_router && !aligned(w_router, 16)) ||
+      !aligned(w_shared_gate, 16) || (residual && !aligned(residual, 16)))
+    return set_error(MOE_ERR_INVALID, "x, out, w_router, w_shared_gate and residual must be 16-byte aligned");
+  if (!aligned(pool, kAlign) || !aligned(shared_blob, kAlign))
+    return set_error(MOE_ERR_INVALID, "pool and shared_blob must be 256-byte aligned");
+  DecodeArgs a;
+  if ((st = fill_decode_args(shape, T, ws, ws_bytes, &a)) != MOE_OK) return st;
+  a.x = static_cast<const uint16_t*>(x);
+  a.wr = static_cast<const uint16_t*>(w_router);
+  a.rbias = router_bias;
+  a.wsg = static_cast<const uint16_t*>(w_shared_gate);
+  a.pool = pool;
+  a.slot_table = slot_table;
+  a.n_slots = n_slots;
+  a.shared_blob = shared_blob;
+  a.residual = static_cast<const uint16_t*>(residual);
+  a.out = static_cast<uint16_t*>(out);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  prof_mark(0, false, s);
+  if (!topk_idx_in) {
+    if (topk_idx_out) {
+      a.topk_idx = topk_idx_out;
+      a.topk_w = topk_w_out;
+    }
+    e = launch_router_decode(a, true, s);
+    if (e != cudaSuccess) return cuda_fail(e, "router launch");
+  } else {
+    a.topk_idx = const_cast<int32_t*>(topk_idx_in);
+    a.topk_w = const_cast<float*>(topk_w_in);
+    e = launch_plan_decode(a, s);
+    if (e != cudaSuccess) return cuda_fail(e, "plan launch");
+  }
+  prof_mark(0, true, s);
+  bool ok = true;
+  prof_mark(1, false, s);
+  e = launch_gateup_decode(a, shape->bits, s, &ok);
+  if (e != cudaSuccess) return cuda_fail(e, "gate/up launch");
+  prof_mark(1, true, s);
+  prof_mark(2, false, s);
+  e = launch_down_decode(a, shape->bits, s, &ok);
+  if (e != cudaSuccess) return cuda_fail(e, "down launch");
+  prof_mark(2, true, s);
+  return MOE_OK;
+}
+
+moe_status moe_profile_events(void* const* events, int32_t n) {
+  if (events && n < 0) return set_error(MOE_ERR_INVALID, "n must be >= 0");
+  g_prof_events = events;
+  g_prof_n = events ? n : 0;
+  return MOE_OK;
+}
+
+moe_status moe_ws_check(void* ws, void* stream, uint32_t* flags) {
+  if (!ws || !flags) return set_error(MOE_ERR_INVALID, "ws and flags must be non-NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  uint32_t v = 0;
+  e = cudaMemcpy(&v, ws, sizeof v, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "error word read");
+  if (v) {
+    const uint32_t zero = 0;
+    e = cudaMemcpy(ws, &zero, sizeof zero, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "error word clear");
+  }
+  *flags = v;
+  if (v) return set_error(MOE_ERR_DEVICE, "device error bits 0x%x", v);
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,122 @@
+// Internal declarations shared by the sm_100a kernels and the C-ABI layer.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stddef.h>
+
+namespace moe {
+
+constexpr int kGroup = 64;      // quantisation group along the input dimension
+constexpr int kAlign = 256;     // blob section / workspace alignment
+constexpr int kMaxDecodeT = 8;  // tokens per call on the GEMV (decode) path
+constexpr int kMaxTopK = 32;
+constexpr int kMaxExperts = 1024;
+
+// Device error-word bits (mirrors MOE_DEVERR_* in include/moe.h).
+constexpr uint32_t kErrBadExpert = 0x1u;
+constexpr uint32_t kErrBadSlot = 0x2u;
+constexpr uint32_t kErrNonFinite = 0x4u;
+constexpr uint32_t kErrTimeout = 0x8u;
+
+// ---------------------------------------------------------------------------------------
+// Fixed-stride expert blob: nine 256-byte aligned sections (gate/up/down codes, then
+// gate scale, gate bias, up scale, up bias, down scale, down bias).
+// ---------------------------------------------------------------------------------------
+struct BlobLayout {
+  int64_t off[9];
+  int64_t stride;
+};
+
+inline int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+inline BlobLayout make_blob_layout(int H, int I, int bits) {
+  BlobLayout L{};
+  const int64_t codes_gu = (int64_t)I * H * bits / 8;
+  const int64_t codes_d = (int64_t)H * I * bits / 8;
+  const int64_t sb_gu = (int64_t)I * (H / kGroup) * 2;
+  const int64_t sb_d = (int64_t)H * (I / kGroup) * 2;
+  const int64_t size[9] = {codes_gu, codes_gu, codes_d, sb_gu, sb_gu, sb_gu, sb_gu, sb_d, sb_d};
+  int64_t pos = 0;
+  for (int i = 0; i < 9; ++i) {
+    pos = round_up(pos, kAlign);
+    L.off[i] = pos;
+    pos += size[i];
+  }
+  L.stride = round_up(pos, kAlign);
+  return L;
+}
+
+// ---------------------------------------------------------------------------------------
+// Workspace: a control block, then fixed-size arrays, each 256-byte aligned.
+// ---------------------------------------------------------------------------------------
+struct Ctrl {
+  uint32_t err;     // sticky MOE_DEVERR_* bits (cleared by moe_ws_check)
+  uint32_t ticket;  // last-block-done counter of the router (always returns to 0)
+  int32_t act_n;    // number of distinct routed experts of the current call
+  int32_t n_valid;  // number of (token, k) pairs with a valid expert id
+  uint32_t pad[60];
+};
+static_assert(sizeof(Ctrl) == 256, "ctrl block is 256 bytes");
+
+struct WsLayout {
+  size_t ctrl, logits, topk_idx, topk_w, gate, order, act_e, act_begin, h, hs, total;
+};
+
+inline WsLayout make_ws_layout(int T, int E, int k, int I, int Is) {
+  WsLayout W{};
+  size_t pos = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = (size_t)round_up((int64_t)pos, kAlign);
+    pos = at + bytes;
+    return at;
+  };
+  W.ctrl = take(sizeof(Ctrl));
+  W.logits = take(sizeof(double) * (size_t)T * (E + 1));
+  W.topk_idx = take(sizeof(int32_t) * (size_t)T * k);
+  W.topk_w = take(sizeof(float) * (size_t)T * k);
+  W.gate = take(sizeof(float) * (size_t)T);
+  W.order = take(sizeof(int32_t) * (size_t)T * k);
+  W.act_e = take(sizeof(int32_t) * (size_t)T * k);
+  W.act_begin = take(sizeof(int32_t) * ((size_t)T * k + 1));
+  W.h = take(sizeof(float) * (size_t)T * k * I);
+  W.hs = take(sizeof(float) * (size_t)T * Is);
+  W.total = (size_t)round_up((int64_t)pos, kAlign);
+  return W;
+}
+
+// Everything one decode-path layer call needs, as raw pointers.
+struct DecodeArgs {
+  int H, I, Is, E, k, T;
+  const uint16_t* x;         // bf16 [T, H]
+  const uint16_t* wr;        // bf16 [E, H]
+  const float* rbias;        // fp32 [E] or null
+  const uint16_t* wsg;       // bf16 [H]
+  const uint8_t* pool;       // n_slots * stride
+  const int32_t* slot_table; // [E]
+  int64_t n_slots;
+  const uint8_t* shared_blob;
+  const uint16_t* residual;  // bf16 [T, H] or null
+  uint16_t* out;             // bf16 [T, H]
+  int32_t* topk_idx;         // [T, k]  (router output, or caller-given input)
+  float* topk_w;             // [T, k]
+  BlobLayout L, Ls;
+  // workspace
+  Ctrl* ctrl;
+  double* logits;            // [T, E+1] (column E: shared-gate logit)
+  float* gate;               // [T]
+  int32_t* order;            // [T*k] pair numbers sorted by expert (stable)
+  int32_t* act_e;            // [T*k] distinct experts, ascending
+  int32_t* act_begin;        // [T*k+1] first sorted position of each distinct expert
+  float* h;                  // [T*k, I]  SwiGLU intermediate per sorted pair
+  float* hs;                 // [T, Is]   shared-expert intermediate per token
+};
+
+// Kernel launchers (decode.cu).  Return cudaError_t of the launch.
+cudaError_t launch_router_decode(const DecodeArgs& a, bool build_plan, cudaStream_t s);
+cudaError_t launch_plan_decode(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_gateup_decode(const DecodeArgs& a, int bits, cudaStream_t s, bool* supported);
+cudaError_t launch_down_decode(const DecodeArgs& a, int bits, cudaStream_t s, bool* supported);
+bool decode_shape_supported(int H, int I, int bits);
+
+}  // namespace moe

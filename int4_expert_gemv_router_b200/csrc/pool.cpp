@@ -1,0 +1,241 @@
+// Bounded expert slot pool with LFU + recency eviction (host side).
+//
+// The Swiftlet pages describe a bounded pool of slots that caches the popular routed
+// experts, evicting with LFU combined with recency, and a fixed-stride container so that
+// fetching one expert is a single read («Paquets Swiftlet 80B Qwen dans Mac…», paragraph
+// 5; «Swiftlet: 在 Mac 和 iPhone 上執行 80B 與 35B Qwen 模型», section 記憶體管理與權重串流).
+// Here the backing store is pinned host memory and a fetch is one cudaMemcpyAsync of one
+// blob on the pool's side stream.
+//
+// Policy (the pages give only "LFU + recency"; this is the plain reading):
+//   per slot: resident expert, use count (1 when loaded, +1 for every later step that uses
+//   it), last-use step.  A step's distinct experts are looked up in first-appearance order;
+//   hits refresh count and last use.  Misses are then loaded in the same order into the
+//   lowest-numbered empty slot, else into the slot with the smallest
+//   (count, last use, slot index) among slots whose expert the step does not need.
+#include "../../include/moe.h"
+#include "common.cuh"
+
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <new>
+#include <vector>
+
+namespace moe {
+moe_status set_error(moe_status s, const char* fmt, ...);
+moe_status cuda_fail(cudaError_t e, const char* what);
+moe_status check_shape(const moe_shape* s);
+}  // namespace moe
+
+using namespace moe;
+
+struct moe_pool {
+  moe_shape shape;
+  int32_t n_slots = 0;
+  int64_t stride = 0;
+  const uint8_t* host_blobs = nullptr;
+  uint8_t* dev_pool = nullptr;
+  int32_t* dev_slot_table = nullptr;
+  std::vector<int32_t> slot_of;    // [E] slot of expert, -1 if not resident
+  std::vector<int32_t> expert_in;  // [S] expert in slot, -1 if empty
+  std::vector<int64_t> count;      // [S]
+  std::vector<int64_t> last_use;   // [S]
+  std::vector<uint8_t> needed;     // [E] scratch: expert needed by the current step
+  int64_t step_no = 0;
+  moe_pool_stats_t stats{};
+  int64_t fail_at = -1;            // test hook: copies until an injected failure
+  cudaStream_t side = nullptr;
+  cudaEvent_t ready = nullptr;     // slot table + blobs of the last step are on the device
+  bool ready_recorded = false;
+  int32_t* h_ids = nullptr;        // pinned [kMaxDecodeT * kMaxTopK]
+  int32_t* h_table = nullptr;      // pinned [E]
+};
+
+extern "C" {
+
+moe_status moe_pool_create(const moe_shape* shape, int32_t n_slots, const uint8_t* host_blobs, uint8_t* dev_pool,
+                           int32_t* dev_slot_table, moe_pool** out) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!out) return set_error(MOE_ERR_INVALID, "out is NULL");
+  *out = nullptr;
+  if (n_slots < 1) return set_error(MOE_ERR_INVALID, "n_slots must be >= 1");
+  if (!host_blobs || !dev_pool || !dev_slot_table)
+    return set_error(MOE_ERR_INVALID, "host_blobs, dev_pool and dev_slot_table must be non-NULL");
+  if (((uintptr_t)dev_pool & 255) || ((uintptr_t)host_blobs & 15))
+    return set_error(MOE_ERR_INVALID, "dev_pool must be 256-byte and host_blobs 16-byte aligned");
+  cudaPointerAttributes attr{};
+  if (cudaPointerGetAttributes(&attr, host_blobs) != cudaSuccess || attr.type != cudaMemoryTypeHost) {
+    cudaGetLastError();
+    return set_error(MOE_ERR_INVALID, "host_blobs must be pinned host memory (cudaHostAlloc / pin_memory)");
+  }
+  moe_pool* p = new (std::nothrow) moe_pool();
+  if (!p) return set_error(MOE_ERR_INVALID, "out of host memory");
+  p->shape = *shape;
+  p->n_slots = n_slots;
+  p->stride = make_blob_layout(shape->hidden, shape->inter, shape->bits).stride;
+  p->host_blobs = host_blobs;
+  p->dev_pool = dev_pool;
+  p->dev_slot_table = dev_slot_table;
+  const int E = shape->n_experts;
+  p->slot_of.assign(E, -1);
+  p->expert_in.assign(n_slots, -1);
+  p->count.assign(n_slots, 0);
+  p->last_use.assign(n_slots, -1);
+  p->needed.assign(E, 0);
+  cudaError_t e;
+  if ((e = cudaStreamCreateWithFlags(&p->side, cudaStreamNonBlocking)) != cudaSuccess ||
+      (e = cudaEventCreateWithFlags(&p->ready, cudaEventDisableTiming)) != cudaSuccess ||
+      (e = cudaHostAlloc((void**)&p->h_ids, sizeof(int32_t) * kMaxDecodeT * kMaxTopK, cudaHostAllocDefault)) !=
+          cudaSuccess ||
+      (e = cudaHostAlloc((void**)&p->h_table, sizeof(int32_t) * E, cudaHostAllocDefault)) != cudaSuccess) {
+    moe_pool_destroy(p);
+    return cuda_fail(e, "pool create");
+  }
+  for (int i = 0; i < E; ++i) p->h_table[i] = -1;
+  e = cudaMemcpyAsync(dev_slot_table, p->h_table, sizeof(int32_t) * E, cudaMemcpyHostToDevice, p->side);
+  if (e == cudaSuccess) e = cudaEventRecord(p->ready, p->side);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(p->side);
+  if (e != cudaSuccess) {
+    moe_pool_destroy(p);
+    return cuda_fail(e, "pool slot table init");
+  }
+  p->ready_recorded = true;
+  *out = p;
+  return MOE_OK;
+}
+
+moe_status moe_expert_pool_load(moe_pool* p, const int32_t* topk_idx, int32_t T, void* stream) {
+  if (!p || !topk_idx) return set_error(MOE_ERR_INVALID, "pool and topk_idx must be non-NULL");
+  const int k = p->shape.top_k, E = p->shape.n_experts;
+  if (T < 1 || T > kMaxDecodeT) return set_error(MOE_ERR_INVALID, "T must be in [1, %d]", kMaxDecodeT);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int n = T * k;
+  // The ids are needed on the host.  Synchronising the caller stream also guarantees that
+  // every earlier forward on it has finished reading the slots this step may overwrite.
+  cudaError_t e = cudaMemcpyAsync(p->h_ids, topk_idx, sizeof(int32_t) * n, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "top-k read-back");
+  // The previous step's table upload reads h_table: let it finish before editing it.
+  if (p->ready_recorded && (e = cudaEventSynchronize(p->ready)) != cudaSuccess) return cuda_fail(e, "pool event");
+  // distinct ids in first-appearance order
+  std::vector<int32_t> uniq;
+  uniq.reserve(n);
+  for (int i = 0; i < n; ++i) {
+    const int32_t id = p->h_ids[i];
+    if (id < 0 || id >= E) {
+      for (int32_t u : uniq) p->needed[u] = 0;
+      return set_error(MOE_ERR_INVALID, "expert id %d outside [0, %d)", id, E);
+    }
+    if (!p->needed[id]) {
+      p->needed[id] = 1;
+      uniq.push_back(id);
+    }
+  }
+  if ((int)uniq.size() > p->n_slots) {
+    for (int32_t u : uniq) p->needed[u] = 0;
+    return set_error(MOE_ERR_CAPACITY, "step needs %zu distinct experts, pool has %d slots", uniq.size(),
+                     p->n_slots);
+  }
+  const int64_t now = p->step_no;
+  moe_status result = MOE_OK;
+  for (int32_t id : uniq) {
+    p->stats.lookups++;
+    const int32_t sl = p->slot_of[id];
+    if (sl >= 0) {
+      p->stats.hits++;
+      p->count[sl]++;
+      p->last_use[sl] = now;
+    }
+  }
+  for (int32_t id : uniq) {
+    if (p->slot_of[id] >= 0) continue;
+    p->stats.misses++;
+    int32_t victim = -1;
+    for (int32_t sl = 0; sl < p->n_slots; ++sl)
+      if (p->expert_in[sl] < 0) {
+        victim = sl;
+        break;
+      }
+    bool evicting = false;
+    if (victim < 0) {
+      for (int32_t sl = 0; sl < p->n_slots; ++sl) {
+        if (p->needed[p->expert_in[sl]]) continue;
+        if (victim < 0 || p->count[sl] < p->count[victim] ||
+            (p->count[sl] == p->count[victim] && p->last_use[sl] < p->last_use[victim]))
+          victim = sl;  // ascending scan keeps the lowest slot index on full ties
+      }
+      evicting = true;
+    }
+    if (evicting) {
+      p->slot_of[p->expert_in[victim]] = -1;
+      p->expert_in[victim] = -1;
+      p->stats.evictions++;
+    }
+    bool failed = false;
+    if (p->fail_at == 0) {
+      failed = true;
+      p->fail_at = -1;
+    } else {
+      if (p->fail_at > 0) p->fail_at--;
+      e = cudaMemcpyAsync(p->dev_pool + (int64_t)victim * p->stride, p->host_blobs + (int64_t)id * p->stride,
+                          (size_t)p->stride, cudaMemcpyHostToDevice, p->side);
+      failed = (e != cudaSuccess);
+    }
+    if (failed) {
+      // slot stays empty; the expert stays non-resident
+      result = (e != cudaSuccess) ? cuda_fail(e, "blob copy") : set_error(MOE_ERR_CUDA, "blob copy failed (injected)");
+      e = cudaSuccess;
+      continue;
+    }
+    p->expert_in[victim] = id;
+    p->slot_of[id] = victim;
+    p->count[victim] = 1;
+    p->last_use[victim] = now;
+    p->stats.h2d_bytes += p->stride;
+  }
+  for (int32_t u : uniq) p->needed[u] = 0;
+  for (int i = 0; i < E; ++i) p->h_table[i] = p->slot_of[i];
+  e = cudaMemcpyAsync(p->dev_slot_table, p->h_table, sizeof(int32_t) * E, cudaMemcpyHostToDevice, p->side);
+  if (e == cudaSuccess) e = cudaEventRecord(p->ready, p->side);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, p->ready, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "slot table upload");
+  p->ready_recorded = true;
+  p->step_no++;
+  if (result == MOE_OK) p->stats.steps++;
+  return result;
+}
+
+moe_status moe_pool_stats(const moe_pool* p, moe_pool_stats_t* stats) {
+  if (!p || !stats) return set_error(MOE_ERR_INVALID, "pool and stats must be non-NULL");
+  *stats = p->stats;
+  return MOE_OK;
+}
+
+moe_status moe_pool_slot_table(const moe_pool* p, int32_t* slot_of_expert, int32_t* expert_in_slot) {
+  if (!p) return set_error(MOE_ERR_INVALID, "pool is NULL");
+  if (slot_of_expert) memcpy(slot_of_expert, p->slot_of.data(), sizeof(int32_t) * p->slot_of.size());
+  if (expert_in_slot) memcpy(expert_in_slot, p->expert_in.data(), sizeof(int32_t) * p->expert_in.size());
+  return MOE_OK;
+}
+
+moe_status moe_pool_inject_copy_failure(moe_pool* p, int64_t nth) {
+  if (!p) return set_error(MOE_ERR_INVALID, "pool is NULL");
+  p->fail_at = nth < 0 ? -1 : nth;
+  return MOE_OK;
+}
+
+void moe_pool_destroy(moe_pool* p) {
+  if (!p) return;
+  if (p->side) {
+    cudaStreamSynchronize(p->side);
+    cudaStreamDestroy(p->side);
+  }
+  if (p->ready) cudaEventDestroy(p->ready);
+  if (p->h_ids) cudaFreeHost(p->h_ids);
+  if (p->h_table) cudaFreeHost(p->h_table);
+  delete p;
+}
+
+}  // extern "C"

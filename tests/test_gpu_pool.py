@@ -1,0 +1,130 @@
+"""GPU checks of the bounded slot pool (moe_expert_pool_load): slot decisions equal the
+oracle's LFU + recency simulation step by step, missed blobs land byte-for-byte, the
+pool-mode forward is bit-identical to the all-resident forward, and failures leave the
+pool consistent."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import forward, ws_for
+from int4_expert_gemv_router_b200 import abi, build
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build.build()
+
+
+class Pool:
+    def __init__(self, w, n_slots, layer=0):
+        self.w = w
+        self.L = synth.make_layer(w, layer, DEV)  # all-resident copy (reference path)
+        self.host = self.L.pool.cpu().pin_memory()
+        self.stride = self.L.pool.shape[1]
+        self.dev = torch.zeros(n_slots, self.stride, dtype=torch.uint8, device=DEV)
+        self.table = torch.empty(w.n_experts, dtype=torch.int32, device=DEV)
+        self.n_slots = n_slots
+        self.shape = abi.shape_of(w)
+        self.h = abi.moe_pool_create(self.shape, n_slots, self.host, self.dev, self.table)
+
+    def close(self):
+        abi.moe_pool_destroy(self.h)
+
+
+def _route(P, x):
+    w = P.w
+    T = x.shape[0]
+    ws = ws_for(P.shape, T)
+    idx = torch.empty(T, w.top_k, dtype=torch.int32, device=DEV)
+    p = torch.empty(T, w.top_k, dtype=torch.float32, device=DEV)
+    abi.moe_router_topk(P.shape, x, T, P.L.w_router, P.L.router_bias, idx, p, ws)
+    return idx, p
+
+
+@pytest.mark.parametrize("wname,steps,T", [("pool_int4", 48, 1), ("pool_int8", 32, 1), ("pool_int4", 12, 8)])
+def test_pool_matches_oracle_cache_and_resident_forward(wname, steps, T):
+    w = synth.WORKLOADS[wname]
+    P = Pool(w, w.n_slots)
+    sim = oracle.SlotCache(w.n_experts, w.n_slots)
+    try:
+        assert torch.all(P.table == -1)
+        for s in range(steps):
+            x = synth.activations(w, s, tokens=T, device=DEV)
+            idx, p = _route(P, x)
+            abi.moe_expert_pool_load(P.h, idx, T)
+            sim.step(idx.cpu().numpy().reshape(-1).tolist())
+            slot_of, expert_in = abi.moe_pool_slot_table(P.h, w.n_experts, w.n_slots)
+            assert slot_of == sim.slot_of.tolist()
+            assert expert_in == sim.expert_in.tolist()
+            torch.cuda.synchronize()
+            assert P.table.cpu().tolist() == slot_of
+            # the selected experts' slots hold their blobs byte for byte
+            for e in set(idx.cpu().numpy().reshape(-1).tolist()):
+                assert torch.equal(P.dev[slot_of[e]].cpu(), P.host[e])
+            out_pool, *_ = forward(w, P.L, x, residual=x, pool=P.dev, slot_table=P.table, n_slots=P.n_slots,
+                                   topk=(idx, p))
+            out_res, *_ = forward(w, P.L, x, residual=x, topk=(idx, p))
+            assert torch.equal(out_pool, out_res)
+        st = abi.moe_pool_stats(P.h)
+        assert (st["lookups"], st["hits"], st["misses"], st["evictions"]) == (sim.lookups, sim.hits, sim.misses,
+                                                                              sim.evictions)
+        assert st["h2d_bytes"] == sim.misses * P.stride
+        assert st["steps"] == steps
+    finally:
+        P.close()
+
+
+def test_pool_capacity_error_changes_nothing():
+    w = synth.WORKLOADS["tiny"].with_(n_experts=16, top_k=4, seed=31)
+    P = Pool(w, 3)
+    try:
+        x = synth.activations(w, 0, tokens=1, device=DEV)
+        idx, _ = _route(P, x)
+        with pytest.raises(abi.MoeError) as ei:
+            abi.moe_expert_pool_load(P.h, idx, 1)
+        assert ei.value.status == -3
+        slot_of, expert_in = abi.moe_pool_slot_table(P.h, 16, 3)
+        assert all(s == -1 for s in slot_of) and all(e == -1 for e in expert_in)
+        assert abi.moe_pool_stats(P.h)["lookups"] == 0
+    finally:
+        P.close()
+
+
+def test_pool_bad_id_rejected():
+    w = synth.WORKLOADS["tiny"].with_(seed=32)
+    P = Pool(w, 8)
+    try:
+        bad = torch.tensor([[3, 16]], dtype=torch.int32, device=DEV)
+        with pytest.raises(abi.MoeError) as ei:
+            abi.moe_expert_pool_load(P.h, bad, 1)
+        assert ei.value.status == -1
+    finally:
+        P.close()
+
+
+def test_pool_injected_copy_failure_leaves_consistent_state():
+    w = synth.WORKLOADS["tiny"].with_(n_experts=16, top_k=2, seed=33)
+    P = Pool(w, 4)
+    try:
+        ids = torch.tensor([[5, 9]], dtype=torch.int32, device=DEV)
+        abi.moe_pool_inject_copy_failure(P.h, 1)  # the second copy fails
+        with pytest.raises(abi.MoeError) as ei:
+            abi.moe_expert_pool_load(P.h, ids, 1)
+        assert ei.value.status == -2
+        slot_of, expert_in = abi.moe_pool_slot_table(P.h, 16, 4)
+        assert slot_of[5] == 0 and slot_of[9] == -1 and expert_in == [5, -1, -1, -1]
+        torch.cuda.synchronize()
+        assert P.table.cpu().tolist() == slot_of
+        # retry succeeds and lands the blob
+        abi.moe_expert_pool_load(P.h, ids, 1)
+        slot_of, _ = abi.moe_pool_slot_table(P.h, 16, 4)
+        assert slot_of[9] == 1
+        torch.cuda.synchronize()
+        assert torch.equal(P.dev[1].cpu(), P.host[9])
+    finally:
+        P.close()
