@@ -8,7 +8,9 @@ Default workload: the 80B-like decode stack -- hidden 2048, 512 experts, top-10,
 intermediate 512, shared expert 512, int4 group 64, one token per step through 48
 stacked layers with independent seeded weights, a router bias giving Zipf(1.0)
 popularity, all 512 x 48 experts resident (43.5 GB of blobs).  A step is one token
-through all 48 layers (input of layer l+1 = bf16(x_l + moe_l)).
+through all 48 layers; the input of layer l+1 is bf16(x_0 + moe_l(x_l)) (x_0 = the step's
+token), which keeps the serial dependence between layers and unit-scale activations (a plain
+residual chain x_l + moe_l(x_l) grows without bound under random weights).
 
 Timing: W untimed warm-up steps, then K steps timed with CUDA events on the launching
 stream, bracketed by a barrier and a device synchronize; the max over ranks is taken.
@@ -137,6 +139,11 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def event_ms(a: torch.cuda.Event, b: torch.cuda.Event) -> float:
+    """Elapsed ms between two events (recorded by the library's profiling hook)."""
+    return float(a.elapsed_time(b))
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -190,7 +197,7 @@ class DecodeStack:
         a, w = self.abi, self.w
         for l, L in enumerate(self.layers):
             a.moe_layer_forward(self.shape, self.bufs[l], self.T, L.w_router, L.router_bias, None, None, L.pool,
-                                self.slot_table, w.n_experts, L.shared, L.w_sg, self.bufs[l], self.bufs[l + 1],
+                                self.slot_table, w.n_experts, L.shared, L.w_sg, self.bufs[0], self.bufs[l + 1],
                                 self.idx[l], self.p[l], self.ws)
 
     def unique_experts(self):
@@ -256,26 +263,30 @@ def run_decode(args, w, T, device, rank, ws_n):
     uniq = st.unique_experts()
     flags = abi.moe_ws_check(st.ws, stream)
 
-    # per-kernel durations: the same step with the profiling hook, graph-captured
+    # per-kernel durations: the same step, eager, with the library's profiling hook recording
+    # events around each kernel on the launching stream.  A GPU sleep issued first lets the
+    # host enqueue the whole step before the device reaches it, so consecutive launches run
+    # back to back as in the graph; each interval is one kernel plus its launch gap.
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(w.layers)]
-    g2 = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g2, stream=stream):
-        for l, L in enumerate(st.layers):
-            abi.moe_profile_events(evs[l], 3)
-            abi.moe_layer_forward(st.shape, st.bufs[l], T, L.w_router, L.router_bias, None, None, L.pool,
-                                  st.slot_table, w.n_experts, L.shared, L.w_sg, st.bufs[l], st.bufs[l + 1],
-                                  st.idx[l], st.p[l], st.ws)
-        abi.moe_profile_events(None)
+    for row in evs:  # torch creates the CUDA event lazily, on its first record
+        for ev in row:
+            ev.record(stream)
     kern_ms = {0: [], 1: [], 2: []}
-    reps = 5
+    reps = 3
     for r in range(reps):
         with torch.cuda.stream(stream):
             st.bufs[0].copy_(st.inputs[r % (K + W)], non_blocking=True)
-            g2.replay()
+            torch.cuda._sleep(100_000_000)
+            for l, L in enumerate(st.layers):
+                abi.moe_profile_events(evs[l], 3)
+                abi.moe_layer_forward(st.shape, st.bufs[l], T, L.w_router, L.router_bias, None, None, L.pool,
+                                      st.slot_table, w.n_experts, L.shared, L.w_sg, st.bufs[0], st.bufs[l + 1],
+                                      st.idx[l], st.p[l], st.ws)
+            abi.moe_profile_events(None)
         stream.synchronize()
         for l in range(w.layers):
             for kk in range(3):
-                kern_ms[kk].append(evs[l][2 * kk].elapsed_time(evs[l][2 * kk + 1]))
+                kern_ms[kk].append(event_ms(evs[l][2 * kk], evs[l][2 * kk + 1]))
     kern_avg_us = {kk: 1e3 * statistics.mean(v) for kk, v in kern_ms.items()}
 
     # end to end through the public call with host buffers: pinned H2D of the token(s),
@@ -311,6 +322,7 @@ def cpu_baseline_decode(w, T, device, stack, budget_s=12.0):
     Copying the layer's bytes to the host is not timed."""
     import oracle
     x = stack.inputs[0]
+    x0b = _bits(x)
     t_total, n = 0.0, 0
     for l in range(w.layers):
         L = stack.layers[l]
@@ -321,7 +333,7 @@ def cpu_baseline_decode(w, T, device, stack, budget_s=12.0):
         blobs = {int(e): L.pool[int(e)].cpu().numpy() for e in set(pre.reshape(-1).tolist())}
         t0 = time.perf_counter()
         r = oracle.layer_forward(xb, wr, b, w.top_k, lambda e: blobs[e], shared, wsg, w.hidden, w.inter,
-                                 w.shared_inter, w.bits, residual_bits=xb)
+                                 w.shared_inter, w.bits, residual_bits=x0b)
         t_total += time.perf_counter() - t0
         n += 1
         x = torch.from_numpy(oracle.f64_to_bf16_bits(r["out"]).view(np.int16)).view(torch.bfloat16).to(device)

@@ -73,15 +73,16 @@ def test_full_size_layer_parity(wname, T, layers):
 
 
 def test_stacked_layers_chain_80b():
-    """Three chained 80B-like layers (input of layer l+1 = bf16(x_l + moe_l)); each layer is
-    checked against the oracle on the GPU's own x_l, so rounding does not compound into
-    routing flips."""
+    """Three chained 80B-like layers as the benchmark chains them (input of layer l+1 =
+    bf16(x_0 + moe_l(x_l))); each layer is checked against the oracle on the GPU's own x_l,
+    so rounding does not compound into routing flips."""
     w = synth.WORKLOADS["decode80b"]
-    x = synth.activations(w, 7, device=DEV)
+    x0 = synth.activations(w, 7, device=DEV)
+    x = x0
     for l in range(3):
         L = synth.make_layer(w, l, DEV)
-        out, idx, p, ws = forward(w, L, x, residual=x)
-        ref = oracle_forward(w, L, x, residual=x)
+        out, idx, p, ws = forward(w, L, x, residual=x0)
+        ref = oracle_forward(w, L, x, residual=x0)
         assert_routing(idx, ref["idx"], ref["logits"])
         assert_close(out, ref["out"])
         x = out
