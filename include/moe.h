@@ -150,6 +150,39 @@ MOE_API moe_status moe_layer_forward(const moe_shape* shape, const void* x, int3
                              float* topk_w_out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * moe_layer_forward_static -- moe_layer_forward for callers that cannot allocate device
+ * memory.  The Swiftlet pages have no counterpart of this call.
+ *
+ * Some callers cannot call cudaMalloc: hosts that fix every device allocation up front
+ * under a memory budget, code that runs where a new allocation would fail or stall the
+ * device, and plain C callers with no device allocator of their own for scratch.  This call
+ * takes the same inputs and outputs as moe_layer_forward (the caller still passes x, the
+ * weights, the pool, the slot table and out) but no workspace.  Its scratch is one fixed
+ * 1 MiB device array inside the library, which every GPU that loads the library holds
+ * until the process exits; the call itself allocates nothing.
+ *   - Shapes whose scratch need (moe_workspace_size) exceeds 1 MiB are rejected with
+ *     MOE_ERR_INVALID and a message; T is limited to 1..8 as on the decode path.
+ *   - The first call on each device looks up that device's scratch address (with the
+ *     device current) and caches it; make that first call before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents: each call
+ *     clears the array's control block (on `stream`, before its kernels) and writes the
+ *     rest before reading it.  Calls whose work overlaps on the GPU (other streams, other
+ *     threads) race on the array and must not be issued.
+ *   - Device-detected errors (bad slot or expert id) are skipped as in moe_layer_forward,
+ *     but cannot be read back: the control block is cleared by the next call.
+ *   - The control-block clear may already be enqueued when a later argument check fails;
+ *     it touches only the library's own array.
+ */
+MOE_API moe_status moe_layer_forward_static(const moe_shape* shape, const void* x, int32_t T,
+                                            const void* w_router, const float* router_bias,
+                                            const int32_t* topk_idx_in, const float* topk_w_in,
+                                            const uint8_t* pool, const int32_t* slot_table,
+                                            int64_t n_slots, const uint8_t* shared_blob,
+                                            const void* w_shared_gate, const void* residual,
+                                            void* out, int32_t* topk_idx_out, float* topk_w_out,
+                                            void* stream);
+
+/*
  * moe_ws_check -- synchronise `stream`, read and clear the workspace's device error word.
  *   *flags (host) receives the MOE_DEVERR_* bits.  Returns MOE_ERR_DEVICE if any bit was
  *   set, MOE_OK otherwise.

@@ -52,6 +52,8 @@ _SIGS = {
     "moe_router_topk": (ctypes.c_int, [ctypes.POINTER(moe_shape), _P, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_layer_forward": (ctypes.c_int, [ctypes.POINTER(moe_shape), _P, _I32, _P, _P, _P, _P, _P, _P, _I64,
                                          _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_layer_forward_static": (ctypes.c_int, [ctypes.POINTER(moe_shape), _P, _I32, _P, _P, _P, _P, _P, _P,
+                                                _I64, _P, _P, _P, _P, _P, _P, _P]),
     "moe_ws_check": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "moe_pool_create": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, _P, _P, _P, ctypes.POINTER(_P)]),
     "moe_expert_pool_load": (ctypes.c_int, [_P, _P, _I32, _P]),
@@ -150,6 +152,15 @@ def moe_layer_forward(shape, x, T, w_router, router_bias, topk_idx_in, topk_w_in
                                    _ptr(shared_blob), _ptr(w_shared_gate), _ptr(residual), _ptr(out),
                                    _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(ws),
                                    ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_layer_forward_static(shape, x, T, w_router, router_bias, topk_idx_in, topk_w_in, pool, slot_table, n_slots,
+                             shared_blob, w_shared_gate, residual, out, topk_idx_out, topk_w_out, stream=None):
+    """moe_layer_forward without a workspace argument (the library's fixed device scratch)."""
+    _check(lib().moe_layer_forward_static(ctypes.byref(shape), _ptr(x), T, _ptr(w_router), _ptr(router_bias),
+                                          _ptr(topk_idx_in), _ptr(topk_w_in), _ptr(pool), _ptr(slot_table),
+                                          n_slots, _ptr(shared_blob), _ptr(w_shared_gate), _ptr(residual),
+                                          _ptr(out), _ptr(topk_idx_out), _ptr(topk_w_out), _stream(stream)))
 
 
 def moe_ws_check(ws, stream=None, raise_on_error: bool = False) -> int:

@@ -1,0 +1,56 @@
+"""moe_layer_forward_static: the workspace-free variant of the layer forward, for callers
+that cannot allocate device memory (their allocations are fixed up front, or allocating
+would fail or stall the device).  It must give the same result as moe_layer_forward with a
+caller workspace, call after call, although every call reuses the library's one scratch
+array.  This file is collected last so that a failure here comes after every other test.
+"""
+import pytest
+import torch
+
+import synth
+from helpers import REL, ABS, forward
+from int4_expert_gemv_router_b200 import abi, build
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build.build()
+
+
+def _static(w, L, x, residual):
+    shape = abi.shape_of(w)
+    T = x.shape[0]
+    out = torch.empty(T, w.hidden, dtype=torch.bfloat16, device=DEV)
+    idx = torch.empty(T, w.top_k, dtype=torch.int32, device=DEV)
+    p = torch.empty(T, w.top_k, dtype=torch.float32, device=DEV)
+    slots = torch.arange(w.n_experts, dtype=torch.int32, device=DEV)
+    abi.moe_layer_forward_static(shape, x, T, L.w_router, L.router_bias, None, None, L.pool, slots, w.n_experts,
+                                 L.shared, L.w_sg, residual, out, idx, p)
+    torch.cuda.synchronize()
+    return out, idx, p
+
+
+@pytest.mark.parametrize("wname,T", [("decode80b", 1), ("decode35b", 8), ("tiny", 4)])
+def test_static_scratch_matches_workspace_path_twice(wname, T):
+    w = synth.WORKLOADS[wname]
+    L = synth.make_layer(w, 0, DEV)
+    for call in range(2):  # two calls in a row share the scratch array
+        x = synth.activations(w, 50 + call, tokens=T, device=DEV)
+        ref_out, ref_idx, ref_p, _ = forward(w, L, x, residual=x)
+        out, idx, p = _static(w, L, x, x)
+        assert torch.equal(idx, ref_idx)
+        assert torch.allclose(p, ref_p, rtol=1e-6, atol=0)
+        r, o = ref_out.float(), out.float()
+        assert (r - o).abs().max().item() <= REL * r.abs().max().item() + ABS
+
+
+def test_static_scratch_rejects_oversized_shape():
+    w = synth.WORKLOADS["tiny"].with_(hidden=4096, inter=1024, shared_inter=1024, n_experts=1024, top_k=32)
+    shape = abi.shape_of(w)
+    t = torch.zeros(16, dtype=torch.uint8, device=DEV)
+    with pytest.raises(abi.MoeError) as ei:
+        abi.moe_layer_forward_static(shape, t, 8, t, None, None, None, t, t, 1, t, t, None, t, None, None)
+    assert ei.value.status == -1 and "static scratch" in str(ei.value)
