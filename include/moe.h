@@ -150,6 +150,42 @@ MOE_API moe_status moe_layer_forward(const moe_shape* shape, const void* x, int3
                              float* topk_w_out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * One layer of a stack for moe_stack_forward (all pointers device pointers, as in
+ * moe_layer_forward).  x may be NULL for layers after the first: the layer then reads the
+ * previous layer's out.
+ */
+typedef struct {
+  const void* x;                /* bf16 [T, H] layer input, or NULL (previous layer's out)   */
+  const void* w_router;         /* bf16 [E, H] (unused when topk_idx_in != NULL)             */
+  const float* router_bias;     /* fp32 [E] or NULL                                          */
+  const int32_t* topk_idx_in;   /* int32 [T, k] or NULL (route inside)                       */
+  const float* topk_w_in;       /* fp32 [T, k] (with topk_idx_in)                            */
+  const uint8_t* pool;          /* u8 [n_slots * stride]                                     */
+  const int32_t* slot_table;    /* int32 [E]                                                 */
+  int64_t n_slots;
+  const uint8_t* shared_blob;   /* shared-expert blob                                        */
+  const void* w_shared_gate;    /* bf16 [H]                                                  */
+  const void* residual;         /* bf16 [T, H] or NULL                                       */
+  void* out;                    /* bf16 [T, H] out                                           */
+  int32_t* topk_idx_out;        /* int32 [T, k] or NULL                                      */
+  float* topk_w_out;            /* fp32 [T, k] or NULL                                       */
+} moe_layer_desc;
+
+/*
+ * moe_stack_forward -- n_layers (1..64) routed-MoE layers in sequence, layer l+1 reading
+ * layer l's output (decode: T = 1..8 tokens; the per-layer token decode loop of the pages,
+ * «Swiftlet — это Swift + Metal рантайм…» paragraph 2, whose speed is bound by dispatch).
+ *   layers (host) array of n_layers descriptors; every layer has the same shape.
+ *   ws, ws_bytes as for moe_layer_forward (one workspace serves every layer).
+ * Same results as calling moe_layer_forward once per layer.  For the shapes it supports
+ * (hidden/inter 256/64, 512/128, 1024/256, 2048/512, 4096/1024; E <= 512) the whole stack
+ * is one persistent cooperative kernel with grid-wide barriers between its phases; other
+ * shapes run layer by layer.
+ */
+MOE_API moe_status moe_stack_forward(const moe_shape* shape, int32_t T, const moe_layer_desc* layers,
+                                     int32_t n_layers, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * moe_layer_forward_static -- moe_layer_forward for callers that cannot allocate device
  * memory.  The Swiftlet pages have no counterpart of this call.
  *

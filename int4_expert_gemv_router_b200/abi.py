@@ -44,6 +44,14 @@ class moe_pool_stats_t(ctypes.Structure):
         return {k: int(getattr(self, k)) for k, _ in self._fields_}
 
 
+class moe_layer_desc(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("w_router", ctypes.c_void_p), ("router_bias", ctypes.c_void_p),
+                ("topk_idx_in", ctypes.c_void_p), ("topk_w_in", ctypes.c_void_p), ("pool", ctypes.c_void_p),
+                ("slot_table", ctypes.c_void_p), ("n_slots", ctypes.c_int64), ("shared_blob", ctypes.c_void_p),
+                ("w_shared_gate", ctypes.c_void_p), ("residual", ctypes.c_void_p), ("out", ctypes.c_void_p),
+                ("topk_idx_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p)]
+
+
 _P = ctypes.c_void_p
 _I32, _I64, _SZ = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
 _SIGS = {
@@ -54,6 +62,8 @@ _SIGS = {
                                          _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_layer_forward_static": (ctypes.c_int, [ctypes.POINTER(moe_shape), _P, _I32, _P, _P, _P, _P, _P, _P,
                                                 _I64, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_stack_forward": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, ctypes.POINTER(moe_layer_desc), _I32, _P,
+                                         _SZ, _P]),
     "moe_ws_check": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "moe_pool_create": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, _P, _P, _P, ctypes.POINTER(_P)]),
     "moe_expert_pool_load": (ctypes.c_int, [_P, _P, _I32, _P]),
@@ -151,6 +161,22 @@ def moe_layer_forward(shape, x, T, w_router, router_bias, topk_idx_in, topk_w_in
                                    _ptr(topk_idx_in), _ptr(topk_w_in), _ptr(pool), _ptr(slot_table), n_slots,
                                    _ptr(shared_blob), _ptr(w_shared_gate), _ptr(residual), _ptr(out),
                                    _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def layer_desc(x=None, w_router=None, router_bias=None, topk_idx_in=None, topk_w_in=None, pool=None,
+               slot_table=None, n_slots=0, shared_blob=None, w_shared_gate=None, residual=None, out=None,
+               topk_idx_out=None, topk_w_out=None) -> moe_layer_desc:
+    """A moe_layer_desc from tensors (None -> NULL)."""
+    return moe_layer_desc(_ptr(x), _ptr(w_router), _ptr(router_bias), _ptr(topk_idx_in), _ptr(topk_w_in), _ptr(pool),
+                          _ptr(slot_table), int(n_slots), _ptr(shared_blob), _ptr(w_shared_gate), _ptr(residual),
+                          _ptr(out), _ptr(topk_idx_out), _ptr(topk_w_out))
+
+
+def moe_stack_forward(shape, T, layers, ws, stream=None):
+    """layers: a list of moe_layer_desc (see layer_desc)."""
+    arr = (moe_layer_desc * len(layers))(*layers)
+    _check(lib().moe_stack_forward(ctypes.byref(shape), T, arr, len(layers), _ptr(ws),
                                    ws.numel() * ws.element_size(), _stream(stream)))
 
 

@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 namespace moe {
@@ -141,6 +142,69 @@ moe_status moe_router_topk(const moe_shape* shape, const void* x, int32_t T, con
   return MOE_OK;
 }
 
+static moe_status run_fused_stack(const moe_shape* shape, int32_t T, const moe_layer_desc* L, int32_t n,
+                                  const DecodeArgs& a, cudaStream_t s) {
+  static FusedArgs f;  // large (kMaxFusedLayers descriptors); filled per call under g_fused_mu
+  static std::mutex g_fused_mu;
+  std::lock_guard<std::mutex> lock(g_fused_mu);
+  memset(&f, 0, sizeof f);
+  f.H = shape->hidden;
+  f.I = shape->inter;
+  f.E = shape->n_experts;
+  f.k = shape->top_k;
+  f.T = T;
+  f.bits = shape->bits;
+  f.n_layers = n;
+  f.L = a.L;
+  f.ctrl = a.ctrl;
+  f.logits = a.logits;
+  f.h = a.h;
+  f.hs = a.hs;
+  for (int l = 0; l < n; ++l) {
+    FusedLayer& d = f.layer[l];
+    d.pool = L[l].pool;
+    d.slot_table = L[l].slot_table;
+    d.n_slots = L[l].n_slots;
+    d.wr = static_cast<const uint16_t*>(L[l].w_router);
+    d.rbias = L[l].router_bias;
+    d.shared = L[l].shared_blob;
+    d.wsg = static_cast<const uint16_t*>(L[l].w_shared_gate);
+    d.x = static_cast<const uint16_t*>(L[l].x ? L[l].x : L[l - 1].out);
+    d.residual = static_cast<const uint16_t*>(L[l].residual);
+    d.out = static_cast<uint16_t*>(L[l].out);
+    d.topk_idx_out = L[l].topk_idx_out;
+    d.topk_w_out = L[l].topk_w_out;
+    d.topk_idx_in = L[l].topk_idx_in;
+    d.topk_w_in = L[l].topk_w_in;
+  }
+  bool ok = true;
+  prof_mark(0, false, s);
+  cudaError_t e = launch_fused_decode(f, s, &ok);
+  if (e != cudaSuccess) return cuda_fail(e, "fused decode launch");
+  if (!ok) return set_error(MOE_ERR_UNSUPPORTED, "no fused decode kernel for this shape");
+  prof_mark(0, true, s);
+  return MOE_OK;
+}
+
+// Argument checks of one layer descriptor (everything but the shape).
+static moe_status check_layer(const moe_shape* shape, const moe_layer_desc* d, bool first) {
+  if (!d->pool || !d->slot_table || !d->shared_blob || !d->w_shared_gate || !d->out)
+    return set_error(MOE_ERR_INVALID, "pool, slot_table, shared_blob, w_shared_gate and out must be non-NULL");
+  if (first && !d->x) return set_error(MOE_ERR_INVALID, "the first layer needs x");
+  if (!d->topk_idx_in && !d->w_router) return set_error(MOE_ERR_INVALID, "w_router is NULL and no topk_idx_in given");
+  if (d->topk_idx_in && !d->topk_w_in) return set_error(MOE_ERR_INVALID, "topk_idx_in given without topk_w_in");
+  if ((d->topk_idx_out == nullptr) != (d->topk_w_out == nullptr))
+    return set_error(MOE_ERR_INVALID, "topk_idx_out and topk_w_out must both be given or both be NULL");
+  if (d->n_slots < 1) return set_error(MOE_ERR_INVALID, "n_slots must be >= 1");
+  if ((d->x && !aligned(d->x, 16)) || !aligned(d->out, 16) || (d->w_router && !aligned(d->w_router, 16)) ||
+      !aligned(d->w_shared_gate, 16) || (d->residual && !aligned(d->residual, 16)))
+    return set_error(MOE_ERR_INVALID, "x, out, w_router, w_shared_gate and residual must be 16-byte aligned");
+  if (!aligned(d->pool, kAlign) || !aligned(d->shared_blob, kAlign))
+    return set_error(MOE_ERR_INVALID, "pool and shared_blob must be 256-byte aligned");
+  (void)shape;
+  return MOE_OK;
+}
+
 moe_status moe_layer_forward(const moe_shape* shape, const void* x, int32_t T, const void* w_router,
                              const float* router_bias, const int32_t* topk_idx_in, const float* topk_w_in,
                              const uint8_t* pool, const int32_t* slot_table, int64_t n_slots,
@@ -182,6 +246,24 @@ moe_status moe_layer_forward(const moe_shape* shape, const void* x, int32_t T, c
   a.out = static_cast<uint16_t*>(out);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
+  if (fused_shape_supported(shape->hidden, shape->inter, shape->bits, shape->n_experts)) {
+    moe_layer_desc d{};
+    d.x = x;
+    d.w_router = w_router;
+    d.router_bias = router_bias;
+    d.topk_idx_in = topk_idx_in;
+    d.topk_w_in = topk_w_in;
+    d.pool = pool;
+    d.slot_table = slot_table;
+    d.n_slots = n_slots;
+    d.shared_blob = shared_blob;
+    d.w_shared_gate = w_shared_gate;
+    d.residual = residual;
+    d.out = out;
+    d.topk_idx_out = topk_idx_out;
+    d.topk_w_out = topk_w_out;
+    return run_fused_stack(shape, T, &d, 1, a, s);
+  }
   prof_mark(0, false, s);
   if (!topk_idx_in) {
     if (topk_idx_out) {
@@ -206,6 +288,35 @@ moe_status moe_layer_forward(const moe_shape* shape, const void* x, int32_t T, c
   e = launch_down_decode(a, shape->bits, s, &ok);
   if (e != cudaSuccess) return cuda_fail(e, "down launch");
   prof_mark(2, true, s);
+  return MOE_OK;
+}
+
+moe_status moe_stack_forward(const moe_shape* shape, int32_t T, const moe_layer_desc* layers, int32_t n_layers,
+                             void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!layers) return set_error(MOE_ERR_INVALID, "layers is NULL");
+  if (n_layers < 1 || n_layers > kMaxFusedLayers)
+    return set_error(MOE_ERR_INVALID, "n_layers must be in [1, %d] (got %d)", kMaxFusedLayers, n_layers);
+  if (shape->shared_inter != shape->inter)
+    return set_error(MOE_ERR_UNSUPPORTED, "this build needs shared_inter == inter");
+  if (!decode_shape_supported(shape->hidden, shape->inter, shape->bits))
+    return set_error(MOE_ERR_UNSUPPORTED, "no decode kernel for hidden=%d inter=%d bits=%d", shape->hidden,
+                     shape->inter, shape->bits);
+  for (int l = 0; l < n_layers; ++l)
+    if ((st = check_layer(shape, &layers[l], l == 0)) != MOE_OK) return st;
+  DecodeArgs a;
+  if ((st = fill_decode_args(shape, T, ws, ws_bytes, &a)) != MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (fused_shape_supported(shape->hidden, shape->inter, shape->bits, shape->n_experts))
+    return run_fused_stack(shape, T, layers, n_layers, a, s);
+  for (int l = 0; l < n_layers; ++l) {
+    const moe_layer_desc& d = layers[l];
+    st = moe_layer_forward(shape, d.x ? d.x : layers[l - 1].out, T, d.w_router, d.router_bias, d.topk_idx_in,
+                           d.topk_w_in, d.pool, d.slot_table, d.n_slots, d.shared_blob, d.w_shared_gate, d.residual,
+                           d.out, d.topk_idx_out, d.topk_w_out, ws, ws_bytes, stream);
+    if (st != MOE_OK) return st;
+  }
   return MOE_OK;
 }
 

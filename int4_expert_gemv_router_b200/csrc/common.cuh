@@ -55,7 +55,9 @@ struct Ctrl {
   uint32_t ticket;  // last-block-done counter of the router (always returns to 0)
   int32_t act_n;    // number of distinct routed experts of the current call
   int32_t n_valid;  // number of (token, k) pairs with a valid expert id
-  uint32_t pad[60];
+  uint32_t bar_count;  // grid barrier of the fused decode kernel: arrivals (returns to 0)
+  uint32_t bar_gen;    // grid barrier generation (monotonic)
+  uint32_t pad[58];
 };
 static_assert(sizeof(Ctrl) == 256, "ctrl block is 256 bytes");
 
@@ -112,11 +114,80 @@ struct DecodeArgs {
   float* hs;                 // [T, Is]   shared-expert intermediate per token
 };
 
+// Shared-memory carve of the fused kernel (byte offsets from the dynamic base), used by the
+// host to size the launch and by the kernel to find its arrays.
+struct FusedSmem {
+  uint32_t xs4, xsum, partial, ids, pw, order, pos_of, act_e, act_slot, act_begin, gate, scratch, cand_v, cand_e,
+      total;
+};
+__host__ __device__ inline FusedSmem fused_smem_layout(int T, int H, int bits, int k, int jmax, int n_stages,
+                                                       int stage_bytes, int n_cons) {
+  FusedSmem m{};
+  size_t off = (size_t)n_stages * stage_bytes;
+  auto carve = [&](size_t bytes) {
+    off = (off + 15) / 16 * 16;
+    const uint32_t at = (uint32_t)off;
+    off += bytes;
+    return at;
+  };
+  const int CC = 128 / bits, NC = H / CC, TK = T * k;
+  m.xs4 = carve((size_t)T * H * 4);
+  m.xsum = carve((size_t)T * NC * 4);
+  m.partial = carve((size_t)(TK + T) * jmax * 4);
+  m.ids = carve((size_t)TK * 4);
+  m.pw = carve((size_t)TK * 4);
+  m.order = carve((size_t)TK * 4);
+  m.pos_of = carve((size_t)TK * 4);
+  m.act_e = carve((size_t)TK * 4);
+  m.act_slot = carve((size_t)TK * 4);
+  m.act_begin = carve((size_t)(TK + 1) * 4);
+  m.gate = carve((size_t)T * 4);
+  m.scratch = carve((size_t)2 * TK * 4);
+  m.cand_v = carve((size_t)n_cons * 32 * 8);
+  m.cand_e = carve((size_t)n_cons * 32 * 4);
+  m.total = (uint32_t)((off + 127) / 128 * 128);
+  return m;
+}
+
+// One layer of a fused decode stack (see decode_fused.cu).
+struct FusedLayer {
+  const uint8_t* pool;
+  const int32_t* slot_table;
+  int64_t n_slots;
+  const uint16_t* wr;
+  const float* rbias;
+  const uint8_t* shared;
+  const uint16_t* wsg;
+  const uint16_t* x;
+  const uint16_t* residual;
+  uint16_t* out;
+  int32_t* topk_idx_out;
+  float* topk_w_out;
+  const int32_t* topk_idx_in;
+  const float* topk_w_in;
+};
+constexpr int kMaxFusedLayers = 64;
+
+struct FusedArgs {
+  int H, I, E, k, T, n_layers, bits;
+  int n_stages, stage_bytes, jmax;
+  FusedSmem sm;  // shared-memory carve (host-computed)
+  BlobLayout L;
+  Ctrl* ctrl;
+  double* logits;
+  float* h;
+  float* hs;
+  FusedLayer layer[kMaxFusedLayers];
+};
+
 // Kernel launchers (decode.cu).  Return cudaError_t of the launch.
 cudaError_t launch_router_decode(const DecodeArgs& a, bool build_plan, cudaStream_t s);
 cudaError_t launch_plan_decode(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_gateup_decode(const DecodeArgs& a, int bits, cudaStream_t s, bool* supported);
 cudaError_t launch_down_decode(const DecodeArgs& a, int bits, cudaStream_t s, bool* supported);
 bool decode_shape_supported(int H, int I, int bits);
+// Fused decode stack (decode_fused.cu).
+bool fused_shape_supported(int H, int I, int bits, int E);
+cudaError_t launch_fused_decode(const FusedArgs& a, cudaStream_t s, bool* supported);
 
 }  // namespace moe

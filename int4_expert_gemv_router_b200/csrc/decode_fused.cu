@@ -1,0 +1,866 @@
+// Fused persistent decode kernel: a stack of routed-MoE layers (T <= 8 tokens) in one
+// cooperative launch on sm_100a.
+//
+// One CTA per SM, 16 warps: warps 0..14 compute, warp 15 streams weights.  Per layer:
+//
+//   phase R  router logits (E rows + the shared-gate row; fp64 sums of exact bf16 products)
+//            and the shared expert's gate/up + SwiGLU rows, spread over every compute warp
+//            of the grid; activations staged once per CTA in shared memory.
+//   -- grid barrier --
+//   phase T  every CTA selects the top-k per token from the logits (threshold + warp
+//            bitonic sort; ties to the lower id), forms the softmax weights and the shared
+//            gate, and groups the (token, k) pairs by expert.  CTA 0 writes the top-k.
+//   phase G  the routed experts' gate/up rows, split evenly over CTAs, stream into a shared-
+//            memory ring through cp.async.bulk (one elected thread of warp 15, mbarrier
+//            transaction counts) and are reduced to h = silu(Wg x) * (Wu x); right behind
+//            them the same warp streams this CTA's rows of every selected expert's down
+//            matrix (and the shared expert's), so they are on chip before they are needed.
+//   -- grid barrier --
+//   phase D  each CTA owns a slice of output rows: per expert one warp multiplies its staged
+//            down rows with the expert's h (registers), the per-pair partial sums meet in
+//            shared memory and are added in a fixed order (top-k slot order, then the shared
+//            expert, then the residual) and rounded to bf16.
+//   -- grid barrier --
+//
+// While a layer runs, warp 15 also prefetches the next layer's routing-independent rows
+// (router matrix and shared expert) into L2 with cp.async.bulk.prefetch.
+//
+// The sums run in a fixed order, so the output bits do not depend on where experts sit in
+// the pool.  Every wait (grid barrier, mbarrier) is bounded: on timeout the kernel sets
+// MOE_DEVERR_TIMEOUT, lets its in-flight copies land and returns.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kFThreads = 512;
+constexpr int kCons = 15;          // compute warps
+constexpr int kConsThreads = kCons * 32;
+constexpr int kProd = 15;          // streaming warp
+constexpr int kMaxStages = 8;
+constexpr int kFusedMaxE = 512;  // experts per layer on the fused path (larger E: unfused kernels)
+constexpr int kLaneE = kFusedMaxE / 32;
+constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s bound on any wait
+
+constexpr int cgcd(int a, int b) { return b == 0 ? a : cgcd(b, a % b); }
+constexpr int clcm(int a, int b) { return a / cgcd(a, b) * b; }
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t tx) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(tx) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for the phase of the given parity to complete.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
+  if (mbar_try_wait(b, parity)) return true;
+  const unsigned long long t0 = now_ns();
+  for (;;) {
+    if (mbar_try_wait(b, parity)) return true;
+    if (now_ns() - t0 > kWaitNs) return false;
+  }
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void bar_cons() { asm volatile("bar.sync 1, %0;" ::"n"(kConsThreads) : "memory"); }
+
+// Grid-wide barrier among the CTAs of a cooperative launch (called by one thread per CTA).
+// Sense by generation: the last arriver resets the count and bumps the generation.
+__device__ bool grid_barrier(Ctrl* c, uint32_t nblocks) {
+  const uint32_t gen = ld_acquire(&c->bar_gen);
+  __threadfence();
+  const uint32_t arrived = atomicAdd(&c->bar_count, 1u);
+  if (arrived == nblocks - 1) {
+    atomicExch(&c->bar_count, 0u);
+    __threadfence();
+    atomicAdd(&c->bar_gen, 1u);
+    return true;
+  }
+  const unsigned long long t0 = now_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (ld_acquire(&c->bar_gen) != gen) {
+      __threadfence();
+      return true;
+    }
+    if ((it & 255u) == 255u && now_ns() - t0 > kWaitNs) {
+      atomicOr(&c->err, kErrTimeout);
+      return false;
+    }
+  }
+}
+
+// Key order of the top-k: larger logit first, ties to the lower id.
+__device__ __forceinline__ bool key_better(double av, int ae, double bv, int be) {
+  return av > bv || (av == bv && ae < be);
+}
+
+// Sorts one key per lane across the warp, best key to lane 0 (bitonic network).
+__device__ __forceinline__ void warp_sort_keys(double& v, int& e) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const double pv = __shfl_xor_sync(0xffffffffu, v, stride);
+      const int pe = __shfl_xor_sync(0xffffffffu, e, stride);
+      const bool keep_better = (((lane & stride) == 0) == ((lane & size) == 0));
+      const bool pb = key_better(pv, pe, v, e);
+      if (keep_better == pb) {
+        v = pv;
+        e = pe;
+      }
+    }
+  }
+}
+
+
+// Top-k of one token's logits by one warp.  Lane i (i < k) receives the i-th best key
+// (sv, se): larger logit first, ties to the lower id.  A threshold (the k-th best of the 32
+// lane maxima bounds the k-th best key from below) leaves few candidates, which one bitonic
+// sort orders; with more than 32 candidates (many equal keys) k rounds of warp arg-max run.
+__device__ __noinline__ void warp_topk(const double* lt, int E, int k, double* cv_base, int* ce_base,
+                                       uint32_t* err, double& sv, int& se) {
+  const int lane = threadIdx.x & 31;
+  double v[kLaneE];
+  double bv = -INFINITY;
+  int be = 0x7fffffff;
+#pragma unroll
+  for (int m = 0; m < kLaneE; ++m) {
+    const int e = lane + 32 * m;
+    double x = -INFINITY;
+    if (e < E) {
+      x = __ldcg(lt + e);
+      if (!(x == x)) {
+        atomicOr(err, kErrNonFinite);
+        x = -INFINITY;
+      }
+    }
+    v[m] = x;
+    if (e < E && key_better(x, e, bv, be)) {
+      bv = x;
+      be = e;
+    }
+  }
+  // threshold: the k-th best lane maximum bounds the k-th best key from below
+  double tv = bv;
+  int te = be;
+  warp_sort_keys(tv, te);
+  const double thr_v = __shfl_sync(0xffffffffu, tv, k - 1);
+  const int thr_e = __shfl_sync(0xffffffffu, te, k - 1);
+  int cnt = 0;
+#pragma unroll
+  for (int m = 0; m < kLaneE; ++m) {
+    const int e = lane + 32 * m;
+    cnt += (e < E && !key_better(thr_v, thr_e, v[m], e)) ? 1 : 0;
+  }
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  if (total <= 32) {
+    double* cv = cv_base;
+    int* ce = ce_base;
+    int pos = incl - cnt;
+#pragma unroll
+    for (int m = 0; m < kLaneE; ++m) {
+      const int e = lane + 32 * m;
+      if (e < E && !key_better(thr_v, thr_e, v[m], e)) {
+        cv[pos] = v[m];
+        ce[pos] = e;
+        ++pos;
+      }
+    }
+    __syncwarp();
+    sv = lane < total ? cv[lane] : -INFINITY;
+    se = lane < total ? ce[lane] : 0x7fffffff;
+    __syncwarp();
+    warp_sort_keys(sv, se);
+  } else {
+    // many near-equal keys: k rounds of warp arg-max over the candidates
+    uint32_t taken = 0;
+    sv = -INFINITY;
+    se = 0x7fffffff;
+    for (int r = 0; r < k; ++r) {
+      double rv = -INFINITY;
+      int re = 0x7fffffff;
+#pragma unroll
+      for (int m = 0; m < kLaneE; ++m) {
+        const int e = lane + 32 * m;
+        if (e < E && !((taken >> m) & 1u) && key_better(v[m], e, rv, re)) {
+          rv = v[m];
+          re = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ov = __shfl_xor_sync(0xffffffffu, rv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, re, o);
+        if (key_better(ov, oe, rv, re)) {
+          rv = ov;
+          re = oe;
+        }
+      }
+      if (re != 0x7fffffff && (re & 31) == lane) taken |= 1u << (re >> 5);
+      if (lane == r) {
+        sv = rv;
+        se = re;
+      }
+    }
+  }
+}
+
+template <int BITS, int H, int I, int TM>
+__global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_constant__ FusedArgs a) {
+  // ---- constants ----
+  constexpr int CC = 128 / BITS, V4 = CC / 4;
+  constexpr int NCg = H / CC, NCLg = NCg < 32 ? NCg : 32, RPWg = 32 / NCLg, CPLg = NCg / NCLg;
+  constexpr int ROWBg = H * BITS / 8, NGg = H / kGroup, SRg = NGg * 2;
+  constexpr int NCd = I / CC, NCLd = NCd < 32 ? NCd : 32, RPWd = 32 / NCLd, CPLd = NCd / NCLd;
+  constexpr int ROWBd = I * BITS / 8, NGd = I / kGroup, SRd = NGd * 2;
+  constexpr int gG = clcm(16 / cgcd(16, SRg), RPWg);
+  constexpr int gD = clcm(16 / cgcd(16, SRd), RPWd);
+  constexpr int ROWG_BYTES = 2 * ROWBg + 4 * SRg;  // one gate/up row with its scales
+  constexpr int ROWD_BYTES = ROWBd + 2 * SRd;      // one down row with its scales
+
+  const int T = a.T, E = a.E, k = a.k, G = gridDim.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int NS = a.n_stages, SB = a.stage_bytes;
+  const int RG = (SB / ROWG_BYTES) / gG * gG;  // gate/up rows per stage
+
+  // ---- shared memory ----
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(8) uint64_t full_bar[kMaxStages], empty_bar[kMaxStages], plan_bar;
+  __shared__ int s_act_n, s_n_valid, s_abort;
+  uint8_t* ring = smem;
+  float4* xs4 = reinterpret_cast<float4*>(smem + a.sm.xs4);
+  float* xsum = reinterpret_cast<float*>(smem + a.sm.xsum);
+  float* partial = reinterpret_cast<float*>(smem + a.sm.partial);  // [(T*k + T) * jmax]
+  const int TK = T * k;
+#define P_IDS reinterpret_cast<int*>(smem + a.sm.ids)
+#define P_PW reinterpret_cast<float*>(smem + a.sm.pw)
+#define P_ORDER reinterpret_cast<int*>(smem + a.sm.order)
+#define P_POS reinterpret_cast<int*>(smem + a.sm.pos_of)
+#define P_ACTE reinterpret_cast<int*>(smem + a.sm.act_e)
+#define P_SLOT reinterpret_cast<int*>(smem + a.sm.act_slot)
+#define P_BEGIN reinterpret_cast<int*>(smem + a.sm.act_begin)
+#define P_GATE reinterpret_cast<float*>(smem + a.sm.gate)
+#define P_SCRATCH reinterpret_cast<int*>(smem + a.sm.scratch)
+#define P_CANDV reinterpret_cast<double*>(smem + a.sm.cand_v)
+#define P_CANDE reinterpret_cast<int*>(smem + a.sm.cand_e)
+
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kCons);
+    }
+    mbar_init(&plan_bar, 1);
+    s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  // This CTA's slice of output rows (phase D), in granules of gD rows.
+  const int nGranD = H / gD;
+  const int j0 = (int)((long long)blockIdx.x * nGranD / G) * gD;
+  const int j1 = (int)((long long)(blockIdx.x + 1) * nGranD / G) * gD;
+  const int nJ = j1 - j0;
+
+  // =====================================================================================
+  // streaming warp
+  // =====================================================================================
+  if (warp == kProd) {
+    uint32_t q = 0;  // stage sequence number, shared convention with the compute warps
+    bool ok = true;
+    for (int l = 0; l < a.n_layers && ok; ++l) {
+      const FusedLayer& Lc = a.layer[l];
+      // L2 prefetch of the next layer's routing-independent rows this CTA's warps will read
+      if (l + 1 < a.n_layers && lane == 0) {
+        const FusedLayer& Ln = a.layer[l + 1];
+        const int n_router = (Ln.topk_idx_in ? 0 : E) + 1;
+        const int n_items = n_router + I / RPWg;
+        for (int it = blockIdx.x * kCons; it < min(n_items, (blockIdx.x + 1) * kCons); ++it) {
+          if (it < n_router) {
+            const bool gate_row = (it == n_router - 1);
+            const uint16_t* row = gate_row ? Ln.wsg : Ln.wr + (size_t)it * H;
+            prefetch_l2(row, H * 2);
+          } else {
+            const int r = (it - n_router) * RPWg;
+            prefetch_l2(Ln.shared + a.L.off[0] + (int64_t)r * ROWBg, RPWg * ROWBg);
+            prefetch_l2(Ln.shared + a.L.off[1] + (int64_t)r * ROWBg, RPWg * ROWBg);
+          }
+        }
+      }
+      // wait for this layer's plan
+      if (!mbar_wait(&plan_bar, l & 1)) {
+        ok = false;
+        break;
+      }
+      if (*(volatile int*)&s_abort) break;
+      const int act_n = s_act_n;
+      // ---- phase G pieces ----
+      const int nGranG = act_n * I / gG;
+      const int f0 = (int)((long long)blockIdx.x * nGranG / G) * gG;
+      const int f1 = (int)((long long)(blockIdx.x + 1) * nGranG / G) * gG;
+      for (int f = f0; f < f1 && ok;) {
+        const int u = f / I, r0 = f - u * I;
+        const int n = min(min(RG, f1 - f), I - r0);
+        const int s = q % NS;
+        if (!mbar_wait(&empty_bar[s], ((q / NS) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          uint8_t* st = ring + (size_t)s * SB;
+          const int slot = P_SLOT[u];
+          if (slot < 0) {
+            mbar_arrive(&full_bar[s]);
+          } else {
+            const uint8_t* b = Lc.pool + (int64_t)slot * a.L.stride;
+            mbar_expect_tx(&full_bar[s], (uint32_t)(n * ROWG_BYTES));
+            bulk_g2s(st, b + a.L.off[0] + (int64_t)r0 * ROWBg, n * ROWBg, &full_bar[s]);
+            bulk_g2s(st + n * ROWBg, b + a.L.off[1] + (int64_t)r0 * ROWBg, n * ROWBg, &full_bar[s]);
+            uint8_t* sc = st + 2 * n * ROWBg;
+            for (int z = 0; z < 4; ++z)
+              bulk_g2s(sc + z * n * SRg, b + a.L.off[3 + z] + (int64_t)r0 * SRg, n * SRg, &full_bar[s]);
+          }
+        }
+        __syncwarp();
+        ++q;
+        f += n;
+      }
+      // ---- phase D pieces: this CTA's down rows of every selected expert, then the shared one ----
+      if (nJ > 0) {
+        const int per_stage = SB / (nJ * ROWD_BYTES);
+        for (int u = 0; u <= act_n && ok;) {
+          const int cnt = min(per_stage, act_n + 1 - u);
+          const int s = q % NS;
+          if (!mbar_wait(&empty_bar[s], ((q / NS) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            uint8_t* st = ring + (size_t)s * SB;
+            uint32_t bytes = 0;
+            for (int z = 0; z < cnt; ++z) {
+              const int uu = u + z;
+              const int slot = (uu < act_n) ? P_SLOT[uu] : 0;
+              if (uu < act_n && slot < 0) continue;
+              bytes += nJ * ROWD_BYTES;
+            }
+            mbar_expect_tx(&full_bar[s], bytes);
+            for (int z = 0; z < cnt; ++z) {
+              const int uu = u + z;
+              const uint8_t* b;
+              if (uu < act_n) {
+                const int slot = P_SLOT[uu];
+                if (slot < 0) continue;
+                b = Lc.pool + (int64_t)slot * a.L.stride;
+              } else {
+                b = Lc.shared;
+              }
+              uint8_t* d = st + (size_t)z * nJ * ROWD_BYTES;
+              bulk_g2s(d, b + a.L.off[2] + (int64_t)j0 * ROWBd, nJ * ROWBd, &full_bar[s]);
+              bulk_g2s(d + nJ * ROWBd, b + a.L.off[7] + (int64_t)j0 * SRd, nJ * SRd, &full_bar[s]);
+              bulk_g2s(d + nJ * ROWBd + nJ * SRd, b + a.L.off[8] + (int64_t)j0 * SRd, nJ * SRd, &full_bar[s]);
+            }
+          }
+          __syncwarp();
+          ++q;
+          u += cnt;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      atomicOr(&a.ctrl->err, kErrTimeout);
+      s_abort = 1;
+    }
+    // let every issued copy land before the CTA may exit
+    if (lane == 0) {
+      const uint32_t first = q > (uint32_t)NS ? q - NS : 0;
+      for (uint32_t qq = first; qq < q; ++qq) mbar_wait(&full_bar[qq % NS], (qq / NS) & 1);
+    }
+    return;
+  }
+
+  // =====================================================================================
+  // compute warps
+  // =====================================================================================
+  const int cw = warp;  // 0..14
+  const int gw = blockIdx.x * kCons + cw, NW = G * kCons;
+  uint32_t q = 0;
+  bool ok = true;
+
+  for (int l = 0; l < a.n_layers; ++l) {
+    const FusedLayer& Lc = a.layer[l];
+    const bool routed = (Lc.topk_idx_in == nullptr);
+
+    // ---- stage x: chunk-interleaved, pre-scaled fp32 + chunk sums ----
+    stage_vectors<BITS, H>(xs4, xsum, T, tid, kConsThreads, [&](int r, int i) {
+      const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(Lc.x + (size_t)r * H + i));
+      return make_float4(bf_lo(raw.x), bf_hi(raw.x), bf_lo(raw.y), bf_hi(raw.y));
+    });
+    bar_cons();
+
+    // ---- phase R: router rows, shared-gate row, shared gate/up rows ----
+    {
+      const int n_router = (routed ? E : 0) + 1;
+      const int n_items = n_router + I / RPWg;
+      for (int it = gw; it < n_items; it += NW) {
+        if (it < n_router) {
+          const bool gate_row = (it == n_router - 1);
+          const int e = gate_row ? E : it;
+          const uint16_t* row = gate_row ? Lc.wsg : Lc.wr + (size_t)e * H;
+          double acc[TM];
+#pragma unroll
+          for (int t = 0; t < TM; ++t) acc[t] = 0.0;
+          for (int c8 = lane; c8 < H / 8; c8 += 32) {
+            const uint4 w = ld_stream(row + c8 * 8);
+            const float wv[8] = {bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y),
+                                 bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w)};
+            const int c = c8 / (CC / 8), v0 = (c8 % (CC / 8)) * 2;
+#pragma unroll
+            for (int t = 0; t < TM; ++t) {
+              if (t < T) {
+                const float4 xa = xs4[((size_t)t * V4 + v0) * NCg + c];
+                const float4 xb = xs4[((size_t)t * V4 + v0 + 1) * NCg + c];
+                const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+                double s = 0.0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  // undo the staging scale (a power of two): the product stays exact
+                  const float xr = xv[i] * stage_unscale<BITS>(v0 * 4 + i);
+                  s += (double)(wv[i] * xr);
+                }
+                acc[t] += s;
+              }
+            }
+          }
+#pragma unroll
+          for (int t = 0; t < TM; ++t) {
+            if (t < T) {
+              double v = acc[t];
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+              if (lane == 0) {
+                if (!gate_row && Lc.rbias) v += (double)Lc.rbias[e];
+                a.logits[(size_t)t * (E + 1) + e] = v;
+              }
+            }
+          }
+        } else {
+          // shared expert gate/up row(s)
+          const int r = (it - n_router) * RPWg + lane / NCLg;
+          const int sub = lane % NCLg;
+          const uint8_t* b = Lc.shared;
+          uint4 qg[CPLg], qu[CPLg];
+          float sg[CPLg], bg[CPLg], su[CPLg], bu[CPLg];
+#pragma unroll
+          for (int m = 0; m < CPLg; ++m) {
+            const int c = sub + NCLg * m, g = c * CC / kGroup;
+            qg[m] = ld_stream(b + a.L.off[0] + (int64_t)r * ROWBg + c * 16);
+            qu[m] = ld_stream(b + a.L.off[1] + (int64_t)r * ROWBg + c * 16);
+            sg[m] = bf1(ld_u16(b + a.L.off[3] + (int64_t)r * SRg + g * 2));
+            bg[m] = bf1(ld_u16(b + a.L.off[4] + (int64_t)r * SRg + g * 2));
+            su[m] = bf1(ld_u16(b + a.L.off[5] + (int64_t)r * SRg + g * 2));
+            bu[m] = bf1(ld_u16(b + a.L.off[6] + (int64_t)r * SRg + g * 2));
+          }
+          for (int t = 0; t < T; ++t) {
+            float ag = 0.f, au = 0.f;
+#pragma unroll
+            for (int m = 0; m < CPLg; ++m) {
+              const int c = sub + NCLg * m;
+              float dg, du;
+              dot_chunk2<BITS>(qg[m], qu[m], xs4 + (size_t)t * V4 * NCg + c, NCg, dg, du);
+              const float xc = xsum[t * NCg + c];
+              ag = fmaf(sg[m], dg, fmaf(bg[m], xc, ag));
+              au = fmaf(su[m], du, fmaf(bu[m], xc, au));
+            }
+#pragma unroll
+            for (int o = NCLg / 2; o > 0; o >>= 1) {
+              ag += __shfl_xor_sync(0xffffffffu, ag, o);
+              au += __shfl_xor_sync(0xffffffffu, au, o);
+            }
+            if (sub == 0) a.hs[(size_t)t * I + r] = ag / (1.0f + expf(-ag)) * au;
+          }
+        }
+      }
+    }
+    bar_cons();
+    if (tid == 0 && !grid_barrier(a.ctrl, G)) s_abort = 1;
+    bar_cons();
+    if (s_abort) ok = false;
+
+    // ---- phase T: top-k, softmax, shared gate, grouping (every CTA) ----
+    if (ok) {
+      for (int t = cw; t < T; t += kCons) {
+        const double* lt = a.logits + (size_t)t * (E + 1);
+        if (routed) {
+          double sv;
+          int se;
+          warp_topk(lt, E, k, P_CANDV + cw * 32, P_CANDE + cw * 32, &a.ctrl->err, sv, se);
+          // lanes 0..k-1 hold the selection in order
+          const double v0 = __shfl_sync(0xffffffffu, sv, 0);
+          const bool valid = lane < k && se != 0x7fffffff && sv != -INFINITY;
+          const double ex = valid ? exp(sv - v0) : 0.0;
+          double den = ex;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+          if (lane < k) {
+            if (!valid) atomicOr(&a.ctrl->err, kErrNonFinite);
+            const int id = valid ? se : -1;
+            const float pw = valid ? (float)(ex / den) : 0.f;
+            P_IDS[t * k + lane] = id;
+            P_PW[t * k + lane] = pw;
+            if (blockIdx.x == 0 && Lc.topk_idx_out) {
+              Lc.topk_idx_out[t * k + lane] = id;
+              Lc.topk_w_out[t * k + lane] = pw;
+            }
+          }
+        } else if (lane < k) {
+          P_IDS[t * k + lane] = Lc.topk_idx_in[t * k + lane];
+          P_PW[t * k + lane] = Lc.topk_w_in[t * k + lane];
+        }
+        if (lane == 0) P_GATE[t] = (float)(1.0 / (1.0 + exp(-__ldcg(lt + E))));
+      }
+    }
+    bar_cons();
+    // grouping: pairs sorted by (expert, pair number); invalid ids left out
+    if (ok) {
+      int* key = P_SCRATCH;
+      int* first = P_SCRATCH + TK;
+      for (int i = tid; i < TK; i += kConsThreads) {
+        const int e = P_IDS[i];
+        const bool valid = e >= 0 && e < E;
+        if (!valid && blockIdx.x == 0) atomicOr(&a.ctrl->err, kErrBadExpert);
+        key[i] = valid ? e : E;
+      }
+      bar_cons();
+      for (int i = tid; i < TK; i += kConsThreads) {
+        const int ki = key[i];
+        int rank = 0, fst = 1;
+        for (int j = 0; j < TK; ++j) {
+          const int kj = key[j];
+          rank += (kj < ki) || (kj == ki && j < i);
+          if (kj == ki && j < i) fst = 0;
+        }
+        P_ORDER[rank] = i;
+        P_POS[i] = (ki < E) ? rank : -1;
+        first[i] = (fst && ki < E) ? 1 : 0;
+      }
+      bar_cons();
+      for (int i = tid; i < TK; i += kConsThreads) {
+        if (first[i]) {
+          const int ki = key[i];
+          int act = 0, before = 0;
+          for (int j = 0; j < TK; ++j) {
+            act += (first[j] && key[j] < ki);
+            before += (key[j] < ki);
+          }
+          P_ACTE[act] = ki;
+          P_BEGIN[act] = before;
+          const int slot = Lc.slot_table[ki];
+          const bool sok = slot >= 0 && slot < Lc.n_slots;
+          if (!sok) atomicOr(&a.ctrl->err, kErrBadSlot);
+          P_SLOT[act] = sok ? slot : -1;
+        }
+      }
+      if (tid == 0) {
+        int an = 0, nv = 0;
+        for (int i = 0; i < TK; ++i) {
+          an += first[i];
+          nv += key[i] < E;
+        }
+        s_act_n = an;
+        s_n_valid = nv;
+        P_BEGIN[an] = nv;
+      }
+    }
+    bar_cons();
+    if (tid == 0) mbar_arrive(&plan_bar);  // the streaming warp may issue this layer's pieces
+    if (!ok) break;
+    const int act_n = s_act_n, n_valid = s_n_valid;
+
+    // ---- phase G: routed gate/up + SwiGLU from the ring ----
+    {
+      const int nGranG = act_n * I / gG;
+      const int f0 = (int)((long long)blockIdx.x * nGranG / G) * gG;
+      const int f1 = (int)((long long)(blockIdx.x + 1) * nGranG / G) * gG;
+      const int sub = lane % NCLg, rsub = lane / NCLg;
+      for (int f = f0; f < f1;) {
+        const int u = f / I, r0 = f - u * I;
+        const int n = min(min(RG, f1 - f), I - r0);
+        const int s = q % NS;
+        if (!mbar_wait(&full_bar[s], (q / NS) & 1)) {
+          ok = false;
+          atomicOr(&a.ctrl->err, kErrTimeout);
+          break;
+        }
+        const uint8_t* st = ring + (size_t)s * SB;
+        if (P_SLOT[u] >= 0) {
+          const int pb = P_BEGIN[u], pe = P_BEGIN[u + 1];
+          for (int step = cw; step < n / RPWg; step += kCons) {
+            const int rl = step * RPWg + rsub;
+            const uint8_t* gq = st + rl * ROWBg;
+            const uint8_t* uq = st + n * ROWBg + rl * ROWBg;
+            const uint8_t* sc = st + 2 * n * ROWBg + rl * SRg;
+            uint4 qg[CPLg], qu[CPLg];
+            float sg[CPLg], bg[CPLg], su[CPLg], bu[CPLg];
+#pragma unroll
+            for (int m = 0; m < CPLg; ++m) {
+              const int c = sub + NCLg * m, g = c * CC / kGroup;
+              qg[m] = *reinterpret_cast<const uint4*>(gq + c * 16);
+              qu[m] = *reinterpret_cast<const uint4*>(uq + c * 16);
+              sg[m] = bf1(*reinterpret_cast<const uint16_t*>(sc + g * 2));
+              bg[m] = bf1(*reinterpret_cast<const uint16_t*>(sc + n * SRg + g * 2));
+              su[m] = bf1(*reinterpret_cast<const uint16_t*>(sc + 2 * n * SRg + g * 2));
+              bu[m] = bf1(*reinterpret_cast<const uint16_t*>(sc + 3 * n * SRg + g * 2));
+            }
+            for (int p = pb; p < pe; ++p) {
+              const int t = P_ORDER[p] / k;
+              float ag = 0.f, au = 0.f;
+#pragma unroll
+              for (int m = 0; m < CPLg; ++m) {
+                const int c = sub + NCLg * m;
+                float dg, du;
+                dot_chunk2<BITS>(qg[m], qu[m], xs4 + (size_t)t * V4 * NCg + c, NCg, dg, du);
+                const float xc = xsum[t * NCg + c];
+                ag = fmaf(sg[m], dg, fmaf(bg[m], xc, ag));
+                au = fmaf(su[m], du, fmaf(bu[m], xc, au));
+              }
+#pragma unroll
+              for (int o = NCLg / 2; o > 0; o >>= 1) {
+                ag += __shfl_xor_sync(0xffffffffu, ag, o);
+                au += __shfl_xor_sync(0xffffffffu, au, o);
+              }
+              if (sub == 0) a.h[(size_t)p * I + r0 + rl] = ag / (1.0f + expf(-ag)) * au;
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[s]);
+        ++q;
+        f += n;
+      }
+    }
+    bar_cons();
+    if (tid == 0 && (!ok || !grid_barrier(a.ctrl, G))) s_abort = 1;
+    bar_cons();
+    if (s_abort) break;
+
+    // ---- phase D: down rows j0..j1 of every selected expert and the shared expert ----
+    if (nJ > 0) {
+      const int per_stage = SB / (nJ * ROWD_BYTES);
+      const int sub = lane % NCLd, rsub = lane / NCLd;
+      for (int u0 = 0; u0 <= act_n;) {
+        const int cnt = min(per_stage, act_n + 1 - u0);
+        const int s = q % NS;
+        if (!mbar_wait(&full_bar[s], (q / NS) & 1)) {
+          ok = false;
+          atomicOr(&a.ctrl->err, kErrTimeout);
+          break;
+        }
+        const uint8_t* st = ring + (size_t)s * SB;
+        for (int z = cw; z < cnt; z += kCons) {
+          const int u = u0 + z;
+          const bool shared = (u == act_n);
+          const uint8_t* dq = st + (size_t)z * nJ * ROWD_BYTES;
+          const uint8_t* ds = dq + nJ * ROWBd;
+          const uint8_t* db = ds + nJ * SRd;
+          const bool have = shared || P_SLOT[u] >= 0;
+          const int pb = shared ? n_valid : P_BEGIN[u];
+          const int pe = shared ? n_valid + T : P_BEGIN[u + 1];
+          for (int p = pb; p < pe; ++p) {
+            int t;
+            float w;
+            const float* hsrc;
+            if (!shared) {
+              const int nn = P_ORDER[p];
+              t = nn / k;
+              w = P_PW[nn];
+              hsrc = a.h + (size_t)p * I;
+            } else {
+              t = p - n_valid;
+              w = P_GATE[t];
+              hsrc = a.hs + (size_t)t * I;
+            }
+            (void)t;
+            // this pair's h chunks in registers, pre-scaled like staged activations
+            float4 hr[CPLd][V4];
+            float hsum[CPLd];
+#pragma unroll
+            for (int m = 0; m < CPLd; ++m) {
+              const int c = sub + NCLd * m;
+              float sum = 0.f;
+#pragma unroll
+              for (int v = 0; v < V4; ++v) {
+                const float4 f4 = __ldcg(reinterpret_cast<const float4*>(hsrc + c * CC + 4 * v));
+                sum += (f4.x + f4.y) + (f4.z + f4.w);
+                hr[m][v] = make_float4(f4.x * stage_scale<BITS>(4 * v), f4.y * stage_scale<BITS>(4 * v + 1),
+                                       f4.z * stage_scale<BITS>(4 * v + 2), f4.w * stage_scale<BITS>(4 * v + 3));
+              }
+              hsum[m] = sum;
+            }
+            for (int rs = 0; rs < nJ / RPWd; ++rs) {
+              const int jl = rs * RPWd + rsub;
+              float part = 0.f;
+              if (have) {
+#pragma unroll
+                for (int m = 0; m < CPLd; ++m) {
+                  const int c = sub + NCLd * m, g = c * CC / kGroup;
+                  const uint4 qd = *reinterpret_cast<const uint4*>(dq + jl * ROWBd + c * 16);
+                  const float sd = bf1(*reinterpret_cast<const uint16_t*>(ds + jl * SRd + g * 2));
+                  const float bd = bf1(*reinterpret_cast<const uint16_t*>(db + jl * SRd + g * 2));
+                  const float d = dot_chunk<BITS>(qd, hr[m], 1);
+                  part = fmaf(sd, d, fmaf(bd, hsum[m], part));
+                }
+              }
+#pragma unroll
+              for (int o = NCLd / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+              if (sub == 0) partial[(size_t)p * a.jmax + jl] = w * part;
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[s]);
+        ++q;
+        u0 += cnt;
+      }
+      bar_cons();
+      // combine in a fixed order: top-k slots, then the shared expert, then the residual
+      if (ok) {
+        for (int i = tid; i < T * nJ; i += kConsThreads) {
+          const int t = i / nJ, jl = i - t * nJ;
+          float v = 0.f;
+          for (int kk = 0; kk < k; ++kk) {
+            const int p = P_POS[t * k + kk];
+            if (p >= 0) v += partial[(size_t)p * a.jmax + jl];
+          }
+          v += partial[(size_t)(n_valid + t) * a.jmax + jl];
+          if (Lc.residual) v += bf1(__ldcg(Lc.residual + (size_t)t * H + j0 + jl));
+          Lc.out[(size_t)t * H + j0 + jl] = f2bf(v);
+        }
+      }
+    }
+    bar_cons();
+    if (tid == 0 && (!ok || !grid_barrier(a.ctrl, G))) s_abort = 1;
+    bar_cons();
+    if (s_abort) break;
+  }
+  // on an early exit make sure the streaming warp is not left waiting for a plan
+  if (tid == 0 && s_abort) {
+    s_abort = 1;
+    mbar_arrive(&plan_bar);
+  }
+}
+
+}  // namespace
+
+static size_t fused_smem_bytes(const FusedArgs& a, int stages) {
+  return fused_smem_layout(a.T, a.H, a.bits, a.k, a.jmax, stages, a.stage_bytes, kCons).total;
+}
+
+template <int BITS, int H, int I, int TM>
+static cudaError_t run_fused(FusedArgs a, cudaStream_t s) {
+  static int n_sm = 0;
+  if (!n_sm) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  }
+  int max_smem = 0, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  max_smem -= 2048;  // static shared memory and reserve
+  // output-row slice of a CTA (granule gD rows)
+  constexpr int CC = 128 / BITS, NCd = I / CC, NCLd = NCd < 32 ? NCd : 32, RPWd = 32 / NCLd;
+  constexpr int SRd = (I / kGroup) * 2;
+  constexpr int gD = clcm(16 / cgcd(16, SRd), RPWd);
+  const int nGran = H / gD;
+  a.jmax = ((nGran + n_sm - 1) / n_sm) * gD;
+  a.stage_bytes = 32768;
+  int stages = kMaxStages;
+  while (stages > 2 && fused_smem_bytes(a, stages) > (size_t)max_smem) --stages;
+  a.n_stages = stages;
+  a.sm = fused_smem_layout(a.T, a.H, a.bits, a.k, a.jmax, stages, a.stage_bytes, kCons);
+  const size_t smem = a.sm.total;
+  if (smem > (size_t)max_smem) return cudaErrorInvalidConfiguration;
+  // one stage must hold one gate/up row and one expert's down slice
+  if ((size_t)a.jmax * ((I * BITS / 8) + 2 * SRd) > (size_t)a.stage_bytes) return cudaErrorInvalidConfiguration;
+  auto fn = k_fused_decode<BITS, H, I, TM>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int bps = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, fn, kFThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (bps < 1) return cudaErrorInvalidConfiguration;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_sm);
+  cfg.blockDim = dim3(kFThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fn, a);
+}
+
+bool fused_shape_supported(int H, int I, int bits, int E) {
+  return E <= kFusedMaxE && (bits == 4 || bits == 8) && ((H == 2048 && I == 512) || (H == 256 && I == 64) ||
+                                      (H == 512 && I == 128) || (H == 1024 && I == 256) ||
+                                      (H == 4096 && I == 1024));
+}
+
+cudaError_t launch_fused_decode(const FusedArgs& a, cudaStream_t s, bool* supported) {
+  *supported = true;
+#define MOE_FD(B, HH, II)                                            \
+  if (a.bits == B && a.H == HH && a.I == II) {                       \
+    if (a.T == 1) return run_fused<B, HH, II, 1>(a, s);              \
+    return run_fused<B, HH, II, kMaxDecodeT>(a, s);                  \
+  }
+  MOE_FD(4, 2048, 512) MOE_FD(8, 2048, 512) MOE_FD(4, 256, 64) MOE_FD(8, 256, 64)
+  MOE_FD(4, 512, 128) MOE_FD(8, 512, 128) MOE_FD(4, 1024, 256) MOE_FD(8, 1024, 256)
+  MOE_FD(4, 4096, 1024) MOE_FD(8, 4096, 1024)
+#undef MOE_FD
+  *supported = false;
+  return cudaSuccess;
+}
+
+}  // namespace moe

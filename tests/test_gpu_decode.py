@@ -148,3 +148,55 @@ def test_device_error_flags():
     ref = oracle_forward(w, L, x, idx=np.where(bad.cpu().numpy() < w.n_experts, bad.cpu().numpy(), 0),
                          p=np.where(bad.cpu().numpy() < w.n_experts, p.cpu().numpy(), 0.0))
     assert_close(out, ref["out"])
+
+
+def test_stack_forward_equals_layer_by_layer():
+    """moe_stack_forward (one launch for the stack) gives the same bits as one
+    moe_layer_forward per layer, and each layer matches the oracle on its own input."""
+    w = synth.WORKLOADS["decode80b"].with_(layers=3)
+    T = 1
+    layers = [synth.make_layer(w, l, DEV) for l in range(3)]
+    shape = abi.shape_of(w)
+    x0 = synth.activations(w, 11, tokens=T, device=DEV)
+    bufs = [x0] + [torch.empty(T, w.hidden, dtype=torch.bfloat16, device=DEV) for _ in range(3)]
+    idx = [torch.empty(T, w.top_k, dtype=torch.int32, device=DEV) for _ in range(3)]
+    p = [torch.empty(T, w.top_k, dtype=torch.float32, device=DEV) for _ in range(3)]
+    slots = torch.arange(w.n_experts, dtype=torch.int32, device=DEV)
+    descs = [abi.layer_desc(x=bufs[l] if l == 0 else None, w_router=L.w_router, router_bias=L.router_bias,
+                            pool=L.pool, slot_table=slots, n_slots=w.n_experts, shared_blob=L.shared,
+                            w_shared_gate=L.w_sg, residual=x0, out=bufs[l + 1], topk_idx_out=idx[l],
+                            topk_w_out=p[l]) for l, L in enumerate(layers)]
+    ws = ws_for(shape, T)
+    abi.moe_stack_forward(shape, T, descs, ws)
+    torch.cuda.synchronize()
+    assert abi.moe_ws_check(ws) == 0
+    x = x0
+    for l, L in enumerate(layers):
+        out, i2, p2, _ = forward(w, L, x, residual=x0)
+        assert torch.equal(out, bufs[l + 1]) and torch.equal(i2, idx[l]) and torch.equal(p2, p[l])
+        ref = oracle_forward(w, L, x, residual=x0)
+        assert_routing(idx[l], ref["idx"], ref["logits"])
+        assert_close(bufs[l + 1], ref["out"])
+        x = bufs[l + 1]
+
+
+@pytest.mark.parametrize("T", [1, 3, 8])
+def test_stack_forward_unfused_shape_falls_back(T):
+    """A shape without a fused kernel (E > 512) runs layer by layer with the same results."""
+    w = TINY.with_(n_experts=600, top_k=6, seed=41, layers=2)
+    layers = [synth.make_layer(w, l, DEV) for l in range(2)]
+    shape = abi.shape_of(w)
+    x0 = synth.activations(w, 12, tokens=T, device=DEV)
+    outs = [torch.empty(T, w.hidden, dtype=torch.bfloat16, device=DEV) for _ in range(2)]
+    slots = torch.arange(w.n_experts, dtype=torch.int32, device=DEV)
+    descs = [abi.layer_desc(x=x0 if l == 0 else None, w_router=L.w_router, router_bias=L.router_bias, pool=L.pool,
+                            slot_table=slots, n_slots=w.n_experts, shared_blob=L.shared, w_shared_gate=L.w_sg,
+                            residual=None, out=outs[l]) for l, L in enumerate(layers)]
+    ws = ws_for(shape, T)
+    abi.moe_stack_forward(shape, T, descs, ws)
+    torch.cuda.synchronize()
+    x = x0
+    for l, L in enumerate(layers):
+        ref = oracle_forward(w, L, x)
+        assert_close(outs[l], ref["out"])
+        x = outs[l]
