@@ -43,8 +43,8 @@
  *     [0, n_slots), non-finite router logits) set bits in the workspace's error word
  *     and the offending term is skipped; read them with moe_ws_check().
  *   - The workspace must be zero-filled once before its first use; every call leaves
- *     its internal counters at zero again.  Calls that share a workspace must not run
- *     concurrently.
+ *     its internal counters at zero again (after a MOE_DEVERR_TIMEOUT, zero it again).
+ *     Calls that share a workspace must not run concurrently.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H

@@ -55,8 +55,8 @@ struct Ctrl {
   uint32_t ticket;  // last-block-done counter of the router (always returns to 0)
   int32_t act_n;    // number of distinct routed experts of the current call
   int32_t n_valid;  // number of (token, k) pairs with a valid expert id
-  uint32_t bar_count;  // grid barrier of the fused decode kernel: arrivals (returns to 0)
-  uint32_t bar_gen;    // grid barrier generation (monotonic)
+  uint32_t bar_count;  // fused decode kernel: grid-barrier arrivals (back to 0 at exit)
+  uint32_t bar_gen;    // fused decode kernel: CTAs that have exited (back to 0 at exit)
   uint32_t pad[58];
 };
 static_assert(sizeof(Ctrl) == 256, "ctrl block is 256 bytes");
@@ -117,11 +117,14 @@ struct DecodeArgs {
 // Shared-memory carve of the fused kernel (byte offsets from the dynamic base), used by the
 // host to size the launch and by the kernel to find its arrays.
 struct FusedSmem {
-  uint32_t xs4, xsum, partial, ids, pw, order, pos_of, act_e, act_slot, act_begin, gate, scratch, cand_v, cand_e,
+  uint32_t xs4, xsum, partial, ids, pw, order, pos_of, act_e, act_slot, act_begin, gate, scratch, slot, topk, red,
       total;
 };
-__host__ __device__ inline FusedSmem fused_smem_layout(int T, int H, int bits, int k, int jmax, int n_stages,
-                                                       int stage_bytes, int n_cons) {
+// Per-token top-k scratch of the fused kernel: 32 lane maxima (double + id), 64 candidates
+// (double + id), a counter and the threshold lane.
+constexpr int kTopkScratchBytes = 32 * 8 + 32 * 4 + 64 * 8 + 64 * 4 + 16;
+__host__ __device__ inline FusedSmem fused_smem_layout(int T, int H, int I, int E, int bits, int k, int jmax,
+                                                       int n_stages, int stage_bytes, int n_cons) {
   FusedSmem m{};
   size_t off = (size_t)n_stages * stage_bytes;
   auto carve = [&](size_t bytes) {
@@ -131,6 +134,7 @@ __host__ __device__ inline FusedSmem fused_smem_layout(int T, int H, int bits, i
     return at;
   };
   const int CC = 128 / bits, NC = H / CC, TK = T * k;
+  const int NCd = I / CC, NCLd = NCd < 32 ? NCd : 32;
   m.xs4 = carve((size_t)T * H * 4);
   m.xsum = carve((size_t)T * NC * 4);
   m.partial = carve((size_t)(TK + T) * jmax * 4);
@@ -143,8 +147,9 @@ __host__ __device__ inline FusedSmem fused_smem_layout(int T, int H, int bits, i
   m.act_begin = carve((size_t)(TK + 1) * 4);
   m.gate = carve((size_t)T * 4);
   m.scratch = carve((size_t)2 * TK * 4);
-  m.cand_v = carve((size_t)n_cons * 32 * 8);
-  m.cand_e = carve((size_t)n_cons * 32 * 4);
+  m.slot = carve((size_t)E * 4);
+  m.topk = carve((size_t)T * kTopkScratchBytes);
+  m.red = carve((size_t)n_cons * jmax * (NCLd + 1) * 4);
   m.total = (uint32_t)((off + 127) / 128 * 128);
   return m;
 }

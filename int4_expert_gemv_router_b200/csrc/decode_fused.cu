@@ -98,20 +98,20 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
 __device__ __forceinline__ void bar_cons() { asm volatile("bar.sync 1, %0;" ::"n"(kConsThreads) : "memory"); }
 
 // Grid-wide barrier among the CTAs of a cooperative launch (called by one thread per CTA).
-// Sense by generation: the last arriver resets the count and bumps the generation.
-__device__ bool grid_barrier(Ctrl* c, uint32_t nblocks) {
-  const uint32_t gen = ld_acquire(&c->bar_gen);
+// bar_count only grows during a launch: barrier number b (0, 1, 2, ...) completes when it
+// reaches (b + 1) * nblocks, so a barrier costs one atomic and the polls.  grid_exit()
+// returns it to zero once every CTA has passed its last barrier.
+__device__ bool grid_barrier(Ctrl* c, uint32_t nblocks, uint32_t b) {
+  const uint32_t target = (b + 1) * nblocks;
   __threadfence();
-  const uint32_t arrived = atomicAdd(&c->bar_count, 1u);
-  if (arrived == nblocks - 1) {
-    atomicExch(&c->bar_count, 0u);
+  const uint32_t arrived = atomicAdd(&c->bar_count, 1u) + 1;
+  if (arrived >= target) {
     __threadfence();
-    atomicAdd(&c->bar_gen, 1u);
     return true;
   }
   const unsigned long long t0 = now_ns();
   for (uint32_t it = 0;; ++it) {
-    if (ld_acquire(&c->bar_gen) != gen) {
+    if (ld_acquire(&c->bar_count) >= target) {
       __threadfence();
       return true;
     }
@@ -122,101 +122,114 @@ __device__ bool grid_barrier(Ctrl* c, uint32_t nblocks) {
   }
 }
 
+// Called once per CTA after its last barrier: the last CTA out resets the barrier counters
+// (no CTA reads bar_count any more by then).
+__device__ void grid_exit(Ctrl* c, uint32_t nblocks) {
+  __threadfence();
+  if (atomicAdd(&c->bar_gen, 1u) + 1 == nblocks) {
+    atomicExch(&c->bar_count, 0u);
+    atomicExch(&c->bar_gen, 0u);
+  }
+}
+
 // Key order of the top-k: larger logit first, ties to the lower id.
 __device__ __forceinline__ bool key_better(double av, int ae, double bv, int be) {
   return av > bv || (av == bv && ae < be);
 }
 
-// Sorts one key per lane across the warp, best key to lane 0 (bitonic network).
-__device__ __forceinline__ void warp_sort_keys(double& v, int& e) {
+// Top-k of one token's logits by one warp, through shared memory instead of shuffle chains.
+// Lane i (i < k) receives the i-th best key (sv, se): larger logit first, ties to the lower
+// id.  The k-th best of the 32 lane maxima bounds the k-th best key from below; the keys at
+// or above it (at least k, usually few) are ranked by counting; with more than 64 of them
+// (many equal keys) k rounds of warp arg-max run instead.
+__device__ __noinline__ void warp_topk(const double* lt, int E, int k, uint8_t* scratch, uint32_t* err,
+                                       double& sv, int& se) {
   const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      const double pv = __shfl_xor_sync(0xffffffffu, v, stride);
-      const int pe = __shfl_xor_sync(0xffffffffu, e, stride);
-      const bool keep_better = (((lane & stride) == 0) == ((lane & size) == 0));
-      const bool pb = key_better(pv, pe, v, e);
-      if (keep_better == pb) {
-        v = pv;
-        e = pe;
-      }
-    }
-  }
-}
-
-
-// Top-k of one token's logits by one warp.  Lane i (i < k) receives the i-th best key
-// (sv, se): larger logit first, ties to the lower id.  A threshold (the k-th best of the 32
-// lane maxima bounds the k-th best key from below) leaves few candidates, which one bitonic
-// sort orders; with more than 32 candidates (many equal keys) k rounds of warp arg-max run.
-__device__ __noinline__ void warp_topk(const double* lt, int E, int k, double* cv_base, int* ce_base,
-                                       uint32_t* err, double& sv, int& se) {
-  const int lane = threadIdx.x & 31;
+  double* lmv = reinterpret_cast<double*>(scratch);          // [32]
+  int* lme = reinterpret_cast<int*>(lmv + 32);               // [32]
+  double* cv = reinterpret_cast<double*>(lme + 32);          // [64]
+  int* ce = reinterpret_cast<int*>(cv + 64);                 // [64]
+  int* cnt = ce + 64;                                        // [2]: candidates, threshold lane
   double v[kLaneE];
   double bv = -INFINITY;
   int be = 0x7fffffff;
+  // all loads first (no side effects in between, so they are in flight together)
 #pragma unroll
   for (int m = 0; m < kLaneE; ++m) {
     const int e = lane + 32 * m;
-    double x = -INFINITY;
-    if (e < E) {
-      x = __ldcg(lt + e);
-      if (!(x == x)) {
-        atomicOr(err, kErrNonFinite);
-        x = -INFINITY;
-      }
+    v[m] = (e < E) ? __ldcg(lt + e) : -INFINITY;
+  }
+  bool nan_seen = false;
+#pragma unroll
+  for (int m = 0; m < kLaneE; ++m) {
+    const int e = lane + 32 * m;
+    if (!(v[m] == v[m])) {
+      nan_seen = true;
+      v[m] = -INFINITY;
     }
-    v[m] = x;
-    if (e < E && key_better(x, e, bv, be)) {
-      bv = x;
+    if (e < E && key_better(v[m], e, bv, be)) {
+      bv = v[m];
       be = e;
     }
   }
-  // threshold: the k-th best lane maximum bounds the k-th best key from below
-  double tv = bv;
-  int te = be;
-  warp_sort_keys(tv, te);
-  const double thr_v = __shfl_sync(0xffffffffu, tv, k - 1);
-  const int thr_e = __shfl_sync(0xffffffffu, te, k - 1);
-  int cnt = 0;
+  if (nan_seen) atomicOr(err, kErrNonFinite);
+  lmv[lane] = bv;
+  lme[lane] = be;
+  if (lane == 0) cnt[0] = 0;
+  __syncwarp();
+  int r = 0;
+#pragma unroll 8
+  for (int j = 0; j < 32; ++j) r += key_better(lmv[j], lme[j], bv, be) ? 1 : 0;
+  if (r == k - 1 && be != 0x7fffffff) cnt[1] = lane;
+  __syncwarp();
+  const double thr_v = lmv[cnt[1]];
+  const int thr_e = lme[cnt[1]];
 #pragma unroll
   for (int m = 0; m < kLaneE; ++m) {
     const int e = lane + 32 * m;
-    cnt += (e < E && !key_better(thr_v, thr_e, v[m], e)) ? 1 : 0;
-  }
-  int incl = cnt;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  const int total = __shfl_sync(0xffffffffu, incl, 31);
-  if (total <= 32) {
-    double* cv = cv_base;
-    int* ce = ce_base;
-    int pos = incl - cnt;
-#pragma unroll
-    for (int m = 0; m < kLaneE; ++m) {
-      const int e = lane + 32 * m;
-      if (e < E && !key_better(thr_v, thr_e, v[m], e)) {
+    if (e < E && !key_better(thr_v, thr_e, v[m], e)) {
+      const int pos = atomicAdd(&cnt[0], 1);
+      if (pos < 64) {
         cv[pos] = v[m];
         ce[pos] = e;
-        ++pos;
+      }
+    }
+  }
+  __syncwarp();
+  const int n = cnt[0];
+  if (n <= 64) {
+    double mv[2];
+    int me[2], mr[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = lane + 32 * h;
+      mv[h] = i < n ? cv[i] : -INFINITY;
+      me[h] = i < n ? ce[i] : 0x7fffffff;
+      mr[h] = 0;
+    }
+    for (int j = 0; j < n; ++j) {
+      const double jv = cv[j];
+      const int je = ce[j];
+      mr[0] += key_better(jv, je, mv[0], me[0]) ? 1 : 0;
+      mr[1] += key_better(jv, je, mv[1], me[1]) ? 1 : 0;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (lane + 32 * h < n && mr[h] < k) {
+        lmv[mr[h]] = mv[h];
+        lme[mr[h]] = me[h];
       }
     }
     __syncwarp();
-    sv = lane < total ? cv[lane] : -INFINITY;
-    se = lane < total ? ce[lane] : 0x7fffffff;
+    sv = lane < k ? lmv[lane] : -INFINITY;
+    se = lane < k ? lme[lane] : 0x7fffffff;
     __syncwarp();
-    warp_sort_keys(sv, se);
   } else {
-    // many near-equal keys: k rounds of warp arg-max over the candidates
     uint32_t taken = 0;
     sv = -INFINITY;
     se = 0x7fffffff;
-    for (int r = 0; r < k; ++r) {
+    for (int rr = 0; rr < k; ++rr) {
       double rv = -INFINITY;
       int re = 0x7fffffff;
 #pragma unroll
@@ -237,7 +250,7 @@ __device__ __noinline__ void warp_topk(const double* lt, int E, int k, double* c
         }
       }
       if (re != 0x7fffffff && (re & 31) == lane) taken |= 1u << (re >> 5);
-      if (lane == r) {
+      if (lane == rr) {
         sv = rv;
         se = re;
       }
@@ -281,8 +294,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
 #define P_BEGIN reinterpret_cast<int*>(smem + a.sm.act_begin)
 #define P_GATE reinterpret_cast<float*>(smem + a.sm.gate)
 #define P_SCRATCH reinterpret_cast<int*>(smem + a.sm.scratch)
-#define P_CANDV reinterpret_cast<double*>(smem + a.sm.cand_v)
-#define P_CANDE reinterpret_cast<int*>(smem + a.sm.cand_e)
+#define S_SLOT reinterpret_cast<int*>(smem + a.sm.slot)
 
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -424,6 +436,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
   const int cw = warp;  // 0..14
   const int gw = blockIdx.x * kCons + cw, NW = G * kCons;
   uint32_t q = 0;
+  uint32_t nb = 0;  // grid barriers passed in this launch
   bool ok = true;
 
   for (int l = 0; l < a.n_layers; ++l) {
@@ -435,6 +448,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
       const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(Lc.x + (size_t)r * H + i));
       return make_float4(bf_lo(raw.x), bf_hi(raw.x), bf_lo(raw.y), bf_hi(raw.y));
     });
+    for (int e = tid; e < E; e += kConsThreads) S_SLOT[e] = __ldg(Lc.slot_table + e);
     bar_cons();
 
     // ---- phase R: router rows, shared-gate row, shared gate/up rows ----
@@ -449,6 +463,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
           double acc[TM];
 #pragma unroll
           for (int t = 0; t < TM; ++t) acc[t] = 0.0;
+#pragma unroll 4
           for (int c8 = lane; c8 < H / 8; c8 += 32) {
             const uint4 w = ld_stream(row + c8 * 8);
             const float wv[8] = {bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y),
@@ -484,45 +499,51 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
             }
           }
         } else {
-          // shared expert gate/up row(s)
+          // shared expert gate/up row(s): chunk by chunk, every token against each chunk
           const int r = (it - n_router) * RPWg + lane / NCLg;
           const int sub = lane % NCLg;
           const uint8_t* b = Lc.shared;
-          uint4 qg[CPLg], qu[CPLg];
-          float sg[CPLg], bg[CPLg], su[CPLg], bu[CPLg];
+          float ag[TM], au[TM];
 #pragma unroll
+          for (int t = 0; t < TM; ++t) ag[t] = au[t] = 0.f;
+#pragma unroll 1
           for (int m = 0; m < CPLg; ++m) {
             const int c = sub + NCLg * m, g = c * CC / kGroup;
-            qg[m] = ld_stream(b + a.L.off[0] + (int64_t)r * ROWBg + c * 16);
-            qu[m] = ld_stream(b + a.L.off[1] + (int64_t)r * ROWBg + c * 16);
-            sg[m] = bf1(ld_u16(b + a.L.off[3] + (int64_t)r * SRg + g * 2));
-            bg[m] = bf1(ld_u16(b + a.L.off[4] + (int64_t)r * SRg + g * 2));
-            su[m] = bf1(ld_u16(b + a.L.off[5] + (int64_t)r * SRg + g * 2));
-            bu[m] = bf1(ld_u16(b + a.L.off[6] + (int64_t)r * SRg + g * 2));
+            const uint4 qg = ld_stream(b + a.L.off[0] + (int64_t)r * ROWBg + c * 16);
+            const uint4 qu = ld_stream(b + a.L.off[1] + (int64_t)r * ROWBg + c * 16);
+            const float sg = bf1(ld_u16(b + a.L.off[3] + (int64_t)r * SRg + g * 2));
+            const float bg = bf1(ld_u16(b + a.L.off[4] + (int64_t)r * SRg + g * 2));
+            const float su = bf1(ld_u16(b + a.L.off[5] + (int64_t)r * SRg + g * 2));
+            const float bu = bf1(ld_u16(b + a.L.off[6] + (int64_t)r * SRg + g * 2));
+#pragma unroll
+            for (int t = 0; t < TM; ++t) {
+              if (t < T) {
+                float dg, du;
+                dot_chunk2<BITS>(qg, qu, xs4 + (size_t)t * V4 * NCg + c, NCg, dg, du);
+                const float xc = xsum[t * NCg + c];
+                ag[t] = fmaf(sg, dg, fmaf(bg, xc, ag[t]));
+                au[t] = fmaf(su, du, fmaf(bu, xc, au[t]));
+              }
+            }
           }
-          for (int t = 0; t < T; ++t) {
-            float ag = 0.f, au = 0.f;
 #pragma unroll
-            for (int m = 0; m < CPLg; ++m) {
-              const int c = sub + NCLg * m;
-              float dg, du;
-              dot_chunk2<BITS>(qg[m], qu[m], xs4 + (size_t)t * V4 * NCg + c, NCg, dg, du);
-              const float xc = xsum[t * NCg + c];
-              ag = fmaf(sg[m], dg, fmaf(bg[m], xc, ag));
-              au = fmaf(su[m], du, fmaf(bu[m], xc, au));
-            }
+          for (int t = 0; t < TM; ++t) {
+            if (t < T) {
+              float g2 = ag[t], u2 = au[t];
 #pragma unroll
-            for (int o = NCLg / 2; o > 0; o >>= 1) {
-              ag += __shfl_xor_sync(0xffffffffu, ag, o);
-              au += __shfl_xor_sync(0xffffffffu, au, o);
+              for (int o = NCLg / 2; o > 0; o >>= 1) {
+                g2 += __shfl_xor_sync(0xffffffffu, g2, o);
+                u2 += __shfl_xor_sync(0xffffffffu, u2, o);
+              }
+              if (sub == 0) a.hs[(size_t)t * I + r] = g2 / (1.0f + expf(-g2)) * u2;
             }
-            if (sub == 0) a.hs[(size_t)t * I + r] = ag / (1.0f + expf(-ag)) * au;
           }
         }
       }
     }
     bar_cons();
-    if (tid == 0 && !grid_barrier(a.ctrl, G)) s_abort = 1;
+    if (tid == 0 && !grid_barrier(a.ctrl, G, nb)) s_abort = 1;
+    ++nb;
     bar_cons();
     if (s_abort) ok = false;
 
@@ -533,7 +554,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
         if (routed) {
           double sv;
           int se;
-          warp_topk(lt, E, k, P_CANDV + cw * 32, P_CANDE + cw * 32, &a.ctrl->err, sv, se);
+          warp_topk(lt, E, k, smem + a.sm.topk + (size_t)t * kTopkScratchBytes, &a.ctrl->err, sv, se);
           // lanes 0..k-1 hold the selection in order
           const double v0 = __shfl_sync(0xffffffffu, sv, 0);
           const bool valid = lane < k && se != 0x7fffffff && sv != -INFINITY;
@@ -594,7 +615,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
           }
           P_ACTE[act] = ki;
           P_BEGIN[act] = before;
-          const int slot = Lc.slot_table[ki];
+          const int slot = S_SLOT[ki];
           const bool sok = slot >= 0 && slot < Lc.n_slots;
           if (!sok) atomicOr(&a.ctrl->err, kErrBadSlot);
           P_SLOT[act] = sok ? slot : -1;
@@ -634,34 +655,30 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
         const uint8_t* st = ring + (size_t)s * SB;
         if (P_SLOT[u] >= 0) {
           const int pb = P_BEGIN[u], pe = P_BEGIN[u + 1];
-          for (int step = cw; step < n / RPWg; step += kCons) {
+          // row steps are dealt to warps round-robin over the CTA's whole row range
+          const int step0 = (f - f0) / RPWg;
+          for (int step = (cw - step0 % kCons + kCons) % kCons; step < n / RPWg; step += kCons) {
             const int rl = step * RPWg + rsub;
             const uint8_t* gq = st + rl * ROWBg;
             const uint8_t* uq = st + n * ROWBg + rl * ROWBg;
             const uint8_t* sc = st + 2 * n * ROWBg + rl * SRg;
-            uint4 qg[CPLg], qu[CPLg];
-            float sg[CPLg], bg[CPLg], su[CPLg], bu[CPLg];
-#pragma unroll
-            for (int m = 0; m < CPLg; ++m) {
-              const int c = sub + NCLg * m, g = c * CC / kGroup;
-              qg[m] = *reinterpret_cast<const uint4*>(gq + c * 16);
-              qu[m] = *reinterpret_cast<const uint4*>(uq + c * 16);
-              sg[m] = bf1(*reinterpret_cast<const uint16_t*>(sc + g * 2));
-              bg[m] = bf1(*reinterpret_cast<const uint16_t*>(sc + n * SRg + g * 2));
-              su[m] = bf1(*reinterpret_cast<const uint16_t*>(sc + 2 * n * SRg + g * 2));
-              bu[m] = bf1(*reinterpret_cast<const uint16_t*>(sc + 3 * n * SRg + g * 2));
-            }
             for (int p = pb; p < pe; ++p) {
               const int t = P_ORDER[p] / k;
               float ag = 0.f, au = 0.f;
-#pragma unroll
+#pragma unroll 1
               for (int m = 0; m < CPLg; ++m) {
-                const int c = sub + NCLg * m;
+                const int c = sub + NCLg * m, g = c * CC / kGroup;
+                const uint4 qg = *reinterpret_cast<const uint4*>(gq + c * 16);
+                const uint4 qu = *reinterpret_cast<const uint4*>(uq + c * 16);
                 float dg, du;
-                dot_chunk2<BITS>(qg[m], qu[m], xs4 + (size_t)t * V4 * NCg + c, NCg, dg, du);
+                dot_chunk2<BITS>(qg, qu, xs4 + (size_t)t * V4 * NCg + c, NCg, dg, du);
                 const float xc = xsum[t * NCg + c];
-                ag = fmaf(sg[m], dg, fmaf(bg[m], xc, ag));
-                au = fmaf(su[m], du, fmaf(bu[m], xc, au));
+                const float sg = bf1(*reinterpret_cast<const uint16_t*>(sc + g * 2));
+                const float bg = bf1(*reinterpret_cast<const uint16_t*>(sc + n * SRg + g * 2));
+                const float su = bf1(*reinterpret_cast<const uint16_t*>(sc + 2 * n * SRg + g * 2));
+                const float bu = bf1(*reinterpret_cast<const uint16_t*>(sc + 3 * n * SRg + g * 2));
+                ag = fmaf(sg, dg, fmaf(bg, xc, ag));
+                au = fmaf(su, du, fmaf(bu, xc, au));
               }
 #pragma unroll
               for (int o = NCLg / 2; o > 0; o >>= 1) {
@@ -679,7 +696,8 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
       }
     }
     bar_cons();
-    if (tid == 0 && (!ok || !grid_barrier(a.ctrl, G))) s_abort = 1;
+    if (tid == 0 && (!ok || !grid_barrier(a.ctrl, G, nb))) s_abort = 1;
+    ++nb;
     bar_cons();
     if (s_abort) break;
 
@@ -687,6 +705,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
     if (nJ > 0) {
       const int per_stage = SB / (nJ * ROWD_BYTES);
       const int sub = lane % NCLd, rsub = lane / NCLd;
+      float* red = reinterpret_cast<float*>(smem + a.sm.red) + (size_t)cw * a.jmax * (NCLd + 1);
       for (int u0 = 0; u0 <= act_n;) {
         const int cnt = min(per_stage, act_n + 1 - u0);
         const int s = q % NS;
@@ -696,7 +715,8 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
           break;
         }
         const uint8_t* st = ring + (size_t)s * SB;
-        for (int z = cw; z < cnt; z += kCons) {
+        // expert slices are dealt to warps round-robin over the layer
+        for (int z = (cw - u0 % kCons + kCons) % kCons; z < cnt; z += kCons) {
           const int u = u0 + z;
           const bool shared = (u == act_n);
           const uint8_t* dq = st + (size_t)z * nJ * ROWD_BYTES;
@@ -736,6 +756,8 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
               }
               hsum[m] = sum;
             }
+            // per-lane partial dots of every row, then a fixed-order sum per row through
+            // shared memory (no shuffle chain per row)
             for (int rs = 0; rs < nJ / RPWd; ++rs) {
               const int jl = rs * RPWd + rsub;
               float part = 0.f;
@@ -750,10 +772,16 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
                   part = fmaf(sd, d, fmaf(bd, hsum[m], part));
                 }
               }
-#pragma unroll
-              for (int o = NCLd / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-              if (sub == 0) partial[(size_t)p * a.jmax + jl] = w * part;
+              red[jl * (NCLd + 1) + sub] = part;
             }
+            __syncwarp();
+            for (int jl = lane; jl < nJ; jl += 32) {
+              float sum = 0.f;
+#pragma unroll
+              for (int qq = 0; qq < NCLd; ++qq) sum += red[jl * (NCLd + 1) + qq];
+              partial[(size_t)p * a.jmax + jl] = w * sum;
+            }
+            __syncwarp();
           }
         }
         __syncwarp();
@@ -778,7 +806,8 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
       }
     }
     bar_cons();
-    if (tid == 0 && (!ok || !grid_barrier(a.ctrl, G))) s_abort = 1;
+    if (tid == 0 && (!ok || !grid_barrier(a.ctrl, G, nb))) s_abort = 1;
+    ++nb;
     bar_cons();
     if (s_abort) break;
   }
@@ -787,12 +816,13 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
     s_abort = 1;
     mbar_arrive(&plan_bar);
   }
+  if (tid == 0 && !s_abort) grid_exit(a.ctrl, G);
 }
 
 }  // namespace
 
 static size_t fused_smem_bytes(const FusedArgs& a, int stages) {
-  return fused_smem_layout(a.T, a.H, a.bits, a.k, a.jmax, stages, a.stage_bytes, kCons).total;
+  return fused_smem_layout(a.T, a.H, a.I, a.E, a.bits, a.k, a.jmax, stages, a.stage_bytes, kCons).total;
 }
 
 template <int BITS, int H, int I, int TM>
@@ -817,7 +847,7 @@ static cudaError_t run_fused(FusedArgs a, cudaStream_t s) {
   int stages = kMaxStages;
   while (stages > 2 && fused_smem_bytes(a, stages) > (size_t)max_smem) --stages;
   a.n_stages = stages;
-  a.sm = fused_smem_layout(a.T, a.H, a.bits, a.k, a.jmax, stages, a.stage_bytes, kCons);
+  a.sm = fused_smem_layout(a.T, a.H, a.I, a.E, a.bits, a.k, a.jmax, stages, a.stage_bytes, kCons);
   const size_t smem = a.sm.total;
   if (smem > (size_t)max_smem) return cudaErrorInvalidConfiguration;
   // one stage must hold one gate/up row and one expert's down slice
