@@ -457,6 +457,8 @@ def parse(argv=None):
     ap.add_argument("--workload", default="decode80b", choices=["decode80b", "decode35b"])
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the stack depth (profiling of a small case only; not a bench value)")
     return ap.parse_args(argv)
 
 
@@ -465,6 +467,8 @@ def main(argv=None):
     if args.warmup < 3:
         args.warmup = 3
     w = synth.WORKLOADS[args.workload]
+    if args.layers:
+        w = w.with_(layers=args.layers)
     T = args.tokens or w.tokens
     if args.impl == "reference":
         line = run_reference(args, w, T)
