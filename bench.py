@@ -41,6 +41,11 @@ import synth  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per layer-token of the kernel the
+# bench times, from the ncu capture summarised in profiles/k_fused_decode_decode80b_2layer_full.md
+# (2-layer case, scaled by layers).  Must be re-captured whenever the kernel changes.
+NCU_TRAFFIC_PER_LAYER = {("k_fused_decode", "decode80b", 1): 21_639_120}
+
 
 # --------------------------------------------------------------------------------------
 # distributed plumbing (host-side helpers are importable for the CPU tests)
@@ -382,7 +387,8 @@ def decode_line(args, w, T, r, n_gpus, peaks, peak_kind, cpu_base):
                      "mean_distinct_experts_per_layer": round(float(np.mean(r["uniq"])), 2)},
         "roofline": {"bound": "hbm", "kernel": "k_fused_decode (whole 48-layer step, one launch)",
                      "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                     "traffic": None, "launch_us": round(k_us, 3), "bytes_per_launch": int(k_bytes),
+                     "traffic": (NCU_TRAFFIC_PER_LAYER.get(("k_fused_decode", w.name, T), 0) * w.layers) or None,
+                     "launch_us": round(k_us, 3), "bytes_per_launch": int(k_bytes),
                      "peak_kind": f"{peak_kind} hbm_gbs (burst copy)"},
         "clocks": r["clocks"],
         "e2e": {"value": round(tok / (r["e2e_ms"] / 1e3), 2), "unit": "tokens/s",
