@@ -139,8 +139,12 @@ MOE_API moe_status moe_router_topk(const moe_shape* shape, const void* x, int32_
  *   out          (dev) bf16 [T, H] out (round-to-nearest-even of the fp32 sum)
  *   topk_idx_out, topk_w_out (dev) [T, k] or NULL: the routing used (when routed inside)
  *   ws, ws_bytes workspace (see moe_workspace_size)
- * T: 1..8 (decode path).  Deterministic: the same inputs give the same bits, whichever
- * slots the experts sit in.
+ * T: 1..8 runs the decode path (fused GEMV kernels): deterministic, the same inputs give
+ * the same bits whichever slots the experts sit in.  T > 8 runs the many-token (prefill)
+ * path: router on the tensor cores with every near-boundary logit recomputed exactly, the
+ * pairs grouped by expert, and per-expert tcgen05 GEMMs on weights dequantised to bf16
+ * (hidden % 128 == 0, E <= 512); its down products are summed with fp32 atomics, so the
+ * last bits of out may vary from run to run.
  */
 MOE_API moe_status moe_layer_forward(const moe_shape* shape, const void* x, int32_t T, const void* w_router,
                              const float* router_bias, const int32_t* topk_idx_in,
@@ -217,6 +221,19 @@ MOE_API moe_status moe_layer_forward_static(const moe_shape* shape, const void* 
                                             const void* w_shared_gate, const void* residual,
                                             void* out, int32_t* topk_idx_out, float* topk_w_out,
                                             void* stream);
+
+/*
+ * moe_group_pairs -- stable counting sort of the T*k (token, slot) pairs by expert: the
+ * grouping step of the many-token path (each expert then sees its tokens as one matrix;
+ * «Swiftlet: 在 Mac 和 iPhone 上執行…», 社群觀點, on prefill).
+ *   topk_idx (dev) int32 [T, k]; pair n = t*k + slot refers to topk_idx[n]
+ *   order    (dev) int32 [T*k] out: pair numbers sorted by expert, ties in pair order
+ *   offsets  (dev) int32 [E+1] out: pairs of expert e are order[offsets[e] .. offsets[e+1])
+ *   ws, ws_bytes: workspace of moe_workspace_size(shape, T) bytes
+ * Ids outside [0, E) are left out (MOE_DEVERR_BAD_EXPERT); then offsets[E] < T*k.  E <= 512.
+ */
+MOE_API moe_status moe_group_pairs(const moe_shape* shape, int32_t T, const int32_t* topk_idx, int32_t* order,
+                                   int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * moe_ws_check -- synchronise `stream`, read and clear the workspace's device error word.

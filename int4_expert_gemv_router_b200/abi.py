@@ -64,6 +64,7 @@ _SIGS = {
                                                 _I64, _P, _P, _P, _P, _P, _P, _P]),
     "moe_stack_forward": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, ctypes.POINTER(moe_layer_desc), _I32, _P,
                                          _SZ, _P]),
+    "moe_group_pairs": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, _P, _P, _P, _P, _SZ, _P]),
     "moe_ws_check": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "moe_pool_create": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, _P, _P, _P, ctypes.POINTER(_P)]),
     "moe_expert_pool_load": (ctypes.c_int, [_P, _P, _I32, _P]),
@@ -187,6 +188,11 @@ def moe_layer_forward_static(shape, x, T, w_router, router_bias, topk_idx_in, to
                                           _ptr(topk_idx_in), _ptr(topk_w_in), _ptr(pool), _ptr(slot_table),
                                           n_slots, _ptr(shared_blob), _ptr(w_shared_gate), _ptr(residual),
                                           _ptr(out), _ptr(topk_idx_out), _ptr(topk_w_out), _stream(stream)))
+
+
+def moe_group_pairs(shape, T, topk_idx, order, offsets, ws, stream=None):
+    _check(lib().moe_group_pairs(ctypes.byref(shape), T, _ptr(topk_idx), _ptr(order), _ptr(offsets), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def moe_ws_check(ws, stream=None, raise_on_error: bool = False) -> int:

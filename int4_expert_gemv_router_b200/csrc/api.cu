@@ -81,7 +81,11 @@ moe_status moe_workspace_size(const moe_shape* shape, int32_t T, size_t* bytes) 
   if (st != MOE_OK) return st;
   if (!bytes) return set_error(MOE_ERR_INVALID, "bytes is NULL");
   if (T < 1) return set_error(MOE_ERR_INVALID, "T must be >= 1 (got %d)", T);
-  *bytes = make_ws_layout(T, shape->n_experts, shape->top_k, shape->inter, shape->shared_inter).total;
+  // one size serves every call on T tokens: the decode layout (T <= 8), the prefill layout,
+  // and moe_group_pairs (which uses the prefill layout at any T)
+  const size_t dec = make_ws_layout(T, shape->n_experts, shape->top_k, shape->inter, shape->shared_inter).total;
+  const size_t pre = make_prefill_layout(T, shape->n_experts, shape->top_k, shape->hidden, shape->inter).total;
+  *bytes = dec > pre ? dec : pre;
   return MOE_OK;
 }
 
@@ -205,6 +209,89 @@ static moe_status check_layer(const moe_shape* shape, const moe_layer_desc* d, b
   return MOE_OK;
 }
 
+// Many tokens: router GEMM + certified top-k, grouping, tcgen05 grouped GEMMs (prefill.cu).
+static moe_status prefill_forward(const moe_shape* shape, const void* x, int32_t T, const void* w_router,
+                                  const float* router_bias, const int32_t* topk_idx_in, const float* topk_w_in,
+                                  const uint8_t* pool, const int32_t* slot_table, int64_t n_slots,
+                                  const uint8_t* shared_blob, const void* w_shared_gate, const void* residual,
+                                  void* out, int32_t* topk_idx_out, float* topk_w_out, void* ws, size_t ws_bytes,
+                                  cudaStream_t s) {
+  if (!prefill_shape_supported(shape->hidden, shape->inter, shape->bits, shape->n_experts))
+    return set_error(MOE_ERR_UNSUPPORTED,
+                     "no prefill kernel for hidden=%d inter=%d bits=%d E=%d (hidden %% 128 == 0, E <= 512)",
+                     shape->hidden, shape->inter, shape->bits, shape->n_experts);
+  if (!ws || !aligned(ws, kAlign)) return set_error(MOE_ERR_INVALID, "ws must be non-NULL and 256-byte aligned");
+  const int E = shape->n_experts, k = shape->top_k, H = shape->hidden, I = shape->inter;
+  const PrefillLayout W = make_prefill_layout(T, E, k, H, I);
+  if (ws_bytes < W.total) return set_error(MOE_ERR_INVALID, "ws_bytes %zu < required %zu", ws_bytes, W.total);
+  char* b = static_cast<char*>(ws);
+  PrefillArgs p{};
+  p.T = T;
+  p.E = E;
+  p.k = k;
+  p.H = H;
+  p.I = I;
+  p.x = static_cast<const uint16_t*>(x);
+  p.wr = static_cast<const uint16_t*>(w_router);
+  p.wsg = static_cast<const uint16_t*>(w_shared_gate);
+  p.rbias = router_bias;
+  p.residual = static_cast<const uint16_t*>(residual);
+  p.out = static_cast<uint16_t*>(out);
+  p.route = (topk_idx_in == nullptr);
+  p.ctrl = reinterpret_cast<Ctrl*>(b + W.ctrl);
+  p.xnorm = reinterpret_cast<double*>(b + W.xnorm);
+  p.wnorm = reinterpret_cast<double*>(b + W.wnorm);
+  p.logits = reinterpret_cast<float*>(b + W.logits);
+  if (topk_idx_in) {
+    p.topk_idx = const_cast<int32_t*>(topk_idx_in);
+    p.topk_w = const_cast<float*>(topk_w_in);
+  } else if (topk_idx_out) {
+    p.topk_idx = topk_idx_out;
+    p.topk_w = topk_w_out;
+  } else {
+    p.topk_idx = reinterpret_cast<int32_t*>(b + W.topk_idx);
+    p.topk_w = reinterpret_cast<float*>(b + W.topk_w);
+  }
+  p.gate = reinterpret_cast<float*>(b + W.gate);
+  p.order = reinterpret_cast<int32_t*>(b + W.order);
+  p.offsets = reinterpret_cast<int32_t*>(b + W.offsets);
+  p.counts = reinterpret_cast<int32_t*>(b + W.counts);
+  p.units_rt = reinterpret_cast<GemmUnit*>(b + W.units_rt);
+  p.units_gu = reinterpret_cast<GemmUnit*>(b + W.units_gu);
+  p.units_dn = reinterpret_cast<GemmUnit*>(b + W.units_dn);
+  p.n_units = reinterpret_cast<int*>(b + W.n_units);
+  p.acc = reinterpret_cast<float*>(b + W.acc);
+  p.h = reinterpret_cast<uint16_t*>(b + W.h);
+  p.hs = reinterpret_cast<uint16_t*>(b + W.hs);
+  GemmArgs& g = p.g;
+  g.H = H;
+  g.I = I;
+  g.E = E;
+  g.k = k;
+  g.T = T;
+  g.pool = pool;
+  g.slot_table = slot_table;
+  g.n_slots = n_slots;
+  g.shared = shared_blob;
+  g.L = make_blob_layout(H, I, shape->bits);
+  g.x = p.x;
+  g.wr = p.wr;
+  g.wsg = p.wsg;
+  g.order = p.order;
+  g.topk_w = p.topk_w;
+  g.gate = p.gate;
+  g.h = p.h;
+  g.hs = p.hs;
+  g.acc = p.acc;
+  g.logits = p.logits;
+  g.ctrl = p.ctrl;
+  prof_mark(0, false, s);
+  cudaError_t e = launch_prefill(p, shape->bits, s);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  prof_mark(0, true, s);
+  return MOE_OK;
+}
+
 moe_status moe_layer_forward(const moe_shape* shape, const void* x, int32_t T, const void* w_router,
                              const float* router_bias, const int32_t* topk_idx_in, const float* topk_w_in,
                              const uint8_t* pool, const int32_t* slot_table, int64_t n_slots,
@@ -232,6 +319,10 @@ moe_status moe_layer_forward(const moe_shape* shape, const void* x, int32_t T, c
     return set_error(MOE_ERR_INVALID, "x, out, w_router, w_shared_gate and residual must be 16-byte aligned");
   if (!aligned(pool, kAlign) || !aligned(shared_blob, kAlign))
     return set_error(MOE_ERR_INVALID, "pool and shared_blob must be 256-byte aligned");
+  if (T > kMaxDecodeT)
+    return prefill_forward(shape, x, T, w_router, router_bias, topk_idx_in, topk_w_in, pool, slot_table, n_slots,
+                           shared_blob, w_shared_gate, residual, out, topk_idx_out, topk_w_out, ws, ws_bytes,
+                           static_cast<cudaStream_t>(stream));
   DecodeArgs a;
   if ((st = fill_decode_args(shape, T, ws, ws_bytes, &a)) != MOE_OK) return st;
   a.x = static_cast<const uint16_t*>(x);
@@ -317,6 +408,37 @@ moe_status moe_stack_forward(const moe_shape* shape, int32_t T, const moe_layer_
                            d.out, d.topk_idx_out, d.topk_w_out, ws, ws_bytes, stream);
     if (st != MOE_OK) return st;
   }
+  return MOE_OK;
+}
+
+moe_status moe_group_pairs(const moe_shape* shape, int32_t T, const int32_t* topk_idx, int32_t* order,
+                           int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (T < 1) return set_error(MOE_ERR_INVALID, "T must be >= 1 (got %d)", T);
+  if (!topk_idx || !order || !offsets) return set_error(MOE_ERR_INVALID, "topk_idx, order and offsets must be non-NULL");
+  if (shape->n_experts > 512) return set_error(MOE_ERR_UNSUPPORTED, "grouping supports E <= 512");
+  if (!ws || !aligned(ws, kAlign)) return set_error(MOE_ERR_INVALID, "ws must be non-NULL and 256-byte aligned");
+  const int E = shape->n_experts, k = shape->top_k;
+  const PrefillLayout W = make_prefill_layout(T, E, k, shape->hidden, shape->inter);
+  if (ws_bytes < W.total) return set_error(MOE_ERR_INVALID, "ws_bytes %zu < required %zu", ws_bytes, W.total);
+  char* b = static_cast<char*>(ws);
+  PrefillArgs p{};
+  p.T = T;
+  p.E = E;
+  p.k = k;
+  p.H = shape->hidden;
+  p.I = shape->inter;
+  p.ctrl = reinterpret_cast<Ctrl*>(b + W.ctrl);
+  p.topk_idx = const_cast<int32_t*>(topk_idx);
+  p.order = order;
+  p.offsets = offsets;
+  p.counts = reinterpret_cast<int32_t*>(b + W.counts);
+  p.units_gu = reinterpret_cast<GemmUnit*>(b + W.units_gu);
+  p.units_dn = reinterpret_cast<GemmUnit*>(b + W.units_dn);
+  p.n_units = reinterpret_cast<int*>(b + W.n_units);
+  cudaError_t e = launch_group(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "grouping launch");
   return MOE_OK;
 }
 

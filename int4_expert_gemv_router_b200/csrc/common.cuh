@@ -185,6 +185,108 @@ struct FusedArgs {
   FusedLayer layer[kMaxFusedLayers];
 };
 
+// ---------------------------------------------------------------------------------------
+// Prefill path (prefill.cu)
+// ---------------------------------------------------------------------------------------
+constexpr int kModeRouter = 0, kModeGateUp = 1, kModeDown = 2;
+
+// One tcgen05 GEMM work unit: expert e (-1: shared expert, -2: router), row tile mt, first
+// column p0 (pair position, or token for the shared expert / router) and column count n.
+struct GemmUnit {
+  int e, mt, p0, n;
+};
+
+struct GemmArgs {
+  int H, I, E, k, T;
+  const uint8_t* pool;
+  const int32_t* slot_table;
+  int64_t n_slots;
+  const uint8_t* shared;
+  BlobLayout L;
+  const uint16_t* x;    // bf16 [T, H]
+  const uint16_t* wr;   // bf16 [E, H]
+  const uint16_t* wsg;  // bf16 [H]
+  const int32_t* order; // [T*k] pair numbers sorted by expert
+  const float* topk_w;  // [T*k]
+  const float* gate;    // [T]
+  uint16_t* h;          // bf16 [T*k, I] per sorted pair
+  uint16_t* hs;         // bf16 [T, I] shared expert
+  float* acc;           // fp32 [T, H]
+  float* logits;        // fp32 [T, E+1] (no bias)
+  const GemmUnit* units;
+  const int* n_units;
+  Ctrl* ctrl;
+};
+
+struct PrefillArgs {
+  int T, E, k, H, I;
+  const uint16_t* x;
+  const uint16_t* wr;
+  const uint16_t* wsg;
+  const float* rbias;
+  const uint16_t* residual;
+  uint16_t* out;
+  bool route;           // false: topk_idx / topk_w hold the caller's routing
+  double* xnorm;        // [T]
+  double* wnorm;        // [E+1]
+  float* logits;
+  int32_t* topk_idx;
+  float* topk_w;
+  float* gate;
+  int32_t* order;
+  int32_t* offsets;     // [E+1]
+  int32_t* counts;      // [E]
+  GemmUnit* units_rt;
+  GemmUnit* units_gu;
+  GemmUnit* units_dn;
+  int* n_units;         // [3]: gate/up, down, router
+  float* acc;
+  uint16_t* h;
+  uint16_t* hs;
+  Ctrl* ctrl;
+  GemmArgs g;           // shared GEMM arguments (units filled per launch)
+};
+
+struct PrefillLayout {
+  size_t ctrl, xnorm, wnorm, logits, topk_idx, topk_w, gate, order, offsets, counts, units_rt, units_gu,
+      units_dn, n_units, acc, h, hs, total;
+};
+
+inline PrefillLayout make_prefill_layout(int T, int E, int k, int H, int I) {
+  PrefillLayout W{};
+  size_t pos = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = (size_t)round_up((int64_t)pos, kAlign);
+    pos = at + bytes;
+    return at;
+  };
+  const size_t tiles = (size_t)E + ((size_t)T * k + 255) / 256 + ((size_t)T + 255) / 256 + 1;
+  const size_t rt_units = (size_t)((E + 1 + 127) / 128) * ((T + 127) / 128);
+  W.ctrl = take(sizeof(Ctrl));
+  W.xnorm = take(sizeof(double) * T);
+  W.wnorm = take(sizeof(double) * (E + 1));
+  W.logits = take(sizeof(float) * (size_t)T * (E + 1));
+  W.topk_idx = take(sizeof(int32_t) * (size_t)T * k);
+  W.topk_w = take(sizeof(float) * (size_t)T * k);
+  W.gate = take(sizeof(float) * T);
+  W.order = take(sizeof(int32_t) * (size_t)T * k);
+  W.offsets = take(sizeof(int32_t) * (E + 1));
+  W.counts = take(sizeof(int32_t) * E);
+  W.units_rt = take(sizeof(GemmUnit) * rt_units);
+  W.units_gu = take(sizeof(GemmUnit) * tiles * (I / 64));
+  W.units_dn = take(sizeof(GemmUnit) * tiles * (H / 128));
+  W.n_units = take(sizeof(int) * 4);
+  W.acc = take(sizeof(float) * (size_t)T * H);
+  W.h = take(2 * (size_t)T * k * I);
+  W.hs = take(2 * (size_t)T * I);
+  W.total = (size_t)round_up((int64_t)pos, kAlign);
+  return W;
+}
+
+bool prefill_shape_supported(int H, int I, int bits, int E);
+cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s);
+cudaError_t launch_group(const PrefillArgs& p, cudaStream_t s);
+
 // Kernel launchers (decode.cu).  Return cudaError_t of the launch.
 cudaError_t launch_router_decode(const DecodeArgs& a, bool build_plan, cudaStream_t s);
 cudaError_t launch_plan_decode(const DecodeArgs& a, cudaStream_t s);

@@ -1,0 +1,842 @@
+// Prefill path of the routed-MoE layer (many tokens per call), sm_100a.
+//
+// The multi-token case the pages single out as the slow part («Swiftlet: 在 Mac 和 iPhone
+// 上執行…», section 社群觀點: prefill is the bottleneck for long prompts).  With T·k pairs
+// spread over E experts (about 80 tokens per expert at T = 4096, k = 10, E = 512) every
+// expert sees a real matrix product, so the expert matmuls run on the tensor cores:
+//
+//   k_norms        ||x_t|| and ||w_e|| (fp64) for the routing error bound
+//   k_gemm ROUTER  fp32 router logits on tcgen05 (bf16 x bf16 -> fp32 in TMEM)
+//   k_route        top-k with certification: every expert whose fp32 logit is within the
+//                  fp32 error bound of the k-th is recomputed exactly (fp64 sums of exact
+//                  bf16 products) and the selection is made on the exact values; softmax
+//                  over the selected logits; shared-expert gate
+//   k_group        stable counting sort of the (token, k) pairs by expert and the list of
+//                  GEMM work units (expert, row tile, token tile)
+//   k_gemm GATEUP  per unit: [gate; up] rows of one expert (dequantised to bf16 in shared
+//                  memory) x the expert's tokens (gathered), SwiGLU in the epilogue -> h
+//   k_gemm DOWN    per unit: down rows x the expert's h, weighted scatter-add into an fp32
+//                  accumulator (the shared expert is one more "expert" over all tokens)
+//   k_finalize     out = bf16(acc + residual)
+//
+// GEMM kernel ("swap-AB": the weight rows are the MMA's M = 128, the tokens its N <= 256):
+//   warp 0       TMEM allocation; lane 0 issues tcgen05.mma (kind::f16, cta_group::1)
+//   warps 1..3   gather the tokens' activation rows with cp.async (zero rows beyond N)
+//   warps 4..11  dequantise the weight rows (w = s*q + b, rounded to bf16) into shared memory
+//   warps 12..15 epilogue: tcgen05.ld of the fp32 accumulator, then SwiGLU / scatter / store
+// Operands are K-major with no swizzle: 8-row x 16-byte core matrices, k-octets 128 bytes
+// apart (LBO) and 8-row groups 1024 bytes apart (SBO) for a 64-wide K stage.  Four stages,
+// two TMEM accumulators of 256 columns so the epilogue of one unit overlaps the next.
+// Every wait is bounded; on timeout the kernel flags MOE_DEVERR_TIMEOUT, drains and frees
+// its TMEM.
+#include "common.cuh"
+#include "kernels.cuh"
+#include "sync.cuh"
+
+#include <cuda_bf16.h>
+
+namespace moe {
+namespace {
+
+constexpr int kKC = 64;                   // K per stage
+constexpr int kStagesG = 4;
+constexpr int kNmax = 256;                // tokens per unit (MMA N)
+constexpr int kABytes = 128 * kKC * 2;    // 16 KB
+constexpr int kBBytes = kNmax * kKC * 2;  // 32 KB
+constexpr int kGemmThreads = 512;
+constexpr int kBWarp0 = 1, kBWarps = 3;
+constexpr int kAWarp0 = 4, kAWarps = 8;
+constexpr int kEWarp0 = 12, kEWarps = 4;
+constexpr int kSBO = (kKC / 8) * 128;     // 1024
+
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((128u >> 4) & 0x3FFFu) << 16;   // LBO: next k-octet
+  d |= (uint64_t)(((uint32_t)kSBO >> 4) & 0x3FFFu) << 32;  // SBO: next 8-row group
+  d |= (uint64_t)1 << 46;                         // descriptor version (sm_100)
+  return d;                                       // base offset 0, no swizzle
+}
+
+__device__ __forceinline__ uint32_t umma_idesc(int n) {
+  // kind::f16: D fp32, A bf16, B bf16, both K-major, M = 128
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&p);
+}
+
+// 8 int4 codes (one 32-bit word, element j at bits 4j) -> 8 bf16 values of s*q + b.
+__device__ __forceinline__ uint4 dq8_int4(uint32_t w, float s, float b) {
+  float v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = fmaf(s, (float)((w >> (4 * j)) & 0xFu), b);
+  return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+}
+// 8 int8 codes (two words) -> 8 bf16 values.
+__device__ __forceinline__ uint4 dq8_int8(uint32_t w0, uint32_t w1, float s, float b) {
+  float v[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    v[j] = fmaf(s, (float)((w0 >> (8 * j)) & 0xFFu), b);
+    v[4 + j] = fmaf(s, (float)((w1 >> (8 * j)) & 0xFFu), b);
+  }
+  return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+}
+
+__device__ __forceinline__ int core_off(int row, int koct) {  // byte offset in a stage tile
+  return (row >> 3) * kSBO + koct * 128 + (row & 7) * 16;
+}
+
+__device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, Ctrl* c) {
+  if (mbar_wait(bar, parity)) return true;
+  atomicOr(&c->err, kErrTimeout);
+  return false;
+}
+
+// ---------------------------------------------------------------------------------------
+// GEMM kernel
+// ---------------------------------------------------------------------------------------
+template <int BITS, int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant__ GemmArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ __align__(8) uint64_t a_full[kStagesG], b_full[kStagesG], empty[kStagesG], acc_full[2], acc_empty[2],
+      drain;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int K = (MODE == kModeDown) ? a.I : a.H;
+  const int nK = K / kKC;
+  const int n_units = *a.n_units;
+  const uint32_t smem_base = smem_u32(smem);
+
+  if (tid == 0) {
+    for (int s = 0; s < kStagesG; ++s) {
+      mbar_init(&a_full[s], kAWarps);
+      mbar_init(&b_full[s], kBWarps);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEWarps);
+    }
+    mbar_init(&drain, 1);
+    s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                 "r"(512u));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 0) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      uint32_t q = 0;
+      int it = 0;
+      for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x, ++it) {
+        const GemmUnit U = a.units[u];
+        const int npad = (U.n + 15) & ~15;
+        const uint32_t idesc = umma_idesc(npad);
+        const int buf = it & 1;
+        if (!wait_or_flag(&acc_empty[buf], ((it >> 1) & 1) ^ 1, a.ctrl)) {
+          s_abort = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)buf * 256u;
+        for (int kc = 0; kc < nK; ++kc, ++q) {
+          const int s = q % kStagesG;
+          const uint32_t par = (q / kStagesG) & 1;
+          if (!wait_or_flag(&a_full[s], par, a.ctrl) || !wait_or_flag(&b_full[s], par, a.ctrl)) {
+            s_abort = 1;
+            break;
+          }
+          proxy_fence();
+          tc_fence_after();
+          const uint32_t a_base = smem_base + s * (kABytes + kBBytes);
+          const uint32_t b_base = a_base + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kKC / 16; ++kk)
+            umma_f16(d_tmem, umma_desc(a_base + kk * 256), umma_desc(b_base + kk * 256), idesc,
+                     (kc > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&empty[s]);
+        }
+        if (s_abort) break;
+        umma_commit(&acc_full[buf]);
+      }
+      // every MMA this thread issued has completed once this commit arrives
+      umma_commit(&drain);
+      if (!mbar_wait(&drain, 0)) atomicOr(&a.ctrl->err, kErrTimeout);
+    }
+    __syncwarp();
+  } else if (warp >= kBWarp0 && warp < kBWarp0 + kBWarps) {
+    // ------------------------------ B gather (cp.async) ------------------------------
+    const int bt = tid - kBWarp0 * 32;  // 0..95
+    const int bw = warp - kBWarp0;
+    uint32_t q = 0;
+    for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x) {
+      const GemmUnit U = a.units[u];
+      const int npad = (U.n + 15) & ~15;
+      const uint16_t* src_base;
+      int src_ld;
+      if (MODE == kModeDown) {
+        src_base = (U.e < 0) ? a.hs : a.h;
+        src_ld = a.I;
+      } else {
+        src_base = a.x;
+        src_ld = a.H;
+      }
+      const int n_copies = npad * (kKC / 8);  // 16-byte pieces per stage
+      for (int kc = 0; kc < nK; ++kc, ++q) {
+        const int s = q % kStagesG;
+        if (!wait_or_flag(&empty[s], ((q / kStagesG) & 1) ^ 1, a.ctrl)) {
+          s_abort = 1;
+          break;
+        }
+        const uint32_t b_base = smem_base + s * (kABytes + kBBytes) + kABytes;
+        for (int i = bt; i < n_copies; i += kBWarps * 32) {
+          // consecutive i: consecutive rows within a core matrix (conflict-free smem writes)
+          const int n = (i & 7) | ((i >> 6) << 3);
+          const int j = (i >> 3) & 7;
+          // row (token or pair position) of column n; no row beyond the unit's columns
+          int r = -1;
+          if (n < U.n) {
+            if (MODE == kModeGateUp && U.e >= 0) r = __ldg(a.order + U.p0 + n) / a.k;
+            else r = U.p0 + n;
+          }
+          const uint16_t* src = src_base + (size_t)(r < 0 ? 0 : r) * src_ld + kc * kKC + j * 8;
+          cp_async16(b_base + core_off(n, j), src, r < 0 ? 0u : 16u);
+        }
+        cp_async_commit();
+        // retire the stage issued kStagesG-2 steps ago
+        if (kc >= kStagesG - 2) {
+          cp_async_wait<kStagesG - 2>();
+          proxy_fence();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&b_full[(q - (kStagesG - 2)) % kStagesG]);
+        }
+      }
+      // retire the unit's remaining stages
+      cp_async_wait<0>();
+      proxy_fence();
+      __syncwarp();
+      if (lane == 0 && !s_abort) {
+        const int first = nK >= kStagesG - 2 ? nK - (kStagesG - 2) : 0;
+        for (int kc = first; kc < nK; ++kc) mbar_arrive(&b_full[(q - nK + kc) % kStagesG]);
+      }
+    }
+    cp_async_wait<0>();  // no copy may still be landing when the CTA leaves
+    (void)bw;
+  } else if (warp >= kAWarp0 && warp < kAWarp0 + kAWarps) {
+    // ------------------------------ A producers (dequantise) ------------------------------
+    const int at = tid - kAWarp0 * 32;  // 0..255
+    const int m = at >> 1;              // tile row 0..127
+    const int half = at & 1;            // which 32 columns of the 64-wide stage
+    uint32_t q = 0;
+    for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x) {
+      const GemmUnit U = a.units[u];
+      // this thread's weight row
+      const uint8_t* codes = nullptr;
+      const uint16_t* sc = nullptr;
+      const uint16_t* bi = nullptr;
+      const uint16_t* wrow = nullptr;
+      bool zero = false;
+      if (MODE == kModeRouter) {
+        const int e = U.mt * 128 + m;
+        if (e < a.E) wrow = a.wr + (size_t)e * a.H;
+        else if (e == a.E) wrow = a.wsg;
+        else zero = true;
+      } else {
+        const uint8_t* blob;
+        if (U.e < 0) {
+          blob = a.shared;
+        } else {
+          const int slot = a.slot_table[U.e];
+          if (slot < 0 || slot >= a.n_slots) {
+            atomicOr(&a.ctrl->err, kErrBadSlot);
+            blob = nullptr;
+          } else {
+            blob = a.pool + (int64_t)slot * a.L.stride;
+          }
+        }
+        if (!blob) {
+          zero = true;
+        } else if (MODE == kModeGateUp) {
+          const int r = U.mt * 64 + (m >> 1);
+          const int up = m & 1;  // rows alternate gate, up of the same intermediate row
+          const int rowb = a.H * BITS / 8, ng = a.H / kGroup;
+          codes = blob + a.L.off[up ? 1 : 0] + (int64_t)r * rowb;
+          sc = reinterpret_cast<const uint16_t*>(blob + a.L.off[up ? 5 : 3]) + (int64_t)r * ng;
+          bi = reinterpret_cast<const uint16_t*>(blob + a.L.off[up ? 6 : 4]) + (int64_t)r * ng;
+        } else {
+          const int j = U.mt * 128 + m;
+          const int rowb = a.I * BITS / 8, ng = a.I / kGroup;
+          codes = blob + a.L.off[2] + (int64_t)j * rowb;
+          sc = reinterpret_cast<const uint16_t*>(blob + a.L.off[7]) + (int64_t)j * ng;
+          bi = reinterpret_cast<const uint16_t*>(blob + a.L.off[8]) + (int64_t)j * ng;
+        }
+      }
+      for (int kc = 0; kc < nK; ++kc, ++q) {
+        const int s = q % kStagesG;
+        // load before waiting for the slot, so the global latency overlaps the wait
+        uint4 raw[4];
+        float sv = 0.f, bv = 0.f;
+        if (!zero) {
+          if (MODE == kModeRouter) {
+            const uint4* p = reinterpret_cast<const uint4*>(wrow + kc * kKC + half * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) raw[i] = __ldg(p + i);
+          } else if (BITS == 4) {
+            raw[0] = ld_stream(codes + kc * 32 + half * 16);
+            sv = bf1(ld_u16(sc + kc));
+            bv = bf1(ld_u16(bi + kc));
+          } else {
+            const uint8_t* p = codes + kc * 64 + half * 32;
+            raw[0] = ld_stream(p);
+            raw[1] = ld_stream(p + 16);
+            sv = bf1(ld_u16(sc + kc));
+            bv = bf1(ld_u16(bi + kc));
+          }
+        }
+        if (!wait_or_flag(&empty[s], ((q / kStagesG) & 1) ^ 1, a.ctrl)) {
+          s_abort = 1;
+          break;
+        }
+        uint8_t* a_tile = smem + s * (kABytes + kBBytes);
+#pragma unroll
+        for (int o = 0; o < 4; ++o) {  // 4 k-octets of 8 values = this thread's 32 columns
+          uint4 v;
+          if (zero) {
+            v = make_uint4(0, 0, 0, 0);
+          } else if (MODE == kModeRouter) {
+            v = raw[o];
+          } else if (BITS == 4) {
+            v = dq8_int4(o == 0 ? raw[0].x : o == 1 ? raw[0].y : o == 2 ? raw[0].z : raw[0].w, sv, bv);
+          } else {
+            const uint4 w = raw[o >> 1];
+            v = (o & 1) ? dq8_int8(w.z, w.w, sv, bv) : dq8_int8(w.x, w.y, sv, bv);
+          }
+          *reinterpret_cast<uint4*>(a_tile + core_off(m, half * 4 + o)) = v;
+        }
+        proxy_fence();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[s]);
+      }
+    }
+  } else if (warp >= kEWarp0) {
+    // ------------------------------ epilogue ------------------------------
+    const int quad = warp & 3;       // TMEM lane quadrant of this warp
+    const int m = quad * 32 + lane;  // accumulator row
+    int it = 0;
+    for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x, ++it) {
+      const GemmUnit U = a.units[u];
+      const int buf = it & 1;
+      if (!wait_or_flag(&acc_full[buf], (it >> 1) & 1, a.ctrl)) {
+        s_abort = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)buf * 256u;
+      for (int c0 = 0; c0 < U.n; c0 += 8) {
+        float v[8];
+        tmem_ld8(taddr + c0, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int n = c0 + i;
+          const float val = v[i];
+          if (MODE == kModeGateUp) {
+            const float other = __shfl_xor_sync(0xffffffffu, val, 1);
+            if (n < U.n && !(m & 1)) {
+              const float g = val, up = other;
+              const float hv = g / (1.0f + expf(-g)) * up;
+              const int r = U.mt * 64 + (m >> 1);
+              uint16_t* dst = (U.e < 0) ? a.hs + (size_t)(U.p0 + n) * a.I : a.h + (size_t)(U.p0 + n) * a.I;
+              dst[r] = f2bf(hv);
+            }
+          } else if (MODE == kModeDown) {
+            if (n < U.n) {
+              const int j = U.mt * 128 + m;
+              int t;
+              float w;
+              if (U.e < 0) {
+                t = U.p0 + n;
+                w = a.gate[t];
+              } else {
+                const int pair = a.order[U.p0 + n];
+                t = pair / a.k;
+                w = a.topk_w[pair];
+              }
+              atomicAdd(a.acc + (size_t)t * a.H + j, w * val);
+            }
+          } else {  // router logits (no bias)
+            const int e = U.mt * 128 + m;
+            if (n < U.n && e <= a.E) a.logits[(size_t)(U.p0 + n) * (a.E + 1) + e] = val;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
+  }
+
+  // drain: every role has left its loop; make sure no MMA is still writing TMEM
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512u));
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// norms for the routing error bound
+// ---------------------------------------------------------------------------------------
+__global__ void k_norms(const uint16_t* x, int T, int H, const uint16_t* wr, const uint16_t* wsg, int E,
+                        double* xnorm, double* wnorm) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int rows = T + E + 1;
+  if (warp >= rows) return;
+  const uint16_t* row = warp < T ? x + (size_t)warp * H : (warp < T + E ? wr + (size_t)(warp - T) * H : wsg);
+  double s = 0.0;
+  for (int i = lane; i < H; i += 32) {
+    const double v = (double)bf1(row[i]);
+    s += v * v;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) {
+    if (warp < T) xnorm[warp] = sqrt(s);
+    else wnorm[warp - T] = sqrt(s);
+  }
+}
+
+// Exact-product fp64 dot of two bf16 rows by one warp (fixed order).
+__device__ __forceinline__ double warp_dot_exact(const uint16_t* a, const uint16_t* b, int H) {
+  const int lane = threadIdx.x & 31;
+  double s = 0.0;
+  for (int i = lane * 8; i < H; i += 256) {
+    const uint4 va = *reinterpret_cast<const uint4*>(a + i);
+    const uint4 vb = *reinterpret_cast<const uint4*>(b + i);
+    s += (double)(bf_lo(va.x) * bf_lo(vb.x));
+    s += (double)(bf_hi(va.x) * bf_hi(vb.x));
+    s += (double)(bf_lo(va.y) * bf_lo(vb.y));
+    s += (double)(bf_hi(va.y) * bf_hi(vb.y));
+    s += (double)(bf_lo(va.z) * bf_lo(vb.z));
+    s += (double)(bf_hi(va.z) * bf_hi(vb.z));
+    s += (double)(bf_lo(va.w) * bf_lo(vb.w));
+    s += (double)(bf_hi(va.w) * bf_hi(vb.w));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
+}
+
+// ---------------------------------------------------------------------------------------
+// certified top-k: one warp per token
+// ---------------------------------------------------------------------------------------
+constexpr int kRouteCand = 96;
+
+__global__ void __launch_bounds__(256) k_gate(PrefillArgs a) {
+  const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + wl;
+  if (t >= a.T) return;
+  const double gl = warp_dot_exact(a.x + (size_t)t * a.H, a.wsg, a.H);
+  if (lane == 0) a.gate[t] = (float)(1.0 / (1.0 + exp(-gl)));
+}
+
+__global__ void __launch_bounds__(256) k_route(PrefillArgs a) {
+  __shared__ double s_cv[8][kRouteCand];
+  __shared__ int s_ce[8][kRouteCand];
+  __shared__ int s_cnt[8];
+  const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + wl;
+  if (t >= a.T) return;
+  const int E = a.E, k = a.k, H = a.H;
+  const float* lt = a.logits + (size_t)t * (E + 1);
+  const uint16_t* xt = a.x + (size_t)t * H;
+  // error bound of an fp32 sum of H exact products: |err| <= H * 2^-22 * ||x|| * ||w||
+  const double cb = (double)H * 0x1p-22 * a.xnorm[t];
+  // lower bound of the k-th best value: the k-th best lane maximum of (l - err)
+  double lmax = -INFINITY;
+  for (int e = lane; e < E; e += 32) {
+    const double b = a.rbias ? (double)a.rbias[e] : 0.0;
+    const double lo = (double)lt[e] + b - cb * a.wnorm[e];
+    lmax = fmax(lmax, lo);
+  }
+  // k-th largest of the 32 lane maxima (rank by counting; ties resolved by lane id)
+  int rank = 0;
+  for (int j = 0; j < 32; ++j) {
+    const double o = __shfl_sync(0xffffffffu, lmax, j);
+    rank += (o > lmax || (o == lmax && j < lane)) ? 1 : 0;
+  }
+  const unsigned sel = __ballot_sync(0xffffffffu, rank == k - 1);
+  const double thr = __shfl_sync(0xffffffffu, lmax, __ffs(sel) - 1);
+  // candidates: upper bound reaches the threshold
+  if (lane == 0) s_cnt[wl] = 0;
+  __syncwarp();
+  bool overflow = false;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int e = e0 + lane;
+    bool c = false;
+    if (e < E) {
+      const double b = a.rbias ? (double)a.rbias[e] : 0.0;
+      c = ((double)lt[e] + b + cb * a.wnorm[e]) >= thr || !((double)lt[e] == (double)lt[e]);
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, c);
+    const int base = s_cnt[wl];
+    if (c) {
+      const int pos = base + __popc(m & ((1u << lane) - 1));
+      if (pos < kRouteCand) s_ce[wl][pos] = e;
+    }
+    __syncwarp();
+    if (lane == 0) s_cnt[wl] = base + __popc(m);
+    __syncwarp();
+  }
+  int n = s_cnt[wl];
+  if (n > kRouteCand) {
+    overflow = true;  // recompute everything exactly (rare: many near-equal logits)
+    n = E;
+  }
+  // exact values of the candidates (fp64 sums of exact products, fixed order)
+  if (!overflow) {
+    for (int i = 0; i < n; ++i) {
+      const int e = s_ce[wl][i];
+      const double v = warp_dot_exact(xt, a.wr + (size_t)e * H, H) + (a.rbias ? (double)a.rbias[e] : 0.0);
+      if (lane == 0) s_cv[wl][i] = v;
+    }
+  }
+  __syncwarp();
+  // select the k best exact keys (value desc, id asc) by k rounds over the candidates
+  double sv = -INFINITY;
+  int se = 0x7fffffff;
+  if (!overflow) {
+    uint32_t taken[(kRouteCand + 31) / 32] = {0, 0, 0};
+    for (int r = 0; r < k; ++r) {
+      double bv = -INFINITY;
+      int be = 0x7fffffff, bi = -1;
+      for (int i = lane; i < n; i += 32) {
+        if ((taken[i >> 5] >> (i & 31)) & 1u) continue;
+        const double v = s_cv[wl][i];
+        const int e = s_ce[wl][i];
+        if (v > bv || (v == bv && e < be) || bi < 0) {
+          if (v == v) {
+            bv = v;
+            be = e;
+            bi = i;
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (oi >= 0 && (bi < 0 || ov > bv || (ov == bv && oe < be))) {
+          bv = ov;
+          be = oe;
+          bi = oi;
+        }
+      }
+      if (bi >= 0) taken[bi >> 5] |= 1u << (bi & 31);
+      if (lane == r) {
+        sv = bv;
+        se = bi >= 0 ? be : 0x7fffffff;
+      }
+    }
+  } else {
+    // exact value of every expert, k rounds of warp arg-max
+    uint32_t taken[kMaxExperts / 32] = {};
+    for (int r = 0; r < k; ++r) {
+      double bv = -INFINITY;
+      int be = 0x7fffffff;
+      for (int e = 0; e < E; ++e) {
+        if ((taken[e >> 5] >> (e & 31)) & 1u) continue;
+        const double v = warp_dot_exact(xt, a.wr + (size_t)e * H, H) + (a.rbias ? (double)a.rbias[e] : 0.0);
+        if (v == v && (be == 0x7fffffff || v > bv || (v == bv && e < be))) {
+          bv = v;
+          be = e;
+        }
+      }
+      if (be != 0x7fffffff) taken[be >> 5] |= 1u << (be & 31);
+      if (lane == r) {
+        sv = bv;
+        se = be;
+      }
+    }
+  }
+  const double v0 = __shfl_sync(0xffffffffu, sv, 0);
+  const bool valid = lane < k && se != 0x7fffffff;
+  const double ex = valid ? exp(sv - v0) : 0.0;
+  double den = ex;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  if (lane < k) {
+    if (!valid) atomicOr(&a.ctrl->err, kErrNonFinite);
+    a.topk_idx[t * k + lane] = valid ? se : -1;
+    a.topk_w[t * k + lane] = valid ? (float)(ex / den) : 0.f;
+  }
+  const double gl = warp_dot_exact(xt, a.wsg, H);
+  if (lane == 0) a.gate[t] = (float)(1.0 / (1.0 + exp(-gl)));
+}
+
+// ---------------------------------------------------------------------------------------
+// stable counting sort of the pairs by expert, and the GEMM work units (one CTA)
+// ---------------------------------------------------------------------------------------
+constexpr int kGroupThreads = 1024;
+
+__global__ void __launch_bounds__(kGroupThreads) k_group(PrefillArgs a) {
+  extern __shared__ int gsm[];
+  const int E = a.E, n = a.T * a.k;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, NWp = kGroupThreads / 32;
+  int* hist = gsm;             // [NWp][E] per-warp counts, then per-warp running positions
+  int* cnt = gsm + NWp * E;    // [E]
+  int* off = cnt + E;          // [E + 1]
+  for (int i = threadIdx.x; i < NWp * E; i += kGroupThreads) hist[i] = 0;
+  __syncthreads();
+  const int seg = (n + NWp - 1) / NWp;
+  const int p0 = warp * seg, p1 = min(n, p0 + seg);
+  // pass 1: per-warp histograms, in pair order
+  for (int b = p0; b < p1; b += 32) {
+    const int p = b + lane;
+    int e = -1;
+    if (p < p1) {
+      e = a.topk_idx[p];
+      if (e < 0 || e >= E) {
+        atomicOr(&a.ctrl->err, kErrBadExpert);
+        e = -1;
+      }
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) hist[warp * E + e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // counts and offsets
+  for (int e = threadIdx.x; e < E; e += kGroupThreads) {
+    int c = 0;
+    for (int w = 0; w < NWp; ++w) c += hist[w * E + e];
+    cnt[e] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int e = 0; e < E; ++e) {
+      off[e] = acc;
+      acc += cnt[e];
+    }
+    off[E] = acc;
+  }
+  __syncthreads();
+  // running position of each (warp, expert): offset + counts of earlier warps
+  for (int e = threadIdx.x; e < E; e += kGroupThreads) {
+    int pos = off[e];
+    for (int w = 0; w < NWp; ++w) {
+      const int c = hist[w * E + e];
+      hist[w * E + e] = pos;
+      pos += c;
+    }
+  }
+  __syncthreads();
+  // pass 2: stable scatter
+  for (int b = p0; b < p1; b += 32) {
+    const int p = b + lane;
+    int e = -1;
+    if (p < p1) {
+      e = a.topk_idx[p];
+      if (e < 0 || e >= E) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0) {
+      const int rank = __popc(peers & ((1u << lane) - 1));
+      a.order[hist[warp * E + e] + rank] = p;
+    }
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) hist[warp * E + e] += __popc(peers);
+    __syncwarp();
+  }
+  for (int e = threadIdx.x; e <= E; e += kGroupThreads) {
+    a.offsets[e] = off[e];
+    if (e < E) a.counts[e] = cnt[e];
+  }
+  __syncthreads();
+  // work units: per expert, token tiles of <= 256 pairs x row tiles; then the shared expert.
+  // Tile bases by an exclusive scan of the experts' tile counts (one expert per thread).
+  __syncthreads();
+  int* tile_base = hist;  // reuse: [E + 1]
+  for (int e = threadIdx.x; e < E; e += kGroupThreads) tile_base[e] = (cnt[e] + kNmax - 1) / kNmax;
+  __syncthreads();
+  if (threadIdx.x < 32) {  // one warp scans E <= 1024 counts in 32-wide chunks
+    int carry = 0;
+    for (int c0 = 0; c0 < E; c0 += 32) {
+      const int e = c0 + lane;
+      const int v = e < E ? tile_base[e] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (e < E) tile_base[e] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) tile_base[E] = carry;
+  }
+  __syncthreads();
+  const int mt_gu = a.I / 64, mt_dn = a.H / 128;
+  for (int e = threadIdx.x; e < E; e += kGroupThreads) {
+    int tb = tile_base[e];
+    for (int s0 = 0; s0 < cnt[e]; s0 += kNmax, ++tb) {
+      const int nn = min(kNmax, cnt[e] - s0);
+      for (int mt = 0; mt < mt_gu; ++mt) a.units_gu[tb * mt_gu + mt] = GemmUnit{e, mt, off[e] + s0, nn};
+      for (int mt = 0; mt < mt_dn; ++mt) a.units_dn[tb * mt_dn + mt] = GemmUnit{e, mt, off[e] + s0, nn};
+    }
+  }
+  const int tiles_r = tile_base[E];
+  const int st_n = (a.T + kNmax - 1) / kNmax;
+  for (int i = threadIdx.x; i < st_n * mt_gu; i += kGroupThreads) {
+    const int st = i / mt_gu, mt = i - st * mt_gu, t0 = st * kNmax;
+    a.units_gu[(tiles_r + st) * mt_gu + mt] = GemmUnit{-1, mt, t0, min(kNmax, a.T - t0)};
+  }
+  for (int i = threadIdx.x; i < st_n * mt_dn; i += kGroupThreads) {
+    const int st = i / mt_dn, mt = i - st * mt_dn, t0 = st * kNmax;
+    a.units_dn[(tiles_r + st) * mt_dn + mt] = GemmUnit{-1, mt, t0, min(kNmax, a.T - t0)};
+  }
+  if (threadIdx.x == 0) {
+    a.n_units[0] = (tiles_r + st_n) * mt_gu;
+    a.n_units[1] = (tiles_r + st_n) * mt_dn;
+  }
+}
+
+__global__ void k_finalize(const float* acc, const uint16_t* residual, uint16_t* out, size_t n) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = f2bf(acc[i] + (residual ? bf1(residual[i]) : 0.f));
+}
+
+__global__ void k_router_units(GemmUnit* units, int* n_units, int T, int E) {
+  // (E + 1) rows in tiles of 128 x tokens in tiles of 128
+  const int mt_n = (E + 1 + 127) / 128;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int nt = (T + 127) / 128;
+  if (i < mt_n * nt) {
+    const int mt = i % mt_n, tt = i / mt_n;
+    units[i] = GemmUnit{-2, mt, tt * 128, min(128, T - tt * 128)};
+  }
+  if (i == 0) *n_units = mt_n * nt;
+}
+
+template <int BITS, int MODE>
+cudaError_t launch_gemm(const GemmArgs& g, int n_sm, cudaStream_t s) {
+  const size_t smem = (size_t)kStagesG * (kABytes + kBBytes);
+  auto fn = k_gemm<BITS, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  fn<<<n_sm, kGemmThreads, smem, s>>>(g);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_shape_supported(int H, int I, int bits, int E) {
+  return (bits == 4 || bits == 8) && H % 128 == 0 && I % 64 == 0 && E <= 512 && H <= 8192 && I <= 4096;
+}
+
+cudaError_t launch_group(const PrefillArgs& p, cudaStream_t s) {
+  const size_t smem = sizeof(int) * ((size_t)(kGroupThreads / 32) * p.E + 2 * p.E + 2);
+  cudaError_t e = cudaFuncSetAttribute(k_group, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_group<<<1, kGroupThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
+  int dev = 0, n_sm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  const int T = p.T, E = p.E, H = p.H;
+  cudaError_t e;
+  // accumulator of the down products
+  if ((e = cudaMemsetAsync(p.acc, 0, sizeof(float) * (size_t)T * H, s)) != cudaSuccess) return e;
+  // norms, router logits, certified top-k
+  {
+    const int rows = T + E + 1;
+    if (p.route) {
+      k_norms<<<(rows * 32 + 255) / 256, 256, 0, s>>>(p.x, T, H, p.wr, p.wsg, E, p.xnorm, p.wnorm);
+      const int mt_n = (E + 1 + 127) / 128, nt = (T + 127) / 128;
+      k_router_units<<<(mt_n * nt + 255) / 256, 256, 0, s>>>(p.units_rt, p.n_units + 2, T, E);
+      GemmArgs g = p.g;
+      g.units = p.units_rt;
+      g.n_units = p.n_units + 2;
+      if ((e = (bits == 4 ? launch_gemm<4, kModeRouter>(g, n_sm, s) : launch_gemm<8, kModeRouter>(g, n_sm, s))) !=
+          cudaSuccess)
+        return e;
+      k_route<<<(T + 7) / 8, 256, 0, s>>>(p);
+    } else {
+      k_gate<<<(T + 7) / 8, 256, 0, s>>>(p);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // grouping and work units
+  if ((e = launch_group(p, s)) != cudaSuccess) return e;
+  // gate/up + SwiGLU, then down + scatter
+  {
+    GemmArgs g = p.g;
+    g.units = p.units_gu;
+    g.n_units = p.n_units;
+    if ((e = (bits == 4 ? launch_gemm<4, kModeGateUp>(g, n_sm, s) : launch_gemm<8, kModeGateUp>(g, n_sm, s))) !=
+        cudaSuccess)
+      return e;
+    g.units = p.units_dn;
+    g.n_units = p.n_units + 1;
+    if ((e = (bits == 4 ? launch_gemm<4, kModeDown>(g, n_sm, s) : launch_gemm<8, kModeDown>(g, n_sm, s))) !=
+        cudaSuccess)
+      return e;
+  }
+  const size_t n = (size_t)T * H;
+  k_finalize<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p.acc, p.residual, p.out, n);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -88,8 +88,9 @@ def test_layer_forward_rejects_before_any_device_work():
     st = abi.lib().moe_layer_forward(ctypes.byref(s2), 16, 1, 16, None, None, None, 256, 16, 1, 256, 16, None, 16,
                                      None, None, 256, 1 << 20, None)
     assert st == -5
-    # T beyond the decode path
-    st = abi.lib().moe_layer_forward(ctypes.byref(s), 16, 9, 16, None, None, None, 256, 16, 1, 256, 16, None, 16,
+    # many tokens on a shape without a prefill kernel (E > 512)
+    s3 = abi.make_shape(2048, 512, 512, 600, 10, 4)
+    st = abi.lib().moe_layer_forward(ctypes.byref(s3), 16, 9, 16, None, None, None, 256, 16, 1, 256, 16, None, 16,
                                      None, None, 256, 1 << 30, None)
     assert st == -5
     # misaligned x
