@@ -401,6 +401,252 @@ def decode_line(args, w, T, r, n_gpus, peaks, peak_kind, cpu_base):
     return line
 
 
+# ======================================================================================
+# prefill workload (many tokens in one call)
+# ======================================================================================
+def prefill_flops(w, T):
+    """Algorithmic FLOPs of one call (padding excluded): router, routed experts, shared expert."""
+    H, I, Is, E, k = w.hidden, w.inter, w.shared_inter, w.n_experts, w.top_k
+    router = 2 * T * H * (E + 1)
+    gateup = 2 * T * k * 2 * H * I + 2 * T * 2 * H * Is
+    down = 2 * T * k * I * H + 2 * T * Is * H
+    return router, gateup, down
+
+
+def run_prefill(args, w, T, device, rank):
+    from int4_expert_gemv_router_b200 import abi, build
+    build.build()
+    K, W = args.steps, args.warmup
+    L = synth.make_layer(w, 0, device)
+    shape = abi.shape_of(w)
+    n_in = 3
+    xs = [synth.activations(w, rank_step_seed(rank, s), tokens=T, device=device) for s in range(n_in)]
+    xbuf = torch.empty_like(xs[0])
+    out = torch.empty(T, w.hidden, dtype=torch.bfloat16, device=device)
+    idx = torch.empty(T, w.top_k, dtype=torch.int32, device=device)
+    p = torch.empty(T, w.top_k, dtype=torch.float32, device=device)
+    slots = torch.arange(w.n_experts, dtype=torch.int32, device=device)
+    ws = torch.zeros(abi.moe_workspace_size(shape, T), dtype=torch.uint8, device=device)
+    stream = torch.cuda.Stream(device)
+
+    def call():
+        abi.moe_layer_forward(shape, xbuf, T, L.w_router, L.router_bias, None, None, L.pool, slots, w.n_experts,
+                              L.shared, L.w_sg, xbuf, out, idx, p, ws)
+
+    def step(i):
+        xbuf.copy_(xs[i % n_in], non_blocking=True)
+        call()
+
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            step(i)
+    stream.synchronize()
+    barrier(device)
+    clk = ClockSampler(device.index)
+    clk.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(K):
+            step(i)
+        e1.record(stream)
+    e1.synchronize()
+    clocks = clk.stop()
+    barrier(device)
+    ms = reduce_max(e0.elapsed_time(e1), device)
+    flags = abi.moe_ws_check(ws, stream)
+    # per-kernel durations through the library's events hook (5 groups, see moe_profile_events)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+    for ev in evs:
+        ev.record(stream)
+    kern = [[] for _ in range(5)]
+    for r in range(3):
+        with torch.cuda.stream(stream):
+            xbuf.copy_(xs[r % n_in], non_blocking=True)
+            torch.cuda._sleep(20_000_000)
+            abi.moe_profile_events(evs, 5)
+            call()
+            abi.moe_profile_events(None)
+        stream.synchronize()
+        for g in range(5):
+            kern[g].append(event_ms(evs[2 * g], evs[2 * g + 1]))
+    kern_us = [1e3 * statistics.mean(v) for v in kern]
+    # end to end: pinned host x in, out back, every step
+    x_host = [x.cpu().pin_memory() for x in xs]
+    out_host = torch.empty(T, w.hidden, dtype=torch.bfloat16).pin_memory()
+    barrier(device)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for i in range(K):
+            xbuf.copy_(x_host[i % n_in], non_blocking=True)
+            call()
+            out_host.copy_(out, non_blocking=True)
+        f1.record(stream)
+    f1.synchronize()
+    e2e_ms = reduce_max(f0.elapsed_time(f1), device)
+    counts = np.bincount(idx.cpu().numpy().reshape(-1), minlength=w.n_experts)
+    return dict(ms=ms, clocks=clocks, flags=flags, kern_us=kern_us, e2e_ms=e2e_ms, layer=L, x=xs[0],
+                tokens_per_expert=(float(counts.mean()), int(counts.min()), int(counts.max())))
+
+
+def cpu_baseline_prefill(w, T, r, n_sample=32):
+    """The fp64 oracle as it stands on host cores: routing and outputs of a seeded sample of
+    the call's tokens (copies to the host not timed), scaled to tokens/s."""
+    import oracle
+    L = r["layer"]
+    sample = np.sort(np.random.default_rng(0).choice(T, n_sample, replace=False))
+    x = r["x"][torch.from_numpy(sample).to(r["x"].device)]
+    xb, wr, wsg = _bits(x), _bits(L.w_router), _bits(L.w_sg)
+    pre, _ = oracle.route(oracle.router_logits(xb, wr, None), w.top_k)
+    blobs = {int(e): L.pool[int(e)].cpu().numpy() for e in set(pre.reshape(-1).tolist())}
+    shared = L.shared.cpu().numpy()
+    t0 = time.perf_counter()
+    oracle.layer_forward(xb, wr, None, w.top_k, lambda e: blobs[e], shared, wsg, w.hidden, w.inter,
+                         w.shared_inter, w.bits, residual_bits=xb)
+    dt = time.perf_counter() - t0
+    return {"value": round(n_sample / dt, 3), "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{n_sample} of the {T} tokens (seeded), routing + experts + shared expert, fp64 numpy "
+                      f"oracle ({dt:.1f} s), scaled to tokens/s"}
+
+
+def prefill_line(args, w, T, r, n_gpus, peaks, peak_kind, cpu_base):
+    K = args.steps
+    router_f, gu_f, dn_f = prefill_flops(w, T)
+    total_f = router_f + gu_f + dn_f
+    step_s = r["ms"] / 1e3 / K
+    value = n_gpus * T * K / (r["ms"] / 1e3)
+    peak = peaks["bf16_tflops"]
+    gu_us = r["kern_us"][2]
+    achieved = gu_f / (gu_us * 1e-6) / 1e12
+    line = {
+        "metric": "routed-MoE layer tokens/s; tensor % (prefill)",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": n_gpus, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(r["ms"] / K, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": f"int{w.bits} weights dequantised to bf16, bf16 x bf16 -> fp32 (tcgen05)",
+        "data": "synthetic (seeded; weights ~N(0,0.02) quantised, x ~N(0,1))",
+        "config": {"workload": w.name, "hidden": w.hidden, "n_experts": w.n_experts, "top_k": w.top_k,
+                   "inter": w.inter, "shared_inter": w.shared_inter, "bits": w.bits, "group": 64,
+                   "tokens_per_call": T, "layers": 1, "parallelism": f"replicas{n_gpus}",
+                   "l2": "inputs exceed L2 (906 MB of expert blobs per call)",
+                   "tokens_per_expert_mean_min_max": r["tokens_per_expert"]},
+        "tensor_step": {"flops_per_call": total_f, "achieved_tflops": round(total_f / step_s / 1e12, 1),
+                        "frac_of_measured": round(total_f / step_s / 1e12 / peak, 4)},
+        "roofline": {"bound": "tensor", "kernel": "k_gemm<GATEUP> (gate/up grouped GEMM + SwiGLU)",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None, "launch_us": round(gu_us, 2),
+                     "flops_per_launch": gu_f, "peak_kind": f"{peak_kind} bf16_tflops (burst)"},
+        "kernels_us": {"router+topk": round(r["kern_us"][0], 2), "group": round(r["kern_us"][1], 2),
+                       "gateup_gemm": round(r["kern_us"][2], 2), "down_gemm": round(r["kern_us"][3], 2),
+                       "finalize": round(r["kern_us"][4], 2)},
+        "clocks": r["clocks"],
+        "e2e": {"value": round(n_gpus * T * K / (r["e2e_ms"] / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * w.hidden * 2, "d2h_bytes_per_step": T * w.hidden * 2},
+        "gpu_launches": 8 * K,
+        "device_error_flags": r["flags"],
+    }
+    if cpu_base is not None:
+        line["cpu_baseline"] = cpu_base
+    return line
+
+
+# ======================================================================================
+# bounded slot pool (25% of experts resident, LFU + recency, misses from pinned host)
+# ======================================================================================
+def run_pool(args, w, device, rank, total_steps=1024):
+    """Decode steps of one layer through the bounded pool: router -> moe_expert_pool_load (reads
+    the ids back, loads the misses on the pool's side stream) -> layer forward on the slots.
+    W warm-up steps, then the timed steps; at least total_steps steps run for the hit rate."""
+    from int4_expert_gemv_router_b200 import abi, build
+    build.build()
+    K, W = args.steps, args.warmup
+    n_total = max(total_steps, K + W)
+    L = synth.make_layer(w, 0, device)
+    host_blobs = L.pool.cpu().pin_memory()
+    stride = L.pool.shape[1]
+    del L.pool
+    torch.cuda.empty_cache()
+    shape = abi.shape_of(w)
+    dev_pool = torch.zeros(w.n_slots, stride, dtype=torch.uint8, device=device)
+    table = torch.empty(w.n_experts, dtype=torch.int32, device=device)
+    pool = abi.moe_pool_create(shape, w.n_slots, host_blobs, dev_pool, table)
+    T = 1
+    xs = torch.stack([synth.activations(w, rank_step_seed(rank, s), tokens=T, device=device) for s in range(n_total)])
+    out = torch.empty(T, w.hidden, dtype=torch.bfloat16, device=device)
+    idx = torch.empty(T, w.top_k, dtype=torch.int32, device=device)
+    p = torch.empty(T, w.top_k, dtype=torch.float32, device=device)
+    ws = torch.zeros(abi.moe_workspace_size(shape, T), dtype=torch.uint8, device=device)
+    stream = torch.cuda.Stream(device)
+    popularity = np.zeros(w.n_experts, dtype=np.int64)
+
+    def step(i):
+        x = xs[i]
+        abi.moe_router_topk(shape, x, T, L.w_router, L.router_bias, idx, p, ws)
+        abi.moe_expert_pool_load(pool, idx, T)
+        abi.moe_layer_forward(shape, x, T, L.w_router, L.router_bias, idx, p, dev_pool, table, w.n_slots,
+                              L.shared, L.w_sg, x, out, None, None, ws)
+
+    t_start = n_total - K
+    with torch.cuda.stream(stream):
+        for i in range(t_start):
+            step(i)
+            if i >= W:
+                popularity[idx.cpu().numpy().reshape(-1)] += 1
+    stream.synchronize()
+    st0 = abi.moe_pool_stats(pool)
+    barrier(device)
+    clk = ClockSampler(device.index)
+    clk.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(t_start, n_total):
+            step(i)
+        e1.record(stream)
+    e1.synchronize()
+    clocks = clk.stop()
+    ms = reduce_max(e0.elapsed_time(e1), device)
+    st1 = abi.moe_pool_stats(pool)
+    flags = abi.moe_ws_check(ws, stream)
+    abi.moe_pool_destroy(pool)
+    hits = st1["hits"] - st0["hits"]
+    look = st1["lookups"] - st0["lookups"]
+    # Zipf exponent fitted to the measured popularity (log count vs log rank)
+    cnt = np.sort(popularity)[::-1]
+    cnt = cnt[cnt > 0]
+    rk = np.arange(1, len(cnt) + 1)
+    zipf_s = float(-np.polyfit(np.log(rk), np.log(cnt), 1)[0]) if len(cnt) > 2 else None
+    return dict(ms=ms, clocks=clocks, flags=flags, K=K, n_total=n_total, stats=st1,
+                hit_rate_all=st1["hits"] / max(1, st1["lookups"]), hit_rate_timed=hits / max(1, look),
+                h2d_timed=st1["h2d_bytes"] - st0["h2d_bytes"], zipf_s=zipf_s, stride=stride)
+
+
+def pool_line(args, w, r, n_gpus):
+    K = r["K"]
+    value = n_gpus * K / (r["ms"] / 1e3)
+    return {
+        "metric": "routed-MoE layer tokens/s with a bounded slot pool; expert-cache hit rate",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": n_gpus, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(r["ms"] / K, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": f"int{w.bits} weights, bf16 activations, fp32 accumulate",
+        "data": "synthetic (seeded; Zipf(1.0) router bias)",
+        "config": {"workload": w.name, "hidden": w.hidden, "n_experts": w.n_experts, "top_k": w.top_k,
+                   "bits": w.bits, "n_slots": w.n_slots, "slot_fraction": w.n_slots / w.n_experts,
+                   "steps_total": r["n_total"], "tokens_per_step": 1, "policy": "LFU + recency",
+                   "miss_path": "pinned host -> cudaMemcpyAsync on a side stream",
+                   "timing": "events around the timed steps; each step waits on the host for the ids"},
+        "pool": {"hit_rate_all_steps": round(r["hit_rate_all"], 4), "hit_rate_timed": round(r["hit_rate_timed"], 4),
+                 "stats": r["stats"], "h2d_bytes_timed": r["h2d_timed"],
+                 "h2d_gbs_timed": round(r["h2d_timed"] / (r["ms"] / 1e3) / 1e9, 2),
+                 "fitted_zipf_s": None if r["zipf_s"] is None else round(r["zipf_s"], 3)},
+        "clocks": r["clocks"],
+        "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
+                "note": "inputs resident; the per-step D2H of the ids and H2D of misses are inside the timing"},
+        "gpu_launches": 6 * K,
+        "device_error_flags": r["flags"],
+    }
+
+
 # --------------------------------------------------------------------------------------
 # reference arm: the fp64 oracle on host cores
 # --------------------------------------------------------------------------------------
@@ -460,7 +706,8 @@ def parse(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode80b", choices=["decode80b", "decode35b"])
+    ap.add_argument("--workload", default="decode80b",
+                    choices=["decode80b", "decode35b", "prefill", "pool_int4", "pool_int8"])
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
@@ -488,11 +735,21 @@ def main(argv=None):
     device = torch.device("cuda", local)
     init_dist("nccl")
     peaks, peak_kind = load_peaks()
-    r = run_decode(args, w, T, device, rank, ws)
     cpu_base = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        cpu_base = cpu_baseline_decode(w, T, device, r["stack"])
-    line = decode_line(args, w, T, r, ws, peaks, peak_kind, cpu_base)
+    want_cpu = rank == 0 and ws == 1 and not args.no_cpu_baseline
+    if w.name == "prefill":
+        r = run_prefill(args, w, T, device, rank)
+        if want_cpu:
+            cpu_base = cpu_baseline_prefill(w, T, r)
+        line = prefill_line(args, w, T, r, ws, peaks, peak_kind, cpu_base)
+    elif w.name.startswith("pool"):
+        r = run_pool(args, w, device, rank)
+        line = pool_line(args, w, r, ws)
+    else:
+        r = run_decode(args, w, T, device, rank, ws)
+        if want_cpu:
+            cpu_base = cpu_baseline_decode(w, T, device, r["stack"])
+        line = decode_line(args, w, T, r, ws, peaks, peak_kind, cpu_base)
     if rank == 0:
         print(json.dumps(line), flush=True)
     import torch.distributed as dist

@@ -304,8 +304,10 @@ MOE_API void moe_pool_destroy(moe_pool* pool);
  * moe_profile_events -- measurement hook.  While set (events != NULL), each
  * moe_layer_forward / moe_router_topk call on this thread records events[2*i] on its stream
  * just before its i-th kernel launch and events[2*i+1] just after it, for i < n
- * (i = 0: router or grouping, 1: gate/up + SwiGLU, 2: down + combine).  events are
- * cudaEvent_t handles owned by the caller.  Thread-local; NULL disables.
+ * (decode, unfused: 0 router or grouping, 1 gate/up + SwiGLU, 2 down + combine; decode,
+ * fused: 0 the persistent kernel; many tokens: 0 norms + router GEMM + certified top-k,
+ * 1 grouping, 2 gate/up GEMM, 3 down GEMM, 4 final sum).  events are cudaEvent_t handles
+ * owned by the caller.  Thread-local; NULL disables.
  */
 MOE_API moe_status moe_profile_events(void* const* events, int32_t n);
 

@@ -284,6 +284,8 @@ inline PrefillLayout make_prefill_layout(int T, int E, int k, int H, int I) {
 }
 
 bool prefill_shape_supported(int H, int I, int bits, int E);
+// Profiling hook of moe_profile_events (api.cu): event pair i around kernel group i.
+void prof_mark(int i, bool end, cudaStream_t s);
 cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s);
 cudaError_t launch_group(const PrefillArgs& p, cudaStream_t s);
 

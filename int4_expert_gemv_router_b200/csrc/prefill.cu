@@ -800,6 +800,7 @@ cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
   // accumulator of the down products
   if ((e = cudaMemsetAsync(p.acc, 0, sizeof(float) * (size_t)T * H, s)) != cudaSuccess) return e;
   // norms, router logits, certified top-k
+  prof_mark(0, false, s);
   {
     const int rows = T + E + 1;
     if (p.route) {
@@ -818,24 +819,33 @@ cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  prof_mark(0, true, s);
   // grouping and work units
+  prof_mark(1, false, s);
   if ((e = launch_group(p, s)) != cudaSuccess) return e;
+  prof_mark(1, true, s);
   // gate/up + SwiGLU, then down + scatter
   {
     GemmArgs g = p.g;
     g.units = p.units_gu;
     g.n_units = p.n_units;
+    prof_mark(2, false, s);
     if ((e = (bits == 4 ? launch_gemm<4, kModeGateUp>(g, n_sm, s) : launch_gemm<8, kModeGateUp>(g, n_sm, s))) !=
         cudaSuccess)
       return e;
+    prof_mark(2, true, s);
     g.units = p.units_dn;
     g.n_units = p.n_units + 1;
+    prof_mark(3, false, s);
     if ((e = (bits == 4 ? launch_gemm<4, kModeDown>(g, n_sm, s) : launch_gemm<8, kModeDown>(g, n_sm, s))) !=
         cudaSuccess)
       return e;
+    prof_mark(3, true, s);
   }
   const size_t n = (size_t)T * H;
+  prof_mark(4, false, s);
   k_finalize<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p.acc, p.residual, p.out, n);
+  prof_mark(4, true, s);
   return cudaGetLastError();
 }
 
