@@ -319,51 +319,67 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
           bi = reinterpret_cast<const uint16_t*>(blob + a.L.off[8]) + (int64_t)j * ng;
         }
       }
-      for (int kc = 0; kc < nK; ++kc, ++q) {
-        const int s = q % kStagesG;
-        // load before waiting for the slot, so the global latency overlaps the wait
-        uint4 raw[4];
-        float sv = 0.f, bv = 0.f;
-        if (!zero) {
-          if (MODE == kModeRouter) {
-            const uint4* p = reinterpret_cast<const uint4*>(wrow + kc * kKC + half * 32);
+      // loads run kRing stages ahead of the shared-memory stores (register ring), so each
+      // stage's global latency overlaps the dequantisation of the stages before it
+      constexpr int kRing = 4;
+      uint4 rr[kRing][4];
+      float rs[kRing], rb[kRing];
+      auto load = [&](int kc, int d) {
+        if (zero) return;
+        if (MODE == kModeRouter) {
+          const uint4* p = reinterpret_cast<const uint4*>(wrow + kc * kKC + half * 32);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) raw[i] = __ldg(p + i);
-          } else if (BITS == 4) {
-            raw[0] = ld_stream(codes + kc * 32 + half * 16);
-            sv = bf1(ld_u16(sc + kc));
-            bv = bf1(ld_u16(bi + kc));
-          } else {
-            const uint8_t* p = codes + kc * 64 + half * 32;
-            raw[0] = ld_stream(p);
-            raw[1] = ld_stream(p + 16);
-            sv = bf1(ld_u16(sc + kc));
-            bv = bf1(ld_u16(bi + kc));
-          }
+          for (int i = 0; i < 4; ++i) rr[d][i] = __ldg(p + i);
+        } else if (BITS == 4) {
+          rr[d][0] = ld_stream(codes + kc * 32 + half * 16);
+          rs[d] = bf1(ld_u16(sc + kc));
+          rb[d] = bf1(ld_u16(bi + kc));
+        } else {
+          const uint8_t* p = codes + kc * 64 + half * 32;
+          rr[d][0] = ld_stream(p);
+          rr[d][1] = ld_stream(p + 16);
+          rs[d] = bf1(ld_u16(sc + kc));
+          rb[d] = bf1(ld_u16(bi + kc));
         }
-        if (!wait_or_flag(&empty[s], ((q / kStagesG) & 1) ^ 1, a.ctrl)) {
-          s_abort = 1;
-          break;
-        }
-        uint8_t* a_tile = smem + s * (kABytes + kBBytes);
+      };
 #pragma unroll
-        for (int o = 0; o < 4; ++o) {  // 4 k-octets of 8 values = this thread's 32 columns
-          uint4 v;
-          if (zero) {
-            v = make_uint4(0, 0, 0, 0);
-          } else if (MODE == kModeRouter) {
-            v = raw[o];
-          } else if (BITS == 4) {
-            v = dq8_int4(o == 0 ? raw[0].x : o == 1 ? raw[0].y : o == 2 ? raw[0].z : raw[0].w, sv, bv);
-          } else {
-            const uint4 w = raw[o >> 1];
-            v = (o & 1) ? dq8_int8(w.z, w.w, sv, bv) : dq8_int8(w.x, w.y, sv, bv);
+      for (int d = 0; d < kRing; ++d)
+        if (d < nK) load(d, d);
+      bool stop = false;
+      for (int kc0 = 0; kc0 < nK && !stop; kc0 += kRing) {
+#pragma unroll
+        for (int d = 0; d < kRing; ++d) {
+          const int kc = kc0 + d;
+          if (kc >= nK || stop) continue;
+          const int s = q % kStagesG;
+          if (!wait_or_flag(&empty[s], ((q / kStagesG) & 1) ^ 1, a.ctrl)) {
+            s_abort = 1;
+            stop = true;
+            continue;
           }
-          *reinterpret_cast<uint4*>(a_tile + core_off(m, half * 4 + o)) = v;
+          uint8_t* a_tile = smem + s * (kABytes + kBBytes);
+#pragma unroll
+          for (int o = 0; o < 4; ++o) {  // 4 k-octets of 8 values = this thread's 32 columns
+            uint4 v;
+            if (zero) {
+              v = make_uint4(0, 0, 0, 0);
+            } else if (MODE == kModeRouter) {
+              v = rr[d][o];
+            } else if (BITS == 4) {
+              const uint4 w = rr[d][0];
+              v = dq8_int4(o == 0 ? w.x : o == 1 ? w.y : o == 2 ? w.z : w.w, rs[d], rb[d]);
+            } else {
+              const uint4 w = rr[d][o >> 1];
+              v = (o & 1) ? dq8_int8(w.z, w.w, rs[d], rb[d]) : dq8_int8(w.x, w.y, rs[d], rb[d]);
+            }
+            *reinterpret_cast<uint4*>(a_tile + core_off(m, half * 4 + o)) = v;
+          }
+          if (kc + kRing < nK) load(kc + kRing, d);
+          proxy_fence();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a_full[s]);
+          ++q;
         }
-        proxy_fence();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[s]);
       }
     }
   } else if (warp >= kEWarp0) {
@@ -638,20 +654,28 @@ __global__ void __launch_bounds__(kGroupThreads) k_group(PrefillArgs a) {
   __syncthreads();
   const int seg = (n + NWp - 1) / NWp;
   const int p0 = warp * seg, p1 = min(n, p0 + seg);
-  // pass 1: per-warp histograms, in pair order
-  for (int b = p0; b < p1; b += 32) {
-    const int p = b + lane;
-    int e = -1;
-    if (p < p1) {
-      e = a.topk_idx[p];
-      if (e < 0 || e >= E) {
+  // pass 1: per-warp histograms, in pair order; ids are loaded 8 batches at a time so the
+  // loads are in flight together
+  constexpr int kB = 8;
+  for (int b0 = p0; b0 < p1; b0 += 32 * kB) {
+    int ev[kB];
+#pragma unroll
+    for (int j = 0; j < kB; ++j) {
+      const int p = b0 + 32 * j + lane;
+      ev[j] = (p < p1) ? __ldg(a.topk_idx + p) : -1;
+    }
+#pragma unroll
+    for (int j = 0; j < kB; ++j) {
+      int e = ev[j];
+      const int p = b0 + 32 * j + lane;
+      if (p < p1 && (e < 0 || e >= E)) {
         atomicOr(&a.ctrl->err, kErrBadExpert);
         e = -1;
       }
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      if (e >= 0 && lane == __ffs(peers) - 1) hist[warp * E + e] += __popc(peers);
+      __syncwarp();
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && lane == __ffs(peers) - 1) hist[warp * E + e] += __popc(peers);
-    __syncwarp();
   }
   __syncthreads();
   // counts and offsets
@@ -681,21 +705,26 @@ __global__ void __launch_bounds__(kGroupThreads) k_group(PrefillArgs a) {
   }
   __syncthreads();
   // pass 2: stable scatter
-  for (int b = p0; b < p1; b += 32) {
-    const int p = b + lane;
-    int e = -1;
-    if (p < p1) {
-      e = a.topk_idx[p];
-      if (e < 0 || e >= E) e = -1;
+  for (int b0 = p0; b0 < p1; b0 += 32 * kB) {
+    int ev[kB];
+#pragma unroll
+    for (int j = 0; j < kB; ++j) {
+      const int p = b0 + 32 * j + lane;
+      ev[j] = (p < p1) ? __ldg(a.topk_idx + p) : -1;
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0) {
-      const int rank = __popc(peers & ((1u << lane) - 1));
-      a.order[hist[warp * E + e] + rank] = p;
+#pragma unroll
+    for (int j = 0; j < kB; ++j) {
+      const int p = b0 + 32 * j + lane;
+      const int e = (ev[j] >= 0 && ev[j] < E) ? ev[j] : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      if (e >= 0) {
+        const int rank = __popc(peers & ((1u << lane) - 1));
+        a.order[hist[warp * E + e] + rank] = p;
+      }
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) hist[warp * E + e] += __popc(peers);
+      __syncwarp();
     }
-    __syncwarp();
-    if (e >= 0 && lane == __ffs(peers) - 1) hist[warp * E + e] += __popc(peers);
-    __syncwarp();
   }
   for (int e = threadIdx.x; e <= E; e += kGroupThreads) {
     a.offsets[e] = off[e];
