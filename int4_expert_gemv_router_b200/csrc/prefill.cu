@@ -103,21 +103,35 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 // 8 int4 codes (one 32-bit word, element j at bits 4j) -> 8 bf16 values of s*q + b.
-__device__ __forceinline__ uint4 dq8_int4(uint32_t w, float s, float b) {
-  float v[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) v[j] = fmaf(s, (float)((w >> (4 * j)) & 0xFu), b);
-  return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+// The code at bit position p is turned into the exact float q*2^p by OR-ing it into the
+// mantissa of 2^23 and subtracting 2^23; multiplying by s*2^-p (exact) then gives s*q, so
+// every value is round(s*q + b) as from a direct conversion, without integer-to-float
+// instructions.  Two codes per packed fp32x2 add and FMA.
+__device__ __forceinline__ float2 ffma2p(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(reinterpret_cast<unsigned long long&>(d))
+      : "l"(reinterpret_cast<const unsigned long long&>(a)), "l"(reinterpret_cast<const unsigned long long&>(b)),
+        "l"(reinterpret_cast<const unsigned long long&>(c)));
+  return d;
 }
-// 8 int8 codes (two words) -> 8 bf16 values.
+__device__ __forceinline__ uint32_t dq2(uint32_t m0, uint32_t m1, float s0, float s1, float b) {
+  const float2 v = codes2(m0, m1);  // exact q0*2^p0, q1*2^p1
+  const float2 r = ffma2p(v, make_float2(s0, s1), make_float2(b, b));
+  return pack_bf16(r.x, r.y);
+}
+__device__ __forceinline__ uint4 dq8_int4(uint32_t w, float s, float b) {
+  const uint32_t wh = w >> 12;
+  const float s4 = s * 0x1p-4f, s8 = s * 0x1p-8f, s12 = s * 0x1p-12f, s16 = s * 0x1p-16f;
+  return make_uint4(dq2(w & 0xFu, w & 0xF0u, s, s4, b), dq2(w & 0xF00u, w & 0xF000u, s8, s12, b),
+                    dq2(w & 0xF0000u, wh & 0xF00u, s16, s8, b), dq2(wh & 0xF000u, wh & 0xF0000u, s12, s16, b));
+}
+// 8 int8 codes (two words, byte j at bits 8j) -> 8 bf16 values.
 __device__ __forceinline__ uint4 dq8_int8(uint32_t w0, uint32_t w1, float s, float b) {
-  float v[8];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    v[j] = fmaf(s, (float)((w0 >> (8 * j)) & 0xFFu), b);
-    v[4 + j] = fmaf(s, (float)((w1 >> (8 * j)) & 0xFFu), b);
-  }
-  return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+  const uint32_t h0 = w0 >> 16, h1 = w1 >> 16;
+  const float s8 = s * 0x1p-8f;
+  return make_uint4(dq2(w0 & 0xFFu, w0 & 0xFF00u, s, s8, b), dq2(h0 & 0xFFu, h0 & 0xFF00u, s, s8, b),
+                    dq2(w1 & 0xFFu, w1 & 0xFF00u, s, s8, b), dq2(h1 & 0xFFu, h1 & 0xFF00u, s, s8, b));
 }
 
 __device__ __forceinline__ int core_off(int row, int koct) {  // byte offset in a stage tile
@@ -140,6 +154,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
+  __shared__ int s_rows[kBWarps][kNmax];  // per B warp: source row of each column of the unit
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int K = (MODE == kModeDown) ? a.I : a.H;
@@ -229,6 +244,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         src_base = a.x;
         src_ld = a.H;
       }
+      // source row (token or pair position) of each column, once per unit; -1: zero row
+      for (int n = lane; n < npad; n += 32) {
+        int r = -1;
+        if (n < U.n) r = (MODE == kModeGateUp && U.e >= 0) ? __ldg(a.order + U.p0 + n) / a.k : U.p0 + n;
+        s_rows[bw][n] = r;
+      }
+      __syncwarp();
       const int n_copies = npad * (kKC / 8);  // 16-byte pieces per stage
       for (int kc = 0; kc < nK; ++kc, ++q) {
         const int s = q % kStagesG;
@@ -241,12 +263,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
           // consecutive i: consecutive rows within a core matrix (conflict-free smem writes)
           const int n = (i & 7) | ((i >> 6) << 3);
           const int j = (i >> 3) & 7;
-          // row (token or pair position) of column n; no row beyond the unit's columns
-          int r = -1;
-          if (n < U.n) {
-            if (MODE == kModeGateUp && U.e >= 0) r = __ldg(a.order + U.p0 + n) / a.k;
-            else r = U.p0 + n;
-          }
+          const int r = s_rows[bw][n];
           const uint16_t* src = src_base + (size_t)(r < 0 ? 0 : r) * src_ld + kc * kKC + j * 8;
           cp_async16(b_base + core_off(n, j), src, r < 0 ? 0u : 16u);
         }
@@ -269,7 +286,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       }
     }
     cp_async_wait<0>();  // no copy may still be landing when the CTA leaves
-    (void)bw;
   } else if (warp >= kAWarp0 && warp < kAWarp0 + kAWarps) {
     // ------------------------------ A producers (dequantise) ------------------------------
     const int at = tid - kAWarp0 * 32;  // 0..255
