@@ -189,6 +189,7 @@ struct FusedArgs {
 // Prefill path (prefill.cu)
 // ---------------------------------------------------------------------------------------
 constexpr int kModeRouter = 0, kModeGateUp = 1, kModeDown = 2;
+constexpr int kPrefillN = 128;  // tokens (MMA N) per GEMM work unit
 
 // One tcgen05 GEMM work unit: expert e (-1: shared expert, -2: router), row tile mt, first
 // column p0 (pair position, or token for the shared expert / router) and column count n.
@@ -260,7 +261,8 @@ inline PrefillLayout make_prefill_layout(int T, int E, int k, int H, int I) {
     pos = at + bytes;
     return at;
   };
-  const size_t tiles = (size_t)E + ((size_t)T * k + 255) / 256 + ((size_t)T + 255) / 256 + 1;
+  const size_t tiles = (size_t)E + ((size_t)T * k + kPrefillN - 1) / kPrefillN +
+                       ((size_t)T + kPrefillN - 1) / kPrefillN + 1;
   const size_t rt_units = (size_t)((E + 1 + 127) / 128) * ((T + 127) / 128);
   W.ctrl = take(sizeof(Ctrl));
   W.xnorm = take(sizeof(double) * T);

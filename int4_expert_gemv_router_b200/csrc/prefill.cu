@@ -19,14 +19,18 @@
 //                  accumulator (the shared expert is one more "expert" over all tokens)
 //   k_finalize     out = bf16(acc + residual)
 //
-// GEMM kernel ("swap-AB": the weight rows are the MMA's M = 128, the tokens its N <= 256):
+// GEMM kernel ("swap-AB": the weight rows are the MMA's M = 128, the tokens its N <= 128):
 //   warp 0       TMEM allocation; lane 0 issues tcgen05.mma (kind::f16, cta_group::1)
 //   warps 1..3   gather the tokens' activation rows with cp.async (zero rows beyond N)
-//   warps 4..11  dequantise the weight rows (w = s*q + b, rounded to bf16) into shared memory
+//   warps 4..11  dequantise the weight rows (w = s*q + b, rounded to bf16) into shared memory;
+//                the raw codes stream through a per-thread cp.async ring several stages ahead
+//                and each unit's row scales and biases are copied to shared memory once
 //   warps 12..15 epilogue: tcgen05.ld of the fp32 accumulator, then SwiGLU / scatter / store
 // Operands are K-major with no swizzle: 8-row x 16-byte core matrices, k-octets 128 bytes
-// apart (LBO) and 8-row groups 1024 bytes apart (SBO) for a 64-wide K stage.  Four stages,
-// two TMEM accumulators of 256 columns so the epilogue of one unit overlaps the next.
+// apart (LBO) and 8-row groups 1024 bytes apart (SBO) for a 64-wide K stage.  A and B
+// tiles have rings of their own (the B gather runs six stages ahead, its completion tracked
+// by cp.async mbarrier arrivals); two TMEM accumulators of 128 columns let the epilogue of
+// one unit overlap the next.
 // Every wait is bounded; on timeout the kernel flags MOE_DEVERR_TIMEOUT, drains and frees
 // its TMEM.
 #include "common.cuh"
@@ -39,15 +43,31 @@ namespace moe {
 namespace {
 
 constexpr int kKC = 64;                   // K per stage
-constexpr int kStagesG = 4;
-constexpr int kNmax = 256;                // tokens per unit (MMA N)
+constexpr int kNmax = kPrefillN;          // tokens per unit (MMA N)
 constexpr int kABytes = 128 * kKC * 2;    // 16 KB
-constexpr int kBBytes = kNmax * kKC * 2;  // 32 KB
+constexpr int kBBytes = kNmax * kKC * 2;  // 16 KB
 constexpr int kGemmThreads = 512;
 constexpr int kBWarp0 = 1, kBWarps = 3;
 constexpr int kAWarp0 = 4, kAWarps = 8;
 constexpr int kEWarp0 = 12, kEWarps = 4;
 constexpr int kSBO = (kKC / 8) * 128;     // 1024
+constexpr int kTmemCols = 2 * kNmax;      // two accumulators
+constexpr int kRawBytes = 32 * 1024;      // cp.async ring of raw weight bytes (A producers)
+constexpr int kAThreads = kAWarps * 32;
+// raw bytes per A thread per stage, and ring depth, per mode / width
+template <int BITS, int MODE>
+struct RawRing {
+  static constexpr int kBytes = BITS == 4 ? 16 : 32;
+  static constexpr int kDepth = kRawBytes / (kAThreads * kBytes);
+};
+// A and B tile stages (16 KB each).  The dequantising modes also hold the raw ring and the
+// unit's scales and biases (up to 32 KB at K = 4096), so they keep fewer A stages: the raw
+// ring already runs kDepth stages ahead of the dequantisation.
+template <int MODE>
+struct StageCount {
+  static constexpr int kA = MODE == kModeRouter ? 6 : 3;
+  static constexpr int kB = 6;
+};
 
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
   uint64_t d = 0;
@@ -92,6 +112,11 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// arrival on an mbarrier once every cp.async this thread has issued so far has landed
+// (.noinc: the arrival is one of the barrier's expected count)
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
@@ -144,29 +169,46 @@ __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, Ctr
   return false;
 }
 
+// Every lane of a warp waits, and all take the same branch afterwards (a lane whose wait
+// ran out would otherwise leave the others behind at the next __syncwarp).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Ctrl* c, int lane) {
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, parity) ? 1 : 0);
+  if (!ok && lane == 0) atomicOr(&c->err, kErrTimeout);
+  return ok;
+}
+
 // ---------------------------------------------------------------------------------------
 // GEMM kernel
 // ---------------------------------------------------------------------------------------
 template <int BITS, int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant__ GemmArgs a) {
+  constexpr int kSA = StageCount<MODE>::kA, kSB = StageCount<MODE>::kB;
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ __align__(8) uint64_t a_full[kStagesG], b_full[kStagesG], empty[kStagesG], acc_full[2], acc_empty[2],
-      drain;
+  __shared__ __align__(8) uint64_t a_full[kSA], a_empty[kSA], b_full[kSB], b_empty[kSB], acc_full[2],
+      acc_empty[2], drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_rows[kBWarps][kNmax];  // per B warp: source row of each column of the unit
+  __shared__ int s_colt[kEWarps][kNmax];  // per epilogue warp (down): token of each column
+  __shared__ float s_colw[kEWarps][kNmax];  // and its routing weight
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int K = (MODE == kModeDown) ? a.I : a.H;
   const int nK = K / kKC;
   const int n_units = *a.n_units;
   const uint32_t smem_base = smem_u32(smem);
+  const uint32_t b_area = smem_base + kSA * kABytes;
 
   if (tid == 0) {
-    for (int s = 0; s < kStagesG; ++s) {
-      mbar_init(&a_full[s], kAWarps);
-      mbar_init(&b_full[s], kBWarps);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < kSA; ++s) {
+      // router rows are plain copies whose completion each A thread signals; dequantised
+      // tiles are signalled once per A warp
+      mbar_init(&a_full[s], MODE == kModeRouter ? kAThreads : kAWarps);
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < kSB; ++s) {
+      mbar_init(&b_full[s], kBWarps * 32);  // one cp.async-tracking arrival per B thread
+      mbar_init(&b_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -178,7 +220,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
-                 "r"(512u));
+                 "r"((uint32_t)kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
@@ -201,23 +243,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + (uint32_t)buf * 256u;
+        const uint32_t d_tmem = tmem + (uint32_t)buf * (uint32_t)kNmax;
         for (int kc = 0; kc < nK; ++kc, ++q) {
-          const int s = q % kStagesG;
-          const uint32_t par = (q / kStagesG) & 1;
-          if (!wait_or_flag(&a_full[s], par, a.ctrl) || !wait_or_flag(&b_full[s], par, a.ctrl)) {
+          const int sa = q % kSA, sb = q % kSB;
+          if (!wait_or_flag(&a_full[sa], (q / kSA) & 1, a.ctrl) || !wait_or_flag(&b_full[sb], (q / kSB) & 1, a.ctrl)) {
             s_abort = 1;
             break;
           }
+          // the tiles were written through the generic proxy (st.shared, cp.async)
           proxy_fence();
           tc_fence_after();
-          const uint32_t a_base = smem_base + s * (kABytes + kBBytes);
-          const uint32_t b_base = a_base + kABytes;
+          const uint32_t a_base = smem_base + sa * kABytes;
+          const uint32_t b_base = b_area + sb * kBBytes;
 #pragma unroll
           for (int kk = 0; kk < kKC / 16; ++kk)
             umma_f16(d_tmem, umma_desc(a_base + kk * 256), umma_desc(b_base + kk * 256), idesc,
                      (kc > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&empty[s]);
+          umma_commit(&a_empty[sa]);
+          umma_commit(&b_empty[sb]);
         }
         if (s_abort) break;
         umma_commit(&acc_full[buf]);
@@ -229,6 +272,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     __syncwarp();
   } else if (warp >= kBWarp0 && warp < kBWarp0 + kBWarps) {
     // ------------------------------ B gather (cp.async) ------------------------------
+    // Each thread's copies of a stage are tracked by the stage's mbarrier (an arrival that
+    // fires when they have landed), so the gather runs up to kSB stages ahead of the MMAs.
     const int bt = tid - kBWarp0 * 32;  // 0..95
     const int bw = warp - kBWarp0;
     uint32_t q = 0;
@@ -252,13 +297,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       }
       __syncwarp();
       const int n_copies = npad * (kKC / 8);  // 16-byte pieces per stage
+      bool stop = false;
       for (int kc = 0; kc < nK; ++kc, ++q) {
-        const int s = q % kStagesG;
-        if (!wait_or_flag(&empty[s], ((q / kStagesG) & 1) ^ 1, a.ctrl)) {
+        const int sb = q % kSB;
+        if (!warp_wait(&b_empty[sb], ((q / kSB) & 1) ^ 1, a.ctrl, lane)) {
           s_abort = 1;
+          stop = true;
           break;
         }
-        const uint32_t b_base = smem_base + s * (kABytes + kBBytes) + kABytes;
+        const uint32_t b_base = b_area + sb * kBBytes;
         for (int i = bt; i < n_copies; i += kBWarps * 32) {
           // consecutive i: consecutive rows within a core matrix (conflict-free smem writes)
           const int n = (i & 7) | ((i >> 6) << 3);
@@ -267,137 +314,151 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
           const uint16_t* src = src_base + (size_t)(r < 0 ? 0 : r) * src_ld + kc * kKC + j * 8;
           cp_async16(b_base + core_off(n, j), src, r < 0 ? 0u : 16u);
         }
-        cp_async_commit();
-        // retire the stage issued kStagesG-2 steps ago
-        if (kc >= kStagesG - 2) {
-          cp_async_wait<kStagesG - 2>();
-          proxy_fence();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&b_full[(q - (kStagesG - 2)) % kStagesG]);
-        }
+        cp_async_arrive_noinc(&b_full[sb]);
       }
-      // retire the unit's remaining stages
-      cp_async_wait<0>();
-      proxy_fence();
-      __syncwarp();
-      if (lane == 0 && !s_abort) {
-        const int first = nK >= kStagesG - 2 ? nK - (kStagesG - 2) : 0;
-        for (int kc = first; kc < nK; ++kc) mbar_arrive(&b_full[(q - nK + kc) % kStagesG]);
-      }
+      if (stop) break;
     }
     cp_async_wait<0>();  // no copy may still be landing when the CTA leaves
-  } else if (warp >= kAWarp0 && warp < kAWarp0 + kAWarps) {
-    // ------------------------------ A producers (dequantise) ------------------------------
-    const int at = tid - kAWarp0 * 32;  // 0..255
-    const int m = at >> 1;              // tile row 0..127
-    const int half = at & 1;            // which 32 columns of the 64-wide stage
+  } else if (warp >= kAWarp0 && warp < kAWarp0 + kAWarps && MODE == kModeRouter) {
+    // ------------------------------ A rows of the router (bf16, plain copies) ------------------------------
+    const int at = tid - kAWarp0 * 32;
+    const int m = at >> 1, half = at & 1;
     uint32_t q = 0;
     for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x) {
       const GemmUnit U = a.units[u];
-      // this thread's weight row
-      const uint8_t* codes = nullptr;
-      const uint16_t* sc = nullptr;
-      const uint16_t* bi = nullptr;
-      const uint16_t* wrow = nullptr;
-      bool zero = false;
-      if (MODE == kModeRouter) {
-        const int e = U.mt * 128 + m;
-        if (e < a.E) wrow = a.wr + (size_t)e * a.H;
-        else if (e == a.E) wrow = a.wsg;
-        else zero = true;
-      } else {
-        const uint8_t* blob;
+      const int e = U.mt * 128 + m;
+      const uint16_t* row = e < a.E ? a.wr + (size_t)e * a.H : (e == a.E ? a.wsg : nullptr);
+      bool stop = false;
+      for (int kc = 0; kc < nK; ++kc, ++q) {
+        const int sa = q % kSA;
+        if (!warp_wait(&a_empty[sa], ((q / kSA) & 1) ^ 1, a.ctrl, lane)) {
+          s_abort = 1;
+          stop = true;
+          break;
+        }
+        const uint32_t a_base = smem_base + sa * kABytes;
+#pragma unroll
+        for (int o = 0; o < 4; ++o) {
+          const uint16_t* src = row ? row + kc * kKC + (half * 4 + o) * 8 : a.wsg;
+          cp_async16(a_base + core_off(m, half * 4 + o), src, row ? 16u : 0u);
+        }
+        cp_async_arrive_noinc(&a_full[sa]);
+      }
+      if (stop) break;
+    }
+    cp_async_wait<0>();
+  } else if (warp >= kAWarp0 && warp < kAWarp0 + kAWarps) {
+    // ------------------------------ A producers (dequantise) ------------------------------
+    // Raw weight bytes stream into a per-thread cp.async ring (kDepth stages ahead); each
+    // unit's row scales and biases land once in shared memory (thread pair (m, 0) copies the
+    // scales, (m, 1) the biases).  A thread only ever reads bytes it copied itself, apart from
+    // its partner's half of the scales, which a __syncwarp after both waits makes visible.
+    using RR = RawRing<BITS, MODE>;
+    constexpr int kDepth = RR::kDepth, kRB = RR::kBytes;
+    const int at = tid - kAWarp0 * 32;  // 0..255
+    const int m = at >> 1;              // tile row 0..127
+    const int half = at & 1;            // which 32 columns of the 64-wide stage
+    const int NG = K / kGroup;          // groups (= stages) per row
+    uint8_t* raw_ring = smem + (size_t)kSA * kABytes + (size_t)kSB * kBBytes;
+    uint8_t* my_raw = raw_ring + (size_t)at * kRB * kDepth;
+    uint16_t* sb_area = reinterpret_cast<uint16_t*>(raw_ring + kRawBytes);  // [128][2][NG]
+    uint16_t* my_s = sb_area + (size_t)m * 2 * NG;
+    uint16_t* my_b = my_s + NG;
+    uint32_t q = 0;
+    for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x) {
+      const GemmUnit U = a.units[u];
+      // this thread's weight row (bytes of the row, its scales and biases)
+      const uint8_t* src = nullptr;
+      const uint8_t* sbsrc = nullptr;
+      {
+        const uint8_t* blob = nullptr;
         if (U.e < 0) {
           blob = a.shared;
         } else {
           const int slot = a.slot_table[U.e];
-          if (slot < 0 || slot >= a.n_slots) {
-            atomicOr(&a.ctrl->err, kErrBadSlot);
-            blob = nullptr;
+          if (slot < 0 || slot >= a.n_slots) atomicOr(&a.ctrl->err, kErrBadSlot);
+          else blob = a.pool + (int64_t)slot * a.L.stride;
+        }
+        if (blob) {
+          if (MODE == kModeGateUp) {
+            const int r = U.mt * 64 + (m >> 1);
+            const int up = m & 1;  // rows alternate gate, up of the same intermediate row
+            src = blob + a.L.off[up ? 1 : 0] + (int64_t)r * (a.H * BITS / 8);
+            sbsrc = blob + a.L.off[(up ? 5 : 3) + half] + (int64_t)r * NG * 2;
           } else {
-            blob = a.pool + (int64_t)slot * a.L.stride;
+            const int j = U.mt * 128 + m;
+            src = blob + a.L.off[2] + (int64_t)j * (a.I * BITS / 8);
+            sbsrc = blob + a.L.off[7 + half] + (int64_t)j * NG * 2;
           }
         }
-        if (!blob) {
-          zero = true;
-        } else if (MODE == kModeGateUp) {
-          const int r = U.mt * 64 + (m >> 1);
-          const int up = m & 1;  // rows alternate gate, up of the same intermediate row
-          const int rowb = a.H * BITS / 8, ng = a.H / kGroup;
-          codes = blob + a.L.off[up ? 1 : 0] + (int64_t)r * rowb;
-          sc = reinterpret_cast<const uint16_t*>(blob + a.L.off[up ? 5 : 3]) + (int64_t)r * ng;
-          bi = reinterpret_cast<const uint16_t*>(blob + a.L.off[up ? 6 : 4]) + (int64_t)r * ng;
-        } else {
-          const int j = U.mt * 128 + m;
-          const int rowb = a.I * BITS / 8, ng = a.I / kGroup;
-          codes = blob + a.L.off[2] + (int64_t)j * rowb;
-          sc = reinterpret_cast<const uint16_t*>(blob + a.L.off[7]) + (int64_t)j * ng;
-          bi = reinterpret_cast<const uint16_t*>(blob + a.L.off[8]) + (int64_t)j * ng;
-        }
       }
-      // loads run kRing stages ahead of the shared-memory stores (register ring), so each
-      // stage's global latency overlaps the dequantisation of the stages before it
-      constexpr int kRing = 4;
-      uint4 rr[kRing][4];
-      float rs[kRing], rb[kRing];
-      auto load = [&](int kc, int d) {
-        if (zero) return;
-        if (MODE == kModeRouter) {
-          const uint4* p = reinterpret_cast<const uint4*>(wrow + kc * kKC + half * 32);
+      const bool zero = (src == nullptr);
+      auto issue = [&](int kc) {  // raw bytes of stage kc into ring slot kc % kDepth
+        if (!zero && kc < nK) {
+          const uint8_t* g = src + (size_t)kc * (kKC * BITS / 8) + half * kRB;
+          const uint32_t d = smem_u32(my_raw + (kc % kDepth) * kRB);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) rr[d][i] = __ldg(p + i);
-        } else if (BITS == 4) {
-          rr[d][0] = ld_stream(codes + kc * 32 + half * 16);
-          rs[d] = bf1(ld_u16(sc + kc));
-          rb[d] = bf1(ld_u16(bi + kc));
-        } else {
-          const uint8_t* p = codes + kc * 64 + half * 32;
-          rr[d][0] = ld_stream(p);
-          rr[d][1] = ld_stream(p + 16);
-          rs[d] = bf1(ld_u16(sc + kc));
-          rb[d] = bf1(ld_u16(bi + kc));
+          for (int o = 0; o < kRB / 16; ++o) cp_async16(d + o * 16, g + o * 16, 16u);
         }
+        cp_async_commit();  // one group per stage, empty past the end, so the counts stay uniform
       };
-#pragma unroll
-      for (int d = 0; d < kRing; ++d)
-        if (d < nK) load(d, d);
-      bool stop = false;
-      for (int kc0 = 0; kc0 < nK && !stop; kc0 += kRing) {
-#pragma unroll
-        for (int d = 0; d < kRing; ++d) {
-          const int kc = kc0 + d;
-          if (kc >= nK || stop) continue;
-          const int s = q % kStagesG;
-          if (!wait_or_flag(&empty[s], ((q / kStagesG) & 1) ^ 1, a.ctrl)) {
-            s_abort = 1;
-            stop = true;
-            continue;
-          }
-          uint8_t* a_tile = smem + s * (kABytes + kBBytes);
-#pragma unroll
-          for (int o = 0; o < 4; ++o) {  // 4 k-octets of 8 values = this thread's 32 columns
-            uint4 v;
-            if (zero) {
-              v = make_uint4(0, 0, 0, 0);
-            } else if (MODE == kModeRouter) {
-              v = rr[d][o];
-            } else if (BITS == 4) {
-              const uint4 w = rr[d][0];
-              v = dq8_int4(o == 0 ? w.x : o == 1 ? w.y : o == 2 ? w.z : w.w, rs[d], rb[d]);
-            } else {
-              const uint4 w = rr[d][o >> 1];
-              v = (o & 1) ? dq8_int8(w.z, w.w, rs[d], rb[d]) : dq8_int8(w.x, w.y, rs[d], rb[d]);
-            }
-            *reinterpret_cast<uint4*>(a_tile + core_off(m, half * 4 + o)) = v;
-          }
-          if (kc + kRing < nK) load(kc + kRing, d);
-          proxy_fence();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&a_full[s]);
-          ++q;
+      // scales/biases of the row (one group with stage 0), then the first kDepth stages
+      if (!zero) {
+        uint16_t* dst = half ? my_b : my_s;
+        if ((NG & 7) == 0) {  // rows of 16-byte multiples: 16-byte aligned in the blob
+          for (int o = 0; o < NG * 2; o += 16) cp_async16(smem_u32(dst) + o, sbsrc + o, 16u);
+        } else {  // narrow rows (small K): plain loads, visible after the first __syncwarp
+          const uint16_t* g = reinterpret_cast<const uint16_t*>(sbsrc);
+          for (int o = 0; o < NG; ++o) dst[o] = __ldg(g + o);
         }
       }
+#pragma unroll 1
+      for (int d = 0; d < kDepth; ++d) issue(d);
+      bool stop = false;
+      for (int kc = 0; kc < nK; ++kc, ++q) {
+        const int sa = q % kSA;
+        cp_async_wait<kDepth - 1>();  // this thread's bytes of stage kc have landed
+        __syncwarp();                 // ... and the partner's half of the scales
+        if (!warp_wait(&a_empty[sa], ((q / kSA) & 1) ^ 1, a.ctrl, lane)) {
+          s_abort = 1;
+          stop = true;
+          break;
+        }
+        const uint4* rp = reinterpret_cast<const uint4*>(my_raw + (kc % kDepth) * kRB);
+        uint4 rw[kRB / 16];
+#pragma unroll
+        for (int o = 0; o < kRB / 16; ++o) rw[o] = zero ? make_uint4(0, 0, 0, 0) : rp[o];
+        float sv = 0.f, bv = 0.f;
+        if (!zero) {
+          sv = bf1(my_s[kc]);
+          bv = bf1(my_b[kc]);
+        }
+        uint8_t* a_tile = smem + sa * kABytes;
+#pragma unroll
+        for (int o = 0; o < 4; ++o) {  // 4 k-octets of 8 values = this thread's 32 columns
+          uint4 v;
+          if (zero) {
+            v = make_uint4(0, 0, 0, 0);
+          } else if (BITS == 4) {
+            const uint4 w = rw[0];
+            v = dq8_int4(o == 0 ? w.x : o == 1 ? w.y : o == 2 ? w.z : w.w, sv, bv);
+          } else {
+            const uint4 w = rw[o >> 1];
+            v = (o & 1) ? dq8_int8(w.z, w.w, sv, bv) : dq8_int8(w.x, w.y, sv, bv);
+          }
+          *reinterpret_cast<uint4*>(a_tile + core_off(m, half * 4 + o)) = v;
+        }
+        // the ring slot's bytes and this stage's scales are consumed (the stores above depend
+        // on them): refill the slot, and let the partner go on to overwrite the scales
+        __syncwarp();
+        issue(kc + kDepth);
+        proxy_fence();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[sa]);
+      }
+      if (stop) break;
     }
+    cp_async_wait<0>();  // no copy may still be landing when the CTA leaves
   } else if (warp >= kEWarp0) {
     // ------------------------------ epilogue ------------------------------
     const int quad = warp & 3;       // TMEM lane quadrant of this warp
@@ -406,12 +467,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x, ++it) {
       const GemmUnit U = a.units[u];
       const int buf = it & 1;
-      if (!wait_or_flag(&acc_full[buf], (it >> 1) & 1, a.ctrl)) {
+      if (MODE == kModeDown) {
+        // token and weight of every column, loaded while the unit's MMAs run
+        for (int n = lane; n < U.n; n += 32) {
+          int t;
+          float w;
+          if (U.e < 0) {
+            t = U.p0 + n;
+            w = __ldg(a.gate + t);
+          } else {
+            const int pair = __ldg(a.order + U.p0 + n);
+            t = pair / a.k;
+            w = __ldg(a.topk_w + pair);
+          }
+          s_colt[quad][n] = t;
+          s_colw[quad][n] = w;
+        }
+        __syncwarp();
+      }
+      if (!warp_wait(&acc_full[buf], (it >> 1) & 1, a.ctrl, lane)) {
         s_abort = 1;
         break;
       }
       tc_fence_after();
-      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)buf * 256u;
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)buf * (uint32_t)kNmax;
       for (int c0 = 0; c0 < U.n; c0 += 8) {
         float v[8];
         tmem_ld8(taddr + c0, v);
@@ -431,17 +510,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
           } else if (MODE == kModeDown) {
             if (n < U.n) {
               const int j = U.mt * 128 + m;
-              int t;
-              float w;
-              if (U.e < 0) {
-                t = U.p0 + n;
-                w = a.gate[t];
-              } else {
-                const int pair = a.order[U.p0 + n];
-                t = pair / a.k;
-                w = a.topk_w[pair];
-              }
-              atomicAdd(a.acc + (size_t)t * a.H + j, w * val);
+              atomicAdd(a.acc + (size_t)s_colt[quad][n] * a.H + j, s_colw[quad][n] * val);
             }
           } else {  // router logits (no bias)
             const int e = U.mt * 128 + m;
@@ -459,7 +528,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512u));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)kTmemCols));
   }
 }
 
@@ -747,7 +816,7 @@ __global__ void __launch_bounds__(kGroupThreads) k_group(PrefillArgs a) {
     if (e < E) a.counts[e] = cnt[e];
   }
   __syncthreads();
-  // work units: per expert, token tiles of <= 256 pairs x row tiles; then the shared expert.
+  // work units: per expert, token tiles of <= 128 pairs x row tiles; then the shared expert.
   // Tile bases by an exclusive scan of the experts' tile counts (one expert per thread).
   __syncthreads();
   int* tile_base = hist;  // reuse: [E + 1]
@@ -814,7 +883,9 @@ __global__ void k_router_units(GemmUnit* units, int* n_units, int T, int E) {
 
 template <int BITS, int MODE>
 cudaError_t launch_gemm(const GemmArgs& g, int n_sm, cudaStream_t s) {
-  const size_t smem = (size_t)kStagesG * (kABytes + kBBytes);
+  const int K = (MODE == kModeDown) ? g.I : g.H;
+  size_t smem = (size_t)StageCount<MODE>::kA * kABytes + (size_t)StageCount<MODE>::kB * kBBytes;
+  if (MODE != kModeRouter) smem += kRawBytes + (size_t)128 * (K / kGroup) * 4;
   auto fn = k_gemm<BITS, MODE>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -825,7 +896,7 @@ cudaError_t launch_gemm(const GemmArgs& g, int n_sm, cudaStream_t s) {
 }  // namespace
 
 bool prefill_shape_supported(int H, int I, int bits, int E) {
-  return (bits == 4 || bits == 8) && H % 128 == 0 && I % 64 == 0 && E <= 512 && H <= 8192 && I <= 4096;
+  return (bits == 4 || bits == 8) && H % 128 == 0 && I % 64 == 0 && E <= 512 && H <= 4096 && I <= 4096;
 }
 
 cudaError_t launch_group(const PrefillArgs& p, cudaStream_t s) {
