@@ -256,6 +256,7 @@ static moe_status prefill_forward(const moe_shape* shape, const void* x, int32_t
   p.order = reinterpret_cast<int32_t*>(b + W.order);
   p.offsets = reinterpret_cast<int32_t*>(b + W.offsets);
   p.counts = reinterpret_cast<int32_t*>(b + W.counts);
+  p.chunk_cnt = reinterpret_cast<int32_t*>(b + W.chunk_cnt);
   p.units_rt = reinterpret_cast<GemmUnit*>(b + W.units_rt);
   p.units_gu = reinterpret_cast<GemmUnit*>(b + W.units_gu);
   p.units_dn = reinterpret_cast<GemmUnit*>(b + W.units_dn);
@@ -432,6 +433,7 @@ moe_status moe_group_pairs(const moe_shape* shape, int32_t T, const int32_t* top
   p.order = order;
   p.offsets = offsets;
   p.counts = reinterpret_cast<int32_t*>(b + W.counts);
+  p.chunk_cnt = reinterpret_cast<int32_t*>(b + W.chunk_cnt);
   p.units_gu = reinterpret_cast<GemmUnit*>(b + W.units_gu);
   p.units_dn = reinterpret_cast<GemmUnit*>(b + W.units_dn);
   p.n_units = reinterpret_cast<int*>(b + W.n_units);

@@ -190,6 +190,7 @@ struct FusedArgs {
 // ---------------------------------------------------------------------------------------
 constexpr int kModeRouter = 0, kModeGateUp = 1, kModeDown = 2;
 constexpr int kPrefillN = 128;  // tokens (MMA N) per GEMM work unit
+constexpr int kGroupChunk = 512;  // (token, k) pairs per CTA of the grouping kernels
 
 // One tcgen05 GEMM work unit: expert e (-1: shared expert, -2: router), row tile mt, first
 // column p0 (pair position, or token for the shared expert / router) and column count n.
@@ -237,6 +238,7 @@ struct PrefillArgs {
   int32_t* order;
   int32_t* offsets;     // [E+1]
   int32_t* counts;      // [E]
+  int32_t* chunk_cnt;   // [ceil(T*k / kGroupChunk)][E]: per-chunk counts, then exclusive sums
   GemmUnit* units_rt;
   GemmUnit* units_gu;
   GemmUnit* units_dn;
@@ -249,8 +251,8 @@ struct PrefillArgs {
 };
 
 struct PrefillLayout {
-  size_t ctrl, xnorm, wnorm, logits, topk_idx, topk_w, gate, order, offsets, counts, units_rt, units_gu,
-      units_dn, n_units, acc, h, hs, total;
+  size_t ctrl, xnorm, wnorm, logits, topk_idx, topk_w, gate, order, offsets, counts, chunk_cnt, units_rt,
+      units_gu, units_dn, n_units, acc, h, hs, total;
 };
 
 inline PrefillLayout make_prefill_layout(int T, int E, int k, int H, int I) {
@@ -274,6 +276,7 @@ inline PrefillLayout make_prefill_layout(int T, int E, int k, int H, int I) {
   W.order = take(sizeof(int32_t) * (size_t)T * k);
   W.offsets = take(sizeof(int32_t) * (E + 1));
   W.counts = take(sizeof(int32_t) * E);
+  W.chunk_cnt = take(sizeof(int32_t) * (size_t)E * (((size_t)T * k + kGroupChunk - 1) / kGroupChunk));
   W.units_rt = take(sizeof(GemmUnit) * rt_units);
   W.units_gu = take(sizeof(GemmUnit) * tiles * (I / 64));
   W.units_dn = take(sizeof(GemmUnit) * tiles * (H / 128));

@@ -11,8 +11,10 @@
 //                  fp32 error bound of the k-th is recomputed exactly (fp64 sums of exact
 //                  bf16 products) and the selection is made on the exact values; softmax
 //                  over the selected logits; shared-expert gate
-//   k_group        stable counting sort of the (token, k) pairs by expert and the list of
-//                  GEMM work units (expert, row tile, token tile)
+//   k_ghist, k_gscan, k_gplace
+//                  stable counting sort of the (token, k) pairs by expert (per-chunk counts,
+//                  one scan, per-chunk stable placement) and the list of GEMM work units
+//                  (expert, row tile, token tile)
 //   k_gemm GATEUP  per unit: [gate; up] rows of one expert (dequantised to bf16 in shared
 //                  memory) x the expert's tokens (gathered), SwiGLU in the epilogue -> h
 //   k_gemm DOWN    per unit: down rows x the expert's h, weighted scatter-add into an fp32
@@ -46,10 +48,10 @@ constexpr int kKC = 64;                   // K per stage
 constexpr int kNmax = kPrefillN;          // tokens per unit (MMA N)
 constexpr int kABytes = 128 * kKC * 2;    // 16 KB
 constexpr int kBBytes = kNmax * kKC * 2;  // 16 KB
-constexpr int kGemmThreads = 512;
-constexpr int kBWarp0 = 1, kBWarps = 3;
-constexpr int kAWarp0 = 4, kAWarps = 8;
-constexpr int kEWarp0 = 12, kEWarps = 4;
+constexpr int kBWarp0 = 1, kBWarps = 2;
+constexpr int kAWarp0 = 3, kAWarps = 8;
+constexpr int kEWarp0 = 11, kEWarps = 4;
+constexpr int kGemmThreads = (kEWarp0 + kEWarps) * 32;  // 480
 constexpr int kSBO = (kKC / 8) * 128;     // 1024
 constexpr int kTmemCols = 2 * kNmax;      // two accumulators
 constexpr int kRawBytes = 32 * 1024;      // cp.async ring of raw weight bytes (A producers)
@@ -127,11 +129,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&p);
 }
 
-// 8 int4 codes (one 32-bit word, element j at bits 4j) -> 8 bf16 values of s*q + b.
-// The code at bit position p is turned into the exact float q*2^p by OR-ing it into the
-// mantissa of 2^23 and subtracting 2^23; multiplying by s*2^-p (exact) then gives s*q, so
-// every value is round(s*q + b) as from a direct conversion, without integer-to-float
-// instructions.  Two codes per packed fp32x2 add and FMA.
+// int8 codes -> bf16 on fp32 pairs: the code at bit position p becomes the exact float
+// q*2^p by OR-ing it into the mantissa of 2^23 and subtracting 2^23; multiplying by s*2^-p
+// (exact) then gives s*q, without integer-to-float instructions.  (bf16 has too few mantissa
+// bits for the same trick on 8-bit codes.)
 __device__ __forceinline__ float2 ffma2p(float2 a, float2 b, float2 c) {
   float2 d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;"
@@ -145,12 +146,6 @@ __device__ __forceinline__ uint32_t dq2(uint32_t m0, uint32_t m1, float s0, floa
   const float2 r = ffma2p(v, make_float2(s0, s1), make_float2(b, b));
   return pack_bf16(r.x, r.y);
 }
-__device__ __forceinline__ uint4 dq8_int4(uint32_t w, float s, float b) {
-  const uint32_t wh = w >> 12;
-  const float s4 = s * 0x1p-4f, s8 = s * 0x1p-8f, s12 = s * 0x1p-12f, s16 = s * 0x1p-16f;
-  return make_uint4(dq2(w & 0xFu, w & 0xF0u, s, s4, b), dq2(w & 0xF00u, w & 0xF000u, s8, s12, b),
-                    dq2(w & 0xF0000u, wh & 0xF00u, s16, s8, b), dq2(wh & 0xF000u, wh & 0xF0000u, s12, s16, b));
-}
 // 8 int8 codes (two words, byte j at bits 8j) -> 8 bf16 values.
 __device__ __forceinline__ uint4 dq8_int8(uint32_t w0, uint32_t w1, float s, float b) {
   const uint32_t h0 = w0 >> 16, h1 = w1 >> 16;
@@ -159,12 +154,48 @@ __device__ __forceinline__ uint4 dq8_int8(uint32_t w0, uint32_t w1, float s, flo
                     dq2(w1 & 0xFFu, w1 & 0xFF00u, s, s8, b), dq2(h1 & 0xFFu, h1 & 0xFF00u, s, s8, b));
 }
 
+// A-producer thread -> (tile row m, column half).  Lanes l and l ^ 8 share a row; the
+// eight lanes of each quarter-warp take eight consecutive rows of one half, so that their
+// 16-byte stores of a k-octet fill 128 contiguous bytes of the tile (no bank conflicts).
+__device__ __forceinline__ void a_lane_map(int at, int& m, int& half) {
+  const int w = at >> 5, l = at & 31;
+  m = w * 16 + (l & 7) + ((l >> 4) << 3);
+  half = (l >> 3) & 1;
+}
+
+// 8 int4 codes (one word, element j at bits 4j) -> 8 bf16 values round(s*q + b), on packed
+// bf16 pairs.  OR-ing a code into the low mantissa bits of bf16 128.0 (0x4300) gives the
+// exact value 128 + q; subtracting 128 is exact, and one fused multiply-add rounds s*q + b
+// once.  Pairs come out as (q0, q4), (q1, q5), ... and are re-paired with byte permutes.
+__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+__device__ __forceinline__ uint4 dq8_int4_bf(uint32_t w, uint32_t s2, uint32_t b2) {
+  constexpr uint32_t kMask = 0x000F000Fu, kBias = 0x43004300u;  // bf16 128.0 in both halves
+  constexpr uint32_t kOne = 0x3F803F80u, kNeg128 = 0xC300C300u;  // bf16 1.0, -128.0
+  uint32_t r[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t p = ((w >> (4 * i)) & kMask) | kBias;  // (128 + q_i, 128 + q_{i+4})
+    r[i] = bf2_fma(bf2_fma(p, kOne, kNeg128), s2, b2);
+  }
+  return make_uint4(prmt(r[0], r[1], 0x5410u), prmt(r[2], r[3], 0x5410u), prmt(r[0], r[1], 0x7632u),
+                    prmt(r[2], r[3], 0x7632u));
+}
+
 __device__ __forceinline__ int core_off(int row, int koct) {  // byte offset in a stage tile
   return (row >> 3) * kSBO + koct * 128 + (row & 7) * 16;
 }
 
 __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, Ctrl* c) {
-  if (mbar_wait(bar, parity)) return true;
+  if (mbar_wait_suspend(bar, parity)) return true;
   atomicOr(&c->err, kErrTimeout);
   return false;
 }
@@ -172,7 +203,7 @@ __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, Ctr
 // Every lane of a warp waits, and all take the same branch afterwards (a lane whose wait
 // ran out would otherwise leave the others behind at the next __syncwarp).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Ctrl* c, int lane) {
-  const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, parity) ? 1 : 0);
+  const bool ok = __all_sync(0xffffffffu, mbar_wait_suspend(bar, parity) ? 1 : 0);
   if (!ok && lane == 0) atomicOr(&c->err, kErrTimeout);
   return ok;
 }
@@ -188,7 +219,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       acc_empty[2], drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  __shared__ int s_rows[kBWarps][kNmax];  // per B warp: source row of each column of the unit
   __shared__ int s_colt[kEWarps][kNmax];  // per epilogue warp (down): token of each column
   __shared__ float s_colw[kEWarps][kNmax];  // and its routing weight
 
@@ -272,10 +302,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     __syncwarp();
   } else if (warp >= kBWarp0 && warp < kBWarp0 + kBWarps) {
     // ------------------------------ B gather (cp.async) ------------------------------
-    // Each thread's copies of a stage are tracked by the stage's mbarrier (an arrival that
-    // fires when they have landed), so the gather runs up to kSB stages ahead of the MMAs.
-    const int bt = tid - kBWarp0 * 32;  // 0..95
-    const int bw = warp - kBWarp0;
+    // Thread bt copies columns bt and bt + 64 of the unit (one token or pair row each, 128
+    // bytes per stage).  Each thread's copies of a stage are tracked by the stage's mbarrier
+    // (an arrival that fires when they have landed), so the gather runs up to kSB stages ahead.
+    const int bt = tid - kBWarp0 * 32;  // 0..63
     uint32_t q = 0;
     for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x) {
       const GemmUnit U = a.units[u];
@@ -289,14 +319,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         src_base = a.x;
         src_ld = a.H;
       }
-      // source row (token or pair position) of each column, once per unit; -1: zero row
-      for (int n = lane; n < npad; n += 32) {
+      // source row of each of the thread's two columns; nullptr: zero column (n >= U.n)
+      const uint16_t* rows[2];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int n = bt + c * 64;
         int r = -1;
         if (n < U.n) r = (MODE == kModeGateUp && U.e >= 0) ? __ldg(a.order + U.p0 + n) / a.k : U.p0 + n;
-        s_rows[bw][n] = r;
+        rows[c] = r < 0 ? nullptr : src_base + (size_t)r * src_ld;
       }
-      __syncwarp();
-      const int n_copies = npad * (kKC / 8);  // 16-byte pieces per stage
       bool stop = false;
       for (int kc = 0; kc < nK; ++kc, ++q) {
         const int sb = q % kSB;
@@ -306,13 +337,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
           break;
         }
         const uint32_t b_base = b_area + sb * kBBytes;
-        for (int i = bt; i < n_copies; i += kBWarps * 32) {
-          // consecutive i: consecutive rows within a core matrix (conflict-free smem writes)
-          const int n = (i & 7) | ((i >> 6) << 3);
-          const int j = (i >> 3) & 7;
-          const int r = s_rows[bw][n];
-          const uint16_t* src = src_base + (size_t)(r < 0 ? 0 : r) * src_ld + kc * kKC + j * 8;
-          cp_async16(b_base + core_off(n, j), src, r < 0 ? 0u : 16u);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int n = bt + c * 64;
+          if (n < npad) {  // columns beyond npad are not read by the MMA
+            const uint16_t* src = rows[c] ? rows[c] + kc * kKC : a.x;
+            const uint32_t d = b_base + core_off(n, 0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) cp_async16(d + j * 128, src + j * 8, rows[c] ? 16u : 0u);
+          }
         }
         cp_async_arrive_noinc(&b_full[sb]);
       }
@@ -321,13 +354,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     cp_async_wait<0>();  // no copy may still be landing when the CTA leaves
   } else if (warp >= kAWarp0 && warp < kAWarp0 + kAWarps && MODE == kModeRouter) {
     // ------------------------------ A rows of the router (bf16, plain copies) ------------------------------
-    const int at = tid - kAWarp0 * 32;
-    const int m = at >> 1, half = at & 1;
+    int m, half;
+    a_lane_map(tid - kAWarp0 * 32, m, half);
     uint32_t q = 0;
     for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x) {
       const GemmUnit U = a.units[u];
       const int e = U.mt * 128 + m;
-      const uint16_t* row = e < a.E ? a.wr + (size_t)e * a.H : (e == a.E ? a.wsg : nullptr);
+      const uint16_t* row = e < a.E ? a.wr + (size_t)e * a.H : nullptr;
       bool stop = false;
       for (int kc = 0; kc < nK; ++kc, ++q) {
         const int sa = q % kSA;
@@ -349,20 +382,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     cp_async_wait<0>();
   } else if (warp >= kAWarp0 && warp < kAWarp0 + kAWarps) {
     // ------------------------------ A producers (dequantise) ------------------------------
-    // Raw weight bytes stream into a per-thread cp.async ring (kDepth stages ahead); each
-    // unit's row scales and biases land once in shared memory (thread pair (m, 0) copies the
-    // scales, (m, 1) the biases).  A thread only ever reads bytes it copied itself, apart from
-    // its partner's half of the scales, which a __syncwarp after both waits makes visible.
+    // Raw weight bytes stream into a cp.async ring (kDepth stages ahead); each unit's row
+    // scales and biases land once in shared memory (of the two threads of a row, half 0
+    // copies the scales, half 1 the biases).  A thread only ever reads ring bytes it copied
+    // itself; its partner's half of the scales becomes visible at the __syncwarp that
+    // follows both threads' waits.
     using RR = RawRing<BITS, MODE>;
-    constexpr int kDepth = RR::kDepth, kRB = RR::kBytes;
+    constexpr int kDepth = RR::kDepth, kRB = RR::kBytes, kPieces = kRB / 16;
     const int at = tid - kAWarp0 * 32;  // 0..255
-    const int m = at >> 1;              // tile row 0..127
-    const int half = at & 1;            // which 32 columns of the 64-wide stage
+    int m, half;                        // tile row 0..127, which 32 columns of the stage
+    a_lane_map(at, m, half);
     const int NG = K / kGroup;          // groups (= stages) per row
+    const int sb_ld = 2 * NG + 8;       // uint16 per row of the scale area (16 bytes of padding)
+    // ring: [slot][piece][thread][16 bytes], so a warp's accesses are 512 contiguous bytes
     uint8_t* raw_ring = smem + (size_t)kSA * kABytes + (size_t)kSB * kBBytes;
-    uint8_t* my_raw = raw_ring + (size_t)at * kRB * kDepth;
-    uint16_t* sb_area = reinterpret_cast<uint16_t*>(raw_ring + kRawBytes);  // [128][2][NG]
-    uint16_t* my_s = sb_area + (size_t)m * 2 * NG;
+    uint8_t* my_raw = raw_ring + (size_t)at * 16;
+    uint16_t* sb_area = reinterpret_cast<uint16_t*>(raw_ring + kRawBytes);  // [128][sb_ld]
+    uint16_t* my_s = sb_area + (size_t)m * sb_ld;
     uint16_t* my_b = my_s + NG;
     uint32_t q = 0;
     for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x) {
@@ -396,16 +432,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       auto issue = [&](int kc) {  // raw bytes of stage kc into ring slot kc % kDepth
         if (!zero && kc < nK) {
           const uint8_t* g = src + (size_t)kc * (kKC * BITS / 8) + half * kRB;
-          const uint32_t d = smem_u32(my_raw + (kc % kDepth) * kRB);
+          const uint32_t d = smem_u32(my_raw + (size_t)(kc % kDepth) * kPieces * (kAThreads * 16));
 #pragma unroll
-          for (int o = 0; o < kRB / 16; ++o) cp_async16(d + o * 16, g + o * 16, 16u);
+          for (int o = 0; o < kPieces; ++o) cp_async16(d + o * (kAThreads * 16), g + o * 16, 16u);
         }
         cp_async_commit();  // one group per stage, empty past the end, so the counts stay uniform
       };
       // scales/biases of the row (one group with stage 0), then the first kDepth stages
       if (!zero) {
         uint16_t* dst = half ? my_b : my_s;
-        if ((NG & 7) == 0) {  // rows of 16-byte multiples: 16-byte aligned in the blob
+        if ((NG & 7) == 0) {  // rows of 16-byte multiples: 16-byte aligned in the blob and here
           for (int o = 0; o < NG * 2; o += 16) cp_async16(smem_u32(dst) + o, sbsrc + o, 16u);
         } else {  // narrow rows (small K): plain loads, visible after the first __syncwarp
           const uint16_t* g = reinterpret_cast<const uint16_t*>(sbsrc);
@@ -424,29 +460,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
           stop = true;
           break;
         }
-        const uint4* rp = reinterpret_cast<const uint4*>(my_raw + (kc % kDepth) * kRB);
-        uint4 rw[kRB / 16];
+        const uint8_t* rp = my_raw + (size_t)(kc % kDepth) * kPieces * (kAThreads * 16);
+        uint4 rw[kPieces];
 #pragma unroll
-        for (int o = 0; o < kRB / 16; ++o) rw[o] = zero ? make_uint4(0, 0, 0, 0) : rp[o];
-        float sv = 0.f, bv = 0.f;
-        if (!zero) {
-          sv = bf1(my_s[kc]);
-          bv = bf1(my_b[kc]);
-        }
+        for (int o = 0; o < kPieces; ++o)
+          rw[o] = zero ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4*>(rp + o * (kAThreads * 16));
+        const uint32_t sbits = zero ? 0u : my_s[kc], bbits = zero ? 0u : my_b[kc];
         uint8_t* a_tile = smem + sa * kABytes;
+        if (BITS == 4) {
+          const uint32_t s2 = sbits | (sbits << 16), b2 = bbits | (bbits << 16);
+          const uint32_t w4[4] = {rw[0].x, rw[0].y, rw[0].z, rw[0].w};
 #pragma unroll
-        for (int o = 0; o < 4; ++o) {  // 4 k-octets of 8 values = this thread's 32 columns
-          uint4 v;
-          if (zero) {
-            v = make_uint4(0, 0, 0, 0);
-          } else if (BITS == 4) {
-            const uint4 w = rw[0];
-            v = dq8_int4(o == 0 ? w.x : o == 1 ? w.y : o == 2 ? w.z : w.w, sv, bv);
-          } else {
+          for (int o = 0; o < 4; ++o)  // 4 k-octets of 8 values = this thread's 32 columns
+            *reinterpret_cast<uint4*>(a_tile + core_off(m, half * 4 + o)) = dq8_int4_bf(w4[o], s2, b2);
+        } else {
+          const float sv = __uint_as_float(sbits << 16), bv = __uint_as_float(bbits << 16);
+#pragma unroll
+          for (int o = 0; o < 4; ++o) {
             const uint4 w = rw[o >> 1];
-            v = (o & 1) ? dq8_int8(w.z, w.w, sv, bv) : dq8_int8(w.x, w.y, sv, bv);
+            const uint4 v = (o & 1) ? dq8_int8(w.z, w.w, sv, bv) : dq8_int8(w.x, w.y, sv, bv);
+            *reinterpret_cast<uint4*>(a_tile + core_off(m, half * 4 + o)) = v;
           }
-          *reinterpret_cast<uint4*>(a_tile + core_off(m, half * 4 + o)) = v;
         }
         // the ring slot's bytes and this stage's scales are consumed (the stores above depend
         // on them): refill the slot, and let the partner go on to overwrite the scales
@@ -514,7 +548,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             }
           } else {  // router logits (no bias)
             const int e = U.mt * 128 + m;
-            if (n < U.n && e <= a.E) a.logits[(size_t)(U.p0 + n) * (a.E + 1) + e] = val;
+            if (n < U.n && e < a.E) a.logits[(size_t)(U.p0 + n) * (a.E + 1) + e] = val;
           }
         }
       }
@@ -724,137 +758,142 @@ __global__ void __launch_bounds__(256) k_route(PrefillArgs a) {
 }
 
 // ---------------------------------------------------------------------------------------
-// stable counting sort of the pairs by expert, and the GEMM work units (one CTA)
+// stable counting sort of the pairs by expert, and the GEMM work units.
+//   k_ghist   per chunk of kGroupChunk pairs: its per-expert counts
+//   k_gscan   per expert: exclusive sums over the chunks (in place), the expert's total;
+//             offsets = exclusive scan of the totals; GEMM work units
+//   k_gplace  per chunk: stable ranks (warp match + per-warp counts), order[slot] = pair
+// Pair p of chunk c lands at offsets[e] + (pairs of e in chunks < c) + (pairs of e before it
+// in chunk c): the pairs of one expert keep their pair-index order.
 // ---------------------------------------------------------------------------------------
-constexpr int kGroupThreads = 1024;
+constexpr int kGroupThreads = 256;  // 8 warps; each takes kGroupChunk / 8 consecutive pairs
+constexpr int kScanThreads = 1024;
+static_assert(kGroupChunk % (kGroupThreads / 32 * 32) == 0, "chunk must split into whole warp rounds");
 
-__global__ void __launch_bounds__(kGroupThreads) k_group(PrefillArgs a) {
-  extern __shared__ int gsm[];
+__global__ void __launch_bounds__(kGroupThreads) k_ghist(PrefillArgs a) {
+  extern __shared__ int hsm[];  // [E]
   const int E = a.E, n = a.T * a.k;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, NWp = kGroupThreads / 32;
-  int* hist = gsm;             // [NWp][E] per-warp counts, then per-warp running positions
-  int* cnt = gsm + NWp * E;    // [E]
-  int* off = cnt + E;          // [E + 1]
-  for (int i = threadIdx.x; i < NWp * E; i += kGroupThreads) hist[i] = 0;
+  for (int e = threadIdx.x; e < E; e += kGroupThreads) hsm[e] = 0;
   __syncthreads();
-  const int seg = (n + NWp - 1) / NWp;
-  const int p0 = warp * seg, p1 = min(n, p0 + seg);
-  // pass 1: per-warp histograms, in pair order; ids are loaded 8 batches at a time so the
-  // loads are in flight together
-  constexpr int kB = 8;
-  for (int b0 = p0; b0 < p1; b0 += 32 * kB) {
-    int ev[kB];
+  const int p0 = blockIdx.x * kGroupChunk;
 #pragma unroll
-    for (int j = 0; j < kB; ++j) {
-      const int p = b0 + 32 * j + lane;
-      ev[j] = (p < p1) ? __ldg(a.topk_idx + p) : -1;
+  for (int j = 0; j < kGroupChunk / kGroupThreads; ++j) {
+    const int p = p0 + j * kGroupThreads + threadIdx.x;
+    if (p < n) {
+      const int e = __ldg(a.topk_idx + p);
+      if (e < 0 || e >= E) atomicOr(&a.ctrl->err, kErrBadExpert);
+      else atomicAdd(&hsm[e], 1);
     }
+  }
+  __syncthreads();
+  int* out = a.chunk_cnt + (size_t)blockIdx.x * E;
+  for (int e = threadIdx.x; e < E; e += kGroupThreads) out[e] = hsm[e];
+}
+
+__global__ void __launch_bounds__(kScanThreads) k_gscan(PrefillArgs a) {
+  __shared__ int cnt[kMaxExperts];
+  __shared__ int off[kMaxExperts + 1];
+  __shared__ int wsum[kScanThreads / 32];
+  const int E = a.E, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n_chunks = (a.T * a.k + kGroupChunk - 1) / kGroupChunk;
+  // per expert: running sum down the chunks (8 loads in flight per step)
+  for (int e = threadIdx.x; e < E; e += kScanThreads) {
+    int s = 0;
+    for (int c0 = 0; c0 < n_chunks; c0 += 8) {
+      int v[8];
 #pragma unroll
-    for (int j = 0; j < kB; ++j) {
-      int e = ev[j];
-      const int p = b0 + 32 * j + lane;
-      if (p < p1 && (e < 0 || e >= E)) {
-        atomicOr(&a.ctrl->err, kErrBadExpert);
-        e = -1;
+      for (int j = 0; j < 8; ++j) v[j] = (c0 + j < n_chunks) ? a.chunk_cnt[(size_t)(c0 + j) * E + e] : 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (c0 + j < n_chunks) {
+          a.chunk_cnt[(size_t)(c0 + j) * E + e] = s;
+          s += v[j];
+        }
+    }
+    cnt[e] = s;
+  }
+  __syncthreads();
+  // exclusive scan of the totals (E <= 1024: one value per thread)
+  {
+    const int e = threadIdx.x;
+    const int v = e < E ? cnt[e] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int wv = wsum[lane];
+      int wi = wv;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += y;
       }
-      const unsigned peers = __match_any_sync(0xffffffffu, e);
-      if (e >= 0 && lane == __ffs(peers) - 1) hist[warp * E + e] += __popc(peers);
-      __syncwarp();
+      wsum[lane] = wi - wv;
     }
+    __syncthreads();
+    if (e < E) off[e] = wsum[warp] + incl - v;
+    if (e == E - 1) off[E] = wsum[warp] + incl;
   }
   __syncthreads();
-  // counts and offsets
-  for (int e = threadIdx.x; e < E; e += kGroupThreads) {
-    int c = 0;
-    for (int w = 0; w < NWp; ++w) c += hist[w * E + e];
-    cnt[e] = c;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int e = 0; e < E; ++e) {
-      off[e] = acc;
-      acc += cnt[e];
-    }
-    off[E] = acc;
-  }
-  __syncthreads();
-  // running position of each (warp, expert): offset + counts of earlier warps
-  for (int e = threadIdx.x; e < E; e += kGroupThreads) {
-    int pos = off[e];
-    for (int w = 0; w < NWp; ++w) {
-      const int c = hist[w * E + e];
-      hist[w * E + e] = pos;
-      pos += c;
-    }
-  }
-  __syncthreads();
-  // pass 2: stable scatter
-  for (int b0 = p0; b0 < p1; b0 += 32 * kB) {
-    int ev[kB];
-#pragma unroll
-    for (int j = 0; j < kB; ++j) {
-      const int p = b0 + 32 * j + lane;
-      ev[j] = (p < p1) ? __ldg(a.topk_idx + p) : -1;
-    }
-#pragma unroll
-    for (int j = 0; j < kB; ++j) {
-      const int p = b0 + 32 * j + lane;
-      const int e = (ev[j] >= 0 && ev[j] < E) ? ev[j] : -1;
-      const unsigned peers = __match_any_sync(0xffffffffu, e);
-      if (e >= 0) {
-        const int rank = __popc(peers & ((1u << lane) - 1));
-        a.order[hist[warp * E + e] + rank] = p;
-      }
-      __syncwarp();
-      if (e >= 0 && lane == __ffs(peers) - 1) hist[warp * E + e] += __popc(peers);
-      __syncwarp();
-    }
-  }
-  for (int e = threadIdx.x; e <= E; e += kGroupThreads) {
+  for (int e = threadIdx.x; e <= E; e += kScanThreads) {
     a.offsets[e] = off[e];
     if (e < E) a.counts[e] = cnt[e];
   }
+  if (!a.units_gu) return;  // grouping only
+  // work units: per expert, token tiles of <= kNmax pairs x row tiles; then the shared
+  // expert.  Tile bases by an exclusive scan of the experts' tile counts.
   __syncthreads();
-  // work units: per expert, token tiles of <= 128 pairs x row tiles; then the shared expert.
-  // Tile bases by an exclusive scan of the experts' tile counts (one expert per thread).
+  int* tile_base = off;  // reuse after the offsets are out: [E + 1]
+  __shared__ int offc[kMaxExperts];
+  for (int e = threadIdx.x; e < E; e += kScanThreads) offc[e] = off[e];
   __syncthreads();
-  int* tile_base = hist;  // reuse: [E + 1]
-  for (int e = threadIdx.x; e < E; e += kGroupThreads) tile_base[e] = (cnt[e] + kNmax - 1) / kNmax;
-  __syncthreads();
-  if (threadIdx.x < 32) {  // one warp scans E <= 1024 counts in 32-wide chunks
-    int carry = 0;
-    for (int c0 = 0; c0 < E; c0 += 32) {
-      const int e = c0 + lane;
-      const int v = e < E ? tile_base[e] : 0;
-      int incl = v;
+  {
+    const int e = threadIdx.x;
+    const int v = e < E ? (cnt[e] + kNmax - 1) / kNmax : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int wv = wsum[lane];
+      int wi = wv;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+        const int y = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += y;
       }
-      if (e < E) tile_base[e] = carry + incl - v;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
+      wsum[lane] = wi - wv;
     }
-    if (lane == 0) tile_base[E] = carry;
+    __syncthreads();
+    if (e < E) tile_base[e] = wsum[warp] + incl - v;
+    if (e == E - 1) tile_base[E] = wsum[warp] + incl;
   }
   __syncthreads();
   const int mt_gu = a.I / 64, mt_dn = a.H / 128;
-  for (int e = threadIdx.x; e < E; e += kGroupThreads) {
+  for (int e = threadIdx.x; e < E; e += kScanThreads) {
     int tb = tile_base[e];
     for (int s0 = 0; s0 < cnt[e]; s0 += kNmax, ++tb) {
       const int nn = min(kNmax, cnt[e] - s0);
-      for (int mt = 0; mt < mt_gu; ++mt) a.units_gu[tb * mt_gu + mt] = GemmUnit{e, mt, off[e] + s0, nn};
-      for (int mt = 0; mt < mt_dn; ++mt) a.units_dn[tb * mt_dn + mt] = GemmUnit{e, mt, off[e] + s0, nn};
+      for (int mt = 0; mt < mt_gu; ++mt) a.units_gu[tb * mt_gu + mt] = GemmUnit{e, mt, offc[e] + s0, nn};
+      for (int mt = 0; mt < mt_dn; ++mt) a.units_dn[tb * mt_dn + mt] = GemmUnit{e, mt, offc[e] + s0, nn};
     }
   }
   const int tiles_r = tile_base[E];
   const int st_n = (a.T + kNmax - 1) / kNmax;
-  for (int i = threadIdx.x; i < st_n * mt_gu; i += kGroupThreads) {
+  for (int i = threadIdx.x; i < st_n * mt_gu; i += kScanThreads) {
     const int st = i / mt_gu, mt = i - st * mt_gu, t0 = st * kNmax;
     a.units_gu[(tiles_r + st) * mt_gu + mt] = GemmUnit{-1, mt, t0, min(kNmax, a.T - t0)};
   }
-  for (int i = threadIdx.x; i < st_n * mt_dn; i += kGroupThreads) {
+  for (int i = threadIdx.x; i < st_n * mt_dn; i += kScanThreads) {
     const int st = i / mt_dn, mt = i - st * mt_dn, t0 = st * kNmax;
     a.units_dn[(tiles_r + st) * mt_dn + mt] = GemmUnit{-1, mt, t0, min(kNmax, a.T - t0)};
   }
@@ -864,14 +903,60 @@ __global__ void __launch_bounds__(kGroupThreads) k_group(PrefillArgs a) {
   }
 }
 
+__global__ void __launch_bounds__(kGroupThreads) k_gplace(PrefillArgs a) {
+  extern __shared__ int wc[];  // [8][E]: per-warp counts, then per-warp running slots
+  constexpr int kW = kGroupThreads / 32, kRounds = kGroupChunk / kGroupThreads;
+  const int E = a.E, n = a.T * a.k;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kW * E; i += kGroupThreads) wc[i] = 0;
+  __syncthreads();
+  // warp w takes pairs [p0 + w * 32 * kRounds, ... + 32 * kRounds), round by round
+  const int pw = blockIdx.x * kGroupChunk + warp * 32 * kRounds;
+  int ev[kRounds];
+#pragma unroll
+  for (int r = 0; r < kRounds; ++r) {
+    const int p = pw + r * 32 + lane;
+    const int e = p < n ? __ldg(a.topk_idx + p) : -1;
+    ev[r] = (e >= 0 && e < E) ? e : -1;
+  }
+#pragma unroll
+  for (int r = 0; r < kRounds; ++r) {
+    const unsigned peers = __match_any_sync(0xffffffffu, ev[r]);
+    if (ev[r] >= 0 && lane == __ffs(peers) - 1) wc[warp * E + ev[r]] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  const int* base = a.chunk_cnt + (size_t)blockIdx.x * E;
+  for (int e = threadIdx.x; e < E; e += kGroupThreads) {
+    int pos = a.offsets[e] + base[e];
+#pragma unroll
+    for (int w = 0; w < kW; ++w) {
+      const int c = wc[w * E + e];
+      wc[w * E + e] = pos;
+      pos += c;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < kRounds; ++r) {
+    const int e = ev[r];
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0) a.order[wc[warp * E + e] + __popc(peers & ((1u << lane) - 1))] = pw + r * 32 + lane;
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * E + e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
 __global__ void k_finalize(const float* acc, const uint16_t* residual, uint16_t* out, size_t n) {
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = f2bf(acc[i] + (residual ? bf1(residual[i]) : 0.f));
 }
 
 __global__ void k_router_units(GemmUnit* units, int* n_units, int T, int E) {
-  // (E + 1) rows in tiles of 128 x tokens in tiles of 128
-  const int mt_n = (E + 1 + 127) / 128;
+  // E rows in tiles of 128 x tokens in tiles of 128 (the shared-expert gate logit is
+  // computed exactly by k_route)
+  const int mt_n = (E + 127) / 128;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   const int nt = (T + 127) / 128;
   if (i < mt_n * nt) {
@@ -885,7 +970,7 @@ template <int BITS, int MODE>
 cudaError_t launch_gemm(const GemmArgs& g, int n_sm, cudaStream_t s) {
   const int K = (MODE == kModeDown) ? g.I : g.H;
   size_t smem = (size_t)StageCount<MODE>::kA * kABytes + (size_t)StageCount<MODE>::kB * kBBytes;
-  if (MODE != kModeRouter) smem += kRawBytes + (size_t)128 * (K / kGroup) * 4;
+  if (MODE != kModeRouter) smem += kRawBytes + (size_t)128 * ((K / kGroup) * 4 + 16);
   auto fn = k_gemm<BITS, MODE>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -900,10 +985,11 @@ bool prefill_shape_supported(int H, int I, int bits, int E) {
 }
 
 cudaError_t launch_group(const PrefillArgs& p, cudaStream_t s) {
-  const size_t smem = sizeof(int) * ((size_t)(kGroupThreads / 32) * p.E + 2 * p.E + 2);
-  cudaError_t e = cudaFuncSetAttribute(k_group, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  k_group<<<1, kGroupThreads, smem, s>>>(p);
+  const int n_chunks = (p.T * p.k + kGroupChunk - 1) / kGroupChunk;
+  k_ghist<<<n_chunks, kGroupThreads, sizeof(int) * p.E, s>>>(p);
+  k_gscan<<<1, kScanThreads, 0, s>>>(p);
+  const size_t smem = sizeof(int) * (size_t)(kGroupThreads / 32) * p.E;
+  k_gplace<<<n_chunks, kGroupThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -921,7 +1007,7 @@ cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
     const int rows = T + E + 1;
     if (p.route) {
       k_norms<<<(rows * 32 + 255) / 256, 256, 0, s>>>(p.x, T, H, p.wr, p.wsg, E, p.xnorm, p.wnorm);
-      const int mt_n = (E + 1 + 127) / 128, nt = (T + 127) / 128;
+      const int mt_n = (E + 127) / 128, nt = (T + 127) / 128;
       k_router_units<<<(mt_n * nt + 255) / 256, 256, 0, s>>>(p.units_rt, p.n_units + 2, T, E);
       GemmArgs g = p.g;
       g.units = p.units_rt;

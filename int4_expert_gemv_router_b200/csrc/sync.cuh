@@ -42,6 +42,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
     if (now_ns() - t0 > kWaitNs) return false;
   }
 }
+// As mbar_wait, but each try suspends the thread until the phase completes or about
+// kSuspendNs have passed, so that a role waiting for a long stretch (a whole GEMM work unit)
+// takes no issue slots from the roles that are busy.
+constexpr uint32_t kSuspendNs = 100000;
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity), "r"(kSuspendNs)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_suspend(uint64_t* b, uint32_t parity) {
+  if (mbar_try_wait_suspend(b, parity)) return true;
+  const unsigned long long t0 = now_ns();
+  for (;;) {
+    if (mbar_try_wait_suspend(b, parity)) return true;
+    if (now_ns() - t0 > kWaitNs) return false;
+  }
+}
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
