@@ -264,6 +264,7 @@ static moe_status prefill_forward(const moe_shape* shape, const void* x, int32_t
   p.acc = reinterpret_cast<float*>(b + W.acc);
   p.h = reinterpret_cast<uint16_t*>(b + W.h);
   p.hs = reinterpret_cast<uint16_t*>(b + W.hs);
+  p.xg = reinterpret_cast<uint16_t*>(b + W.xg);
   GemmArgs& g = p.g;
   g.H = H;
   g.I = I;

@@ -1,6 +1,7 @@
 // Internal declarations shared by the sm_100a kernels and the C-ABI layer.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stddef.h>
@@ -218,6 +219,12 @@ struct GemmArgs {
   const GemmUnit* units;
   const int* n_units;
   Ctrl* ctrl;
+  // TMA descriptors (filled by the launcher per GEMM): A operand (router rows, or the raw
+  // codes of the pool and of the shared blob), B operand (x rows by gather or tile, h, hs)
+  alignas(64) CUtensorMap map_a;
+  alignas(64) CUtensorMap map_a_shared;
+  alignas(64) CUtensorMap map_b;
+  alignas(64) CUtensorMap map_b2;
 };
 
 struct PrefillArgs {
@@ -246,13 +253,14 @@ struct PrefillArgs {
   float* acc;
   uint16_t* h;
   uint16_t* hs;
+  uint16_t* xg;         // bf16 [T*k, H]: x rows in grouped pair order
   Ctrl* ctrl;
   GemmArgs g;           // shared GEMM arguments (units filled per launch)
 };
 
 struct PrefillLayout {
   size_t ctrl, xnorm, wnorm, logits, topk_idx, topk_w, gate, order, offsets, counts, chunk_cnt, units_rt,
-      units_gu, units_dn, n_units, acc, h, hs, total;
+      units_gu, units_dn, n_units, acc, h, hs, xg, total;
 };
 
 inline PrefillLayout make_prefill_layout(int T, int E, int k, int H, int I) {
@@ -284,6 +292,7 @@ inline PrefillLayout make_prefill_layout(int T, int E, int k, int H, int I) {
   W.acc = take(sizeof(float) * (size_t)T * H);
   W.h = take(2 * (size_t)T * k * I);
   W.hs = take(2 * (size_t)T * I);
+  W.xg = take(2 * (size_t)T * k * H);
   W.total = (size_t)round_up((int64_t)pos, kAlign);
   return W;
 }

@@ -11,9 +11,9 @@
 //                  fp32 error bound of the k-th is recomputed exactly (fp64 sums of exact
 //                  bf16 products) and the selection is made on the exact values; softmax
 //                  over the selected logits; shared-expert gate
-//   k_ghist, k_gscan, k_gplace
+//   k_ghist, k_gcol, k_gplace
 //                  stable counting sort of the (token, k) pairs by expert (per-chunk counts,
-//                  one scan, per-chunk stable placement) and the list of GEMM work units
+//                  per-expert scans down the chunks, per-chunk stable placement) and the list of GEMM work units
 //                  (expert, row tile, token tile)
 //   k_gemm GATEUP  per unit: [gate; up] rows of one expert (dequantised to bf16 in shared
 //                  memory) x the expert's tokens (gathered), SwiGLU in the epilogue -> h
@@ -41,6 +41,8 @@
 
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 namespace moe {
 namespace {
 
@@ -48,28 +50,65 @@ constexpr int kKC = 64;                   // K per stage
 constexpr int kNmax = kPrefillN;          // tokens per unit (MMA N)
 constexpr int kABytes = 128 * kKC * 2;    // 16 KB
 constexpr int kBBytes = kNmax * kKC * 2;  // 16 KB
-constexpr int kBWarp0 = 1, kBWarps = 2;
-constexpr int kAWarp0 = 3, kAWarps = 8;
-constexpr int kEWarp0 = 11, kEWarps = 4;
+// warp roles
+constexpr int kBLoadWarp = 1;             // lane 0: B tiles by TMA
+constexpr int kALoadWarp = 2;             // lane 0: raw codes (or router rows) by TMA
+constexpr int kAWarp0 = 3, kAWarps = 8;   // dequantisation
+constexpr int kEWarp0 = 11, kEWarps = 4;  // epilogue
 constexpr int kGemmThreads = (kEWarp0 + kEWarps) * 32;  // 480
-constexpr int kSBO = (kKC / 8) * 128;     // 1024
+constexpr int kSBO = (kKC / 8) * 128;     // 1024: 8-row group stride of a no-swizzle K-major tile
 constexpr int kTmemCols = 2 * kNmax;      // two accumulators
-constexpr int kRawBytes = 32 * 1024;      // cp.async ring of raw weight bytes (A producers)
-constexpr int kAThreads = kAWarps * 32;
-// raw bytes per A thread per stage, and ring depth, per mode / width
+constexpr int kBRows = 32;                // rows per B tile load (tile mode)
+constexpr int kStageMax = 6;              // A and B stages: at most 6 each
+
+constexpr int kSmemMax = 227 * 1024 - 8 * 1024;  // dynamic shared memory budget (static part aside)
+// raw codes of one stage (128 rows x 64 codes)
+// (32 KB of them in flight ahead of the dequantisation)
+template <int BITS>
+struct Raw {
+  static constexpr int kRowBytes = kKC * BITS / 8;  // 32 or 64
+  static constexpr int kBytes = 128 * kRowBytes;    // 4 or 8 KB
+  static constexpr int kDepth = 32768 / kBytes;     // 8 or 4 stages
+};
+
+// Position in a ring of n stages and the parity of its current pass.
+struct Ring {
+  int n, s = 0;
+  uint32_t ph = 0;
+  __device__ explicit Ring(int n_) : n(n_) {}
+  __device__ void next() {
+    if (++s == n) {
+      s = 0;
+      ph ^= 1;
+    }
+  }
+};
+
+// Shared-memory plan of one GEMM launch (host and device agree on it).
+struct GemmSmem {
+  int n_sa, n_sb;      // A and B stages
+  uint32_t raw, sb;    // byte offsets of the raw ring and the scale buffers
+  uint32_t sb_ld;      // uint16 per row of a scale buffer
+  uint32_t total;      // dynamic bytes, including 1 KB of alignment slack
+};
 template <int BITS, int MODE>
-struct RawRing {
-  static constexpr int kBytes = BITS == 4 ? 16 : 32;
-  static constexpr int kDepth = kRawBytes / (kAThreads * kBytes);
-};
-// A and B tile stages (16 KB each).  The dequantising modes also hold the raw ring and the
-// unit's scales and biases (up to 32 KB at K = 4096), so they keep fewer A stages: the raw
-// ring already runs kDepth stages ahead of the dequantisation.
-template <int MODE>
-struct StageCount {
-  static constexpr int kA = MODE == kModeRouter ? 6 : 3;
-  static constexpr int kB = 6;
-};
+__host__ __device__ inline GemmSmem gemm_smem(int K) {
+  GemmSmem p{};
+  const int NG = K / kGroup;
+  p.sb_ld = (uint32_t)(2 * NG + 8);  // scales, biases, 16 bytes of padding
+  const uint32_t fixed = MODE == kModeRouter ? 0u : (uint32_t)(Raw<BITS>::kDepth * Raw<BITS>::kBytes + 2 * 128 * p.sb_ld * 2);
+  // A stages first (the dequantisation loop needs about four), then B stages, then the rest to A
+  int na = MODE == kModeRouter ? 2 : 4, nb = 2;
+  auto fits = [&](int a_, int b_) { return (uint32_t)(a_ + b_) * 16384u + fixed + 1024u <= (uint32_t)kSmemMax; };
+  while (nb < kStageMax && fits(na, nb + 1)) ++nb;
+  while (na < kStageMax && fits(na + 1, nb)) ++na;
+  p.n_sa = na;
+  p.n_sb = nb;
+  p.raw = (uint32_t)(na + nb) * 16384u;
+  p.sb = p.raw + (MODE == kModeRouter ? 0u : (uint32_t)(Raw<BITS>::kDepth * Raw<BITS>::kBytes));
+  p.total = (uint32_t)(na + nb) * 16384u + fixed + 1024u;
+  return p;
+}
 
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
   uint64_t d = 0;
@@ -85,6 +124,43 @@ __device__ __forceinline__ uint32_t umma_idesc(int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
+// K-major operand with 128-byte swizzle (rows of 64 bf16 = 128 bytes, 16-byte chunks XOR-ed
+// with the row's position in its 8-row group; the layout TMA writes with SWIZZLE_128B).  The
+// k-step of one MMA (16 elements = 32 bytes) advances the start address; 8-row groups are
+// 1024 bytes apart.  Tiles start on 1024-byte boundaries.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;                         // LBO (unused for swizzled K-major)
+  d |= (uint64_t)((1024u >> 4) & 0x3FFFu) << 32;  // SBO: next 8-row group
+  d |= (uint64_t)1 << 46;                         // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                         // layout: 128-byte swizzle
+  return d;
+}
+
+// TMA loads into this CTA's shared memory, completing on an mbarrier (transaction bytes).
+__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(dst),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                       uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+      "[%6];" ::"r"(dst),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
 __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
@@ -114,11 +190,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// arrival on an mbarrier once every cp.async this thread has issued so far has landed
-// (.noinc: the arrival is one of the barrier's expected count)
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
@@ -200,6 +271,12 @@ __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, Ctr
   return false;
 }
 
+// The abort flag as the whole warp sees it (one value for all lanes, so that no lane
+// leaves a loop whose other lanes go on to a __syncwarp).
+__device__ __forceinline__ bool warp_aborted(const int* flag) {
+  return __any_sync(0xffffffffu, *reinterpret_cast<const volatile int*>(flag) != 0);
+}
+
 // Every lane of a warp waits, and all take the same branch afterwards (a lane whose wait
 // ran out would otherwise leave the others behind at the next __syncwarp).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Ctrl* c, int lane) {
@@ -208,37 +285,54 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Ctrl* 
   return ok;
 }
 
+// Wait (bounded) for the last loads a loader issued into a ring of n full barriers, so that
+// no copy is still landing when the CTA leaves (the consumers normally waited for them).
+__device__ __forceinline__ void drain_ring(uint64_t* full, int n, int issued, Ctrl* c) {
+  for (int q = issued > n ? issued - n : 0; q < issued; ++q)
+    if (!mbar_wait(&full[q % n], (uint32_t)((q / n) & 1))) {
+      atomicOr(&c->err, kErrTimeout);
+      return;
+    }
+}
+
 // ---------------------------------------------------------------------------------------
 // GEMM kernel
 // ---------------------------------------------------------------------------------------
 template <int BITS, int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant__ GemmArgs a) {
-  constexpr int kSA = StageCount<MODE>::kA, kSB = StageCount<MODE>::kB;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ __align__(8) uint64_t a_full[kSA], a_empty[kSA], b_full[kSB], b_empty[kSB], acc_full[2],
-      acc_empty[2], drain;
+  constexpr int kRawB = Raw<BITS>::kBytes, kDepth = Raw<BITS>::kDepth;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t a_full[kStageMax], a_empty[kStageMax], b_full[kStageMax], b_empty[kStageMax],
+      raw_full[8], raw_empty[8], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  __shared__ int s_colt[kEWarps][kNmax];  // per epilogue warp (down): token of each column
-  __shared__ float s_colw[kEWarps][kNmax];  // and its routing weight
+  __shared__ int s_colt[kEWarps][kNmax];       // per epilogue warp (down): token of each column
+  __shared__ float s_colw[kEWarps][kNmax];     // and its routing weight
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int K = (MODE == kModeDown) ? a.I : a.H;
   const int nK = K / kKC;
   const int n_units = *a.n_units;
-  const uint32_t smem_base = smem_u32(smem);
-  const uint32_t b_area = smem_base + kSA * kABytes;
+  const GemmSmem P = gemm_smem<BITS, MODE>(K);
+  // stage tiles start on 1024-byte boundaries (128-byte swizzle atoms)
+  const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (smem_base - smem_u32(smem_raw));
+  const uint32_t b_area = smem_base + P.n_sa * kABytes;
+  const int my_units = n_units > (int)blockIdx.x ? (n_units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (tid == 0) {
-    for (int s = 0; s < kSA; ++s) {
-      // router rows are plain copies whose completion each A thread signals; dequantised
-      // tiles are signalled once per A warp
-      mbar_init(&a_full[s], MODE == kModeRouter ? kAThreads : kAWarps);
+    for (int s = 0; s < P.n_sa; ++s) {
+      // router rows arrive by TMA (one expect-tx arrival); dequantised tiles once per A warp
+      mbar_init(&a_full[s], MODE == kModeRouter ? 1 : kAWarps);
       mbar_init(&a_empty[s], 1);
     }
-    for (int s = 0; s < kSB; ++s) {
-      mbar_init(&b_full[s], kBWarps * 32);  // one cp.async-tracking arrival per B thread
+    for (int s = 0; s < P.n_sb; ++s) {
+      mbar_init(&b_full[s], 1);
       mbar_init(&b_empty[s], 1);
+    }
+    for (int s = 0; s < kDepth; ++s) {
+      mbar_init(&raw_full[s], 1);
+      mbar_init(&raw_empty[s], kAWarps);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -261,7 +355,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
   if (warp == 0) {
     // ------------------------------ MMA issuer ------------------------------
     if (lane == 0) {
-      uint32_t q = 0;
+      Ring ra(P.n_sa), rb(P.n_sb);
       int it = 0;
       for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x, ++it) {
         const GemmUnit U = a.units[u];
@@ -274,23 +368,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)buf * (uint32_t)kNmax;
-        for (int kc = 0; kc < nK; ++kc, ++q) {
-          const int sa = q % kSA, sb = q % kSB;
-          if (!wait_or_flag(&a_full[sa], (q / kSA) & 1, a.ctrl) || !wait_or_flag(&b_full[sb], (q / kSB) & 1, a.ctrl)) {
+        for (int kc = 0; kc < nK; ++kc, ra.next(), rb.next()) {
+          if (!wait_or_flag(&b_full[rb.s], rb.ph, a.ctrl) || !wait_or_flag(&a_full[ra.s], ra.ph, a.ctrl)) {
             s_abort = 1;
             break;
           }
-          // the tiles were written through the generic proxy (st.shared, cp.async)
-          proxy_fence();
+          // dequantised tiles were written through the generic proxy (st.shared)
+          if (MODE != kModeRouter) proxy_fence();
           tc_fence_after();
-          const uint32_t a_base = smem_base + sa * kABytes;
-          const uint32_t b_base = b_area + sb * kBBytes;
+          const uint32_t a_base = smem_base + ra.s * kABytes;
+          const uint32_t b_base = b_area + rb.s * kBBytes;
 #pragma unroll
-          for (int kk = 0; kk < kKC / 16; ++kk)
-            umma_f16(d_tmem, umma_desc(a_base + kk * 256), umma_desc(b_base + kk * 256), idesc,
-                     (kc > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&a_empty[sa]);
-          umma_commit(&b_empty[sb]);
+          for (int kk = 0; kk < kKC / 16; ++kk) {
+            const uint64_t da = MODE == kModeRouter ? umma_desc_sw128(a_base + kk * 32) : umma_desc(a_base + kk * 256);
+            umma_f16(d_tmem, da, umma_desc_sw128(b_base + kk * 32), idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&a_empty[ra.s]);
+          umma_commit(&b_empty[rb.s]);
         }
         if (s_abort) break;
         umma_commit(&acc_full[buf]);
@@ -300,173 +394,184 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       if (!mbar_wait(&drain, 0)) atomicOr(&a.ctrl->err, kErrTimeout);
     }
     __syncwarp();
-  } else if (warp >= kBWarp0 && warp < kBWarp0 + kBWarps) {
-    // ------------------------------ B gather (cp.async) ------------------------------
-    // Thread bt copies columns bt and bt + 64 of the unit (one token or pair row each, 128
-    // bytes per stage).  Each thread's copies of a stage are tracked by the stage's mbarrier
-    // (an arrival that fires when they have landed), so the gather runs up to kSB stages ahead.
-    const int bt = tid - kBWarp0 * 32;  // 0..63
-    uint32_t q = 0;
-    for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x) {
+  } else if (warp == kBLoadWarp) {
+    // ------------------------------ B tiles (TMA) ------------------------------
+    // Every unit's columns are consecutive rows of a bf16 matrix: x for the router and the
+    // shared expert, the expert-ordered copy xg of x for routed gate/up units, h / hs for
+    // down.  Loads of kBRows rows, one per lane; rows from U.n up to the loaded count belong
+    // to other units or lie beyond the matrix (zero filled): their products are never read.
+    Ring rb(P.n_sb);
+    int issued = 0;
+    for (int u = blockIdx.x; u < n_units && !warp_aborted(&s_abort); u += gridDim.x) {
       const GemmUnit U = a.units[u];
       const int npad = (U.n + 15) & ~15;
-      const uint16_t* src_base;
-      int src_ld;
-      if (MODE == kModeDown) {
-        src_base = (U.e < 0) ? a.hs : a.h;
-        src_ld = a.I;
-      } else {
-        src_base = a.x;
-        src_ld = a.H;
-      }
-      // source row of each of the thread's two columns; nullptr: zero column (n >= U.n)
-      const uint16_t* rows[2];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int n = bt + c * 64;
-        int r = -1;
-        if (n < U.n) r = (MODE == kModeGateUp && U.e >= 0) ? __ldg(a.order + U.p0 + n) / a.k : U.p0 + n;
-        rows[c] = r < 0 ? nullptr : src_base + (size_t)r * src_ld;
-      }
       bool stop = false;
-      for (int kc = 0; kc < nK; ++kc, ++q) {
-        const int sb = q % kSB;
-        if (!warp_wait(&b_empty[sb], ((q / kSB) & 1) ^ 1, a.ctrl, lane)) {
-          s_abort = 1;
+      const CUtensorMap* mb = (MODE != kModeRouter && U.e < 0) ? &a.map_b2 : &a.map_b;
+      const int nrt = (npad + kBRows - 1) / kBRows;
+      const uint32_t bytes = (uint32_t)nrt * kBRows * 128u;
+      for (int kc = 0; kc < nK; ++kc, rb.next()) {
+        if (!warp_wait(&b_empty[rb.s], rb.ph ^ 1, a.ctrl, lane)) {
           stop = true;
           break;
         }
-        const uint32_t b_base = b_area + sb * kBBytes;
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int n = bt + c * 64;
-          if (n < npad) {  // columns beyond npad are not read by the MMA
-            const uint16_t* src = rows[c] ? rows[c] + kc * kKC : a.x;
-            const uint32_t d = b_base + core_off(n, 0);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) cp_async16(d + j * 128, src + j * 8, rows[c] ? 16u : 0u);
+        if (lane == 0) mbar_expect_tx(&b_full[rb.s], bytes);
+        __syncwarp();  // the transaction count is registered before any load can land
+        if (lane < nrt)
+          tma_2d(b_area + rb.s * kBBytes + lane * kBRows * 128, mb, kc * kKC, U.p0 + lane * kBRows, &b_full[rb.s]);
+        ++issued;
+      }
+      if (stop) {
+        s_abort = 1;
+        break;
+      }
+    }
+    // drain: the last loads this thread issued have landed before the CTA may leave
+    if (lane == 0) drain_ring(b_full, P.n_sb, issued, a.ctrl);
+  } else if (warp == kALoadWarp) {
+    // ------------------------------ A operand loads (TMA) ------------------------------
+    // Router: 128 router rows x 64 columns per stage straight into the A tile.  Otherwise the
+    // stage's raw codes (128 rows x 64 codes) into the raw ring, for the dequantising warps;
+    // a unit whose expert has no valid slot reads an out-of-range slot, which TMA fills with
+    // zeros (its scales are zero too, so it dequantises to 0).
+    if (lane == 0) {
+      Ring rr(MODE == kModeRouter ? P.n_sa : kDepth);
+      int issued = 0;
+      bool stop = false;
+      // unit descriptors two units ahead and slots one unit ahead, so that the lookups'
+      // latency is hidden behind the previous unit's loads
+      auto unit_at = [&](int j) { return a.units[blockIdx.x + (size_t)j * gridDim.x]; };
+      auto slot_of = [&](const GemmUnit& U) { return (MODE == kModeRouter || U.e < 0) ? 0 : a.slot_table[U.e]; };
+      GemmUnit un1{}, un2{};
+      int slot1 = 0;
+      if (my_units > 0) {
+        un1 = unit_at(0);
+        slot1 = slot_of(un1);
+      }
+      if (my_units > 1) un2 = unit_at(1);
+      for (int j = 0; j < my_units && !stop && !s_abort; ++j) {
+        const GemmUnit U = un1;
+        int slot = slot1;
+        un1 = un2;
+        if (j + 1 < my_units) slot1 = slot_of(un1);
+        if (j + 2 < my_units) un2 = unit_at(j + 2);
+        const CUtensorMap* ma = &a.map_a;
+        if (MODE != kModeRouter) {
+          if (U.e < 0) {
+            ma = &a.map_a_shared;
+            slot = 0;
+          } else {
+            if (slot < 0 || slot >= a.n_slots) {
+              atomicOr(&a.ctrl->err, kErrBadSlot);
+              slot = (int)a.n_slots;  // out of range: zero fill
+            }
           }
         }
-        cp_async_arrive_noinc(&b_full[sb]);
-      }
-      if (stop) break;
-    }
-    cp_async_wait<0>();  // no copy may still be landing when the CTA leaves
-  } else if (warp >= kAWarp0 && warp < kAWarp0 + kAWarps && MODE == kModeRouter) {
-    // ------------------------------ A rows of the router (bf16, plain copies) ------------------------------
-    int m, half;
-    a_lane_map(tid - kAWarp0 * 32, m, half);
-    uint32_t q = 0;
-    for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x) {
-      const GemmUnit U = a.units[u];
-      const int e = U.mt * 128 + m;
-      const uint16_t* row = e < a.E ? a.wr + (size_t)e * a.H : nullptr;
-      bool stop = false;
-      for (int kc = 0; kc < nK; ++kc, ++q) {
-        const int sa = q % kSA;
-        if (!warp_wait(&a_empty[sa], ((q / kSA) & 1) ^ 1, a.ctrl, lane)) {
-          s_abort = 1;
-          stop = true;
-          break;
+        for (int kc = 0; kc < nK; ++kc, rr.next()) {
+          if (MODE == kModeRouter) {
+            if (!wait_or_flag(&a_empty[rr.s], rr.ph ^ 1, a.ctrl)) {
+              stop = true;
+              break;
+            }
+            mbar_expect_tx(&a_full[rr.s], kABytes);
+            tma_2d(smem_base + rr.s * kABytes, ma, kc * kKC, U.mt * 128, &a_full[rr.s]);
+          } else {
+            if (!wait_or_flag(&raw_empty[rr.s], rr.ph ^ 1, a.ctrl)) {
+              stop = true;
+              break;
+            }
+            const uint32_t dst = smem_base + P.raw + rr.s * kRawB;
+            mbar_expect_tx(&raw_full[rr.s], kRawB);
+            if (MODE == kModeGateUp)  // [gate; up] x 64 rows of the row tile
+              tma_4d(dst, ma, kc * Raw<BITS>::kRowBytes, U.mt * 64, 0, slot, &raw_full[rr.s]);
+            else
+              tma_3d(dst, ma, kc * Raw<BITS>::kRowBytes, U.mt * 128, slot, &raw_full[rr.s]);
+          }
+          ++issued;
         }
-        const uint32_t a_base = smem_base + sa * kABytes;
-#pragma unroll
-        for (int o = 0; o < 4; ++o) {
-          const uint16_t* src = row ? row + kc * kKC + (half * 4 + o) * 8 : a.wsg;
-          cp_async16(a_base + core_off(m, half * 4 + o), src, row ? 16u : 0u);
-        }
-        cp_async_arrive_noinc(&a_full[sa]);
       }
-      if (stop) break;
+      if (stop) s_abort = 1;
+      drain_ring(MODE == kModeRouter ? a_full : raw_full, MODE == kModeRouter ? P.n_sa : kDepth, issued, a.ctrl);
     }
-    cp_async_wait<0>();
-  } else if (warp >= kAWarp0 && warp < kAWarp0 + kAWarps) {
-    // ------------------------------ A producers (dequantise) ------------------------------
-    // Raw weight bytes stream into a cp.async ring (kDepth stages ahead); each unit's row
-    // scales and biases land once in shared memory (of the two threads of a row, half 0
-    // copies the scales, half 1 the biases).  A thread only ever reads ring bytes it copied
-    // itself; its partner's half of the scales becomes visible at the __syncwarp that
-    // follows both threads' waits.
-    using RR = RawRing<BITS, MODE>;
-    constexpr int kDepth = RR::kDepth, kRB = RR::kBytes, kPieces = kRB / 16;
+    __syncwarp();
+  } else if (warp >= kAWarp0 && warp < kAWarp0 + kAWarps && MODE != kModeRouter) {
+    // ------------------------------ dequantisation ------------------------------
+    // Thread (m, half) turns 32 codes of tile row m per stage into bf16 in the A tile.  Each
+    // unit's row scales and biases are copied (cp.async) into one of two buffers one unit
+    // ahead (of the two threads of a row, half 0 copies the scales, half 1 the biases).
     const int at = tid - kAWarp0 * 32;  // 0..255
     int m, half;                        // tile row 0..127, which 32 columns of the stage
     a_lane_map(at, m, half);
-    const int NG = K / kGroup;          // groups (= stages) per row
-    const int sb_ld = 2 * NG + 8;       // uint16 per row of the scale area (16 bytes of padding)
-    // ring: [slot][piece][thread][16 bytes], so a warp's accesses are 512 contiguous bytes
-    uint8_t* raw_ring = smem + (size_t)kSA * kABytes + (size_t)kSB * kBBytes;
-    uint8_t* my_raw = raw_ring + (size_t)at * 16;
-    uint16_t* sb_area = reinterpret_cast<uint16_t*>(raw_ring + kRawBytes);  // [128][sb_ld]
-    uint16_t* my_s = sb_area + (size_t)m * sb_ld;
-    uint16_t* my_b = my_s + NG;
-    uint32_t q = 0;
-    for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x) {
-      const GemmUnit U = a.units[u];
-      // this thread's weight row (bytes of the row, its scales and biases)
+    const int NG = K / kGroup;  // groups (= stages) per row
+    const int sb_ld = (int)P.sb_ld;
+    uint16_t* sb_area = reinterpret_cast<uint16_t*>(smem + P.sb);  // [2][128][sb_ld]
+    // offset of this thread's 16-byte pieces in a raw stage (TMA box layout)
+    const uint32_t raw_off = MODE == kModeGateUp
+                                 ? (uint32_t)((m & 1) * 64 + (m >> 1)) * Raw<BITS>::kRowBytes + half * (kRawB / 256)
+                                 : (uint32_t)m * Raw<BITS>::kRowBytes + half * (kRawB / 256);
+    auto unit_at = [&](int j) { return a.units[blockIdx.x + (size_t)j * gridDim.x]; };
+    auto slot_of = [&](const GemmUnit& U) { return U.e < 0 ? 0 : a.slot_table[U.e]; };
+    // scales / biases of unit ordinal j (descriptor U, slot) into buffer j & 1
+    auto load_scales = [&](int j, const GemmUnit& U, int slot) {
+      const uint8_t* blob = a.shared;
+      if (U.e >= 0) blob = (slot < 0 || slot >= a.n_slots) ? nullptr : a.pool + (int64_t)slot * a.L.stride;
       const uint8_t* src = nullptr;
-      const uint8_t* sbsrc = nullptr;
-      {
-        const uint8_t* blob = nullptr;
-        if (U.e < 0) {
-          blob = a.shared;
+      if (blob) {
+        if (MODE == kModeGateUp) {
+          const int r = U.mt * 64 + (m >> 1);
+          src = blob + a.L.off[((m & 1) ? 5 : 3) + half] + (int64_t)r * NG * 2;
         } else {
-          const int slot = a.slot_table[U.e];
-          if (slot < 0 || slot >= a.n_slots) atomicOr(&a.ctrl->err, kErrBadSlot);
-          else blob = a.pool + (int64_t)slot * a.L.stride;
-        }
-        if (blob) {
-          if (MODE == kModeGateUp) {
-            const int r = U.mt * 64 + (m >> 1);
-            const int up = m & 1;  // rows alternate gate, up of the same intermediate row
-            src = blob + a.L.off[up ? 1 : 0] + (int64_t)r * (a.H * BITS / 8);
-            sbsrc = blob + a.L.off[(up ? 5 : 3) + half] + (int64_t)r * NG * 2;
-          } else {
-            const int j = U.mt * 128 + m;
-            src = blob + a.L.off[2] + (int64_t)j * (a.I * BITS / 8);
-            sbsrc = blob + a.L.off[7 + half] + (int64_t)j * NG * 2;
-          }
+          src = blob + a.L.off[7 + half] + (int64_t)(U.mt * 128 + m) * NG * 2;
         }
       }
-      const bool zero = (src == nullptr);
-      auto issue = [&](int kc) {  // raw bytes of stage kc into ring slot kc % kDepth
-        if (!zero && kc < nK) {
-          const uint8_t* g = src + (size_t)kc * (kKC * BITS / 8) + half * kRB;
-          const uint32_t d = smem_u32(my_raw + (size_t)(kc % kDepth) * kPieces * (kAThreads * 16));
-#pragma unroll
-          for (int o = 0; o < kPieces; ++o) cp_async16(d + o * (kAThreads * 16), g + o * 16, 16u);
-        }
-        cp_async_commit();  // one group per stage, empty past the end, so the counts stay uniform
-      };
-      // scales/biases of the row (one group with stage 0), then the first kDepth stages
-      if (!zero) {
-        uint16_t* dst = half ? my_b : my_s;
-        if ((NG & 7) == 0) {  // rows of 16-byte multiples: 16-byte aligned in the blob and here
-          for (int o = 0; o < NG * 2; o += 16) cp_async16(smem_u32(dst) + o, sbsrc + o, 16u);
-        } else {  // narrow rows (small K): plain loads, visible after the first __syncwarp
-          const uint16_t* g = reinterpret_cast<const uint16_t*>(sbsrc);
-          for (int o = 0; o < NG; ++o) dst[o] = __ldg(g + o);
-        }
+      uint16_t* dst = sb_area + (size_t)(j & 1) * 128 * sb_ld + (size_t)m * sb_ld + (half ? NG : 0);
+      if ((NG & 7) == 0) {  // rows of 16-byte multiples: 16-byte aligned in the blob and here
+        for (int o = 0; o < NG * 2; o += 16) cp_async16(smem_u32(dst) + o, src ? src + o : a.pool, src ? 16u : 0u);
+      } else {  // narrow rows (small K): plain loads
+        const uint16_t* g = reinterpret_cast<const uint16_t*>(src);
+        for (int o = 0; o < NG; ++o) dst[o] = g ? __ldg(g + o) : (uint16_t)0;
       }
-#pragma unroll 1
-      for (int d = 0; d < kDepth; ++d) issue(d);
+      cp_async_commit();
+    };
+    GemmUnit un1{}, un2{};
+    int slot1 = 0;
+    if (my_units > 0) {
+      const GemmUnit u0 = unit_at(0);
+      load_scales(0, u0, slot_of(u0));
+      if (my_units > 1) {
+        un1 = unit_at(1);
+        slot1 = slot_of(un1);
+      }
+      if (my_units > 2) un2 = unit_at(2);
+    }
+    Ring ra(P.n_sa), rr(kDepth);
+    for (int j = 0; j < my_units && !warp_aborted(&s_abort); ++j) {
+      cp_async_wait<0>();  // this unit's scales (own half) have landed
+      __syncwarp();        // ... and the partner's half; buffer (j + 1) & 1 is no longer read
+      if (j + 1 < my_units) {
+        load_scales(j + 1, un1, slot1);
+        un1 = un2;
+        if (j + 2 < my_units) slot1 = slot_of(un1);
+        if (j + 3 < my_units) un2 = unit_at(j + 3);
+      }
+      const uint16_t* my_s = sb_area + (size_t)(j & 1) * 128 * sb_ld + (size_t)m * sb_ld;
       bool stop = false;
-      for (int kc = 0; kc < nK; ++kc, ++q) {
-        const int sa = q % kSA;
-        cp_async_wait<kDepth - 1>();  // this thread's bytes of stage kc have landed
-        __syncwarp();                 // ... and the partner's half of the scales
-        if (!warp_wait(&a_empty[sa], ((q / kSA) & 1) ^ 1, a.ctrl, lane)) {
-          s_abort = 1;
+      for (int kc = 0; kc < nK; ++kc, ra.next(), rr.next()) {
+        if (!warp_wait(&raw_full[rr.s], rr.ph, a.ctrl, lane)) {
           stop = true;
           break;
         }
-        const uint8_t* rp = my_raw + (size_t)(kc % kDepth) * kPieces * (kAThreads * 16);
-        uint4 rw[kPieces];
+        const uint8_t* rp = smem + P.raw + rr.s * kRawB + raw_off;
+        uint4 rw[Raw<BITS>::kRowBytes / 32];
 #pragma unroll
-        for (int o = 0; o < kPieces; ++o)
-          rw[o] = zero ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4*>(rp + o * (kAThreads * 16));
-        const uint32_t sbits = zero ? 0u : my_s[kc], bbits = zero ? 0u : my_b[kc];
-        uint8_t* a_tile = smem + sa * kABytes;
+        for (int o = 0; o < Raw<BITS>::kRowBytes / 32; ++o) rw[o] = *reinterpret_cast<const uint4*>(rp + o * 16);
+        const uint32_t sbits = my_s[kc], bbits = my_s[NG + kc];
+        __syncwarp();  // every lane holds its codes: the raw slot can be refilled
+        if (lane == 0) mbar_arrive(&raw_empty[rr.s]);
+        if (!warp_wait(&a_empty[ra.s], ra.ph ^ 1, a.ctrl, lane)) {
+          stop = true;
+          break;
+        }
+        uint8_t* a_tile = smem + ra.s * kABytes;
         if (BITS == 4) {
           const uint32_t s2 = sbits | (sbits << 16), b2 = bbits | (bbits << 16);
           const uint32_t w4[4] = {rw[0].x, rw[0].y, rw[0].z, rw[0].w};
@@ -482,15 +587,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             *reinterpret_cast<uint4*>(a_tile + core_off(m, half * 4 + o)) = v;
           }
         }
-        // the ring slot's bytes and this stage's scales are consumed (the stores above depend
-        // on them): refill the slot, and let the partner go on to overwrite the scales
-        __syncwarp();
-        issue(kc + kDepth);
         proxy_fence();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[sa]);
+        if (lane == 0) mbar_arrive(&a_full[ra.s]);
       }
-      if (stop) break;
+      if (stop) {
+        s_abort = 1;
+        break;
+      }
     }
     cp_async_wait<0>();  // no copy may still be landing when the CTA leaves
   } else if (warp >= kEWarp0) {
@@ -498,7 +602,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     const int quad = warp & 3;       // TMEM lane quadrant of this warp
     const int m = quad * 32 + lane;  // accumulator row
     int it = 0;
-    for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x, ++it) {
+    for (int u = blockIdx.x; u < n_units && !warp_aborted(&s_abort); u += gridDim.x, ++it) {
       const GemmUnit U = a.units[u];
       const int buf = it & 1;
       if (MODE == kModeDown) {
@@ -528,20 +632,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       for (int c0 = 0; c0 < U.n; c0 += 8) {
         float v[8];
         tmem_ld8(taddr + c0, v);
+        if (MODE == kModeGateUp) {
+          // lanes 2i (gate row) and 2i + 1 (up row) hold intermediate row r; the even lane
+          // finishes column c, the odd lane column c + 1 (one exchange per column pair)
+          const bool odd = lane & 1;
+          const int r = U.mt * 64 + (m >> 1);
+          uint16_t* hbase = (U.e < 0) ? a.hs : a.h;
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) {
+            const float recv = __shfl_xor_sync(0xffffffffu, odd ? v[i] : v[i + 1], 1);
+            const float g = odd ? recv : v[i];
+            const float up = odd ? v[i + 1] : recv;
+            const int n = c0 + i + (odd ? 1 : 0);
+            // silu(g) * up; h is rounded to bf16, far coarser than the fast exp / divide
+            if (n < U.n) hbase[(size_t)(U.p0 + n) * a.I + r] = f2bf(__fdividef(g, 1.0f + __expf(-g)) * up);
+          }
+        } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int n = c0 + i;
           const float val = v[i];
-          if (MODE == kModeGateUp) {
-            const float other = __shfl_xor_sync(0xffffffffu, val, 1);
-            if (n < U.n && !(m & 1)) {
-              const float g = val, up = other;
-              const float hv = g / (1.0f + expf(-g)) * up;
-              const int r = U.mt * 64 + (m >> 1);
-              uint16_t* dst = (U.e < 0) ? a.hs + (size_t)(U.p0 + n) * a.I : a.h + (size_t)(U.p0 + n) * a.I;
-              dst[r] = f2bf(hv);
-            }
-          } else if (MODE == kModeDown) {
+          if (MODE == kModeDown) {
             if (n < U.n) {
               const int j = U.mt * 128 + m;
               atomicAdd(a.acc + (size_t)s_colt[quad][n] * a.H + j, s_colw[quad][n] * val);
@@ -550,6 +661,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             const int e = U.mt * 128 + m;
             if (n < U.n && e < a.E) a.logits[(size_t)(U.p0 + n) * (a.E + 1) + e] = val;
           }
+        }
         }
       }
       tc_fence_before();
@@ -760,15 +872,17 @@ __global__ void __launch_bounds__(256) k_route(PrefillArgs a) {
 // ---------------------------------------------------------------------------------------
 // stable counting sort of the pairs by expert, and the GEMM work units.
 //   k_ghist   per chunk of kGroupChunk pairs: its per-expert counts
-//   k_gscan   per expert: exclusive sums over the chunks (in place), the expert's total;
-//             offsets = exclusive scan of the totals; GEMM work units
-//   k_gplace  per chunk: stable ranks (warp match + per-warp counts), order[slot] = pair
+//   k_gcol    one warp per expert: exclusive sums of its counts down the chunks (in
+//             place) and the expert's total
+//   k_gplace  per chunk: offsets = exclusive scan of the totals; stable ranks (warp match
+//             + per-warp counts); order[slot] = pair.  Chunk 0 also writes offsets, counts
+//             and the GEMM work units.
 // Pair p of chunk c lands at offsets[e] + (pairs of e in chunks < c) + (pairs of e before it
 // in chunk c): the pairs of one expert keep their pair-index order.
 // ---------------------------------------------------------------------------------------
 constexpr int kGroupThreads = 256;  // 8 warps; each takes kGroupChunk / 8 consecutive pairs
-constexpr int kScanThreads = 1024;
-static_assert(kGroupChunk % (kGroupThreads / 32 * 32) == 0, "chunk must split into whole warp rounds");
+static_assert(kGroupChunk % kGroupThreads == 0, "chunk must split into whole warp rounds");
+static_assert(kMaxExperts <= 4 * kGroupThreads, "block scan takes 4 experts per thread");
 
 __global__ void __launch_bounds__(kGroupThreads) k_ghist(PrefillArgs a) {
   extern __shared__ int hsm[];  // [E]
@@ -790,127 +904,87 @@ __global__ void __launch_bounds__(kGroupThreads) k_ghist(PrefillArgs a) {
   for (int e = threadIdx.x; e < E; e += kGroupThreads) out[e] = hsm[e];
 }
 
-__global__ void __launch_bounds__(kScanThreads) k_gscan(PrefillArgs a) {
-  __shared__ int cnt[kMaxExperts];
-  __shared__ int off[kMaxExperts + 1];
-  __shared__ int wsum[kScanThreads / 32];
-  const int E = a.E, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int n_chunks = (a.T * a.k + kGroupChunk - 1) / kGroupChunk;
-  // per expert: running sum down the chunks (8 loads in flight per step)
-  for (int e = threadIdx.x; e < E; e += kScanThreads) {
-    int s = 0;
-    for (int c0 = 0; c0 < n_chunks; c0 += 8) {
-      int v[8];
+__global__ void __launch_bounds__(1024) k_gcol(PrefillArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 32 + (threadIdx.x >> 5);
+  if (e >= a.E) return;
+  const int E = a.E, nc = (a.T * a.k + kGroupChunk - 1) / kGroupChunk;
+  int carry = 0;
+  for (int c0 = 0; c0 < nc; c0 += 128) {
+    int v[4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = (c0 + j < n_chunks) ? a.chunk_cnt[(size_t)(c0 + j) * E + e] : 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (c0 + j < n_chunks) {
-          a.chunk_cnt[(size_t)(c0 + j) * E + e] = s;
-          s += v[j];
-        }
+    for (int j = 0; j < 4; ++j) {
+      const int c = c0 + j * 32 + lane;
+      v[j] = c < nc ? a.chunk_cnt[(size_t)c * E + e] : 0;
     }
-    cnt[e] = s;
-  }
-  __syncthreads();
-  // exclusive scan of the totals (E <= 1024: one value per thread)
-  {
-    const int e = threadIdx.x;
-    const int v = e < E ? cnt[e] : 0;
-    int incl = v;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      const int wv = wsum[lane];
-      int wi = wv;
+    for (int j = 0; j < 4; ++j) {
+      int incl = v[j];
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, wi, o);
-        if (lane >= o) wi += y;
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
       }
-      wsum[lane] = wi - wv;
+      const int c = c0 + j * 32 + lane;
+      if (c < nc) a.chunk_cnt[(size_t)c * E + e] = carry + incl - v[j];
+      carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    __syncthreads();
-    if (e < E) off[e] = wsum[warp] + incl - v;
-    if (e == E - 1) off[E] = wsum[warp] + incl;
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e <= E; e += kScanThreads) {
-    a.offsets[e] = off[e];
-    if (e < E) a.counts[e] = cnt[e];
+  if (lane == 0) a.counts[e] = carry;
+}
+
+// Exclusive scan of val(0..E-1) over the block (kGroupThreads threads, 4 values each);
+// out[0..E] (out[E] = total).  Every thread must call it.
+template <class F>
+__device__ void block_scan4(int E, F val, int* out, int* wsum) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int e0 = threadIdx.x * 4;
+  int v[4], s = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    v[j] = (e0 + j < E) ? val(e0 + j) : 0;
+    s += v[j];
   }
-  if (!a.units_gu) return;  // grouping only
-  // work units: per expert, token tiles of <= kNmax pairs x row tiles; then the shared
-  // expert.  Tile bases by an exclusive scan of the experts' tile counts.
+  int incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
   __syncthreads();
-  int* tile_base = off;  // reuse after the offsets are out: [E + 1]
-  __shared__ int offc[kMaxExperts];
-  for (int e = threadIdx.x; e < E; e += kScanThreads) offc[e] = off[e];
-  __syncthreads();
-  {
-    const int e = threadIdx.x;
-    const int v = e < E ? (cnt[e] + kNmax - 1) / kNmax : 0;
-    int incl = v;
+  if (warp == 0) {
+    const int wv = lane < kGroupThreads / 32 ? wsum[lane] : 0;
+    int wi = wv;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
     }
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      const int wv = wsum[lane];
-      int wi = wv;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, wi, o);
-        if (lane >= o) wi += y;
-      }
-      wsum[lane] = wi - wv;
-    }
-    __syncthreads();
-    if (e < E) tile_base[e] = wsum[warp] + incl - v;
-    if (e == E - 1) tile_base[E] = wsum[warp] + incl;
+    if (lane < kGroupThreads / 32) wsum[lane] = wi - wv;
+    if (lane == kGroupThreads / 32 - 1) wsum[kGroupThreads / 32] = wi;
   }
   __syncthreads();
-  const int mt_gu = a.I / 64, mt_dn = a.H / 128;
-  for (int e = threadIdx.x; e < E; e += kScanThreads) {
-    int tb = tile_base[e];
-    for (int s0 = 0; s0 < cnt[e]; s0 += kNmax, ++tb) {
-      const int nn = min(kNmax, cnt[e] - s0);
-      for (int mt = 0; mt < mt_gu; ++mt) a.units_gu[tb * mt_gu + mt] = GemmUnit{e, mt, offc[e] + s0, nn};
-      for (int mt = 0; mt < mt_dn; ++mt) a.units_dn[tb * mt_dn + mt] = GemmUnit{e, mt, offc[e] + s0, nn};
-    }
+  int run = wsum[warp] + incl - s;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    if (e0 + j < E) out[e0 + j] = run;
+    run += v[j];
   }
-  const int tiles_r = tile_base[E];
-  const int st_n = (a.T + kNmax - 1) / kNmax;
-  for (int i = threadIdx.x; i < st_n * mt_gu; i += kScanThreads) {
-    const int st = i / mt_gu, mt = i - st * mt_gu, t0 = st * kNmax;
-    a.units_gu[(tiles_r + st) * mt_gu + mt] = GemmUnit{-1, mt, t0, min(kNmax, a.T - t0)};
-  }
-  for (int i = threadIdx.x; i < st_n * mt_dn; i += kScanThreads) {
-    const int st = i / mt_dn, mt = i - st * mt_dn, t0 = st * kNmax;
-    a.units_dn[(tiles_r + st) * mt_dn + mt] = GemmUnit{-1, mt, t0, min(kNmax, a.T - t0)};
-  }
-  if (threadIdx.x == 0) {
-    a.n_units[0] = (tiles_r + st_n) * mt_gu;
-    a.n_units[1] = (tiles_r + st_n) * mt_dn;
-  }
+  if (threadIdx.x == 0) out[E] = wsum[kGroupThreads / 32];
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kGroupThreads) k_gplace(PrefillArgs a) {
   extern __shared__ int wc[];  // [8][E]: per-warp counts, then per-warp running slots
+  __shared__ int s_off[kMaxExperts + 1];
+  __shared__ int s_wsum[kGroupThreads / 32 + 1];
   constexpr int kW = kGroupThreads / 32, kRounds = kGroupChunk / kGroupThreads;
   const int E = a.E, n = a.T * a.k;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kW * E; i += kGroupThreads) wc[i] = 0;
-  __syncthreads();
-  // warp w takes pairs [p0 + w * 32 * kRounds, ... + 32 * kRounds), round by round
+  block_scan4(E, [&](int e) { return a.counts[e]; }, s_off, s_wsum);
+  // warp w takes pairs [pw, pw + 32 * kRounds), round by round
   const int pw = blockIdx.x * kGroupChunk + warp * 32 * kRounds;
   int ev[kRounds];
 #pragma unroll
@@ -928,7 +1002,7 @@ __global__ void __launch_bounds__(kGroupThreads) k_gplace(PrefillArgs a) {
   __syncthreads();
   const int* base = a.chunk_cnt + (size_t)blockIdx.x * E;
   for (int e = threadIdx.x; e < E; e += kGroupThreads) {
-    int pos = a.offsets[e] + base[e];
+    int pos = s_off[e] + base[e];
 #pragma unroll
     for (int w = 0; w < kW; ++w) {
       const int c = wc[w * E + e];
@@ -946,6 +1020,48 @@ __global__ void __launch_bounds__(kGroupThreads) k_gplace(PrefillArgs a) {
     if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * E + e] += __popc(peers);
     __syncwarp();
   }
+  if (blockIdx.x != 0) return;
+  // chunk 0: offsets, and the GEMM work units: per expert, token tiles of <= kNmax pairs x
+  // row tiles; then the shared expert as one more expert over all tokens
+  for (int e = threadIdx.x; e <= E; e += kGroupThreads) a.offsets[e] = s_off[e];
+  if (!a.units_gu) return;  // grouping only
+  __syncthreads();
+  int* tile_base = wc;  // [E + 1], reused
+  block_scan4(E, [&](int e) { return (a.counts[e] + kNmax - 1) / kNmax; }, tile_base, s_wsum);
+  const int mt_gu = a.I / 64, mt_dn = a.H / 128;
+  for (int e = threadIdx.x; e < E; e += kGroupThreads) {
+    int tb = tile_base[e];
+    const int ce = a.counts[e];
+    for (int s0 = 0; s0 < ce; s0 += kNmax, ++tb) {
+      const int nn = min(kNmax, ce - s0);
+      for (int mt = 0; mt < mt_gu; ++mt) a.units_gu[tb * mt_gu + mt] = GemmUnit{e, mt, s_off[e] + s0, nn};
+      for (int mt = 0; mt < mt_dn; ++mt) a.units_dn[tb * mt_dn + mt] = GemmUnit{e, mt, s_off[e] + s0, nn};
+    }
+  }
+  const int tiles_r = tile_base[E];
+  const int st_n = (a.T + kNmax - 1) / kNmax;
+  for (int i = threadIdx.x; i < st_n * mt_gu; i += kGroupThreads) {
+    const int st = i / mt_gu, mt = i - st * mt_gu, t0 = st * kNmax;
+    a.units_gu[(tiles_r + st) * mt_gu + mt] = GemmUnit{-1, mt, t0, min(kNmax, a.T - t0)};
+  }
+  for (int i = threadIdx.x; i < st_n * mt_dn; i += kGroupThreads) {
+    const int st = i / mt_dn, mt = i - st * mt_dn, t0 = st * kNmax;
+    a.units_dn[(tiles_r + st) * mt_dn + mt] = GemmUnit{-1, mt, t0, min(kNmax, a.T - t0)};
+  }
+  if (threadIdx.x == 0) {
+    a.n_units[0] = (tiles_r + st_n) * mt_gu;
+    a.n_units[1] = (tiles_r + st_n) * mt_dn;
+  }
+}
+
+// xg[p] = x[order[p] / k] for every grouped pair position p < offsets[E]: the routed gate/up
+// GEMM then reads each expert's tokens as consecutive rows.  One warp per row.
+__global__ void __launch_bounds__(256) k_permute(PrefillArgs a) {
+  const int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (p >= a.offsets[a.E]) return;
+  const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)(__ldg(a.order + p) / a.k) * a.H);
+  uint4* dst = reinterpret_cast<uint4*>(a.xg + (size_t)p * a.H);
+  for (int i = lane; i < a.H / 8; i += 32) dst[i] = __ldg(src + i);
 }
 
 __global__ void k_finalize(const float* acc, const uint16_t* residual, uint16_t* out, size_t n) {
@@ -968,14 +1084,68 @@ __global__ void k_router_units(GemmUnit* units, int* n_units, int T, int E) {
 
 template <int BITS, int MODE>
 cudaError_t launch_gemm(const GemmArgs& g, int n_sm, cudaStream_t s) {
-  const int K = (MODE == kModeDown) ? g.I : g.H;
-  size_t smem = (size_t)StageCount<MODE>::kA * kABytes + (size_t)StageCount<MODE>::kB * kBBytes;
-  if (MODE != kModeRouter) smem += kRawBytes + (size_t)128 * ((K / kGroup) * 4 + 16);
+  const GemmSmem P = gemm_smem<BITS, MODE>((MODE == kModeDown) ? g.I : g.H);
+  if (P.total > (uint32_t)kSmemMax) return cudaErrorInvalidConfiguration;
   auto fn = k_gemm<BITS, MODE>;
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.total);
   if (e != cudaSuccess) return e;
-  fn<<<n_sm, kGemmThreads, smem, s>>>(g);
+  fn<<<n_sm, kGemmThreads, P.total, s>>>(g);
   return cudaGetLastError();
+}
+
+// ---- TMA descriptors (host) ----
+// The driver's encoder is looked up through the runtime, so the library does not link the
+// driver library itself (it loads on machines without a GPU driver).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (EncodeTiledFn) nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+cudaError_t encode_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
+                       const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle sw) {
+  const EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  const CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+// bf16 row-major [rows, cols] (row stride ld elements): boxes of 64 columns x box_rows rows,
+// 128-byte swizzle (the operand layout of the MMAs)
+cudaError_t map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {ld * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+// Raw gate/up codes of a pool (or one blob): bytes [slots][gate, up][I][H*b/8]; a box is one
+// stage (64 codes) of 64 rows of both matrices
+cudaError_t map_codes_gu(CUtensorMap* m, const uint8_t* blob0, int64_t n_slots, const BlobLayout& L, int H, int I,
+                         int bits) {
+  const cuuint64_t dims[4] = {(cuuint64_t)H * bits / 8, (cuuint64_t)I, 2, (cuuint64_t)n_slots};
+  const cuuint64_t strides[3] = {(cuuint64_t)H * bits / 8, (cuuint64_t)(L.off[1] - L.off[0]), (cuuint64_t)L.stride};
+  const cuuint32_t box[4] = {(cuuint32_t)(kKC * bits / 8), 64, 2, 1};
+  return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, blob0 + L.off[0], dims, strides, box,
+                    CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+// Raw down codes: bytes [slots][H][I*b/8]; a box is one stage of 128 rows
+cudaError_t map_codes_dn(CUtensorMap* m, const uint8_t* blob0, int64_t n_slots, const BlobLayout& L, int H, int I,
+                         int bits) {
+  const cuuint64_t dims[3] = {(cuuint64_t)I * bits / 8, (cuuint64_t)H, (cuuint64_t)n_slots};
+  const cuuint64_t strides[2] = {(cuuint64_t)I * bits / 8, (cuuint64_t)L.stride};
+  const cuuint32_t box[3] = {(cuuint32_t)(kKC * bits / 8), 128, 1};
+  return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, blob0 + L.off[2], dims, strides, box,
+                    CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 }  // namespace
@@ -987,7 +1157,7 @@ bool prefill_shape_supported(int H, int I, int bits, int E) {
 cudaError_t launch_group(const PrefillArgs& p, cudaStream_t s) {
   const int n_chunks = (p.T * p.k + kGroupChunk - 1) / kGroupChunk;
   k_ghist<<<n_chunks, kGroupThreads, sizeof(int) * p.E, s>>>(p);
-  k_gscan<<<1, kScanThreads, 0, s>>>(p);
+  k_gcol<<<(p.E + 31) / 32, 1024, 0, s>>>(p);
   const size_t smem = sizeof(int) * (size_t)(kGroupThreads / 32) * p.E;
   k_gplace<<<n_chunks, kGroupThreads, smem, s>>>(p);
   return cudaGetLastError();
@@ -1012,6 +1182,8 @@ cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
       GemmArgs g = p.g;
       g.units = p.units_rt;
       g.n_units = p.n_units + 2;
+      if ((e = map_bf16(&g.map_a, p.wr, E, H, H, 128)) != cudaSuccess) return e;
+      if ((e = map_bf16(&g.map_b, p.x, T, H, H, kBRows)) != cudaSuccess) return e;
       if ((e = (bits == 4 ? launch_gemm<4, kModeRouter>(g, n_sm, s) : launch_gemm<8, kModeRouter>(g, n_sm, s))) !=
           cudaSuccess)
         return e;
@@ -1025,12 +1197,18 @@ cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
   // grouping and work units
   prof_mark(1, false, s);
   if ((e = launch_group(p, s)) != cudaSuccess) return e;
+  k_permute<<<(unsigned)(((size_t)T * p.k * 32 + 255) / 256), 256, 0, s>>>(p);
   prof_mark(1, true, s);
   // gate/up + SwiGLU, then down + scatter
   {
     GemmArgs g = p.g;
     g.units = p.units_gu;
     g.n_units = p.n_units;
+    const int I = p.I;
+    if ((e = map_codes_gu(&g.map_a, g.pool, g.n_slots, g.L, H, I, bits)) != cudaSuccess) return e;
+    if ((e = map_codes_gu(&g.map_a_shared, g.shared, 1, g.L, H, I, bits)) != cudaSuccess) return e;
+    if ((e = map_bf16(&g.map_b, p.xg, (uint64_t)T * p.k, H, H, kBRows)) != cudaSuccess) return e;
+    if ((e = map_bf16(&g.map_b2, p.x, T, H, H, kBRows)) != cudaSuccess) return e;
     prof_mark(2, false, s);
     if ((e = (bits == 4 ? launch_gemm<4, kModeGateUp>(g, n_sm, s) : launch_gemm<8, kModeGateUp>(g, n_sm, s))) !=
         cudaSuccess)
@@ -1038,6 +1216,10 @@ cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
     prof_mark(2, true, s);
     g.units = p.units_dn;
     g.n_units = p.n_units + 1;
+    if ((e = map_codes_dn(&g.map_a, g.pool, g.n_slots, g.L, H, I, bits)) != cudaSuccess) return e;
+    if ((e = map_codes_dn(&g.map_a_shared, g.shared, 1, g.L, H, I, bits)) != cudaSuccess) return e;
+    if ((e = map_bf16(&g.map_b, p.h, (uint64_t)T * p.k, I, I, kBRows)) != cudaSuccess) return e;
+    if ((e = map_bf16(&g.map_b2, p.hs, T, I, I, kBRows)) != cudaSuccess) return e;
     prof_mark(3, false, s);
     if ((e = (bits == 4 ? launch_gemm<4, kModeDown>(g, n_sm, s) : launch_gemm<8, kModeDown>(g, n_sm, s))) !=
         cudaSuccess)
