@@ -13,26 +13,27 @@
 //                  over the selected logits; shared-expert gate
 //   k_ghist, k_gcol, k_gplace
 //                  stable counting sort of the (token, k) pairs by expert (per-chunk counts,
-//                  per-expert scans down the chunks, per-chunk stable placement) and the list of GEMM work units
-//                  (expert, row tile, token tile)
+//                  per-expert scans down the chunks, per-chunk stable placement) and the
+//                  list of GEMM work units (expert, row tile, token tile)
+//   k_permute      xg = the tokens' rows of x in grouped pair order
 //   k_gemm GATEUP  per unit: [gate; up] rows of one expert (dequantised to bf16 in shared
-//                  memory) x the expert's tokens (gathered), SwiGLU in the epilogue -> h
+//                  memory) x the expert's rows of xg, SwiGLU in the epilogue -> h
 //   k_gemm DOWN    per unit: down rows x the expert's h, weighted scatter-add into an fp32
 //                  accumulator (the shared expert is one more "expert" over all tokens)
 //   k_finalize     out = bf16(acc + residual)
 //
 // GEMM kernel ("swap-AB": the weight rows are the MMA's M = 128, the tokens its N <= 128):
-//   warp 0       TMEM allocation; lane 0 issues tcgen05.mma (kind::f16, cta_group::1)
-//   warps 1..3   gather the tokens' activation rows with cp.async (zero rows beyond N)
-//   warps 4..11  dequantise the weight rows (w = s*q + b, rounded to bf16) into shared memory;
-//                the raw codes stream through a per-thread cp.async ring several stages ahead
-//                and each unit's row scales and biases are copied to shared memory once
-//   warps 12..15 epilogue: tcgen05.ld of the fp32 accumulator, then SwiGLU / scatter / store
-// Operands are K-major with no swizzle: 8-row x 16-byte core matrices, k-octets 128 bytes
-// apart (LBO) and 8-row groups 1024 bytes apart (SBO) for a 64-wide K stage.  A and B
-// tiles have rings of their own (the B gather runs six stages ahead, its completion tracked
-// by cp.async mbarrier arrivals); two TMEM accumulators of 128 columns let the epilogue of
-// one unit overlap the next.
+//   warp 0        TMEM allocation; lane 0 issues tcgen05.mma (kind::f16, cta_group::1)
+//   warp 1        B tiles by TMA (consecutive rows of x, of the expert-ordered copy xg, h, hs)
+//   warp 2        lane 0: raw codes by TMA (3-D / 4-D boxes over the pool), or router rows
+//   warps 3..18   dequantise the codes (w = s*q + b, rounded to bf16) into the A tile; each
+//                 unit's row scales and biases are copied to shared memory once
+//   warps 19..22  epilogue: tcgen05.ld of the fp32 accumulator, then SwiGLU / scatter / store
+// A tiles written by the dequantising warps are K-major without swizzle (8-row x 16-byte
+// core matrices, k-octets 128 bytes apart, 8-row groups 1024 bytes apart); tiles written by
+// TMA (B, router rows) use the 128-byte swizzle.  Stage s holds one A and one B tile, with
+// one full barrier (TMA bytes plus the producers' arrivals) and one empty barrier (the MMA's
+// commit); two TMEM accumulators of 128 columns let the epilogue of one unit overlap the next.
 // Every wait is bounded; on timeout the kernel flags MOE_DEVERR_TIMEOUT, drains and frees
 // its TMEM.
 #include "common.cuh"
@@ -53,9 +54,9 @@ constexpr int kBBytes = kNmax * kKC * 2;  // 16 KB
 // warp roles
 constexpr int kBLoadWarp = 1;             // lane 0: B tiles by TMA
 constexpr int kALoadWarp = 2;             // lane 0: raw codes (or router rows) by TMA
-constexpr int kAWarp0 = 3, kAWarps = 8;   // dequantisation
-constexpr int kEWarp0 = 11, kEWarps = 4;  // epilogue
-constexpr int kGemmThreads = (kEWarp0 + kEWarps) * 32;  // 480
+constexpr int kAWarp0 = 3, kAWarps = 16;  // dequantisation
+constexpr int kEWarp0 = 19, kEWarps = 4;  // epilogue
+constexpr int kGemmThreads = (kEWarp0 + kEWarps) * 32;  // 736
 constexpr int kSBO = (kKC / 8) * 128;     // 1024: 8-row group stride of a no-swizzle K-major tile
 constexpr int kTmemCols = 2 * kNmax;      // two accumulators
 constexpr int kBRows = 32;                // rows per B tile load (tile mode)
@@ -84,9 +85,11 @@ struct Ring {
   }
 };
 
-// Shared-memory plan of one GEMM launch (host and device agree on it).
+// Shared-memory plan of one GEMM launch (host and device agree on it).  Stage s holds an A
+// tile (16 KB) and a B tile (16 KB); one full and one empty barrier per stage.
 struct GemmSmem {
-  int n_sa, n_sb;      // A and B stages
+  int n_st;            // stages
+  uint32_t b;          // byte offset of the B tiles
   uint32_t raw, sb;    // byte offsets of the raw ring and the scale buffers
   uint32_t sb_ld;      // uint16 per row of a scale buffer
   uint32_t total;      // dynamic bytes, including 1 KB of alignment slack
@@ -97,16 +100,12 @@ __host__ __device__ inline GemmSmem gemm_smem(int K) {
   const int NG = K / kGroup;
   p.sb_ld = (uint32_t)(2 * NG + 8);  // scales, biases, 16 bytes of padding
   const uint32_t fixed = MODE == kModeRouter ? 0u : (uint32_t)(Raw<BITS>::kDepth * Raw<BITS>::kBytes + 2 * 128 * p.sb_ld * 2);
-  // A stages first (the dequantisation loop needs about four), then B stages, then the rest to A
-  int na = MODE == kModeRouter ? 2 : 4, nb = 2;
-  auto fits = [&](int a_, int b_) { return (uint32_t)(a_ + b_) * 16384u + fixed + 1024u <= (uint32_t)kSmemMax; };
-  while (nb < kStageMax && fits(na, nb + 1)) ++nb;
-  while (na < kStageMax && fits(na + 1, nb)) ++na;
-  p.n_sa = na;
-  p.n_sb = nb;
-  p.raw = (uint32_t)(na + nb) * 16384u;
+  int n = (int)(((uint32_t)kSmemMax - fixed - 1024u) / (uint32_t)(kABytes + kBBytes));
+  p.n_st = n > kStageMax ? kStageMax : n;
+  p.b = (uint32_t)p.n_st * kABytes;
+  p.raw = (uint32_t)p.n_st * (kABytes + kBBytes);
   p.sb = p.raw + (MODE == kModeRouter ? 0u : (uint32_t)(Raw<BITS>::kDepth * Raw<BITS>::kBytes));
-  p.total = (uint32_t)(na + nb) * 16384u + fixed + 1024u;
+  p.total = p.raw + fixed + 1024u;
   return p;
 }
 
@@ -176,14 +175,31 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
-  uint32_t r[8];
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr));
+// 16 / 32 consecutive accumulator columns of this warp's 32 TMEM lanes (one row per thread)
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
@@ -225,13 +241,14 @@ __device__ __forceinline__ uint4 dq8_int8(uint32_t w0, uint32_t w1, float s, flo
                     dq2(w1 & 0xFFu, w1 & 0xFF00u, s, s8, b), dq2(h1 & 0xFFu, h1 & 0xFF00u, s, s8, b));
 }
 
-// A-producer thread -> (tile row m, column half).  Lanes l and l ^ 8 share a row; the
-// eight lanes of each quarter-warp take eight consecutive rows of one half, so that their
-// 16-byte stores of a k-octet fill 128 contiguous bytes of the tile (no bank conflicts).
-__device__ __forceinline__ void a_lane_map(int at, int& m, int& half) {
+// Dequantising thread -> (tile row m, column quarter q).  The four threads of a row are
+// lanes l, l + 8, l + 16, l + 24 of one warp; the eight lanes of each quarter-warp take eight
+// consecutive rows of one quarter, so that their 16-byte stores of a k-octet fill 128
+// contiguous bytes of the tile (no bank conflicts).
+__device__ __forceinline__ void a_lane_map(int at, int& m, int& q) {
   const int w = at >> 5, l = at & 31;
-  m = w * 16 + (l & 7) + ((l >> 4) << 3);
-  half = (l >> 3) & 1;
+  m = w * 8 + (l & 7);
+  q = l >> 3;
 }
 
 // 8 int4 codes (one word, element j at bits 4j) -> 8 bf16 values round(s*q + b), on packed
@@ -285,8 +302,10 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Ctrl* 
   return ok;
 }
 
-// Wait (bounded) for the last loads a loader issued into a ring of n full barriers, so that
-// no copy is still landing when the CTA leaves (the consumers normally waited for them).
+// Wait (bounded) for the last stages a loader issued into a ring of n full barriers, so that
+// no copy is still landing when the CTA leaves.  Normally the consumers have already waited
+// for them and this returns at once; after an abort a phase may lack other arrivals, and
+// the bound (far beyond any copy's latency) ends the wait.
 __device__ __forceinline__ void drain_ring(uint64_t* full, int n, int issued, Ctrl* c) {
   for (int q = issued > n ? issued - n : 0; q < issued; ++q)
     if (!mbar_wait(&full[q % n], (uint32_t)((q / n) & 1))) {
@@ -302,7 +321,7 @@ template <int BITS, int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant__ GemmArgs a) {
   constexpr int kRawB = Raw<BITS>::kBytes, kDepth = Raw<BITS>::kDepth;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t a_full[kStageMax], a_empty[kStageMax], b_full[kStageMax], b_empty[kStageMax],
+  __shared__ __align__(8) uint64_t full[kStageMax], empty[kStageMax],
       raw_full[8], raw_empty[8], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
@@ -317,18 +336,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
   // stage tiles start on 1024-byte boundaries (128-byte swizzle atoms)
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (smem_base - smem_u32(smem_raw));
-  const uint32_t b_area = smem_base + P.n_sa * kABytes;
+  const uint32_t b_area = smem_base + P.b;
   const int my_units = n_units > (int)blockIdx.x ? (n_units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (tid == 0) {
-    for (int s = 0; s < P.n_sa; ++s) {
-      // router rows arrive by TMA (one expect-tx arrival); dequantised tiles once per A warp
-      mbar_init(&a_full[s], MODE == kModeRouter ? 1 : kAWarps);
-      mbar_init(&a_empty[s], 1);
-    }
-    for (int s = 0; s < P.n_sb; ++s) {
-      mbar_init(&b_full[s], 1);
-      mbar_init(&b_empty[s], 1);
+    for (int s = 0; s < P.n_st; ++s) {
+      // full: the B loader's expect-tx arrival, plus the A loader's (router rows by TMA) or
+      // one arrival per dequantising warp; empty: the MMA's commit
+      mbar_init(&full[s], MODE == kModeRouter ? 2 : kAWarps + 1);
+      mbar_init(&empty[s], 1);
     }
     for (int s = 0; s < kDepth; ++s) {
       mbar_init(&raw_full[s], 1);
@@ -355,7 +371,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
   if (warp == 0) {
     // ------------------------------ MMA issuer ------------------------------
     if (lane == 0) {
-      Ring ra(P.n_sa), rb(P.n_sb);
+      Ring r(P.n_st);
       int it = 0;
       for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x, ++it) {
         const GemmUnit U = a.units[u];
@@ -368,23 +384,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)buf * (uint32_t)kNmax;
-        for (int kc = 0; kc < nK; ++kc, ra.next(), rb.next()) {
-          if (!wait_or_flag(&b_full[rb.s], rb.ph, a.ctrl) || !wait_or_flag(&a_full[ra.s], ra.ph, a.ctrl)) {
+        for (int kc = 0; kc < nK; ++kc, r.next()) {
+          if (!wait_or_flag(&full[r.s], r.ph, a.ctrl)) {
             s_abort = 1;
             break;
           }
           // dequantised tiles were written through the generic proxy (st.shared)
           if (MODE != kModeRouter) proxy_fence();
           tc_fence_after();
-          const uint32_t a_base = smem_base + ra.s * kABytes;
-          const uint32_t b_base = b_area + rb.s * kBBytes;
+          const uint32_t a_base = smem_base + r.s * kABytes;
+          const uint32_t b_base = b_area + r.s * kBBytes;
 #pragma unroll
           for (int kk = 0; kk < kKC / 16; ++kk) {
             const uint64_t da = MODE == kModeRouter ? umma_desc_sw128(a_base + kk * 32) : umma_desc(a_base + kk * 256);
             umma_f16(d_tmem, da, umma_desc_sw128(b_base + kk * 32), idesc, (kc > 0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(&a_empty[ra.s]);
-          umma_commit(&b_empty[rb.s]);
+          umma_commit(&empty[r.s]);
         }
         if (s_abort) break;
         umma_commit(&acc_full[buf]);
@@ -400,7 +415,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     // shared expert, the expert-ordered copy xg of x for routed gate/up units, h / hs for
     // down.  Loads of kBRows rows, one per lane; rows from U.n up to the loaded count belong
     // to other units or lie beyond the matrix (zero filled): their products are never read.
-    Ring rb(P.n_sb);
+    Ring rb(P.n_st);
     int issued = 0;
     for (int u = blockIdx.x; u < n_units && !warp_aborted(&s_abort); u += gridDim.x) {
       const GemmUnit U = a.units[u];
@@ -410,14 +425,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       const int nrt = (npad + kBRows - 1) / kBRows;
       const uint32_t bytes = (uint32_t)nrt * kBRows * 128u;
       for (int kc = 0; kc < nK; ++kc, rb.next()) {
-        if (!warp_wait(&b_empty[rb.s], rb.ph ^ 1, a.ctrl, lane)) {
+        if (!warp_wait(&empty[rb.s], rb.ph ^ 1, a.ctrl, lane)) {
           stop = true;
           break;
         }
-        if (lane == 0) mbar_expect_tx(&b_full[rb.s], bytes);
+        if (lane == 0) mbar_expect_tx(&full[rb.s], bytes);
         __syncwarp();  // the transaction count is registered before any load can land
         if (lane < nrt)
-          tma_2d(b_area + rb.s * kBBytes + lane * kBRows * 128, mb, kc * kKC, U.p0 + lane * kBRows, &b_full[rb.s]);
+          tma_2d(b_area + rb.s * kBBytes + lane * kBRows * 128, mb, kc * kKC, U.p0 + lane * kBRows, &full[rb.s]);
         ++issued;
       }
       if (stop) {
@@ -426,7 +441,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       }
     }
     // drain: the last loads this thread issued have landed before the CTA may leave
-    if (lane == 0) drain_ring(b_full, P.n_sb, issued, a.ctrl);
+    if (lane == 0) drain_ring(full, P.n_st, issued, a.ctrl);
   } else if (warp == kALoadWarp) {
     // ------------------------------ A operand loads (TMA) ------------------------------
     // Router: 128 router rows x 64 columns per stage straight into the A tile.  Otherwise the
@@ -434,7 +449,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     // a unit whose expert has no valid slot reads an out-of-range slot, which TMA fills with
     // zeros (its scales are zero too, so it dequantises to 0).
     if (lane == 0) {
-      Ring rr(MODE == kModeRouter ? P.n_sa : kDepth);
+      Ring rr(MODE == kModeRouter ? P.n_st : kDepth);
       int issued = 0;
       bool stop = false;
       // unit descriptors two units ahead and slots one unit ahead, so that the lookups'
@@ -468,12 +483,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         }
         for (int kc = 0; kc < nK; ++kc, rr.next()) {
           if (MODE == kModeRouter) {
-            if (!wait_or_flag(&a_empty[rr.s], rr.ph ^ 1, a.ctrl)) {
+            if (!wait_or_flag(&empty[rr.s], rr.ph ^ 1, a.ctrl)) {
               stop = true;
               break;
             }
-            mbar_expect_tx(&a_full[rr.s], kABytes);
-            tma_2d(smem_base + rr.s * kABytes, ma, kc * kKC, U.mt * 128, &a_full[rr.s]);
+            mbar_expect_tx(&full[rr.s], kABytes);
+            tma_2d(smem_base + rr.s * kABytes, ma, kc * kKC, U.mt * 128, &full[rr.s]);
           } else {
             if (!wait_or_flag(&raw_empty[rr.s], rr.ph ^ 1, a.ctrl)) {
               stop = true;
@@ -490,45 +505,59 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         }
       }
       if (stop) s_abort = 1;
-      drain_ring(MODE == kModeRouter ? a_full : raw_full, MODE == kModeRouter ? P.n_sa : kDepth, issued, a.ctrl);
+      drain_ring(MODE == kModeRouter ? full : raw_full, MODE == kModeRouter ? P.n_st : kDepth, issued, a.ctrl);
     }
     __syncwarp();
   } else if (warp >= kAWarp0 && warp < kAWarp0 + kAWarps && MODE != kModeRouter) {
     // ------------------------------ dequantisation ------------------------------
-    // Thread (m, half) turns 32 codes of tile row m per stage into bf16 in the A tile.  Each
-    // unit's row scales and biases are copied (cp.async) into one of two buffers one unit
-    // ahead (of the two threads of a row, half 0 copies the scales, half 1 the biases).
-    const int at = tid - kAWarp0 * 32;  // 0..255
-    int m, half;                        // tile row 0..127, which 32 columns of the stage
-    a_lane_map(at, m, half);
+    // Thread (m, q) turns 16 codes (columns 16q..16q+15 of the stage) of tile row m into bf16
+    // in the A tile.  Each unit's row scales and biases are copied (cp.async) into one of two
+    // buffers one unit ahead, the four threads of a row sharing the copies.
+    const int at = tid - kAWarp0 * 32;  // 0..511
+    int m, q;                           // tile row 0..127, column quarter 0..3
+    a_lane_map(at, m, q);
     const int NG = K / kGroup;  // groups (= stages) per row
     const int sb_ld = (int)P.sb_ld;
     uint16_t* sb_area = reinterpret_cast<uint16_t*>(smem + P.sb);  // [2][128][sb_ld]
-    // offset of this thread's 16-byte pieces in a raw stage (TMA box layout)
+    // offset of this thread's codes in a raw stage (TMA box layout)
+    constexpr int kQB = Raw<BITS>::kRowBytes / 4;  // 8 or 16 bytes
     const uint32_t raw_off = MODE == kModeGateUp
-                                 ? (uint32_t)((m & 1) * 64 + (m >> 1)) * Raw<BITS>::kRowBytes + half * (kRawB / 256)
-                                 : (uint32_t)m * Raw<BITS>::kRowBytes + half * (kRawB / 256);
+                                 ? (uint32_t)((m & 1) * 64 + (m >> 1)) * Raw<BITS>::kRowBytes + q * kQB
+                                 : (uint32_t)m * Raw<BITS>::kRowBytes + q * kQB;
     auto unit_at = [&](int j) { return a.units[blockIdx.x + (size_t)j * gridDim.x]; };
     auto slot_of = [&](const GemmUnit& U) { return U.e < 0 ? 0 : a.slot_table[U.e]; };
-    // scales / biases of unit ordinal j (descriptor U, slot) into buffer j & 1
+    // scales / biases of unit ordinal j (descriptor U, slot) into buffer j & 1; a row's
+    // buffer holds its NG scales, then its NG biases
     auto load_scales = [&](int j, const GemmUnit& U, int slot) {
       const uint8_t* blob = a.shared;
       if (U.e >= 0) blob = (slot < 0 || slot >= a.n_slots) ? nullptr : a.pool + (int64_t)slot * a.L.stride;
-      const uint8_t* src = nullptr;
+      const uint8_t *src_s = nullptr, *src_b = nullptr;
       if (blob) {
         if (MODE == kModeGateUp) {
-          const int r = U.mt * 64 + (m >> 1);
-          src = blob + a.L.off[((m & 1) ? 5 : 3) + half] + (int64_t)r * NG * 2;
+          const int64_t r = (int64_t)(U.mt * 64 + (m >> 1)) * NG * 2;
+          src_s = blob + a.L.off[(m & 1) ? 5 : 3] + r;
+          src_b = blob + a.L.off[(m & 1) ? 6 : 4] + r;
         } else {
-          src = blob + a.L.off[7 + half] + (int64_t)(U.mt * 128 + m) * NG * 2;
+          const int64_t r = (int64_t)(U.mt * 128 + m) * NG * 2;
+          src_s = blob + a.L.off[7] + r;
+          src_b = blob + a.L.off[8] + r;
         }
       }
-      uint16_t* dst = sb_area + (size_t)(j & 1) * 128 * sb_ld + (size_t)m * sb_ld + (half ? NG : 0);
+      uint16_t* dst = sb_area + (size_t)(j & 1) * 128 * sb_ld + (size_t)m * sb_ld;
       if ((NG & 7) == 0) {  // rows of 16-byte multiples: 16-byte aligned in the blob and here
-        for (int o = 0; o < NG * 2; o += 16) cp_async16(smem_u32(dst) + o, src ? src + o : a.pool, src ? 16u : 0u);
+        const int pieces = NG / 8;  // per array
+        for (int i = q; i < 2 * pieces; i += 4) {
+          const bool bias = i >= pieces;
+          const int o = (bias ? i - pieces : i) * 16;
+          const uint8_t* src = bias ? src_b : src_s;
+          cp_async16(smem_u32(dst) + (bias ? NG * 2 : 0) + o, src ? src + o : a.pool, src ? 16u : 0u);
+        }
       } else {  // narrow rows (small K): plain loads
-        const uint16_t* g = reinterpret_cast<const uint16_t*>(src);
-        for (int o = 0; o < NG; ++o) dst[o] = g ? __ldg(g + o) : (uint16_t)0;
+        for (int i = q; i < 2 * NG; i += 4) {
+          const bool bias = i >= NG;
+          const uint16_t* g = reinterpret_cast<const uint16_t*>(bias ? src_b : src_s);
+          dst[i] = g ? __ldg(g + (bias ? i - NG : i)) : (uint16_t)0;
+        }
       }
       cp_async_commit();
     };
@@ -543,10 +572,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       }
       if (my_units > 2) un2 = unit_at(2);
     }
-    Ring ra(P.n_sa), rr(kDepth);
+    Ring ra(P.n_st), rr(kDepth);
     for (int j = 0; j < my_units && !warp_aborted(&s_abort); ++j) {
-      cp_async_wait<0>();  // this unit's scales (own half) have landed
-      __syncwarp();        // ... and the partner's half; buffer (j + 1) & 1 is no longer read
+      cp_async_wait<0>();  // this unit's scales (this thread's copies) have landed
+      __syncwarp();        // ... and the row's other threads'; buffer (j + 1) & 1 is no longer read
       if (j + 1 < my_units) {
         load_scales(j + 1, un1, slot1);
         un1 = un2;
@@ -561,35 +590,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
           break;
         }
         const uint8_t* rp = smem + P.raw + rr.s * kRawB + raw_off;
-        uint4 rw[Raw<BITS>::kRowBytes / 32];
-#pragma unroll
-        for (int o = 0; o < Raw<BITS>::kRowBytes / 32; ++o) rw[o] = *reinterpret_cast<const uint4*>(rp + o * 16);
+        uint32_t w[kQB / 4];
+        if (BITS == 4) {
+          const uint2 v = *reinterpret_cast<const uint2*>(rp);
+          w[0] = v.x;
+          w[1] = v.y;
+        } else {
+          const uint4 v = *reinterpret_cast<const uint4*>(rp);
+          w[0] = v.x;
+          w[1] = v.y;
+          w[kQB / 4 > 2 ? 2 : 0] = v.z;
+          w[kQB / 4 > 3 ? 3 : 0] = v.w;
+        }
         const uint32_t sbits = my_s[kc], bbits = my_s[NG + kc];
         __syncwarp();  // every lane holds its codes: the raw slot can be refilled
         if (lane == 0) mbar_arrive(&raw_empty[rr.s]);
-        if (!warp_wait(&a_empty[ra.s], ra.ph ^ 1, a.ctrl, lane)) {
+        if (!warp_wait(&empty[ra.s], ra.ph ^ 1, a.ctrl, lane)) {
           stop = true;
           break;
         }
         uint8_t* a_tile = smem + ra.s * kABytes;
         if (BITS == 4) {
           const uint32_t s2 = sbits | (sbits << 16), b2 = bbits | (bbits << 16);
-          const uint32_t w4[4] = {rw[0].x, rw[0].y, rw[0].z, rw[0].w};
 #pragma unroll
-          for (int o = 0; o < 4; ++o)  // 4 k-octets of 8 values = this thread's 32 columns
-            *reinterpret_cast<uint4*>(a_tile + core_off(m, half * 4 + o)) = dq8_int4_bf(w4[o], s2, b2);
+          for (int o = 0; o < 2; ++o)  // 2 k-octets of 8 values = this thread's 16 columns
+            *reinterpret_cast<uint4*>(a_tile + core_off(m, q * 2 + o)) = dq8_int4_bf(w[o], s2, b2);
         } else {
           const float sv = __uint_as_float(sbits << 16), bv = __uint_as_float(bbits << 16);
 #pragma unroll
-          for (int o = 0; o < 4; ++o) {
-            const uint4 w = rw[o >> 1];
-            const uint4 v = (o & 1) ? dq8_int8(w.z, w.w, sv, bv) : dq8_int8(w.x, w.y, sv, bv);
-            *reinterpret_cast<uint4*>(a_tile + core_off(m, half * 4 + o)) = v;
-          }
+          for (int o = 0; o < 2; ++o)
+            *reinterpret_cast<uint4*>(a_tile + core_off(m, q * 2 + o)) =
+                dq8_int8(w[(2 * o) % (kQB / 4)], w[(2 * o + 1) % (kQB / 4)], sv, bv);
         }
         proxy_fence();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[ra.s]);
+        if (lane == 0) mbar_arrive(&full[ra.s]);
       }
       if (stop) {
         s_abort = 1;
@@ -629,9 +664,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       }
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)buf * (uint32_t)kNmax;
-      for (int c0 = 0; c0 < U.n; c0 += 8) {
-        float v[8];
-        tmem_ld8(taddr + c0, v);
+      constexpr int kEC = MODE == kModeRouter ? 16 : 32;  // columns per TMEM load
+      for (int c0 = 0; c0 < U.n; c0 += kEC) {
+        float v[kEC];
+        if (kEC == 32) tmem_ld32(taddr + c0, v);
+        else tmem_ld16(taddr + c0, v);
         if (MODE == kModeGateUp) {
           // lanes 2i (gate row) and 2i + 1 (up row) hold intermediate row r; the even lane
           // finishes column c, the odd lane column c + 1 (one exchange per column pair)
@@ -639,7 +676,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
           const int r = U.mt * 64 + (m >> 1);
           uint16_t* hbase = (U.e < 0) ? a.hs : a.h;
 #pragma unroll
-          for (int i = 0; i < 8; i += 2) {
+          for (int i = 0; i < kEC; i += 2) {
             const float recv = __shfl_xor_sync(0xffffffffu, odd ? v[i] : v[i + 1], 1);
             const float g = odd ? recv : v[i];
             const float up = odd ? v[i + 1] : recv;
@@ -649,7 +686,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
           }
         } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < kEC; ++i) {
           const int n = c0 + i;
           const float val = v[i];
           if (MODE == kModeDown) {
