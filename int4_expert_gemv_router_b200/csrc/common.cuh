@@ -219,13 +219,23 @@ struct GemmArgs {
   const GemmUnit* units;
   const int* n_units;
   Ctrl* ctrl;
-  // TMA descriptors (filled by the launcher per GEMM): A operand (router rows, or the raw
-  // codes of the pool and of the shared blob), B operand (x rows by gather or tile, h, hs)
-  alignas(64) CUtensorMap map_a;
-  alignas(64) CUtensorMap map_a_shared;
-  alignas(64) CUtensorMap map_b;
-  alignas(64) CUtensorMap map_b2;
+  int n_rows;           // weight rows per work unit (the MMA's N): 128 or 256
+  int sc_tma;           // 1: scales and biases arrive by TMA in chunks of 8 groups
+  // TMA descriptors (filled by the launcher per GEMM): token rows (routed / shared
+  // units), weight rows (router rows, or raw codes of the pool / of the shared blob), and
+  // the scale + bias chunks (pool / shared blob)
+  alignas(64) CUtensorMap map_tok;
+  alignas(64) CUtensorMap map_tok2;
+  alignas(64) CUtensorMap map_w;
+  alignas(64) CUtensorMap map_w_shared;
+  alignas(64) CUtensorMap map_sc;
+  alignas(64) CUtensorMap map_sc_shared;
 };
+
+// Weight rows per GEMM work unit of the prefill path: gate/up units hold nI intermediate
+// rows of both matrices (2*nI rows), down units NR output rows.
+__host__ __device__ inline int prefill_gu_rows(int I) { return I % 128 == 0 ? 256 : 128; }
+__host__ __device__ inline int prefill_dn_rows(int H) { return H % 256 == 0 ? 256 : 128; }
 
 struct PrefillArgs {
   int T, E, k, H, I;

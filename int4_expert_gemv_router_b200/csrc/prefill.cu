@@ -48,28 +48,29 @@ namespace moe {
 namespace {
 
 constexpr int kKC = 64;                   // K per stage
-constexpr int kNmax = kPrefillN;          // tokens per unit (MMA N)
-constexpr int kABytes = 128 * kKC * 2;    // 16 KB
-constexpr int kBBytes = kNmax * kKC * 2;  // 16 KB
+constexpr int kTok = kPrefillN;           // tokens per unit: the MMA's M (128 TMEM lanes)
+constexpr int kNMax = 256;                // weight rows per unit: the MMA's N
+constexpr int kTBytes = kTok * kKC * 2;   // 16 KB: token tile of a stage
+constexpr int kWBytes = kNMax * kKC * 2;  // 32 KB: weight tile of a stage (room for N = 256)
 // warp roles
-constexpr int kBLoadWarp = 1;             // lane 0: B tiles by TMA
-constexpr int kALoadWarp = 2;             // lane 0: raw codes (or router rows) by TMA
-constexpr int kAWarp0 = 3, kAWarps = 16;  // dequantisation
+constexpr int kTLoadWarp = 1;             // token tiles by TMA
+constexpr int kWLoadWarp = 2;             // lane 0: raw codes + scale chunks (or router rows) by TMA
+constexpr int kDWarp0 = 3, kDWarps = 16;  // dequantisation: 256 weight rows x 2 column halves
 constexpr int kEWarp0 = 19, kEWarps = 4;  // epilogue
 constexpr int kGemmThreads = (kEWarp0 + kEWarps) * 32;  // 736
 constexpr int kSBO = (kKC / 8) * 128;     // 1024: 8-row group stride of a no-swizzle K-major tile
-constexpr int kTmemCols = 2 * kNmax;      // two accumulators
-constexpr int kBRows = 32;                // rows per B tile load (tile mode)
-constexpr int kStageMax = 6;              // A and B stages: at most 6 each
-
+constexpr int kTmemCols = 2 * kNMax;      // two accumulators of up to 256 columns
+constexpr int kTRows = 32;                // rows per token-tile load
+constexpr int kStageMax = 6;
+constexpr int kChunk = 8;                 // groups per scale chunk
+constexpr int kChunkBytes = kNMax * 2 * kChunk * 2;  // 8 KB: scales + biases of 8 groups, 256 rows
 constexpr int kSmemMax = 227 * 1024 - 8 * 1024;  // dynamic shared memory budget (static part aside)
-// raw codes of one stage (128 rows x 64 codes)
-// (32 KB of them in flight ahead of the dequantisation)
+// raw codes of one stage (256 weight rows x 64 codes), and how many stages are in flight
 template <int BITS>
 struct Raw {
   static constexpr int kRowBytes = kKC * BITS / 8;  // 32 or 64
-  static constexpr int kBytes = 128 * kRowBytes;    // 4 or 8 KB
-  static constexpr int kDepth = 32768 / kBytes;     // 8 or 4 stages
+  static constexpr int kBytes = kNMax * kRowBytes;  // 8 or 16 KB
+  static constexpr int kDepth = BITS == 4 ? 4 : 3;
 };
 
 // Position in a ring of n stages and the parity of its current pass.
@@ -85,26 +86,24 @@ struct Ring {
   }
 };
 
-// Shared-memory plan of one GEMM launch (host and device agree on it).  Stage s holds an A
-// tile (16 KB) and a B tile (16 KB); one full and one empty barrier per stage.
+// Shared-memory plan of one GEMM launch (host and device agree on it).  Stage s holds a
+// token tile (16 KB) and a weight tile (up to 32 KB), with one full and one empty barrier.
 struct GemmSmem {
   int n_st;            // stages
-  uint32_t b;          // byte offset of the B tiles
-  uint32_t raw, sb;    // byte offsets of the raw ring and the scale buffers
-  uint32_t sb_ld;      // uint16 per row of a scale buffer
+  uint32_t w;          // byte offset of the weight tiles
+  uint32_t raw, sc;    // byte offsets of the raw ring and the two scale-chunk slots
   uint32_t total;      // dynamic bytes, including 1 KB of alignment slack
 };
 template <int BITS, int MODE>
-__host__ __device__ inline GemmSmem gemm_smem(int K) {
+__host__ __device__ inline GemmSmem gemm_smem() {
   GemmSmem p{};
-  const int NG = K / kGroup;
-  p.sb_ld = (uint32_t)(2 * NG + 8);  // scales, biases, 16 bytes of padding
-  const uint32_t fixed = MODE == kModeRouter ? 0u : (uint32_t)(Raw<BITS>::kDepth * Raw<BITS>::kBytes + 2 * 128 * p.sb_ld * 2);
-  int n = (int)(((uint32_t)kSmemMax - fixed - 1024u) / (uint32_t)(kABytes + kBBytes));
+  const uint32_t wb = MODE == kModeRouter ? (uint32_t)(kTok * kKC * 2) : (uint32_t)kWBytes;
+  const uint32_t fixed = MODE == kModeRouter ? 0u : (uint32_t)(Raw<BITS>::kDepth * Raw<BITS>::kBytes + 2 * kChunkBytes);
+  int n = (int)(((uint32_t)kSmemMax - fixed - 1024u) / ((uint32_t)kTBytes + wb));
   p.n_st = n > kStageMax ? kStageMax : n;
-  p.b = (uint32_t)p.n_st * kABytes;
-  p.raw = (uint32_t)p.n_st * (kABytes + kBBytes);
-  p.sb = p.raw + (MODE == kModeRouter ? 0u : (uint32_t)(Raw<BITS>::kDepth * Raw<BITS>::kBytes));
+  p.w = (uint32_t)p.n_st * kTBytes;
+  p.raw = p.w + (uint32_t)p.n_st * wb;
+  p.sc = p.raw + (MODE == kModeRouter ? 0u : (uint32_t)(Raw<BITS>::kDepth * Raw<BITS>::kBytes));
   p.total = p.raw + fixed + 1024u;
   return p;
 }
@@ -202,15 +201,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&p);
@@ -241,14 +231,13 @@ __device__ __forceinline__ uint4 dq8_int8(uint32_t w0, uint32_t w1, float s, flo
                     dq2(w1 & 0xFFu, w1 & 0xFF00u, s, s8, b), dq2(h1 & 0xFFu, h1 & 0xFF00u, s, s8, b));
 }
 
-// Dequantising thread -> (tile row m, column quarter q).  The four threads of a row are
-// lanes l, l + 8, l + 16, l + 24 of one warp; the eight lanes of each quarter-warp take eight
-// consecutive rows of one quarter, so that their 16-byte stores of a k-octet fill 128
-// contiguous bytes of the tile (no bank conflicts).
-__device__ __forceinline__ void a_lane_map(int at, int& m, int& q) {
+// Dequantising thread -> (weight row m, column half).  Lanes l and l ^ 8 share a row; the
+// eight lanes of each quarter-warp take eight consecutive rows of one half, so that their
+// 16-byte stores of a k-octet fill 128 contiguous bytes of the tile (no bank conflicts).
+__device__ __forceinline__ void w_lane_map(int at, int& m, int& half) {
   const int w = at >> 5, l = at & 31;
-  m = w * 8 + (l & 7);
-  q = l >> 3;
+  m = w * 16 + (l & 7) + ((l >> 4) << 3);
+  half = (l >> 3) & 1;
 }
 
 // 8 int4 codes (one word, element j at bits 4j) -> 8 bf16 values round(s*q + b), on packed
@@ -319,36 +308,36 @@ __device__ __forceinline__ void drain_ring(uint64_t* full, int n, int issued, Ct
 // ---------------------------------------------------------------------------------------
 template <int BITS, int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant__ GemmArgs a) {
-  constexpr int kRawB = Raw<BITS>::kBytes, kDepth = Raw<BITS>::kDepth;
+  constexpr int kRawB = Raw<BITS>::kBytes, kDepth = Raw<BITS>::kDepth, kRowB = Raw<BITS>::kRowBytes;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full[kStageMax], empty[kStageMax],
-      raw_full[8], raw_empty[8], acc_full[2], acc_empty[2], drain;
+  __shared__ __align__(8) uint64_t full[kStageMax], empty[kStageMax], raw_full[4], raw_empty[4], acc_full[2],
+      acc_empty[2], drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  __shared__ int s_colt[kEWarps][kNmax];       // per epilogue warp (down): token of each column
-  __shared__ float s_colw[kEWarps][kNmax];     // and its routing weight
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int K = (MODE == kModeDown) ? a.I : a.H;
   const int nK = K / kKC;
+  const int NR = a.n_rows;  // weight rows per unit (the MMA's N): 128 or 256
   const int n_units = *a.n_units;
-  const GemmSmem P = gemm_smem<BITS, MODE>(K);
+  const GemmSmem P = gemm_smem<BITS, MODE>();
+  const uint32_t wbytes = MODE == kModeRouter ? (uint32_t)(kTok * kKC * 2) : (uint32_t)kWBytes;  // per stage
   // stage tiles start on 1024-byte boundaries (128-byte swizzle atoms)
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (smem_base - smem_u32(smem_raw));
-  const uint32_t b_area = smem_base + P.b;
+  const uint32_t w_area = smem_base + P.w;
   const int my_units = n_units > (int)blockIdx.x ? (n_units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (tid == 0) {
     for (int s = 0; s < P.n_st; ++s) {
-      // full: the B loader's expect-tx arrival, plus the A loader's (router rows by TMA) or
-      // one arrival per dequantising warp; empty: the MMA's commit
-      mbar_init(&full[s], MODE == kModeRouter ? 2 : kAWarps + 1);
+      // full: the token loader's expect-tx arrival, plus the weight loader's (router rows by
+      // TMA) or one arrival per dequantising warp; empty: the MMA's commit
+      mbar_init(&full[s], MODE == kModeRouter ? 2 : kDWarps + 1);
       mbar_init(&empty[s], 1);
     }
     for (int s = 0; s < kDepth; ++s) {
       mbar_init(&raw_full[s], 1);
-      mbar_init(&raw_empty[s], kAWarps);
+      mbar_init(&raw_empty[s], kDWarps);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -371,19 +360,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
   if (warp == 0) {
     // ------------------------------ MMA issuer ------------------------------
     if (lane == 0) {
+      // D[token][row] += X[token][k] * W[row][k]: A = token tile (TMA, 128-byte swizzle),
+      // B = weight tile (dequantised, no swizzle; router rows by TMA, 128-byte swizzle).
+      // A stage or k-step moves only the descriptors' start addresses (bits 0..13 =
+      // address >> 4; shared addresses stay below 256 KB, so nothing carries out).
+      const uint64_t da0 = umma_desc_sw128(smem_base);
+      const uint64_t db0 = MODE == kModeRouter ? umma_desc_sw128(w_area) : umma_desc(w_area);
+      constexpr uint64_t kAStep = 32 >> 4;                                      // per k-step of 16
+      constexpr uint64_t kBStep = MODE == kModeRouter ? (32 >> 4) : (256 >> 4);
+      const uint32_t idesc = umma_idesc(NR);
       Ring r(P.n_st);
       int it = 0;
       for (int u = blockIdx.x; u < n_units && !s_abort; u += gridDim.x, ++it) {
-        const GemmUnit U = a.units[u];
-        const int npad = (U.n + 15) & ~15;
-        const uint32_t idesc = umma_idesc(npad);
         const int buf = it & 1;
         if (!wait_or_flag(&acc_empty[buf], ((it >> 1) & 1) ^ 1, a.ctrl)) {
           s_abort = 1;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + (uint32_t)buf * (uint32_t)kNmax;
+        const uint32_t d_tmem = tmem + (uint32_t)buf * (uint32_t)kNMax;
         for (int kc = 0; kc < nK; ++kc, r.next()) {
           if (!wait_or_flag(&full[r.s], r.ph, a.ctrl)) {
             s_abort = 1;
@@ -392,13 +387,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
           // dequantised tiles were written through the generic proxy (st.shared)
           if (MODE != kModeRouter) proxy_fence();
           tc_fence_after();
-          const uint32_t a_base = smem_base + r.s * kABytes;
-          const uint32_t b_base = b_area + r.s * kBBytes;
+          const uint64_t da = da0 + (uint64_t)(r.s * (kTBytes >> 4));
+          const uint64_t db = db0 + (uint64_t)(r.s * (wbytes >> 4));
+          umma_f16(d_tmem, da, db, idesc, kc > 0 ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < kKC / 16; ++kk) {
-            const uint64_t da = MODE == kModeRouter ? umma_desc_sw128(a_base + kk * 32) : umma_desc(a_base + kk * 256);
-            umma_f16(d_tmem, da, umma_desc_sw128(b_base + kk * 32), idesc, (kc > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 1; kk < kKC / 16; ++kk) umma_f16(d_tmem, da + kk * kAStep, db + kk * kBStep, idesc, 1u);
           umma_commit(&empty[r.s]);
         }
         if (s_abort) break;
@@ -409,30 +402,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       if (!mbar_wait(&drain, 0)) atomicOr(&a.ctrl->err, kErrTimeout);
     }
     __syncwarp();
-  } else if (warp == kBLoadWarp) {
-    // ------------------------------ B tiles (TMA) ------------------------------
-    // Every unit's columns are consecutive rows of a bf16 matrix: x for the router and the
-    // shared expert, the expert-ordered copy xg of x for routed gate/up units, h / hs for
-    // down.  Loads of kBRows rows, one per lane; rows from U.n up to the loaded count belong
-    // to other units or lie beyond the matrix (zero filled): their products are never read.
-    Ring rb(P.n_st);
+  } else if (warp == kTLoadWarp) {
+    // ------------------------------ token tiles (TMA) ------------------------------
+    // A unit's tokens are consecutive rows of a bf16 matrix: x for the router and the shared
+    // expert's gate/up, the expert-ordered copy xg for routed gate/up, h / hs for down.
+    // Loads of kTRows rows, one per lane; rows beyond U.n belong to other units or lie
+    // beyond the matrix (zero filled): their accumulator lanes are never read.
+    Ring r(P.n_st);
     int issued = 0;
     for (int u = blockIdx.x; u < n_units && !warp_aborted(&s_abort); u += gridDim.x) {
       const GemmUnit U = a.units[u];
-      const int npad = (U.n + 15) & ~15;
+      const CUtensorMap* mt = (MODE != kModeRouter && U.e < 0) ? &a.map_tok2 : &a.map_tok;
+      const int nrt = (U.n + kTRows - 1) / kTRows;
+      const uint32_t bytes = (uint32_t)nrt * kTRows * 128u;
       bool stop = false;
-      const CUtensorMap* mb = (MODE != kModeRouter && U.e < 0) ? &a.map_b2 : &a.map_b;
-      const int nrt = (npad + kBRows - 1) / kBRows;
-      const uint32_t bytes = (uint32_t)nrt * kBRows * 128u;
-      for (int kc = 0; kc < nK; ++kc, rb.next()) {
-        if (!warp_wait(&empty[rb.s], rb.ph ^ 1, a.ctrl, lane)) {
+      for (int kc = 0; kc < nK; ++kc, r.next()) {
+        if (!warp_wait(&empty[r.s], r.ph ^ 1, a.ctrl, lane)) {
           stop = true;
           break;
         }
-        if (lane == 0) mbar_expect_tx(&full[rb.s], bytes);
+        if (lane == 0) mbar_expect_tx(&full[r.s], bytes);
         __syncwarp();  // the transaction count is registered before any load can land
         if (lane < nrt)
-          tma_2d(b_area + rb.s * kBBytes + lane * kBRows * 128, mb, kc * kKC, U.p0 + lane * kBRows, &full[rb.s]);
+          tma_2d(smem_base + r.s * kTBytes + lane * kTRows * 128, mt, kc * kKC, U.p0 + lane * kTRows, &full[r.s]);
         ++issued;
       }
       if (stop) {
@@ -440,17 +432,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         break;
       }
     }
-    // drain: the last loads this thread issued have landed before the CTA may leave
     if (lane == 0) drain_ring(full, P.n_st, issued, a.ctrl);
-  } else if (warp == kALoadWarp) {
-    // ------------------------------ A operand loads (TMA) ------------------------------
-    // Router: 128 router rows x 64 columns per stage straight into the A tile.  Otherwise the
-    // stage's raw codes (128 rows x 64 codes) into the raw ring, for the dequantising warps;
-    // a unit whose expert has no valid slot reads an out-of-range slot, which TMA fills with
-    // zeros (its scales are zero too, so it dequantises to 0).
+  } else if (warp == kWLoadWarp) {
+    // ------------------------------ weight operand loads (TMA) ------------------------------
+    // Router: NR router rows x 64 columns per stage straight into the weight tile.
+    // Otherwise the stage's raw codes (NR rows x 64 codes) into the raw ring, and every 8
+    // stages the scales and biases of those 8 groups (a scale chunk), for the dequantising
+    // warps.  A unit whose expert has no valid slot reads an out-of-range slot, which TMA
+    // fills with zeros (zero scales: it dequantises to 0).
     if (lane == 0) {
       Ring rr(MODE == kModeRouter ? P.n_st : kDepth);
-      int issued = 0;
+      int issued = 0, chunks = 0;
       bool stop = false;
       // unit descriptors two units ahead and slots one unit ahead, so that the lookups'
       // latency is hidden behind the previous unit's loads
@@ -463,43 +455,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         slot1 = slot_of(un1);
       }
       if (my_units > 1) un2 = unit_at(1);
+      const uint32_t raw_bytes = (uint32_t)NR * kRowB, chunk_bytes = (uint32_t)NR * 2 * kChunk * 2;
       for (int j = 0; j < my_units && !stop && !s_abort; ++j) {
         const GemmUnit U = un1;
         int slot = slot1;
         un1 = un2;
         if (j + 1 < my_units) slot1 = slot_of(un1);
         if (j + 2 < my_units) un2 = unit_at(j + 2);
-        const CUtensorMap* ma = &a.map_a;
+        const CUtensorMap* mw = &a.map_w;
+        const CUtensorMap* ms = &a.map_sc;
         if (MODE != kModeRouter) {
           if (U.e < 0) {
-            ma = &a.map_a_shared;
+            mw = &a.map_w_shared;
+            ms = &a.map_sc_shared;
             slot = 0;
-          } else {
-            if (slot < 0 || slot >= a.n_slots) {
-              atomicOr(&a.ctrl->err, kErrBadSlot);
-              slot = (int)a.n_slots;  // out of range: zero fill
-            }
+          } else if (slot < 0 || slot >= a.n_slots) {
+            atomicOr(&a.ctrl->err, kErrBadSlot);
+            slot = (int)a.n_slots;  // out of range: zero fill
           }
         }
+        const int row0 = MODE == kModeGateUp ? U.mt * (NR / 2) : U.mt * NR;
         for (int kc = 0; kc < nK; ++kc, rr.next()) {
           if (MODE == kModeRouter) {
             if (!wait_or_flag(&empty[rr.s], rr.ph ^ 1, a.ctrl)) {
               stop = true;
               break;
             }
-            mbar_expect_tx(&full[rr.s], kABytes);
-            tma_2d(smem_base + rr.s * kABytes, ma, kc * kKC, U.mt * 128, &full[rr.s]);
+            mbar_expect_tx(&full[rr.s], (uint32_t)NR * 128u);
+            tma_2d(w_area + rr.s * wbytes, mw, kc * kKC, row0, &full[rr.s]);
           } else {
             if (!wait_or_flag(&raw_empty[rr.s], rr.ph ^ 1, a.ctrl)) {
               stop = true;
               break;
             }
+            const bool chunk = a.sc_tma && (kc % kChunk) == 0;
+            mbar_expect_tx(&raw_full[rr.s], raw_bytes + (chunk ? chunk_bytes : 0u));
             const uint32_t dst = smem_base + P.raw + rr.s * kRawB;
-            mbar_expect_tx(&raw_full[rr.s], kRawB);
-            if (MODE == kModeGateUp)  // [gate; up] x 64 rows of the row tile
-              tma_4d(dst, ma, kc * Raw<BITS>::kRowBytes, U.mt * 64, 0, slot, &raw_full[rr.s]);
+            if (MODE == kModeGateUp)  // [gate; up] x NR/2 rows of the row tile
+              tma_4d(dst, mw, kc * kRowB, row0, 0, slot, &raw_full[rr.s]);
             else
-              tma_3d(dst, ma, kc * Raw<BITS>::kRowBytes, U.mt * 128, slot, &raw_full[rr.s]);
+              tma_3d(dst, mw, kc * kRowB, row0, slot, &raw_full[rr.s]);
+            if (chunk) {  // [scale, bias] (x [gate, up]) x rows x 8 groups
+              tma_4d(smem_base + P.sc + (chunks & 1) * kChunkBytes, ms, kc, row0, 0, slot, &raw_full[rr.s]);
+              ++chunks;
+            }
           }
           ++issued;
         }
@@ -508,119 +507,101 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       drain_ring(MODE == kModeRouter ? full : raw_full, MODE == kModeRouter ? P.n_st : kDepth, issued, a.ctrl);
     }
     __syncwarp();
-  } else if (warp >= kAWarp0 && warp < kAWarp0 + kAWarps && MODE != kModeRouter) {
+  } else if (warp >= kDWarp0 && warp < kDWarp0 + kDWarps && MODE != kModeRouter) {
     // ------------------------------ dequantisation ------------------------------
-    // Thread (m, q) turns 16 codes (columns 16q..16q+15 of the stage) of tile row m into bf16
-    // in the A tile.  Each unit's row scales and biases are copied (cp.async) into one of two
-    // buffers one unit ahead, the four threads of a row sharing the copies.
-    const int at = tid - kAWarp0 * 32;  // 0..511
-    int m, q;                           // tile row 0..127, column quarter 0..3
-    a_lane_map(at, m, q);
+    // Thread (m, half) turns 32 codes (columns 32*half .. +31 of the stage) of weight row m
+    // into bf16 in the weight tile.  Scales and biases come from the stage's scale chunk
+    // (every 8 stages, by TMA) or, for rows of fewer than 8 groups, from global memory.
+    const int at = tid - kDWarp0 * 32;  // 0..511
+    int m, half;                        // weight row 0..255, column half
+    w_lane_map(at, m, half);
+    const bool active = m < NR;
     const int NG = K / kGroup;  // groups (= stages) per row
-    const int sb_ld = (int)P.sb_ld;
-    uint16_t* sb_area = reinterpret_cast<uint16_t*>(smem + P.sb);  // [2][128][sb_ld]
-    // offset of this thread's codes in a raw stage (TMA box layout)
-    constexpr int kQB = Raw<BITS>::kRowBytes / 4;  // 8 or 16 bytes
-    const uint32_t raw_off = MODE == kModeGateUp
-                                 ? (uint32_t)((m & 1) * 64 + (m >> 1)) * Raw<BITS>::kRowBytes + q * kQB
-                                 : (uint32_t)m * Raw<BITS>::kRowBytes + q * kQB;
-    auto unit_at = [&](int j) { return a.units[blockIdx.x + (size_t)j * gridDim.x]; };
-    auto slot_of = [&](const GemmUnit& U) { return U.e < 0 ? 0 : a.slot_table[U.e]; };
-    // scales / biases of unit ordinal j (descriptor U, slot) into buffer j & 1; a row's
-    // buffer holds its NG scales, then its NG biases
-    auto load_scales = [&](int j, const GemmUnit& U, int slot) {
-      const uint8_t* blob = a.shared;
-      if (U.e >= 0) blob = (slot < 0 || slot >= a.n_slots) ? nullptr : a.pool + (int64_t)slot * a.L.stride;
-      const uint8_t *src_s = nullptr, *src_b = nullptr;
-      if (blob) {
-        if (MODE == kModeGateUp) {
-          const int64_t r = (int64_t)(U.mt * 64 + (m >> 1)) * NG * 2;
-          src_s = blob + a.L.off[(m & 1) ? 5 : 3] + r;
-          src_b = blob + a.L.off[(m & 1) ? 6 : 4] + r;
-        } else {
-          const int64_t r = (int64_t)(U.mt * 128 + m) * NG * 2;
-          src_s = blob + a.L.off[7] + r;
-          src_b = blob + a.L.off[8] + r;
-        }
-      }
-      uint16_t* dst = sb_area + (size_t)(j & 1) * 128 * sb_ld + (size_t)m * sb_ld;
-      if ((NG & 7) == 0) {  // rows of 16-byte multiples: 16-byte aligned in the blob and here
-        const int pieces = NG / 8;  // per array
-        for (int i = q; i < 2 * pieces; i += 4) {
-          const bool bias = i >= pieces;
-          const int o = (bias ? i - pieces : i) * 16;
-          const uint8_t* src = bias ? src_b : src_s;
-          cp_async16(smem_u32(dst) + (bias ? NG * 2 : 0) + o, src ? src + o : a.pool, src ? 16u : 0u);
-        }
-      } else {  // narrow rows (small K): plain loads
-        for (int i = q; i < 2 * NG; i += 4) {
-          const bool bias = i >= NG;
-          const uint16_t* g = reinterpret_cast<const uint16_t*>(bias ? src_b : src_s);
-          dst[i] = g ? __ldg(g + (bias ? i - NG : i)) : (uint16_t)0;
-        }
-      }
-      cp_async_commit();
-    };
-    GemmUnit un1{}, un2{};
-    int slot1 = 0;
-    if (my_units > 0) {
-      const GemmUnit u0 = unit_at(0);
-      load_scales(0, u0, slot_of(u0));
-      if (my_units > 1) {
-        un1 = unit_at(1);
-        slot1 = slot_of(un1);
-      }
-      if (my_units > 2) un2 = unit_at(2);
-    }
+    const uint32_t raw_off = (uint32_t)m * kRowB + half * (kRowB / 2);
+    // position of row m's scale and bias in a chunk: [scale, bias](x [gate, up]) x rows x 8
+    const int sec_rows = MODE == kModeGateUp ? NR / 2 : NR;
+    const int sec = MODE == kModeGateUp && m >= NR / 2 ? 2 : 0;
+    const int crow = MODE == kModeGateUp ? m % (NR / 2) : m;
+    const uint32_t c_s = (uint32_t)((sec * sec_rows + crow) * kChunk), c_b = c_s + (uint32_t)(sec_rows * kChunk);
     Ring ra(P.n_st), rr(kDepth);
+    int g = 0;  // stage of the CTA's stream
     for (int j = 0; j < my_units && !warp_aborted(&s_abort); ++j) {
-      cp_async_wait<0>();  // this unit's scales (this thread's copies) have landed
-      __syncwarp();        // ... and the row's other threads'; buffer (j + 1) & 1 is no longer read
-      if (j + 1 < my_units) {
-        load_scales(j + 1, un1, slot1);
-        un1 = un2;
-        if (j + 2 < my_units) slot1 = slot_of(un1);
-        if (j + 3 < my_units) un2 = unit_at(j + 3);
+      // rows of fewer than 8 groups: this row's scales and biases straight from the blob
+      const uint16_t *gs = nullptr, *gb = nullptr;
+      if (!a.sc_tma && active) {
+        const GemmUnit U = a.units[blockIdx.x + (size_t)j * gridDim.x];
+        const uint8_t* blob = a.shared;
+        if (U.e >= 0) {
+          const int slot = a.slot_table[U.e];
+          blob = (slot < 0 || slot >= a.n_slots) ? nullptr : a.pool + (int64_t)slot * a.L.stride;
+        }
+        if (blob) {
+          if (MODE == kModeGateUp) {
+            const int64_t r = (int64_t)(U.mt * (NR / 2) + crow) * NG * 2;
+            gs = reinterpret_cast<const uint16_t*>(blob + a.L.off[m >= NR / 2 ? 5 : 3] + r);
+            gb = reinterpret_cast<const uint16_t*>(blob + a.L.off[m >= NR / 2 ? 6 : 4] + r);
+          } else {
+            const int64_t r = (int64_t)(U.mt * NR + m) * NG * 2;
+            gs = reinterpret_cast<const uint16_t*>(blob + a.L.off[7] + r);
+            gb = reinterpret_cast<const uint16_t*>(blob + a.L.off[8] + r);
+          }
+        }
       }
-      const uint16_t* my_s = sb_area + (size_t)(j & 1) * 128 * sb_ld + (size_t)m * sb_ld;
       bool stop = false;
-      for (int kc = 0; kc < nK; ++kc, ra.next(), rr.next()) {
+      for (int kc = 0; kc < nK; ++kc, ++g, ra.next(), rr.next()) {
         if (!warp_wait(&raw_full[rr.s], rr.ph, a.ctrl, lane)) {
           stop = true;
           break;
         }
-        const uint8_t* rp = smem + P.raw + rr.s * kRawB + raw_off;
-        uint32_t w[kQB / 4];
-        if (BITS == 4) {
-          const uint2 v = *reinterpret_cast<const uint2*>(rp);
-          w[0] = v.x;
-          w[1] = v.y;
-        } else {
-          const uint4 v = *reinterpret_cast<const uint4*>(rp);
-          w[0] = v.x;
-          w[1] = v.y;
-          w[kQB / 4 > 2 ? 2 : 0] = v.z;
-          w[kQB / 4 > 3 ? 3 : 0] = v.w;
+        uint32_t w[kRowB / 8];  // this thread's 32 codes
+        uint32_t sbits = 0, bbits = 0;
+        if (active) {
+          const uint8_t* rp = smem + P.raw + rr.s * kRawB + raw_off;
+          if (BITS == 4) {
+            const uint4 v = *reinterpret_cast<const uint4*>(rp);
+            w[0] = v.x;
+            w[1] = v.y;
+            w[2] = v.z;
+            w[3] = v.w;
+          } else {
+#pragma unroll
+            for (int o = 0; o < 2; ++o) {
+              const uint4 v = *reinterpret_cast<const uint4*>(rp + o * 16);
+              w[(4 * o + 0) % (kRowB / 8)] = v.x;
+              w[(4 * o + 1) % (kRowB / 8)] = v.y;
+              w[(4 * o + 2) % (kRowB / 8)] = v.z;
+              w[(4 * o + 3) % (kRowB / 8)] = v.w;
+            }
+          }
+          if (a.sc_tma) {
+            const uint16_t* ch = reinterpret_cast<const uint16_t*>(smem + P.sc + ((g / kChunk) & 1) * kChunkBytes);
+            sbits = ch[c_s + kc % kChunk];
+            bbits = ch[c_b + kc % kChunk];
+          } else if (gs) {
+            sbits = __ldg(gs + kc);
+            bbits = __ldg(gb + kc);
+          }
         }
-        const uint32_t sbits = my_s[kc], bbits = my_s[NG + kc];
-        __syncwarp();  // every lane holds its codes: the raw slot can be refilled
+        __syncwarp();  // every lane holds its codes and scales: the raw slot can be refilled
         if (lane == 0) mbar_arrive(&raw_empty[rr.s]);
         if (!warp_wait(&empty[ra.s], ra.ph ^ 1, a.ctrl, lane)) {
           stop = true;
           break;
         }
-        uint8_t* a_tile = smem + ra.s * kABytes;
-        if (BITS == 4) {
-          const uint32_t s2 = sbits | (sbits << 16), b2 = bbits | (bbits << 16);
+        if (active) {
+          uint8_t* w_tile = smem + P.w + ra.s * kWBytes;
+          if (BITS == 4) {
+            const uint32_t s2 = sbits | (sbits << 16), b2 = bbits | (bbits << 16);
 #pragma unroll
-          for (int o = 0; o < 2; ++o)  // 2 k-octets of 8 values = this thread's 16 columns
-            *reinterpret_cast<uint4*>(a_tile + core_off(m, q * 2 + o)) = dq8_int4_bf(w[o], s2, b2);
-        } else {
-          const float sv = __uint_as_float(sbits << 16), bv = __uint_as_float(bbits << 16);
+            for (int o = 0; o < 4; ++o)  // 4 k-octets of 8 values = this thread's 32 columns
+              *reinterpret_cast<uint4*>(w_tile + core_off(m, half * 4 + o)) = dq8_int4_bf(w[o], s2, b2);
+          } else {
+            const float sv = __uint_as_float(sbits << 16), bv = __uint_as_float(bbits << 16);
 #pragma unroll
-          for (int o = 0; o < 2; ++o)
-            *reinterpret_cast<uint4*>(a_tile + core_off(m, q * 2 + o)) =
-                dq8_int8(w[(2 * o) % (kQB / 4)], w[(2 * o + 1) % (kQB / 4)], sv, bv);
+            for (int o = 0; o < 4; ++o)
+              *reinterpret_cast<uint4*>(w_tile + core_off(m, half * 4 + o)) =
+                  dq8_int8(w[(2 * o) % (kRowB / 8)], w[(2 * o + 1) % (kRowB / 8)], sv, bv);
+          }
         }
         proxy_fence();
         __syncwarp();
@@ -631,74 +612,78 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         break;
       }
     }
-    cp_async_wait<0>();  // no copy may still be landing when the CTA leaves
   } else if (warp >= kEWarp0) {
     // ------------------------------ epilogue ------------------------------
-    const int quad = warp & 3;       // TMEM lane quadrant of this warp
-    const int m = quad * 32 + lane;  // accumulator row
+    // This warp reads TMEM lanes 32*quad .. +31: the unit's tokens 32*quad + lane.
+    const int quad = warp & 3;
+    const int tok = quad * 32 + lane;
     int it = 0;
     for (int u = blockIdx.x; u < n_units && !warp_aborted(&s_abort); u += gridDim.x, ++it) {
       const GemmUnit U = a.units[u];
       const int buf = it & 1;
-      if (MODE == kModeDown) {
-        // token and weight of every column, loaded while the unit's MMAs run
-        for (int n = lane; n < U.n; n += 32) {
-          int t;
-          float w;
-          if (U.e < 0) {
-            t = U.p0 + n;
-            w = __ldg(a.gate + t);
-          } else {
-            const int pair = __ldg(a.order + U.p0 + n);
-            t = pair / a.k;
-            w = __ldg(a.topk_w + pair);
-          }
-          s_colt[quad][n] = t;
-          s_colw[quad][n] = w;
+      const bool valid = tok < U.n;
+      // down: the token this lane adds into and its weight, loaded while the MMAs run
+      int t = 0;
+      float wt = 0.f;
+      if (MODE == kModeDown && valid) {
+        if (U.e < 0) {
+          t = U.p0 + tok;
+          wt = __ldg(a.gate + t);
+        } else {
+          const int pair = __ldg(a.order + U.p0 + tok);
+          t = pair / a.k;
+          wt = __ldg(a.topk_w + pair);
         }
-        __syncwarp();
       }
       if (!warp_wait(&acc_full[buf], (it >> 1) & 1, a.ctrl, lane)) {
         s_abort = 1;
         break;
       }
       tc_fence_after();
-      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)buf * (uint32_t)kNmax;
-      constexpr int kEC = MODE == kModeRouter ? 16 : 32;  // columns per TMEM load
-      for (int c0 = 0; c0 < U.n; c0 += kEC) {
-        float v[kEC];
-        if (kEC == 32) tmem_ld32(taddr + c0, v);
-        else tmem_ld16(taddr + c0, v);
-        if (MODE == kModeGateUp) {
-          // lanes 2i (gate row) and 2i + 1 (up row) hold intermediate row r; the even lane
-          // finishes column c, the odd lane column c + 1 (one exchange per column pair)
-          const bool odd = lane & 1;
-          const int r = U.mt * 64 + (m >> 1);
-          uint16_t* hbase = (U.e < 0) ? a.hs : a.h;
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)buf * (uint32_t)kNMax;
+      if (MODE == kModeGateUp) {
+        // columns [0, NR/2) are gate rows, [NR/2, NR) the up rows of the same intermediate rows
+        const int nI = NR / 2;
+        uint16_t* hrow = ((U.e < 0) ? a.hs : a.h) + (size_t)(U.p0 + tok) * a.I + U.mt * nI;
+        for (int c0 = 0; c0 < nI; c0 += 16) {
+          float gv[16], uv[16];
+          tmem_ld16(taddr + c0, gv);
+          tmem_ld16(taddr + nI + c0, uv);
+          if (valid) {
+            uint32_t pk[8];
 #pragma unroll
-          for (int i = 0; i < kEC; i += 2) {
-            const float recv = __shfl_xor_sync(0xffffffffu, odd ? v[i] : v[i + 1], 1);
-            const float g = odd ? recv : v[i];
-            const float up = odd ? v[i + 1] : recv;
-            const int n = c0 + i + (odd ? 1 : 0);
-            // silu(g) * up; h is rounded to bf16, far coarser than the fast exp / divide
-            if (n < U.n) hbase[(size_t)(U.p0 + n) * a.I + r] = f2bf(__fdividef(g, 1.0f + __expf(-g)) * up);
-          }
-        } else {
-#pragma unroll
-        for (int i = 0; i < kEC; ++i) {
-          const int n = c0 + i;
-          const float val = v[i];
-          if (MODE == kModeDown) {
-            if (n < U.n) {
-              const int j = U.mt * 128 + m;
-              atomicAdd(a.acc + (size_t)s_colt[quad][n] * a.H + j, s_colw[quad][n] * val);
+            for (int i = 0; i < 8; ++i) {
+              // silu(g) * up; h is rounded to bf16, far coarser than the fast exp / divide
+              const float h0 = __fdividef(gv[2 * i], 1.0f + __expf(-gv[2 * i])) * uv[2 * i];
+              const float h1 = __fdividef(gv[2 * i + 1], 1.0f + __expf(-gv[2 * i + 1])) * uv[2 * i + 1];
+              pk[i] = pack_bf16(h0, h1);
             }
-          } else {  // router logits (no bias)
-            const int e = U.mt * 128 + m;
-            if (n < U.n && e < a.E) a.logits[(size_t)(U.p0 + n) * (a.E + 1) + e] = val;
+            reinterpret_cast<uint4*>(hrow + c0)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            reinterpret_cast<uint4*>(hrow + c0)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
           }
         }
+      } else if (MODE == kModeDown) {
+        float* arow = a.acc + (size_t)t * a.H + U.mt * NR;
+        for (int c0 = 0; c0 < NR; c0 += 32) {
+          float v[32];
+          tmem_ld32(taddr + c0, v);
+          if (valid) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              atomicAdd(reinterpret_cast<float4*>(arow + c0) + i,
+                        make_float4(wt * v[4 * i], wt * v[4 * i + 1], wt * v[4 * i + 2], wt * v[4 * i + 3]));
+          }
+        }
+      } else {  // router logits (no bias)
+        float* lrow = a.logits + (size_t)(U.p0 + tok) * (a.E + 1) + U.mt * NR;
+        for (int c0 = 0; c0 < NR; c0 += 32) {
+          float v[32];
+          tmem_ld32(taddr + c0, v);
+          if (valid) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (U.mt * NR + c0 + i < a.E) lrow[c0 + i] = v[i];
+          }
         }
       }
       tc_fence_before();
@@ -1058,32 +1043,32 @@ __global__ void __launch_bounds__(kGroupThreads) k_gplace(PrefillArgs a) {
     __syncwarp();
   }
   if (blockIdx.x != 0) return;
-  // chunk 0: offsets, and the GEMM work units: per expert, token tiles of <= kNmax pairs x
-  // row tiles; then the shared expert as one more expert over all tokens
+  // chunk 0: offsets, and the GEMM work units: per expert, token tiles of <= kTok pairs x
+  // weight-row tiles; then the shared expert as one more expert over all tokens
   for (int e = threadIdx.x; e <= E; e += kGroupThreads) a.offsets[e] = s_off[e];
   if (!a.units_gu) return;  // grouping only
   __syncthreads();
   int* tile_base = wc;  // [E + 1], reused
-  block_scan4(E, [&](int e) { return (a.counts[e] + kNmax - 1) / kNmax; }, tile_base, s_wsum);
-  const int mt_gu = a.I / 64, mt_dn = a.H / 128;
+  block_scan4(E, [&](int e) { return (a.counts[e] + kTok - 1) / kTok; }, tile_base, s_wsum);
+  const int mt_gu = a.I / (prefill_gu_rows(a.I) / 2), mt_dn = a.H / prefill_dn_rows(a.H);
   for (int e = threadIdx.x; e < E; e += kGroupThreads) {
     int tb = tile_base[e];
     const int ce = a.counts[e];
-    for (int s0 = 0; s0 < ce; s0 += kNmax, ++tb) {
-      const int nn = min(kNmax, ce - s0);
+    for (int s0 = 0; s0 < ce; s0 += kTok, ++tb) {
+      const int nn = min(kTok, ce - s0);
       for (int mt = 0; mt < mt_gu; ++mt) a.units_gu[tb * mt_gu + mt] = GemmUnit{e, mt, s_off[e] + s0, nn};
       for (int mt = 0; mt < mt_dn; ++mt) a.units_dn[tb * mt_dn + mt] = GemmUnit{e, mt, s_off[e] + s0, nn};
     }
   }
   const int tiles_r = tile_base[E];
-  const int st_n = (a.T + kNmax - 1) / kNmax;
+  const int st_n = (a.T + kTok - 1) / kTok;
   for (int i = threadIdx.x; i < st_n * mt_gu; i += kGroupThreads) {
-    const int st = i / mt_gu, mt = i - st * mt_gu, t0 = st * kNmax;
-    a.units_gu[(tiles_r + st) * mt_gu + mt] = GemmUnit{-1, mt, t0, min(kNmax, a.T - t0)};
+    const int st = i / mt_gu, mt = i - st * mt_gu, t0 = st * kTok;
+    a.units_gu[(tiles_r + st) * mt_gu + mt] = GemmUnit{-1, mt, t0, min(kTok, a.T - t0)};
   }
   for (int i = threadIdx.x; i < st_n * mt_dn; i += kGroupThreads) {
-    const int st = i / mt_dn, mt = i - st * mt_dn, t0 = st * kNmax;
-    a.units_dn[(tiles_r + st) * mt_dn + mt] = GemmUnit{-1, mt, t0, min(kNmax, a.T - t0)};
+    const int st = i / mt_dn, mt = i - st * mt_dn, t0 = st * kTok;
+    a.units_dn[(tiles_r + st) * mt_dn + mt] = GemmUnit{-1, mt, t0, min(kTok, a.T - t0)};
   }
   if (threadIdx.x == 0) {
     a.n_units[0] = (tiles_r + st_n) * mt_gu;
@@ -1121,8 +1106,8 @@ __global__ void k_router_units(GemmUnit* units, int* n_units, int T, int E) {
 
 template <int BITS, int MODE>
 cudaError_t launch_gemm(const GemmArgs& g, int n_sm, cudaStream_t s) {
-  const GemmSmem P = gemm_smem<BITS, MODE>((MODE == kModeDown) ? g.I : g.H);
-  if (P.total > (uint32_t)kSmemMax) return cudaErrorInvalidConfiguration;
+  const GemmSmem P = gemm_smem<BITS, MODE>();
+  if (P.total > (uint32_t)kSmemMax || P.n_st < 2) return cudaErrorInvalidConfiguration;
   auto fn = k_gemm<BITS, MODE>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.total);
   if (e != cudaSuccess) return e;
@@ -1166,22 +1151,34 @@ cudaError_t map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
   return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 // Raw gate/up codes of a pool (or one blob): bytes [slots][gate, up][I][H*b/8]; a box is one
-// stage (64 codes) of 64 rows of both matrices
+// stage (64 codes) of nI rows of both matrices
 cudaError_t map_codes_gu(CUtensorMap* m, const uint8_t* blob0, int64_t n_slots, const BlobLayout& L, int H, int I,
-                         int bits) {
+                         int bits, int nI) {
   const cuuint64_t dims[4] = {(cuuint64_t)H * bits / 8, (cuuint64_t)I, 2, (cuuint64_t)n_slots};
   const cuuint64_t strides[3] = {(cuuint64_t)H * bits / 8, (cuuint64_t)(L.off[1] - L.off[0]), (cuuint64_t)L.stride};
-  const cuuint32_t box[4] = {(cuuint32_t)(kKC * bits / 8), 64, 2, 1};
+  const cuuint32_t box[4] = {(cuuint32_t)(kKC * bits / 8), (cuuint32_t)nI, 2, 1};
   return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, blob0 + L.off[0], dims, strides, box,
                     CU_TENSOR_MAP_SWIZZLE_NONE);
 }
-// Raw down codes: bytes [slots][H][I*b/8]; a box is one stage of 128 rows
+// Raw down codes: bytes [slots][H][I*b/8]; a box is one stage of NR rows
 cudaError_t map_codes_dn(CUtensorMap* m, const uint8_t* blob0, int64_t n_slots, const BlobLayout& L, int H, int I,
-                         int bits) {
+                         int bits, int NR) {
   const cuuint64_t dims[3] = {(cuuint64_t)I * bits / 8, (cuuint64_t)H, (cuuint64_t)n_slots};
   const cuuint64_t strides[2] = {(cuuint64_t)I * bits / 8, (cuuint64_t)L.stride};
-  const cuuint32_t box[3] = {(cuuint32_t)(kKC * bits / 8), 128, 1};
+  const cuuint32_t box[3] = {(cuuint32_t)(kKC * bits / 8), (cuuint32_t)NR, 1};
   return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, blob0 + L.off[2], dims, strides, box,
+                    CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+// Scale / bias chunks: bf16 [slots][n_sec sections][rows][NG], the sections n_sec equally
+// spaced blob sections starting at section `first` (gate/up: gate s, gate b, up s, up b;
+// down: s, b); a box is 8 groups of box_rows rows of every section.  Needs NG % 8 == 0.
+cudaError_t map_scales(CUtensorMap* m, const uint8_t* blob0, int64_t n_slots, const BlobLayout& L, int first,
+                       int n_sec, int rows, int NG, int box_rows) {
+  const cuuint64_t dims[4] = {(cuuint64_t)NG, (cuuint64_t)rows, (cuuint64_t)n_sec, (cuuint64_t)n_slots};
+  const cuuint64_t strides[3] = {(cuuint64_t)NG * 2, (cuuint64_t)(L.off[first + 1] - L.off[first]),
+                                 (cuuint64_t)L.stride};
+  const cuuint32_t box[4] = {(cuuint32_t)kChunk, (cuuint32_t)box_rows, (cuuint32_t)n_sec, 1};
+  return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, blob0 + L.off[first], dims, strides, box,
                     CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
@@ -1219,8 +1216,10 @@ cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
       GemmArgs g = p.g;
       g.units = p.units_rt;
       g.n_units = p.n_units + 2;
-      if ((e = map_bf16(&g.map_a, p.wr, E, H, H, 128)) != cudaSuccess) return e;
-      if ((e = map_bf16(&g.map_b, p.x, T, H, H, kBRows)) != cudaSuccess) return e;
+      g.n_rows = 128;
+      g.sc_tma = 0;
+      if ((e = map_bf16(&g.map_w, p.wr, E, H, H, 128)) != cudaSuccess) return e;
+      if ((e = map_bf16(&g.map_tok, p.x, T, H, H, kTRows)) != cudaSuccess) return e;
       if ((e = (bits == 4 ? launch_gemm<4, kModeRouter>(g, n_sm, s) : launch_gemm<8, kModeRouter>(g, n_sm, s))) !=
           cudaSuccess)
         return e;
@@ -1242,10 +1241,17 @@ cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
     g.units = p.units_gu;
     g.n_units = p.n_units;
     const int I = p.I;
-    if ((e = map_codes_gu(&g.map_a, g.pool, g.n_slots, g.L, H, I, bits)) != cudaSuccess) return e;
-    if ((e = map_codes_gu(&g.map_a_shared, g.shared, 1, g.L, H, I, bits)) != cudaSuccess) return e;
-    if ((e = map_bf16(&g.map_b, p.xg, (uint64_t)T * p.k, H, H, kBRows)) != cudaSuccess) return e;
-    if ((e = map_bf16(&g.map_b2, p.x, T, H, H, kBRows)) != cudaSuccess) return e;
+    g.n_rows = prefill_gu_rows(I);
+    g.sc_tma = (H / kGroup) % kChunk == 0;
+    const int nI = g.n_rows / 2;
+    if ((e = map_codes_gu(&g.map_w, g.pool, g.n_slots, g.L, H, I, bits, nI)) != cudaSuccess) return e;
+    if ((e = map_codes_gu(&g.map_w_shared, g.shared, 1, g.L, H, I, bits, nI)) != cudaSuccess) return e;
+    if (g.sc_tma) {
+      if ((e = map_scales(&g.map_sc, g.pool, g.n_slots, g.L, 3, 4, I, H / kGroup, nI)) != cudaSuccess) return e;
+      if ((e = map_scales(&g.map_sc_shared, g.shared, 1, g.L, 3, 4, I, H / kGroup, nI)) != cudaSuccess) return e;
+    }
+    if ((e = map_bf16(&g.map_tok, p.xg, (uint64_t)T * p.k, H, H, kTRows)) != cudaSuccess) return e;
+    if ((e = map_bf16(&g.map_tok2, p.x, T, H, H, kTRows)) != cudaSuccess) return e;
     prof_mark(2, false, s);
     if ((e = (bits == 4 ? launch_gemm<4, kModeGateUp>(g, n_sm, s) : launch_gemm<8, kModeGateUp>(g, n_sm, s))) !=
         cudaSuccess)
@@ -1253,10 +1259,16 @@ cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
     prof_mark(2, true, s);
     g.units = p.units_dn;
     g.n_units = p.n_units + 1;
-    if ((e = map_codes_dn(&g.map_a, g.pool, g.n_slots, g.L, H, I, bits)) != cudaSuccess) return e;
-    if ((e = map_codes_dn(&g.map_a_shared, g.shared, 1, g.L, H, I, bits)) != cudaSuccess) return e;
-    if ((e = map_bf16(&g.map_b, p.h, (uint64_t)T * p.k, I, I, kBRows)) != cudaSuccess) return e;
-    if ((e = map_bf16(&g.map_b2, p.hs, T, I, I, kBRows)) != cudaSuccess) return e;
+    g.n_rows = prefill_dn_rows(H);
+    g.sc_tma = (I / kGroup) % kChunk == 0;
+    if ((e = map_codes_dn(&g.map_w, g.pool, g.n_slots, g.L, H, I, bits, g.n_rows)) != cudaSuccess) return e;
+    if ((e = map_codes_dn(&g.map_w_shared, g.shared, 1, g.L, H, I, bits, g.n_rows)) != cudaSuccess) return e;
+    if (g.sc_tma) {
+      if ((e = map_scales(&g.map_sc, g.pool, g.n_slots, g.L, 7, 2, H, I / kGroup, g.n_rows)) != cudaSuccess) return e;
+      if ((e = map_scales(&g.map_sc_shared, g.shared, 1, g.L, 7, 2, H, I / kGroup, g.n_rows)) != cudaSuccess) return e;
+    }
+    if ((e = map_bf16(&g.map_tok, p.h, (uint64_t)T * p.k, I, I, kTRows)) != cudaSuccess) return e;
+    if ((e = map_bf16(&g.map_tok2, p.hs, T, I, I, kTRows)) != cudaSuccess) return e;
     prof_mark(3, false, s);
     if ((e = (bits == 4 ? launch_gemm<4, kModeDown>(g, n_sm, s) : launch_gemm<8, kModeDown>(g, n_sm, s))) !=
         cudaSuccess)
