@@ -70,8 +70,8 @@ template <int BITS>
 struct Raw {
   static constexpr int kRowBytes = kKC * BITS / 8;  // 32 or 64
   static constexpr int kBytes = kNMax * kRowBytes;  // 8 or 16 KB
-  static constexpr int kDepth = BITS == 4 ? 4 : 3;
 };
+constexpr int kRawMax = 8;  // raw stages in flight: what shared memory leaves, at most 8
 
 // Position in a ring of n stages and the parity of its current pass.
 struct Ring {
@@ -90,6 +90,7 @@ struct Ring {
 // token tile (16 KB) and a weight tile (up to 32 KB), with one full and one empty barrier.
 struct GemmSmem {
   int n_st;            // stages
+  int n_raw;           // raw-code stages in flight (dequantising modes)
   uint32_t w;          // byte offset of the weight tiles
   uint32_t raw, sc;    // byte offsets of the raw ring and the two scale-chunk slots
   uint32_t total;      // dynamic bytes, including 1 KB of alignment slack
@@ -98,13 +99,23 @@ template <int BITS, int MODE>
 __host__ __device__ inline GemmSmem gemm_smem() {
   GemmSmem p{};
   const uint32_t wb = MODE == kModeRouter ? (uint32_t)(kTok * kKC * 2) : (uint32_t)kWBytes;
-  const uint32_t fixed = MODE == kModeRouter ? 0u : (uint32_t)(Raw<BITS>::kDepth * Raw<BITS>::kBytes + 2 * kChunkBytes);
-  int n = (int)(((uint32_t)kSmemMax - fixed - 1024u) / ((uint32_t)kTBytes + wb));
-  p.n_st = n > kStageMax ? kStageMax : n;
+  const uint32_t budget = (uint32_t)kSmemMax - 1024u;
+  if (MODE == kModeRouter) {
+    const int n = (int)(budget / ((uint32_t)kTBytes + wb));
+    p.n_st = n > kStageMax ? kStageMax : n;
+    p.n_raw = 0;
+  } else {
+    // three stages of tiles, then as many raw stages as fit (the dequantisation runs behind
+    // TMA latency otherwise), at least three
+    const uint32_t rest = budget - 2u * kChunkBytes;
+    p.n_st = 3;
+    const int nr = (int)((rest - 3u * ((uint32_t)kTBytes + wb)) / (uint32_t)Raw<BITS>::kBytes);
+    p.n_raw = nr > kRawMax ? kRawMax : nr;
+  }
   p.w = (uint32_t)p.n_st * kTBytes;
   p.raw = p.w + (uint32_t)p.n_st * wb;
-  p.sc = p.raw + (MODE == kModeRouter ? 0u : (uint32_t)(Raw<BITS>::kDepth * Raw<BITS>::kBytes));
-  p.total = p.raw + fixed + 1024u;
+  p.sc = p.raw + (uint32_t)p.n_raw * Raw<BITS>::kBytes;
+  p.total = p.sc + (MODE == kModeRouter ? 0u : 2u * kChunkBytes) + 1024u;
   return p;
 }
 
@@ -308,9 +319,9 @@ __device__ __forceinline__ void drain_ring(uint64_t* full, int n, int issued, Ct
 // ---------------------------------------------------------------------------------------
 template <int BITS, int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant__ GemmArgs a) {
-  constexpr int kRawB = Raw<BITS>::kBytes, kDepth = Raw<BITS>::kDepth, kRowB = Raw<BITS>::kRowBytes;
+  constexpr int kRawB = Raw<BITS>::kBytes, kRowB = Raw<BITS>::kRowBytes;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full[kStageMax], empty[kStageMax], raw_full[4], raw_empty[4], acc_full[2],
+  __shared__ __align__(8) uint64_t full[kStageMax], empty[kStageMax], raw_full[kRawMax], raw_empty[kRawMax], acc_full[2],
       acc_empty[2], drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
@@ -335,7 +346,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       mbar_init(&full[s], MODE == kModeRouter ? 2 : kDWarps + 1);
       mbar_init(&empty[s], 1);
     }
-    for (int s = 0; s < kDepth; ++s) {
+    for (int s = 0; s < P.n_raw; ++s) {
       mbar_init(&raw_full[s], 1);
       mbar_init(&raw_empty[s], kDWarps);
     }
@@ -441,7 +452,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     // warps.  A unit whose expert has no valid slot reads an out-of-range slot, which TMA
     // fills with zeros (zero scales: it dequantises to 0).
     if (lane == 0) {
-      Ring rr(MODE == kModeRouter ? P.n_st : kDepth);
+      Ring rr(MODE == kModeRouter ? P.n_st : P.n_raw);
       int issued = 0, chunks = 0;
       bool stop = false;
       // unit descriptors two units ahead and slots one unit ahead, so that the lookups'
@@ -504,7 +515,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         }
       }
       if (stop) s_abort = 1;
-      drain_ring(MODE == kModeRouter ? full : raw_full, MODE == kModeRouter ? P.n_st : kDepth, issued, a.ctrl);
+      drain_ring(MODE == kModeRouter ? full : raw_full, MODE == kModeRouter ? P.n_st : P.n_raw, issued, a.ctrl);
     }
     __syncwarp();
   } else if (warp >= kDWarp0 && warp < kDWarp0 + kDWarps && MODE != kModeRouter) {
@@ -523,7 +534,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     const int sec = MODE == kModeGateUp && m >= NR / 2 ? 2 : 0;
     const int crow = MODE == kModeGateUp ? m % (NR / 2) : m;
     const uint32_t c_s = (uint32_t)((sec * sec_rows + crow) * kChunk), c_b = c_s + (uint32_t)(sec_rows * kChunk);
-    Ring ra(P.n_st), rr(kDepth);
+    Ring ra(P.n_st), rr(P.n_raw);
     int g = 0;  // stage of the CTA's stream
     for (int j = 0; j < my_units && !warp_aborted(&s_abort); ++j) {
       // rows of fewer than 8 groups: this row's scales and biases straight from the blob
