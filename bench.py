@@ -45,6 +45,9 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # bench times, from the ncu capture summarised in profiles/k_fused_decode_decode80b_2layer_full.md
 # (2-layer case, scaled by layers).  Must be re-captured whenever the kernel changes.
 NCU_TRAFFIC_PER_LAYER = {("k_fused_decode", "decode80b", 1): 21_639_120}
+# DRAM traffic per launch of the prefill gate/up GEMM on the prefill workload (full-size capture,
+# profiles/k_gemm_gateup_prefill_full.md).  Must be re-captured whenever the kernel changes.
+NCU_TRAFFIC_PREFILL_GATEUP = {("prefill", 4096): 834_096_128}
 
 
 # --------------------------------------------------------------------------------------
@@ -534,7 +537,8 @@ def prefill_line(args, w, T, r, n_gpus, peaks, peak_kind, cpu_base):
                         "frac_of_measured": round(total_f / step_s / 1e12 / peak, 4)},
         "roofline": {"bound": "tensor", "kernel": "k_gemm<GATEUP> (gate/up grouped GEMM + SwiGLU)",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None, "launch_us": round(gu_us, 2),
+                     "frac": round(achieved / peak, 4), "traffic": NCU_TRAFFIC_PREFILL_GATEUP.get((w.name, T)),
+                     "launch_us": round(gu_us, 2),
                      "flops_per_launch": gu_f, "peak_kind": f"{peak_kind} bf16_tflops (burst)"},
         "kernels_us": {"router+topk": round(r["kern_us"][0], 2), "group": round(r["kern_us"][1], 2),
                        "gateup_gemm": round(r["kern_us"][2], 2), "down_gemm": round(r["kern_us"][3], 2),
