@@ -513,9 +513,9 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
           double den = ex;
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+          const int id = valid ? se : -1;
           if (lane < k) {
             if (!valid) atomicOr(&a.ctrl->err, kErrNonFinite);
-            const int id = valid ? se : -1;
             const float pw = valid ? (float)(ex / den) : 0.f;
             P_IDS[t * k + lane] = id;
             P_PW[t * k + lane] = pw;
@@ -524,16 +524,48 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
               Lc.topk_w_out[t * k + lane] = pw;
             }
           }
+          if (T == 1) {
+            // one token: the k ids are distinct, so this warp groups them itself (ranks by
+            // shuffles) and the CTA skips the general grouping below
+            const int key = lane < k ? (id >= 0 ? id : E) : 0x7fffffff;
+            int rank = 0, before = 0;
+            for (int j = 0; j < k; ++j) {
+              const int kj = __shfl_sync(0xffffffffu, key, j);
+              rank += (kj < key) || (kj == key && j < lane);
+              before += kj < key;
+            }
+            const bool vld = lane < k && key < E;
+            const unsigned vm = __ballot_sync(0xffffffffu, vld);
+            if (lane < k) {
+              P_ORDER[rank] = lane;
+              P_POS[lane] = vld ? rank : -1;
+            }
+            if (vld) {  // every valid id is the first (and only) pair of its expert
+              P_ACTE[before] = key;
+              P_BEGIN[before] = before;
+              const int slot = S_SLOT[key];
+              const bool sok = slot >= 0 && slot < Lc.n_slots;
+              if (!sok) atomicOr(&a.ctrl->err, kErrBadSlot);
+              P_SLOT[before] = sok ? slot : -1;
+            }
+            if (lane == 0) {
+              s_act_n = __popc(vm);
+              s_n_valid = __popc(vm);
+              P_BEGIN[__popc(vm)] = __popc(vm);
+            }
+          }
         } else if (lane < k) {
           P_IDS[t * k + lane] = Lc.topk_idx_in[t * k + lane];
           P_PW[t * k + lane] = Lc.topk_w_in[t * k + lane];
         }
-        if (lane == 0) P_GATE[t] = (float)(1.0 / (1.0 + exp(-__ldcg(lt + E))));
       }
+      // shared-expert gates on warps other than the top-k ones, in parallel with them
+      for (int t = 0; t < T; ++t)
+        if (cw == (T + t) % kCons && lane == 0) P_GATE[t] = (float)(1.0 / (1.0 + exp(-__ldcg(a.logits + (size_t)t * (E + 1) + E))));
     }
     bar_cons();
     // grouping: pairs sorted by (expert, pair number); invalid ids left out
-    if (ok) {
+    if (ok && !(T == 1 && routed)) {
       int* key = P_SCRATCH;
       int* first = P_SCRATCH + TK;
       for (int i = tid; i < TK; i += kConsThreads) {
