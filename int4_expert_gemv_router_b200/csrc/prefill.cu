@@ -734,24 +734,28 @@ __global__ void k_norms(const uint16_t* x, int T, int H, const uint16_t* wr, con
 }
 
 // Exact-product fp64 dot of two bf16 rows by one warp (fixed order).
+// (eight partial sums per lane, so the additions are not one dependent chain; the order is
+// fixed, and every product is exact, so the value differs from any other summation order
+// only by fp64 rounding)
 __device__ __forceinline__ double warp_dot_exact(const uint16_t* a, const uint16_t* b, int H) {
   const int lane = threadIdx.x & 31;
-  double s = 0.0;
+  double s[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
   for (int i = lane * 8; i < H; i += 256) {
     const uint4 va = *reinterpret_cast<const uint4*>(a + i);
     const uint4 vb = *reinterpret_cast<const uint4*>(b + i);
-    s += (double)(bf_lo(va.x) * bf_lo(vb.x));
-    s += (double)(bf_hi(va.x) * bf_hi(vb.x));
-    s += (double)(bf_lo(va.y) * bf_lo(vb.y));
-    s += (double)(bf_hi(va.y) * bf_hi(vb.y));
-    s += (double)(bf_lo(va.z) * bf_lo(vb.z));
-    s += (double)(bf_hi(va.z) * bf_hi(vb.z));
-    s += (double)(bf_lo(va.w) * bf_lo(vb.w));
-    s += (double)(bf_hi(va.w) * bf_hi(vb.w));
+    s[0] += (double)(bf_lo(va.x) * bf_lo(vb.x));
+    s[1] += (double)(bf_hi(va.x) * bf_hi(vb.x));
+    s[2] += (double)(bf_lo(va.y) * bf_lo(vb.y));
+    s[3] += (double)(bf_hi(va.y) * bf_hi(vb.y));
+    s[4] += (double)(bf_lo(va.z) * bf_lo(vb.z));
+    s[5] += (double)(bf_hi(va.z) * bf_hi(vb.z));
+    s[6] += (double)(bf_lo(va.w) * bf_lo(vb.w));
+    s[7] += (double)(bf_hi(va.w) * bf_hi(vb.w));
   }
+  double t = ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  return s;
+  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  return t;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -1053,16 +1057,17 @@ __global__ void __launch_bounds__(kGroupThreads) k_gplace(PrefillArgs a) {
     if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * E + e] += __popc(peers);
     __syncwarp();
   }
-  if (blockIdx.x != 0) return;
-  // chunk 0: offsets, and the GEMM work units: per expert, token tiles of <= kTok pairs x
-  // weight-row tiles; then the shared expert as one more expert over all tokens
-  for (int e = threadIdx.x; e <= E; e += kGroupThreads) a.offsets[e] = s_off[e];
+  // offsets (chunk 0), and the GEMM work units: per expert, token tiles of <= kTok pairs x
+  // weight-row tiles; then the shared expert as one more expert over all tokens.  Every
+  // chunk's CTA writes the units of experts e = chunk (mod chunks).
+  if (blockIdx.x == 0)
+    for (int e = threadIdx.x; e <= E; e += kGroupThreads) a.offsets[e] = s_off[e];
   if (!a.units_gu) return;  // grouping only
   __syncthreads();
   int* tile_base = wc;  // [E + 1], reused
   block_scan4(E, [&](int e) { return (a.counts[e] + kTok - 1) / kTok; }, tile_base, s_wsum);
   const int mt_gu = a.I / (prefill_gu_rows(a.I) / 2), mt_dn = a.H / prefill_dn_rows(a.H);
-  for (int e = threadIdx.x; e < E; e += kGroupThreads) {
+  for (int e = blockIdx.x + (int)gridDim.x * threadIdx.x; e < E; e += (int)gridDim.x * kGroupThreads) {
     int tb = tile_base[e];
     const int ce = a.counts[e];
     for (int s0 = 0; s0 < ce; s0 += kTok, ++tb) {
@@ -1071,6 +1076,7 @@ __global__ void __launch_bounds__(kGroupThreads) k_gplace(PrefillArgs a) {
       for (int mt = 0; mt < mt_dn; ++mt) a.units_dn[tb * mt_dn + mt] = GemmUnit{e, mt, s_off[e] + s0, nn};
     }
   }
+  if (blockIdx.x != 0) return;
   const int tiles_r = tile_base[E];
   const int st_n = (a.T + kTok - 1) / kTok;
   for (int i = threadIdx.x; i < st_n * mt_gu; i += kGroupThreads) {
