@@ -154,3 +154,46 @@ def test_prefill_matches_token_by_token_decode():
         assert torch.equal(idd, idx[t0:t0 + 8])
         a, b = od.float(), out[t0:t0 + 8].float()
         assert (a - b).abs().max().item() <= 1e-2 * b.abs().max().item() + 1e-3
+
+
+def test_prefill_device_error_flags():
+    """Many-token path: a selected expert with an out-of-range slot is flagged and contributes
+    nothing (its weights read as zeros); a caller-given id out of range is flagged and its pair
+    is skipped.  The rest of the output still matches the oracle."""
+    w = TINY.with_(hidden=512, inter=128, shared_inter=128, n_experts=20, top_k=3, seed=61)
+    L = synth.make_layer(w, 0, DEV)
+    T = 40
+    x = synth.activations(w, 7, tokens=T, device=DEV)
+    _, idx, p, _ = forward(w, L, x, residual=x)
+    bad_e = int(idx[0, 0].item())
+    st = torch.arange(w.n_experts, dtype=torch.int32, device=DEV)
+    st[bad_e] = 10_000
+    out, idx2, p2, ws = forward(w, L, x, residual=x, slot_table=st)
+    assert abi.moe_ws_check(ws) & abi.DEVERR_BAD_SLOT
+    assert torch.equal(idx2, idx)
+    ih, ph = idx.cpu().numpy(), p.cpu().numpy()
+    ref = oracle_forward(w, L, x, residual=x, idx=ih, p=np.where(ih == bad_e, 0.0, ph))
+    assert_close(out, ref["out"])
+    # caller-given routing with one id out of range
+    bad = idx.clone()
+    bad[3, 1] = w.n_experts + 5
+    out, _, _, ws = forward(w, L, x, residual=x, topk=(bad, p))
+    assert abi.moe_ws_check(ws) & abi.DEVERR_BAD_EXPERT
+    bh = bad.cpu().numpy()
+    ref = oracle_forward(w, L, x, residual=x, idx=np.where(bh < w.n_experts, bh, 0),
+                         p=np.where(bh < w.n_experts, ph, 0.0))
+    assert_close(out, ref["out"])
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_prefill_large_hidden(bits):
+    """hidden 4096 / inter 1024: longer K loops, the fewest tile stages shared memory allows."""
+    w = TINY.with_(hidden=4096, inter=1024, shared_inter=1024, n_experts=12, top_k=3, bits=bits, seed=62 + bits)
+    L = synth.make_layer(w, 0, DEV)
+    T = 64
+    x = synth.activations(w, 8, tokens=T, device=DEV)
+    out, idx, p, ws = forward(w, L, x, residual=x)
+    assert abi.moe_ws_check(ws) == 0
+    ref = oracle_forward(w, L, x, residual=x)
+    assert_close(out, ref["out"])
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"])
