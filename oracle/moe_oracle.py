@@ -310,6 +310,9 @@ def group_pairs(idx: np.ndarray, n_experts: int):
 # ----------------------------------------------------------------------------
 # bounded slot pool: LFU + recency
 # ----------------------------------------------------------------------------
+SLOT_POLICIES = ("lfu_recency", "lru", "lfu")
+
+
 class SlotCache:
     """Bounded pool of expert slots with LFU + recency eviction.
 
@@ -321,9 +324,15 @@ class SlotCache:
     the smallest (count, last use, slot index) among slots whose expert this
     step does not need (those are pinned for the step).  A step that needs more
     unique experts than there are slots is a capacity error.
+
+    For the eviction ablation, `policy` may instead be "lru" (smallest (last use, slot))
+    or "lfu" (smallest (count, slot)); "lfu_recency" is the pages' policy and the default.
     """
 
-    def __init__(self, n_experts: int, n_slots: int):
+    def __init__(self, n_experts: int, n_slots: int, policy: str = "lfu_recency"):
+        if policy not in SLOT_POLICIES:
+            raise ValueError(f"unknown policy {policy!r}")
+        self.policy = policy
         self.E, self.S = n_experts, n_slots
         self.slot_of = np.full(n_experts, -1, dtype=np.int32)
         self.expert_in = np.full(n_slots, -1, dtype=np.int32)
@@ -367,10 +376,15 @@ class SlotCache:
                 for c in range(self.S):
                     if int(self.expert_in[c]) in seen:
                         continue
-                    key = (int(self.count[c]), int(self.last[c]), c)
+                    if self.policy == "lru":
+                        key = (int(self.last[c]), c)
+                    elif self.policy == "lfu":
+                        key = (int(self.count[c]), c)
+                    else:
+                        key = (int(self.count[c]), int(self.last[c]), c)
                     if best is None or key < best:
                         best = key
-                s = best[2]
+                s = best[-1]
                 self.slot_of[self.expert_in[s]] = -1
                 self.evictions += 1
             self.expert_in[s] = e

@@ -372,10 +372,25 @@ def test_slot_cache_hand_traces():
             c.step(tr["capacity_error_next"])
 
 
+def test_slot_cache_policies_hand_traces():
+    fx = _gold("slot_cache_policies.json")
+    for tr in fx["traces"]:
+        for policy, want in tr["by_policy"].items():
+            c = oracle.SlotCache(tr["n_experts"], tr["n_slots"], policy)
+            got = [[list(l) for l in c.step(st)] for st in tr["steps"]]
+            assert got == want["loads"], (tr["name"], policy)
+            assert c.slot_of.tolist() == want["final_slot_of"], (tr["name"], policy)
+            assert [c.lookups, c.hits, c.misses, c.evictions] == want["counters"], (tr["name"], policy)
+
+
 def test_slot_cache_invariants_random():
     rng = np.random.default_rng(11)
     E, S, k = 64, 16, 6
-    c = oracle.SlotCache(E, S)
+    for policy in oracle.SLOT_POLICIES:
+        _slot_cache_invariants(oracle.SlotCache(E, S, policy), rng, E, S, k)
+
+
+def _slot_cache_invariants(c, rng, E, S, k):
     for s in range(300):
         need = rng.choice(E, size=k, replace=False, p=None)
         c.step(need)
