@@ -1,8 +1,9 @@
 #!/usr/bin/env python3
 """Benchmark of the routed-MoE layer forward on B200 (one process per GPU).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode80b|decode35b|pool_int4|pool_int8]
-                    [--tokens T] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--workload decode80b|decode35b|prefill|pool_int4|pool_int8]
+                    [--tokens T] [--impl ours|reference] [--policy lfu_recency|lru|lfu] [--slots S]
 
 Default workload: the 80B-like decode stack -- hidden 2048, 512 experts, top-10,
 intermediate 512, shared expert 512, int4 group 64, one token per step through 48
@@ -574,6 +575,7 @@ def run_pool(args, w, device, rank, total_steps=1024):
     dev_pool = torch.zeros(w.n_slots, stride, dtype=torch.uint8, device=device)
     table = torch.empty(w.n_experts, dtype=torch.int32, device=device)
     pool = abi.moe_pool_create(shape, w.n_slots, host_blobs, dev_pool, table)
+    abi.moe_pool_set_policy(pool, args.policy)
     T = 1
     xs = torch.stack([synth.activations(w, rank_step_seed(rank, s), tokens=T, device=device) for s in range(n_total)])
     out = torch.empty(T, w.hidden, dtype=torch.bfloat16, device=device)
@@ -636,7 +638,8 @@ def pool_line(args, w, r, n_gpus):
         "data": "synthetic (seeded; Zipf(1.0) router bias)",
         "config": {"workload": w.name, "hidden": w.hidden, "n_experts": w.n_experts, "top_k": w.top_k,
                    "bits": w.bits, "n_slots": w.n_slots, "slot_fraction": w.n_slots / w.n_experts,
-                   "steps_total": r["n_total"], "tokens_per_step": 1, "policy": "LFU + recency",
+                   "steps_total": r["n_total"], "tokens_per_step": 1,
+                   "policy": {"lfu_recency": "LFU + recency", "lru": "LRU", "lfu": "LFU"}[args.policy],
                    "miss_path": "pinned host -> cudaMemcpyAsync on a side stream",
                    "timing": "events around the timed steps; each step waits on the host for the ids"},
         "pool": {"hit_rate_all_steps": round(r["hit_rate_all"], 4), "hit_rate_timed": round(r["hit_rate_timed"], 4),
@@ -714,6 +717,9 @@ def parse(argv=None):
                     choices=["decode80b", "decode35b", "prefill", "pool_int4", "pool_int8"])
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--policy", choices=["lfu_recency", "lru", "lfu"], default="lfu_recency",
+                    help="pool workloads: eviction policy (the pages' LFU + recency by default)")
+    ap.add_argument("--slots", type=int, default=None, help="pool workloads: number of slots (default 128)")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the stack depth (profiling of a small case only; not a bench value)")
     return ap.parse_args(argv)
@@ -726,6 +732,8 @@ def main(argv=None):
     w = synth.WORKLOADS[args.workload]
     if args.layers:
         w = w.with_(layers=args.layers)
+    if args.slots and w.name.startswith("pool"):
+        w = w.with_(n_slots=args.slots)
     T = args.tokens or w.tokens
     if args.impl == "reference":
         line = run_reference(args, w, T)

@@ -282,6 +282,16 @@ MOE_API moe_status moe_pool_create(const moe_shape* shape, int32_t n_slots, cons
  */
 MOE_API moe_status moe_expert_pool_load(moe_pool* pool, const int32_t* topk_idx, int32_t T, void* stream);
 
+/*
+ * moe_pool_set_policy -- eviction policy of the next loads (for the eviction ablation):
+ *   MOE_POOL_LFU_RECENCY (the pages' policy, the default): smallest (use count, last use, slot)
+ *   MOE_POOL_LRU: smallest (last use, slot);  MOE_POOL_LFU: smallest (use count, slot)
+ * among the slots whose expert the step does not need.  Host-side only; MOE_ERR_INVALID
+ * for another value.
+ */
+enum { MOE_POOL_LFU_RECENCY = 0, MOE_POOL_LRU = 1, MOE_POOL_LFU = 2 };
+MOE_API moe_status moe_pool_set_policy(moe_pool* pool, int32_t policy);
+
 /* moe_pool_stats -- counters since creation (host struct). */
 MOE_API moe_status moe_pool_stats(const moe_pool* pool, moe_pool_stats_t* stats);
 

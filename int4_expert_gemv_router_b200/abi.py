@@ -71,6 +71,7 @@ _SIGS = {
     "moe_pool_stats": (ctypes.c_int, [_P, ctypes.POINTER(moe_pool_stats_t)]),
     "moe_pool_slot_table": (ctypes.c_int, [_P, _P, _P]),
     "moe_pool_inject_copy_failure": (ctypes.c_int, [_P, _I64]),
+    "moe_pool_set_policy": (ctypes.c_int, [_P, ctypes.c_int32]),
     "moe_pool_destroy": (None, [_P]),
     "moe_profile_events": (ctypes.c_int, [_P, _I32]),
     "moe_last_error": (ctypes.c_char_p, []),
@@ -225,6 +226,14 @@ def moe_pool_slot_table(pool: int, n_experts: int, n_slots: int):
     b = (ctypes.c_int32 * n_slots)()
     _check(lib().moe_pool_slot_table(pool, a, b))
     return list(a), list(b)
+
+
+POOL_POLICIES = {"lfu_recency": 0, "lru": 1, "lfu": 2}
+
+
+def moe_pool_set_policy(pool: int, policy: str):
+    """Eviction policy of the pool's next loads: "lfu_recency" (default), "lru" or "lfu"."""
+    _check(lib().moe_pool_set_policy(pool, POOL_POLICIES[policy]))
 
 
 def moe_pool_inject_copy_failure(pool: int, nth: int):

@@ -7,7 +7,8 @@
 // Here the backing store is pinned host memory and a fetch is one cudaMemcpyAsync of one
 // blob on the pool's side stream.
 //
-// Policy (the pages give only "LFU + recency"; this is the plain reading):
+// Policy (the pages give only "LFU + recency"; this is the plain reading; LRU and pure LFU
+// can be selected for the eviction ablation):
 //   per slot: resident expert, use count (1 when loaded, +1 for every later step that uses
 //   it), last-use step.  A step's distinct experts are looked up in first-appearance order;
 //   hits refresh count and last use.  Misses are then loaded in the same order into the
@@ -44,6 +45,7 @@ struct moe_pool {
   std::vector<uint8_t> needed;     // [E] scratch: expert needed by the current step
   int64_t step_no = 0;
   moe_pool_stats_t stats{};
+  int32_t policy = MOE_POOL_LFU_RECENCY;
   int64_t fail_at = -1;            // test hook: copies until an injected failure
   cudaStream_t side = nullptr;
   cudaEvent_t ready = nullptr;     // slot table + blobs of the last step are on the device
@@ -162,9 +164,18 @@ moe_status moe_expert_pool_load(moe_pool* p, const int32_t* topk_idx, int32_t T,
     if (victim < 0) {
       for (int32_t sl = 0; sl < p->n_slots; ++sl) {
         if (p->needed[p->expert_in[sl]]) continue;
-        if (victim < 0 || p->count[sl] < p->count[victim] ||
-            (p->count[sl] == p->count[victim] && p->last_use[sl] < p->last_use[victim]))
-          victim = sl;  // ascending scan keeps the lowest slot index on full ties
+        bool better;
+        if (victim < 0) {
+          better = true;
+        } else if (p->policy == MOE_POOL_LRU) {
+          better = p->last_use[sl] < p->last_use[victim];
+        } else if (p->policy == MOE_POOL_LFU) {
+          better = p->count[sl] < p->count[victim];
+        } else {
+          better = p->count[sl] < p->count[victim] ||
+                   (p->count[sl] == p->count[victim] && p->last_use[sl] < p->last_use[victim]);
+        }
+        if (better) victim = sl;  // ascending scan keeps the lowest slot index on full ties
       }
       evicting = true;
     }
@@ -217,6 +228,14 @@ moe_status moe_pool_slot_table(const moe_pool* p, int32_t* slot_of_expert, int32
   if (!p) return set_error(MOE_ERR_INVALID, "pool is NULL");
   if (slot_of_expert) memcpy(slot_of_expert, p->slot_of.data(), sizeof(int32_t) * p->slot_of.size());
   if (expert_in_slot) memcpy(expert_in_slot, p->expert_in.data(), sizeof(int32_t) * p->expert_in.size());
+  return MOE_OK;
+}
+
+moe_status moe_pool_set_policy(moe_pool* p, int32_t policy) {
+  if (!p) return set_error(MOE_ERR_INVALID, "pool is NULL");
+  if (policy != MOE_POOL_LFU_RECENCY && policy != MOE_POOL_LRU && policy != MOE_POOL_LFU)
+    return set_error(MOE_ERR_INVALID, "unknown pool policy %d", policy);
+  p->policy = policy;
   return MOE_OK;
 }
 

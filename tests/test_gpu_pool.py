@@ -1,5 +1,6 @@
 """GPU checks of the bounded slot pool (moe_expert_pool_load): slot decisions equal the
-oracle's LFU + recency simulation step by step, missed blobs land byte-for-byte, the
+oracle's LFU + recency simulation step by step (and its LRU / pure LFU variants for the
+eviction ablation), missed blobs land byte-for-byte, the
 pool-mode forward is bit-identical to the all-resident forward, and failures leave the
 pool consistent."""
 import numpy as np
@@ -75,6 +76,37 @@ def test_pool_matches_oracle_cache_and_resident_forward(wname, steps, T):
                                                                               sim.evictions)
         assert st["h2d_bytes"] == sim.misses * P.stride
         assert st["steps"] == steps
+    finally:
+        P.close()
+
+
+@pytest.mark.parametrize("policy", ["lru", "lfu", "lfu_recency"])
+def test_pool_policies_match_oracle(policy):
+    """Eviction ablation: each policy's slot decisions equal the oracle's simulation of the
+    same policy, step by step, on Zipf routing with a small pool (many evictions)."""
+    w = synth.WORKLOADS["pool_int4"]
+    n_slots = 24
+    P = Pool(w, n_slots)
+    sim = oracle.SlotCache(w.n_experts, n_slots, policy)
+    try:
+        abi.moe_pool_set_policy(P.h, policy)
+        with pytest.raises(abi.MoeError):
+            abi.lib()  # the binding maps names; an out-of-range code is rejected by the library
+            abi._check(abi.lib().moe_pool_set_policy(P.h, 7))
+        for s in range(40):
+            x = synth.activations(w, 1000 + s, tokens=1, device=DEV)
+            idx, _ = _route(P, x)
+            abi.moe_expert_pool_load(P.h, idx, 1)
+            sim.step(idx.cpu().numpy().reshape(-1).tolist())
+            slot_of, expert_in = abi.moe_pool_slot_table(P.h, w.n_experts, n_slots)
+            assert slot_of == sim.slot_of.tolist()
+            assert expert_in == sim.expert_in.tolist()
+        torch.cuda.synchronize()
+        assert P.table.cpu().tolist() == slot_of
+        st = abi.moe_pool_stats(P.h)
+        assert (st["lookups"], st["hits"], st["misses"], st["evictions"]) == (sim.lookups, sim.hits, sim.misses,
+                                                                              sim.evictions)
+        assert sim.evictions > 0
     finally:
         P.close()
 
