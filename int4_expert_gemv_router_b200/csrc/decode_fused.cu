@@ -308,19 +308,25 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
           ok = false;
           break;
         }
-        if (lane == 0) {
+        {
+          // lane 0 announces the bytes, then lanes 0..5 issue the stage's six copies at once
+          // (gate codes, up codes, then the four scale/bias sections)
           uint8_t* st = ring + (size_t)s * SB;
           const int slot = P_SLOT[u];
-          if (slot < 0) {
-            mbar_arrive(&full_bar[s]);
-          } else {
+          if (lane == 0) {
+            if (slot < 0)
+              mbar_arrive(&full_bar[s]);
+            else
+              mbar_expect_tx(&full_bar[s], (uint32_t)(n * ROWG_BYTES));
+          }
+          __syncwarp();
+          if (slot >= 0 && lane < 6) {
             const uint8_t* b = Lc.pool + (int64_t)slot * a.L.stride;
-            mbar_expect_tx(&full_bar[s], (uint32_t)(n * ROWG_BYTES));
-            bulk_g2s(st, b + a.L.off[0] + (int64_t)r0 * ROWBg, n * ROWBg, &full_bar[s]);
-            bulk_g2s(st + n * ROWBg, b + a.L.off[1] + (int64_t)r0 * ROWBg, n * ROWBg, &full_bar[s]);
-            uint8_t* sc = st + 2 * n * ROWBg;
-            for (int z = 0; z < 4; ++z)
-              bulk_g2s(sc + z * n * SRg, b + a.L.off[3 + z] + (int64_t)r0 * SRg, n * SRg, &full_bar[s]);
+            if (lane < 2)
+              bulk_g2s(st + lane * n * ROWBg, b + a.L.off[lane] + (int64_t)r0 * ROWBg, n * ROWBg, &full_bar[s]);
+            else
+              bulk_g2s(st + 2 * n * ROWBg + (lane - 2) * n * SRg, b + a.L.off[lane + 1] + (int64_t)r0 * SRg,
+                       n * SRg, &full_bar[s]);
           }
         }
         __syncwarp();
@@ -337,8 +343,8 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
             ok = false;
             break;
           }
+          uint8_t* st = ring + (size_t)s * SB;
           if (lane == 0) {
-            uint8_t* st = ring + (size_t)s * SB;
             uint32_t bytes = 0;
             for (int z = 0; z < cnt; ++z) {
               const int uu = u + z;
@@ -347,21 +353,25 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
               bytes += nJ * ROWD_BYTES;
             }
             mbar_expect_tx(&full_bar[s], bytes);
-            for (int z = 0; z < cnt; ++z) {
-              const int uu = u + z;
-              const uint8_t* b;
-              if (uu < act_n) {
-                const int slot = P_SLOT[uu];
-                if (slot < 0) continue;
-                b = Lc.pool + (int64_t)slot * a.L.stride;
-              } else {
-                b = Lc.shared;
-              }
-              uint8_t* d = st + (size_t)z * nJ * ROWD_BYTES;
-              bulk_g2s(d, b + a.L.off[2] + (int64_t)j0 * ROWBd, nJ * ROWBd, &full_bar[s]);
-              bulk_g2s(d + nJ * ROWBd, b + a.L.off[7] + (int64_t)j0 * SRd, nJ * SRd, &full_bar[s]);
-              bulk_g2s(d + nJ * ROWBd + nJ * SRd, b + a.L.off[8] + (int64_t)j0 * SRd, nJ * SRd, &full_bar[s]);
+          }
+          __syncwarp();
+          // three copies per expert (down codes, scales, biases), spread over the lanes
+          for (int ci = lane; ci < 3 * cnt; ci += 32) {
+            const int z = ci / 3, part = ci - 3 * z, uu = u + z;
+            const uint8_t* b;
+            if (uu < act_n) {
+              const int slot = P_SLOT[uu];
+              if (slot < 0) continue;
+              b = Lc.pool + (int64_t)slot * a.L.stride;
+            } else {
+              b = Lc.shared;
             }
+            uint8_t* d = st + (size_t)z * nJ * ROWD_BYTES;
+            if (part == 0)
+              bulk_g2s(d, b + a.L.off[2] + (int64_t)j0 * ROWBd, nJ * ROWBd, &full_bar[s]);
+            else
+              bulk_g2s(d + nJ * ROWBd + (part - 1) * nJ * SRd, b + a.L.off[6 + part] + (int64_t)j0 * SRd, nJ * SRd,
+                       &full_bar[s]);
           }
           __syncwarp();
           ++q;
