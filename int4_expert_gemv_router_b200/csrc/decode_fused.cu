@@ -221,6 +221,8 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
   constexpr int gD = clcm(16 / cgcd(16, SRd), RPWd);
   constexpr int ROWG_BYTES = 2 * ROWBg + 4 * SRg;  // one gate/up row with its scales
   constexpr int ROWD_BYTES = ROWBd + 2 * SRd;      // one down row with its scales
+  // phase D: the RPWd lanes that share an h chunk; with two of them each loads half
+  constexpr int HS = (RPWd == 2 && V4 % 2 == 0) ? 2 : 1, VH = V4 / HS;
 
   const int T = a.T, E = a.E, k = a.k, G = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -696,6 +698,9 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
 
     // ---- phase D: down rows j0..j1 of every selected expert and the shared expert ----
     if (nJ > 0) {
+      // the first residual element this thread adds in the combine, loaded now
+      float res_v = 0.f;
+      if (Lc.residual && tid < T * nJ) res_v = bf1(__ldcg(Lc.residual + (size_t)(tid / nJ) * H + j0 + tid % nJ));
       const int per_stage = SB / (nJ * ROWD_BYTES);
       const int sub = lane % NCLd, rsub = lane / NCLd;
       float* red = reinterpret_cast<float*>(smem + a.sm.red) + (size_t)cw * a.jmax * (NCLd + 1);
@@ -733,16 +738,35 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
               hsrc = a.hs + (size_t)t * I;
             }
             (void)t;
-            // this pair's h chunks in registers, pre-scaled like staged activations
+            // this pair's h chunks in registers, pre-scaled like staged activations.  With two
+            // lanes per chunk (lane, lane ^ NCLd) each loads one half and they swap halves.
             float4 hr[CPLd][V4];
             float hsum[CPLd];
 #pragma unroll
             for (int m = 0; m < CPLd; ++m) {
               const int c = sub + NCLd * m;
+              if constexpr (HS == 2) {
+#pragma unroll
+                for (int vv = 0; vv < VH; ++vv)
+                  hr[m][vv] = __ldcg(reinterpret_cast<const float4*>(hsrc + c * CC + 4 * (rsub * VH + vv)));
+#pragma unroll
+                for (int vv = 0; vv < VH; ++vv) {
+                  const float4 own = hr[m][vv];
+                  const float4 oth = make_float4(__shfl_xor_sync(0xffffffffu, own.x, NCLd),
+                                                 __shfl_xor_sync(0xffffffffu, own.y, NCLd),
+                                                 __shfl_xor_sync(0xffffffffu, own.z, NCLd),
+                                                 __shfl_xor_sync(0xffffffffu, own.w, NCLd));
+                  hr[m][vv] = rsub ? oth : own;
+                  hr[m][VH + vv] = rsub ? own : oth;
+                }
+              } else {
+#pragma unroll
+                for (int v = 0; v < V4; ++v) hr[m][v] = __ldcg(reinterpret_cast<const float4*>(hsrc + c * CC + 4 * v));
+              }
               float sum = 0.f;
 #pragma unroll
               for (int v = 0; v < V4; ++v) {
-                const float4 f4 = __ldcg(reinterpret_cast<const float4*>(hsrc + c * CC + 4 * v));
+                const float4 f4 = hr[m][v];
                 sum += (f4.x + f4.y) + (f4.z + f4.w);
                 hr[m][v] = make_float4(f4.x * stage_scale<BITS>(4 * v), f4.y * stage_scale<BITS>(4 * v + 1),
                                        f4.z * stage_scale<BITS>(4 * v + 2), f4.w * stage_scale<BITS>(4 * v + 3));
@@ -793,7 +817,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
             if (p >= 0) v += partial[(size_t)p * a.jmax + jl];
           }
           v += partial[(size_t)(n_valid + t) * a.jmax + jl];
-          if (Lc.residual) v += bf1(__ldcg(Lc.residual + (size_t)t * H + j0 + jl));
+          if (Lc.residual) v += (i == tid) ? res_v : bf1(__ldcg(Lc.residual + (size_t)t * H + j0 + jl));
           Lc.out[(size_t)t * H + j0 + jl] = f2bf(v);
         }
       }

@@ -22,20 +22,22 @@
 //                  accumulator (the shared expert is one more "expert" over all tokens)
 //   k_finalize     out = bf16(acc + residual)
 //
-// GEMM kernel ("swap-AB": the weight rows are the MMA's M = 128, the tokens its N <= 128):
+// GEMM kernel (the unit's tokens are the MMA's M = 128 TMEM lanes, its weight rows the N <= 256
+// columns; one kind::f16 MMA per 16-deep k-step):
 //   warp 0        TMEM allocation; lane 0 issues tcgen05.mma (kind::f16, cta_group::1)
-//   warp 1        B tiles by TMA (consecutive rows of x, of the expert-ordered copy xg, h, hs)
-//   warp 2        lane 0: raw codes by TMA (3-D / 4-D boxes over the pool), or router rows
-//   warps 3..18   dequantise the codes (w = s*q + b, rounded to bf16) into the A tile; each
-//                 unit's row scales and biases are copied to shared memory once
+//   warp 1        token tiles by TMA (consecutive rows of x, of the expert-ordered copy xg,
+//                 of h, hs)
+//   warp 2        lane 0: raw codes by TMA (3-D / 4-D boxes over the pool) into a raw ring,
+//                 with the scales and biases of every 8 stages; or router rows
+//   warps 3..18   dequantise the codes (w = s*q + b, rounded to bf16) into the weight tile
 //   warps 19..22  epilogue: tcgen05.ld of the fp32 accumulator, then SwiGLU / scatter / store
-// A tiles written by the dequantising warps are K-major without swizzle (8-row x 16-byte
+// Weight tiles written by the dequantising warps are K-major without swizzle (8-row x 16-byte
 // core matrices, k-octets 128 bytes apart, 8-row groups 1024 bytes apart); tiles written by
-// TMA (B, router rows) use the 128-byte swizzle.  Stage s holds one A and one B tile, with
-// one full barrier (TMA bytes plus the producers' arrivals) and one empty barrier (the MMA's
-// commit); two TMEM accumulators of 128 columns let the epilogue of one unit overlap the next.
-// Every wait is bounded; on timeout the kernel flags MOE_DEVERR_TIMEOUT, drains and frees
-// its TMEM.
+// TMA (tokens, router rows) use the 128-byte swizzle.  Stage s holds one token and one weight
+// tile, with one full barrier (TMA bytes plus the producers' arrivals) and one empty barrier
+// (the MMA's commit); two TMEM accumulators of 256 columns let the epilogue of one unit
+// overlap the next.  Every wait is bounded; on timeout the kernel flags MOE_DEVERR_TIMEOUT,
+// drains and frees its TMEM.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "sync.cuh"
