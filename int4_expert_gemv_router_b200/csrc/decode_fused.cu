@@ -4,8 +4,8 @@
 // One CTA per SM, 16 warps: warps 0..14 compute, warp 15 streams weights.  Per layer:
 //
 //   phase R  router logits (E rows + the shared-gate row; fp64 sums of exact bf16 products)
-//            and the shared expert's gate/up + SwiGLU rows, spread over every compute warp
-//            of the grid; activations staged once per CTA in shared memory.
+//            and the shared expert's gate/up + SwiGLU rows, dealt round-robin over the CTAs
+//            and their compute warps; activations staged once per CTA in shared memory.
 //   -- grid barrier --
 //   phase T  every CTA selects the top-k per token from the logits (threshold + warp
 //            bitonic sort; ties to the lower id), forms the softmax weights and the shared
@@ -275,11 +275,12 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
     for (int l = 0; l < a.n_layers && ok; ++l) {
       const FusedLayer& Lc = a.layer[l];
       // L2 prefetch of the next layer's routing-independent rows this CTA's warps will read
-      if (l + 1 < a.n_layers && lane == 0) {
+      // (phase-R item i belongs to CTA i % G), one lane per item
+      if (l + 1 < a.n_layers) {
         const FusedLayer& Ln = a.layer[l + 1];
         const int n_router = (Ln.topk_idx_in ? 0 : E) + 1;
         const int n_items = n_router + I / RPWg;
-        for (int it = blockIdx.x * kCons; it < min(n_items, (blockIdx.x + 1) * kCons); ++it) {
+        for (int it = blockIdx.x + G * lane; it < n_items; it += G * 32) {
           if (it < n_router) {
             const bool gate_row = (it == n_router - 1);
             const uint16_t* row = gate_row ? Ln.wsg : Ln.wr + (size_t)it * H;
@@ -397,7 +398,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
   // compute warps
   // =====================================================================================
   const int cw = warp;  // 0..14
-  const int gw = blockIdx.x * kCons + cw, NW = G * kCons;
+  const int NW = G * kCons;
   uint32_t q = 0;
   uint32_t nb = 0;  // grid barriers passed in this launch
   bool ok = true;
@@ -418,7 +419,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
     {
       const int n_router = (routed ? E : 0) + 1;
       const int n_items = n_router + I / RPWg;
-      for (int it = gw; it < n_items; it += NW) {
+      for (int it = blockIdx.x + G * cw; it < n_items; it += NW) {  // item i: CTA i % G
         if (it < n_router) {
           const bool gate_row = (it == n_router - 1);
           const int e = gate_row ? E : it;
