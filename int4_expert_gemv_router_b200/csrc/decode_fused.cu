@@ -52,20 +52,21 @@ __device__ __forceinline__ void bar_cons() { asm volatile("bar.sync 1, %0;" ::"n
 // bar_count only grows during a launch: barrier number b (0, 1, 2, ...) completes when it
 // reaches (b + 1) * nblocks, so a barrier costs one atomic and the polls.  grid_exit()
 // returns it to zero once every CTA has passed its last barrier.
+// The arrival is an acq_rel atomic and the polls are acquire loads: the CTA's writes before
+// the barrier (ordered before this thread's arrival by the CTA barrier that precedes it) are
+// visible to every CTA that has seen the count complete, with no separate fence.
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
 __device__ bool grid_barrier(Ctrl* c, uint32_t nblocks, uint32_t b) {
   const uint32_t target = (b + 1) * nblocks;
-  __threadfence();
-  const uint32_t arrived = atomicAdd(&c->bar_count, 1u) + 1;
-  if (arrived >= target) {
-    __threadfence();
-    return true;
-  }
+  const uint32_t arrived = atom_add_acq_rel(&c->bar_count, 1u) + 1;
+  if (arrived >= target) return true;
   const unsigned long long t0 = now_ns();
   for (uint32_t it = 0;; ++it) {
-    if (ld_acquire(&c->bar_count) >= target) {
-      __threadfence();
-      return true;
-    }
+    if (ld_acquire(&c->bar_count) >= target) return true;
     if ((it & 255u) == 255u && now_ns() - t0 > kWaitNs) {
       atomicOr(&c->err, kErrTimeout);
       return false;
