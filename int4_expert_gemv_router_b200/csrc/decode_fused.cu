@@ -210,6 +210,16 @@ __device__ __noinline__ void warp_topk(const double* lt, int E, int k, uint8_t* 
   }
 }
 
+// Rows per phase-G block: the CTAs' equal share of the rows in as few blocks of at most
+// RG rows as it takes, rounded up to the granule gG.
+__device__ __forceinline__ int gate_block_rows(int rows, int G, int RG, int gG) {
+  if (rows <= 0) return gG;
+  const int per_cta = (rows + G - 1) / G;
+  const int n_blocks = (per_cta + RG - 1) / RG;
+  const int br = (per_cta + n_blocks - 1) / n_blocks;
+  return max(gG, (br + gG - 1) / gG * gG);
+}
+
 template <int BITS, int H, int I, int TM>
 __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_constant__ FusedArgs a) {
   // ---- constants ----
@@ -301,12 +311,13 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
       if (*(volatile int*)&s_abort) break;
       const int act_n = s_act_n;
       // ---- phase G pieces ----
-      const int nGranG = act_n * I / gG;
-      const int f0 = (int)((long long)blockIdx.x * nGranG / G) * gG;
-      const int f1 = (int)((long long)(blockIdx.x + 1) * nGranG / G) * gG;
-      for (int f = f0; f < f1 && ok;) {
+      // blocks of BR rows dealt round-robin over the CTAs (block b on CTA b % G), so that at
+      // any moment the grid reads one contiguous stretch of the experts' rows; a block that
+      // crosses into the next expert is two stages
+      const int rows_g = act_n * I, BR = gate_block_rows(rows_g, G, RG, gG);
+      for (int b0 = blockIdx.x * BR, b1 = min(b0 + BR, rows_g), f = b0; f < rows_g && ok;) {
         const int u = f / I, r0 = f - u * I;
-        const int n = min(min(RG, f1 - f), I - r0);
+        const int n = min(b1 - f, I - r0);
         const int s = q % NS;
         if (!mbar_wait(&empty_bar[s], ((q / NS) & 1) ^ 1)) {
           ok = false;
@@ -336,6 +347,11 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
         __syncwarp();
         ++q;
         f += n;
+        if (f == b1) {
+          b0 += G * BR;
+          b1 = min(b0 + BR, rows_g);
+          f = b0;
+        }
       }
       // ---- phase D pieces: this CTA's down rows of every selected expert, then the shared one ----
       if (nJ > 0) {
@@ -636,13 +652,12 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
 
     // ---- phase G: routed gate/up + SwiGLU from the ring ----
     {
-      const int nGranG = act_n * I / gG;
-      const int f0 = (int)((long long)blockIdx.x * nGranG / G) * gG;
-      const int f1 = (int)((long long)(blockIdx.x + 1) * nGranG / G) * gG;
+      const int rows_g = act_n * I, BR = gate_block_rows(rows_g, G, RG, gG);
       const int sub = lane % NCLg, rsub = lane / NCLg;
-      for (int f = f0; f < f1;) {
+      int done = 0;  // rows of this CTA already processed
+      for (int b0 = blockIdx.x * BR, b1 = min(b0 + BR, rows_g), f = b0; f < rows_g;) {
         const int u = f / I, r0 = f - u * I;
-        const int n = min(min(RG, f1 - f), I - r0);
+        const int n = min(b1 - f, I - r0);
         const int s = q % NS;
         if (!mbar_wait(&full_bar[s], (q / NS) & 1)) {
           ok = false;
@@ -653,7 +668,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
         if (P_SLOT[u] >= 0) {
           const int pb = P_BEGIN[u], pe = P_BEGIN[u + 1];
           // row steps are dealt to warps round-robin over the CTA's whole row range
-          const int step0 = (f - f0) / RPWg;
+          const int step0 = done / RPWg;
           for (int step = (cw - step0 % kCons + kCons) % kCons; step < n / RPWg; step += kCons) {
             const int rl = step * RPWg + rsub;
             const uint8_t* gq = st + rl * ROWBg;
@@ -690,6 +705,12 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
         if (lane == 0) mbar_arrive(&empty_bar[s]);
         ++q;
         f += n;
+        done += n;
+        if (f == b1) {
+          b0 += G * BR;
+          b1 = min(b0 + BR, rows_g);
+          f = b0;
+        }
       }
     }
     bar_cons();
