@@ -296,10 +296,23 @@ __device__ __forceinline__ bool warp_aborted(const int* flag) {
   return __any_sync(0xffffffffu, *reinterpret_cast<const volatile int*>(flag) != 0);
 }
 
+// Bounded wait that sleeps between tries (32 ns doubling to 256 ns), so that a warp waiting
+// for its next stage leaves the issue slots to the warps that are converting one.
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* b, uint32_t parity) {
+  if (mbar_try_wait(b, parity)) return true;
+  const unsigned long long t0 = now_ns();
+  uint32_t ns = 32;
+  for (;;) {
+    __nanosleep(ns);
+    if (mbar_try_wait(b, parity)) return true;
+    if (now_ns() - t0 > kWaitNs) return false;
+    ns = ns < 256 ? 2 * ns : 256;
+  }
+}
 // Every lane of a warp waits, and all take the same branch afterwards (a lane whose wait
 // ran out would otherwise leave the others behind at the next __syncwarp).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Ctrl* c, int lane) {
-  const bool ok = __all_sync(0xffffffffu, mbar_wait_suspend(bar, parity) ? 1 : 0);
+  const bool ok = __all_sync(0xffffffffu, mbar_wait_backoff(bar, parity) ? 1 : 0);
   if (!ok && lane == 0) atomicOr(&c->err, kErrTimeout);
   return ok;
 }
