@@ -265,6 +265,8 @@ static moe_status prefill_forward(const moe_shape* shape, const void* x, int32_t
   p.h = reinterpret_cast<uint16_t*>(b + W.h);
   p.hs = reinterpret_cast<uint16_t*>(b + W.hs);
   p.xg = reinterpret_cast<uint16_t*>(b + W.xg);
+  p.xp = reinterpret_cast<uint16_t*>(b + W.xp);
+  p.perm = shape->bits == 4 ? 1 : 0;
   GemmArgs& g = p.g;
   g.H = H;
   g.I = I;

@@ -220,6 +220,7 @@ struct GemmArgs {
   const int* n_units;
   Ctrl* ctrl;
   int n_rows;           // weight rows per work unit (the MMA's N): 128 or 256
+  int perm;             // the gate/up epilogue writes h in k-octet order
   int sc_tma;           // 1: scales and biases arrive by TMA in chunks of 8 groups
   // TMA descriptors (filled by the launcher per GEMM): token rows (routed / shared
   // units), weight rows (router rows, or raw codes of the pool / of the shared blob), and
@@ -264,13 +265,15 @@ struct PrefillArgs {
   uint16_t* h;
   uint16_t* hs;
   uint16_t* xg;         // bf16 [T*k, H]: x rows in grouped pair order
+  uint16_t* xp;         // bf16 [T, H]: x for the shared expert's gate/up (k-octet order, int4)
+  int perm;             // int4: operands of the expert GEMMs in k-octet order (see prefill.cu)
   Ctrl* ctrl;
   GemmArgs g;           // shared GEMM arguments (units filled per launch)
 };
 
 struct PrefillLayout {
   size_t ctrl, xnorm, wnorm, logits, topk_idx, topk_w, gate, order, offsets, counts, chunk_cnt, units_rt,
-      units_gu, units_dn, n_units, acc, h, hs, xg, total;
+      units_gu, units_dn, n_units, acc, h, hs, xg, xp, total;
 };
 
 inline PrefillLayout make_prefill_layout(int T, int E, int k, int H, int I) {
@@ -303,6 +306,7 @@ inline PrefillLayout make_prefill_layout(int T, int E, int k, int H, int I) {
   W.h = take(2 * (size_t)T * k * I);
   W.hs = take(2 * (size_t)T * I);
   W.xg = take(2 * (size_t)T * k * H);
+  W.xp = take(2 * (size_t)T * H);
   W.total = (size_t)round_up((int64_t)pos, kAlign);
   return W;
 }

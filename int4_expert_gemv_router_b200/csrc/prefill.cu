@@ -15,7 +15,8 @@
 //                  stable counting sort of the (token, k) pairs by expert (per-chunk counts,
 //                  per-expert scans down the chunks, per-chunk stable placement) and the
 //                  list of GEMM work units (expert, row tile, token tile)
-//   k_permute      xg = the tokens' rows of x in grouped pair order
+//   k_permute      xg = the tokens' rows of x in grouped pair order (int4: in k-octet order,
+//                  and xp = x in that order for the shared expert; see dq8_int4_bf)
 //   k_gemm GATEUP  per unit: [gate; up] rows of one expert (dequantised to bf16 in shared
 //                  memory) x the expert's rows of xg, SwiGLU in the epilogue -> h
 //   k_gemm DOWN    per unit: down rows x the expert's h, weighted scatter-add into an fp32
@@ -256,7 +257,11 @@ __device__ __forceinline__ void w_lane_map(int at, int& m, int& half) {
 // 8 int4 codes (one word, element j at bits 4j) -> 8 bf16 values round(s*q + b), on packed
 // bf16 pairs.  OR-ing a code into the low mantissa bits of bf16 128.0 (0x4300) gives the
 // exact value 128 + q; subtracting 128 is exact, and one fused multiply-add rounds s*q + b
-// once.  Pairs come out as (q0, q4), (q1, q5), ... and are re-paired with byte permutes.
+// once.  The pairs come out as (q0, q4), (q1, q5), (q2, q6), (q3, q7) and are stored in that
+// order: the int4 expert GEMMs take both operands with every k-octet in the order
+// 0, 4, 1, 5, 2, 6, 3, 7 (the token rows are written so by k_permute and by the gate/up
+// epilogue, see perm_octet), which leaves each dot product unchanged and saves re-pairing
+// the values with byte permutes here.
 __device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
   asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
@@ -276,8 +281,13 @@ __device__ __forceinline__ uint4 dq8_int4_bf(uint32_t w, uint32_t s2, uint32_t b
     const uint32_t p = ((w >> (4 * i)) & kMask) | kBias;  // (128 + q_i, 128 + q_{i+4})
     r[i] = bf2_fma(bf2_fma(p, kOne, kNeg128), s2, b2);
   }
-  return make_uint4(prmt(r[0], r[1], 0x5410u), prmt(r[2], r[3], 0x5410u), prmt(r[0], r[1], 0x7632u),
-                    prmt(r[2], r[3], 0x7632u));
+  return make_uint4(r[0], r[1], r[2], r[3]);
+}
+// Eight consecutive bf16 values (x0 .. x7) -> the k-octet order of the int4 GEMM operands:
+// (x0, x4), (x1, x5), (x2, x6), (x3, x7).
+__device__ __forceinline__ uint4 perm_octet(const uint4& v) {
+  return make_uint4(prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u), prmt(v.y, v.w, 0x5410u),
+                    prmt(v.y, v.w, 0x7632u));
 }
 
 __device__ __forceinline__ int core_off(int row, int koct) {  // byte offset in a stage tile
@@ -684,8 +694,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
               const float h1 = __fdividef(gv[2 * i + 1], 1.0f + __expf(-gv[2 * i + 1])) * uv[2 * i + 1];
               pk[i] = pack_bf16(h0, h1);
             }
-            reinterpret_cast<uint4*>(hrow + c0)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            reinterpret_cast<uint4*>(hrow + c0)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            uint4 o0 = make_uint4(pk[0], pk[1], pk[2], pk[3]), o1 = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            if (a.perm) {  // h is the down GEMM's token operand: k-octet order
+              o0 = perm_octet(o0);
+              o1 = perm_octet(o1);
+            }
+            reinterpret_cast<uint4*>(hrow + c0)[0] = o0;
+            reinterpret_cast<uint4*>(hrow + c0)[1] = o1;
           }
         }
       } else if (MODE == kModeDown) {
@@ -1111,11 +1126,25 @@ __global__ void __launch_bounds__(kGroupThreads) k_gplace(PrefillArgs a) {
 // xg[p] = x[order[p] / k] for every grouped pair position p < offsets[E]: the routed gate/up
 // GEMM then reads each expert's tokens as consecutive rows.  One warp per row.
 __global__ void __launch_bounds__(256) k_permute(PrefillArgs a) {
+  // warps [0, T*k): xg row p (valid pairs only); with perm, warps [T*k, T*k + T): xp row t
   const int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (p >= a.offsets[a.E]) return;
-  const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)(__ldg(a.order + p) / a.k) * a.H);
-  uint4* dst = reinterpret_cast<uint4*>(a.xg + (size_t)p * a.H);
-  for (int i = lane; i < a.H / 8; i += 32) dst[i] = __ldg(src + i);
+  const int n_pairs = a.T * a.k;
+  const uint4* src;
+  uint4* dst;
+  if (p < n_pairs) {
+    if (p >= a.offsets[a.E]) return;
+    src = reinterpret_cast<const uint4*>(a.x + (size_t)(__ldg(a.order + p) / a.k) * a.H);
+    dst = reinterpret_cast<uint4*>(a.xg + (size_t)p * a.H);
+  } else {
+    if (!a.perm || p >= n_pairs + a.T) return;
+    src = reinterpret_cast<const uint4*>(a.x + (size_t)(p - n_pairs) * a.H);
+    dst = reinterpret_cast<uint4*>(a.xp + (size_t)(p - n_pairs) * a.H);
+  }
+  if (a.perm) {
+    for (int i = lane; i < a.H / 8; i += 32) dst[i] = perm_octet(__ldg(src + i));
+  } else {
+    for (int i = lane; i < a.H / 8; i += 32) dst[i] = __ldg(src + i);
+  }
 }
 
 __global__ void k_finalize(const float* acc, const uint16_t* residual, uint16_t* out, size_t n) {
@@ -1265,7 +1294,7 @@ cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
   // grouping and work units
   prof_mark(1, false, s);
   if ((e = launch_group(p, s)) != cudaSuccess) return e;
-  k_permute<<<(unsigned)(((size_t)T * p.k * 32 + 255) / 256), 256, 0, s>>>(p);
+  k_permute<<<(unsigned)((((size_t)T * p.k + (p.perm ? T : 0)) * 32 + 255) / 256), 256, 0, s>>>(p);
   prof_mark(1, true, s);
   // gate/up + SwiGLU, then down + scatter
   {
@@ -1283,7 +1312,8 @@ cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
       if ((e = map_scales(&g.map_sc_shared, g.shared, 1, g.L, 3, 4, I, H / kGroup, nI)) != cudaSuccess) return e;
     }
     if ((e = map_bf16(&g.map_tok, p.xg, (uint64_t)T * p.k, H, H, kTRows)) != cudaSuccess) return e;
-    if ((e = map_bf16(&g.map_tok2, p.x, T, H, H, kTRows)) != cudaSuccess) return e;
+    if ((e = map_bf16(&g.map_tok2, p.perm ? p.xp : p.x, T, H, H, kTRows)) != cudaSuccess) return e;
+    g.perm = p.perm;
     prof_mark(2, false, s);
     if ((e = (bits == 4 ? launch_gemm<4, kModeGateUp>(g, n_sm, s) : launch_gemm<8, kModeGateUp>(g, n_sm, s))) !=
         cudaSuccess)
