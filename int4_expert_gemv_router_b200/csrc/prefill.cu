@@ -58,7 +58,8 @@ constexpr int kWBytes = kNMax * kKC * 2;  // 32 KB: weight tile of a stage (room
 // warp roles
 constexpr int kTLoadWarp = 1;             // token tiles by TMA
 constexpr int kWLoadWarp = 2;             // lane 0: raw codes + scale chunks (or router rows) by TMA
-constexpr int kDWarp0 = 3, kDWarps = 16;  // dequantisation: 256 weight rows x 2 column halves
+constexpr int kDWarp0 = 3, kDWarps = 16;  // dequantisation: two groups of 8 warps, 256 weight rows each
+constexpr int kDGroup = kDWarps / 2;      // warps per dequantising group (one stage each)
 constexpr int kEWarp0 = 19, kEWarps = 4;  // epilogue
 constexpr int kGemmThreads = (kEWarp0 + kEWarps) * 32;  // 736
 constexpr int kSBO = (kKC / 8) * 128;     // 1024: 8-row group stride of a no-swizzle K-major tile
@@ -245,15 +246,6 @@ __device__ __forceinline__ uint4 dq8_int8(uint32_t w0, uint32_t w1, float s, flo
                     dq2(w1 & 0xFFu, w1 & 0xFF00u, s, s8, b), dq2(h1 & 0xFFu, h1 & 0xFF00u, s, s8, b));
 }
 
-// Dequantising thread -> (weight row m, column half).  Lanes l and l ^ 8 share a row; the
-// eight lanes of each quarter-warp take eight consecutive rows of one half, so that their
-// 16-byte stores of a k-octet fill 128 contiguous bytes of the tile (no bank conflicts).
-__device__ __forceinline__ void w_lane_map(int at, int& m, int& half) {
-  const int w = at >> 5, l = at & 31;
-  m = w * 16 + (l & 7) + ((l >> 4) << 3);
-  half = (l >> 3) & 1;
-}
-
 // 8 int4 codes (one word, element j at bits 4j) -> 8 bf16 values round(s*q + b), on packed
 // bf16 pairs.  OR-ing a code into the low mantissa bits of bf16 128.0 (0x4300) gives the
 // exact value 128 + q; subtracting 128 is exact, and one fused multiply-add rounds s*q + b
@@ -346,8 +338,8 @@ template <int BITS, int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant__ GemmArgs a) {
   constexpr int kRawB = Raw<BITS>::kBytes, kRowB = Raw<BITS>::kRowBytes;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full[kStageMax], empty[kStageMax], raw_full[kRawMax], raw_empty[kRawMax], acc_full[2],
-      acc_empty[2], drain;
+  __shared__ __align__(8) uint64_t full[kStageMax], empty[kStageMax], raw_full[kRawMax], raw_empty[kRawMax],
+      chunk_full[2], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -367,14 +359,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
   if (tid == 0) {
     for (int s = 0; s < P.n_st; ++s) {
       // full: the token loader's expect-tx arrival, plus the weight loader's (router rows by
-      // TMA) or one arrival per dequantising warp; empty: the MMA's commit
-      mbar_init(&full[s], MODE == kModeRouter ? 2 : kDWarps + 1);
+      // TMA) or one arrival per warp of the dequantising group that owns the stage; empty: the
+      // MMA's commit
+      mbar_init(&full[s], MODE == kModeRouter ? 2 : kDGroup + 1);
       mbar_init(&empty[s], 1);
     }
     for (int s = 0; s < P.n_raw; ++s) {
       mbar_init(&raw_full[s], 1);
-      mbar_init(&raw_empty[s], kDWarps);
+      mbar_init(&raw_empty[s], kDGroup);
     }
+    for (int c = 0; c < 2; ++c) mbar_init(&chunk_full[c], 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kEWarps);
@@ -525,14 +519,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
               break;
             }
             const bool chunk = a.sc_tma && (kc % kChunk) == 0;
-            mbar_expect_tx(&raw_full[rr.s], raw_bytes + (chunk ? chunk_bytes : 0u));
+            mbar_expect_tx(&raw_full[rr.s], raw_bytes);
             const uint32_t dst = smem_base + P.raw + rr.s * kRawB;
             if (MODE == kModeGateUp)  // [gate; up] x NR/2 rows of the row tile
               tma_4d(dst, mw, kc * kRowB, row0, 0, slot, &raw_full[rr.s]);
             else
               tma_3d(dst, mw, kc * kRowB, row0, slot, &raw_full[rr.s]);
             if (chunk) {  // [scale, bias] (x [gate, up]) x rows x 8 groups
-              tma_4d(smem_base + P.sc + (chunks & 1) * kChunkBytes, ms, kc, row0, 0, slot, &raw_full[rr.s]);
+              // its own barrier: the two dequantising groups read it from different stages
+              mbar_expect_tx(&chunk_full[chunks & 1], chunk_bytes);
+              tma_4d(smem_base + P.sc + (chunks & 1) * kChunkBytes, ms, kc, row0, 0, slot, &chunk_full[chunks & 1]);
               ++chunks;
             }
           }
@@ -541,19 +537,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       }
       if (stop) s_abort = 1;
       drain_ring(MODE == kModeRouter ? full : raw_full, MODE == kModeRouter ? P.n_st : P.n_raw, issued, a.ctrl);
+      if (MODE != kModeRouter) drain_ring(chunk_full, 2, chunks, a.ctrl);
     }
     __syncwarp();
   } else if (warp >= kDWarp0 && warp < kDWarp0 + kDWarps && MODE != kModeRouter) {
     // ------------------------------ dequantisation ------------------------------
-    // Thread (m, half) turns 32 codes (columns 32*half .. +31 of the stage) of weight row m
-    // into bf16 in the weight tile.  Scales and biases come from the stage's scale chunk
-    // (every 8 stages, by TMA) or, for rows of fewer than 8 groups, from global memory.
-    const int at = tid - kDWarp0 * 32;  // 0..511
-    int m, half;                        // weight row 0..255, column half
-    w_lane_map(at, m, half);
+    // Two groups of eight warps take alternate stages (group 0 the even ones), so that two
+    // stages are converted at once.  In its group, thread m turns the 64 codes of weight row m
+    // into bf16 in the weight tile (eight consecutive rows per quarter-warp: each 16-byte store
+    // of a k-octet fills 128 contiguous bytes, no bank conflicts).  Scales and biases come
+    // from the stage's scale chunk (every 8 stages, by TMA) or, for rows of fewer than 8
+    // groups, from global memory.
+    const int grp = (warp - kDWarp0) / kDGroup;
+    const int m = ((warp - kDWarp0) % kDGroup) * 32 + lane;  // weight row 0..255
     const bool active = m < NR;
     const int NG = K / kGroup;  // groups (= stages) per row
-    const uint32_t raw_off = (uint32_t)m * kRowB + half * (kRowB / 2);
+    const uint32_t raw_off = (uint32_t)m * kRowB;
     // position of row m's scale and bias in a chunk: [scale, bias](x [gate, up]) x rows x 8
     const int sec_rows = MODE == kModeGateUp ? NR / 2 : NR;
     const int sec = MODE == kModeGateUp && m >= NR / 2 ? 2 : 0;
@@ -585,31 +584,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       }
       bool stop = false;
       for (int kc = 0; kc < nK; ++kc, ++g, ra.next(), rr.next()) {
+        if ((g & 1) != grp) continue;  // the other group's stage
         if (!warp_wait(&raw_full[rr.s], rr.ph, a.ctrl, lane)) {
           stop = true;
           break;
         }
-        uint32_t w[kRowB / 8];  // this thread's 32 codes
+        uint32_t w[kRowB / 4];  // this thread's 64 codes
         uint32_t sbits = 0, bbits = 0;
         if (active) {
           const uint8_t* rp = smem + P.raw + rr.s * kRawB + raw_off;
-          if (BITS == 4) {
-            const uint4 v = *reinterpret_cast<const uint4*>(rp);
-            w[0] = v.x;
-            w[1] = v.y;
-            w[2] = v.z;
-            w[3] = v.w;
-          } else {
 #pragma unroll
-            for (int o = 0; o < 2; ++o) {
-              const uint4 v = *reinterpret_cast<const uint4*>(rp + o * 16);
-              w[(4 * o + 0) % (kRowB / 8)] = v.x;
-              w[(4 * o + 1) % (kRowB / 8)] = v.y;
-              w[(4 * o + 2) % (kRowB / 8)] = v.z;
-              w[(4 * o + 3) % (kRowB / 8)] = v.w;
-            }
+          for (int o = 0; o < kRowB / 16; ++o) {
+            const uint4 v = *reinterpret_cast<const uint4*>(rp + o * 16);
+            w[4 * o + 0] = v.x;
+            w[4 * o + 1] = v.y;
+            w[4 * o + 2] = v.z;
+            w[4 * o + 3] = v.w;
           }
           if (a.sc_tma) {
+            // chunk g / 8 sits in slot (g / 8) & 1, on that slot's ((g / 8) >> 1)-th fill
+            if (!mbar_wait_backoff(&chunk_full[(g / kChunk) & 1], ((g / kChunk) >> 1) & 1)) {
+              atomicOr(&a.ctrl->err, kErrTimeout);
+              s_abort = 1;
+            }
             const uint16_t* ch = reinterpret_cast<const uint16_t*>(smem + P.sc + ((g / kChunk) & 1) * kChunkBytes);
             sbits = ch[c_s + kc % kChunk];
             bbits = ch[c_b + kc % kChunk];
@@ -629,14 +626,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
           if (BITS == 4) {
             const uint32_t s2 = sbits | (sbits << 16), b2 = bbits | (bbits << 16);
 #pragma unroll
-            for (int o = 0; o < 4; ++o)  // 4 k-octets of 8 values = this thread's 32 columns
-              *reinterpret_cast<uint4*>(w_tile + core_off(m, half * 4 + o)) = dq8_int4_bf(w[o], s2, b2);
+            for (int o = 0; o < 8; ++o)  // 8 k-octets of 8 values = the stage's 64 columns
+              *reinterpret_cast<uint4*>(w_tile + core_off(m, o)) = dq8_int4_bf(w[o], s2, b2);
           } else {
             const float sv = __uint_as_float(sbits << 16), bv = __uint_as_float(bbits << 16);
 #pragma unroll
-            for (int o = 0; o < 4; ++o)
-              *reinterpret_cast<uint4*>(w_tile + core_off(m, half * 4 + o)) =
-                  dq8_int8(w[(2 * o) % (kRowB / 8)], w[(2 * o + 1) % (kRowB / 8)], sv, bv);
+            for (int o = 0; o < 8; ++o)
+              *reinterpret_cast<uint4*>(w_tile + core_off(m, o)) = dq8_int8(w[2 * o], w[2 * o + 1], sv, bv);
           }
         }
         proxy_fence();
