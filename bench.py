@@ -48,7 +48,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC_PER_LAYER = {("k_fused_decode", "decode80b", 1): 21_743_360}
 # DRAM traffic per launch of the prefill gate/up GEMM on the prefill workload (full-size capture,
 # profiles/k_gemm_gateup_prefill_full.md).  Must be re-captured whenever the kernel changes.
-NCU_TRAFFIC_PREFILL_GATEUP = {("prefill", 4096): 832_873_216}
+NCU_TRAFFIC_PREFILL_GATEUP = {("prefill", 4096): 830_150_912}
 
 
 # --------------------------------------------------------------------------------------
