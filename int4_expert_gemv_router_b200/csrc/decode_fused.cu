@@ -7,14 +7,16 @@
 //            and the shared expert's gate/up + SwiGLU rows, dealt round-robin over the CTAs
 //            and their compute warps; activations staged once per CTA in shared memory.
 //   -- grid barrier --
-//   phase T  every CTA selects the top-k per token from the logits (threshold + warp
-//            bitonic sort; ties to the lower id), forms the softmax weights and the shared
-//            gate, and groups the (token, k) pairs by expert.  CTA 0 writes the top-k.
-//   phase G  the routed experts' gate/up rows, split evenly over CTAs, stream into a shared-
-//            memory ring through cp.async.bulk (one elected thread of warp 15, mbarrier
-//            transaction counts) and are reduced to h = silu(Wg x) * (Wu x); right behind
-//            them the same warp streams this CTA's rows of every selected expert's down
-//            matrix (and the shared expert's), so they are on chip before they are needed.
+//   phase T  every CTA selects the top-k per token from the logits (the k-th best lane
+//            maximum as a threshold, then ranking of the keys above it; ties to the lower
+//            id), forms the softmax weights and the shared gate, and groups the (token, k)
+//            pairs by expert.  CTA 0 writes the top-k.
+//   phase G  the routed experts' gate/up rows, in blocks dealt round-robin over the CTAs,
+//            stream into a shared-memory ring through cp.async.bulk (issued by the lanes of
+//            warp 15, mbarrier transaction counts) and are reduced to h = silu(Wg x) * (Wu x);
+//            right behind them the same warp streams this CTA's rows of every selected
+//            expert's down matrix (and the shared expert's), so they are on chip before they
+//            are needed.
 //   -- grid barrier --
 //   phase D  each CTA owns a slice of output rows: per expert one warp multiplies its staged
 //            down rows with the expert's h (registers), the per-pair partial sums meet in
