@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W]
                     [--workload decode80b|decode35b|prefill|pool_int4|pool_int8]
-                    [--tokens T] [--impl ours|reference] [--policy lfu_recency|lru|lfu] [--slots S]
+                    [--tokens T] [--impl ours|reference] [--policy lfu_recency|lru|lfu] [--slots S] [--overlap]
 
 Default workload: the 80B-like decode stack -- hidden 2048, 512 experts, top-10,
 intermediate 512, shared expert 512, int4 group 64, one token per step through 48
@@ -576,6 +576,7 @@ def run_pool(args, w, device, rank, total_steps=1024):
     table = torch.empty(w.n_experts, dtype=torch.int32, device=device)
     pool = abi.moe_pool_create(shape, w.n_slots, host_blobs, dev_pool, table)
     abi.moe_pool_set_policy(pool, args.policy)
+    abi.moe_pool_set_overlap(pool, args.overlap)
     T = 1
     xs = torch.stack([synth.activations(w, rank_step_seed(rank, s), tokens=T, device=device) for s in range(n_total)])
     out = torch.empty(T, w.hidden, dtype=torch.bfloat16, device=device)
@@ -641,6 +642,7 @@ def pool_line(args, w, r, n_gpus):
                    "steps_total": r["n_total"], "tokens_per_step": 1,
                    "policy": {"lfu_recency": "LFU + recency", "lru": "LRU", "lfu": "LFU"}[args.policy],
                    "miss_path": "pinned host -> cudaMemcpyAsync on a side stream",
+                   "overlap": bool(args.overlap),
                    "timing": "events around the timed steps; each step waits on the host for the ids"},
         "pool": {"hit_rate_all_steps": round(r["hit_rate_all"], 4), "hit_rate_timed": round(r["hit_rate_timed"], 4),
                  "stats": r["stats"], "h2d_bytes_timed": r["h2d_timed"],
@@ -720,6 +722,8 @@ def parse(argv=None):
     ap.add_argument("--policy", choices=["lfu_recency", "lru", "lfu"], default="lfu_recency",
                     help="pool workloads: eviction policy (the pages' LFU + recency by default)")
     ap.add_argument("--slots", type=int, default=None, help="pool workloads: number of slots (default 128)")
+    ap.add_argument("--overlap", action="store_true",
+                    help="pool workloads: the forward starts while the step's misses are still being copied")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the stack depth (profiling of a small case only; not a bench value)")
     return ap.parse_args(argv)

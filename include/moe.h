@@ -292,6 +292,22 @@ MOE_API moe_status moe_expert_pool_load(moe_pool* pool, const int32_t* topk_idx,
 enum { MOE_POOL_LFU_RECENCY = 0, MOE_POOL_LRU = 1, MOE_POOL_LFU = 2 };
 MOE_API moe_status moe_pool_set_policy(moe_pool* pool, int32_t policy);
 
+/*
+ * moe_pool_set_overlap -- overlap mode of the next loads (0: off, the default).  Off, the
+ * caller's stream waits until the step's misses have landed, then the layer forward runs.
+ * On, moe_expert_pool_load uploads the slot table with every miss of the step marked
+ * pending (-2), the caller's stream waits for that upload only, and each miss's blob copy is
+ * followed on the side stream by a copy of its slot over the pending entry: the fused decode
+ * kernel (moe_layer_forward / moe_stack_forward with T <= 8) starts at once, computes with the
+ * resident experts and waits, per expert, for a pending entry to settle before it streams
+ * that blob (the NEXT item of the Swiftlet pages' streaming design: compute on hits while the
+ * misses are in flight).  Results are bit-identical to overlap off.  While overlap is on, the
+ * slot table may hold -2 entries between a load and the end of the forward that follows it:
+ * run that forward before the next load, and only the fused decode path may read the table.
+ * MOE_ERR_UNSUPPORTED for shapes without a fused decode kernel.  Host-side only.
+ */
+MOE_API moe_status moe_pool_set_overlap(moe_pool* pool, int32_t on);
+
 /* moe_pool_stats -- counters since creation (host struct). */
 MOE_API moe_status moe_pool_stats(const moe_pool* pool, moe_pool_stats_t* stats);
 

@@ -72,6 +72,7 @@ _SIGS = {
     "moe_pool_slot_table": (ctypes.c_int, [_P, _P, _P]),
     "moe_pool_inject_copy_failure": (ctypes.c_int, [_P, _I64]),
     "moe_pool_set_policy": (ctypes.c_int, [_P, ctypes.c_int32]),
+    "moe_pool_set_overlap": (ctypes.c_int, [_P, ctypes.c_int32]),
     "moe_pool_destroy": (None, [_P]),
     "moe_profile_events": (ctypes.c_int, [_P, _I32]),
     "moe_last_error": (ctypes.c_char_p, []),
@@ -234,6 +235,11 @@ POOL_POLICIES = {"lfu_recency": 0, "lru": 1, "lfu": 2}
 def moe_pool_set_policy(pool: int, policy: str):
     """Eviction policy of the pool's next loads: "lfu_recency" (default), "lru" or "lfu"."""
     _check(lib().moe_pool_set_policy(pool, POOL_POLICIES[policy]))
+
+
+def moe_pool_set_overlap(pool: int, on: bool):
+    """Overlap mode: the forward starts before the step's misses have landed (see moe.h)."""
+    _check(lib().moe_pool_set_overlap(pool, 1 if on else 0))
 
 
 def moe_pool_inject_copy_failure(pool: int, nth: int):

@@ -14,6 +14,10 @@ constexpr int kMaxDecodeT = 8;  // tokens per call on the GEMV (decode) path
 constexpr int kMaxTopK = 32;
 constexpr int kMaxExperts = 1024;
 
+// Slot-table entry of an expert whose blob is still being copied into its slot (a pool in
+// overlap mode); the copy stream overwrites it with the slot once the blob has landed.
+constexpr int32_t kSlotPending = -2;
+
 // Device error-word bits (mirrors MOE_DEVERR_* in include/moe.h).
 constexpr uint32_t kErrBadExpert = 0x1u;
 constexpr uint32_t kErrBadSlot = 0x2u;

@@ -285,6 +285,34 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
   if (warp == kProd) {
     uint32_t q = 0;  // stage sequence number, shared convention with the compute warps
     bool ok = true;
+    // The slot of distinct expert u of layer Lc.  An entry that was pending when phase X read
+    // the table (the blob was still being copied) is polled until the copy stream has written
+    // the slot; the result goes back to the plan, where the compute warps read it after the
+    // stage's full barrier.  Whole warp; bounded (-1 and MOE_DEVERR_TIMEOUT after kWaitNs).
+    const auto slot_of_unit = [&](const FusedLayer& L, int u) {
+      int v = P_SLOT[u];
+      if (v != kSlotPending) return v;
+      if (lane == 0) {
+        const int* entry = L.slot_table + P_ACTE[u];
+        const unsigned long long t0 = now_ns();
+        uint32_t ns = 64;
+        for (;;) {
+          v = ld_acquire_s32(entry);
+          if (v != kSlotPending) break;
+          if (now_ns() - t0 > kWaitNs) {
+            atomicOr(&a.ctrl->err, kErrTimeout);
+            v = -1;
+            break;
+          }
+          __nanosleep(ns);
+          ns = ns < 1024 ? 2 * ns : 1024;
+        }
+        if (v != -1 && (v < 0 || v >= L.n_slots)) v = -1;
+        if (v < 0) atomicOr(&a.ctrl->err, kErrBadSlot);
+        P_SLOT[u] = v;
+      }
+      return __shfl_sync(0xffffffffu, v, 0);
+    };
     for (int l = 0; l < a.n_layers && ok; ++l) {
       const FusedLayer& Lc = a.layer[l];
       // L2 prefetch of the next layer's routing-independent rows this CTA's warps will read
@@ -329,7 +357,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
           // lane 0 announces the bytes, then lanes 0..5 issue the stage's six copies at once
           // (gate codes, up codes, then the four scale/bias sections)
           uint8_t* st = ring + (size_t)s * SB;
-          const int slot = P_SLOT[u];
+          const int slot = slot_of_unit(Lc, u);
           if (lane == 0) {
             if (slot < 0)
               mbar_arrive(&full_bar[s]);
@@ -357,6 +385,8 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
       }
       // ---- phase D pieces: this CTA's down rows of every selected expert, then the shared one ----
       if (nJ > 0) {
+        for (int u = 0; u < act_n; ++u) slot_of_unit(Lc, u);  // every pending slot settled
+        __syncwarp();
         const int per_stage = SB / (nJ * ROWD_BYTES);
         for (int u = 0; u <= act_n && ok;) {
           const int cnt = min(per_stage, act_n + 1 - u);
@@ -576,7 +606,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
               P_ACTE[before] = key;
               P_BEGIN[before] = before;
               const int slot = S_SLOT[key];
-              const bool sok = slot >= 0 && slot < Lc.n_slots;
+              const bool sok = (slot >= 0 && slot < Lc.n_slots) || slot == kSlotPending;
               if (!sok) atomicOr(&a.ctrl->err, kErrBadSlot);
               P_SLOT[before] = sok ? slot : -1;
             }
@@ -631,7 +661,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
           P_ACTE[act] = ki;
           P_BEGIN[act] = before;
           const int slot = S_SLOT[ki];
-          const bool sok = slot >= 0 && slot < Lc.n_slots;
+          const bool sok = (slot >= 0 && slot < Lc.n_slots) || slot == kSlotPending;
           if (!sok) atomicOr(&a.ctrl->err, kErrBadSlot);
           P_SLOT[act] = sok ? slot : -1;
         }

@@ -17,6 +17,7 @@
 #include "../../include/moe.h"
 #include "common.cuh"
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstring>
@@ -30,6 +31,24 @@ moe_status check_shape(const moe_shape* s);
 }  // namespace moe
 
 using namespace moe;
+
+namespace {
+// cuStreamWriteValue32 through the runtime's driver entry point (the library does not link
+// libcuda): a 4-byte write done by the stream itself once its earlier work has finished,
+// far cheaper than a 4-byte host-to-device copy.  Null if the driver does not offer it.
+using WriteValue32Fn = CUresult (*)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
+WriteValue32Fn write_value32_fn() {
+  static WriteValue32Fn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuStreamWriteValue32", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (WriteValue32Fn) nullptr;
+    return reinterpret_cast<WriteValue32Fn>(p);
+  }();
+  return fn;
+}
+}  // namespace
 
 struct moe_pool {
   moe_shape shape;
@@ -46,12 +65,14 @@ struct moe_pool {
   int64_t step_no = 0;
   moe_pool_stats_t stats{};
   int32_t policy = MOE_POOL_LFU_RECENCY;
+  bool overlap = false;            // forward may start before the misses have landed
   int64_t fail_at = -1;            // test hook: copies until an injected failure
   cudaStream_t side = nullptr;
   cudaEvent_t ready = nullptr;     // slot table + blobs of the last step are on the device
   bool ready_recorded = false;
   int32_t* h_ids = nullptr;        // pinned [kMaxDecodeT * kMaxTopK]
   int32_t* h_table = nullptr;      // pinned [E]
+  int32_t* h_final = nullptr;      // pinned [E]: the slot an overlap-mode miss resolves to
 };
 
 extern "C" {
@@ -91,7 +112,8 @@ moe_status moe_pool_create(const moe_shape* shape, int32_t n_slots, const uint8_
       (e = cudaEventCreateWithFlags(&p->ready, cudaEventDisableTiming)) != cudaSuccess ||
       (e = cudaHostAlloc((void**)&p->h_ids, sizeof(int32_t) * kMaxDecodeT * kMaxTopK, cudaHostAllocDefault)) !=
           cudaSuccess ||
-      (e = cudaHostAlloc((void**)&p->h_table, sizeof(int32_t) * E, cudaHostAllocDefault)) != cudaSuccess) {
+      (e = cudaHostAlloc((void**)&p->h_table, sizeof(int32_t) * E, cudaHostAllocDefault)) != cudaSuccess ||
+      (e = cudaHostAlloc((void**)&p->h_final, sizeof(int32_t) * E, cudaHostAllocDefault)) != cudaSuccess) {
     moe_pool_destroy(p);
     return cuda_fail(e, "pool create");
   }
@@ -119,8 +141,10 @@ moe_status moe_expert_pool_load(moe_pool* p, const int32_t* topk_idx, int32_t T,
   cudaError_t e = cudaMemcpyAsync(p->h_ids, topk_idx, sizeof(int32_t) * n, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "top-k read-back");
-  // The previous step's table upload reads h_table: let it finish before editing it.
+  // The previous step's table upload reads h_table (and, in overlap mode, its per-miss entry
+  // copies read h_final): let them finish before editing either.
   if (p->ready_recorded && (e = cudaEventSynchronize(p->ready)) != cudaSuccess) return cuda_fail(e, "pool event");
+  if (p->overlap && (e = cudaStreamSynchronize(p->side)) != cudaSuccess) return cuda_fail(e, "pool side stream");
   // distinct ids in first-appearance order
   std::vector<int32_t> uniq;
   uniq.reserve(n);
@@ -142,6 +166,10 @@ moe_status moe_expert_pool_load(moe_pool* p, const int32_t* topk_idx, int32_t T,
   }
   const int64_t now = p->step_no;
   moe_status result = MOE_OK;
+  struct Load {
+    int32_t id, slot;
+  };
+  std::vector<Load> loads;  // overlap mode: the misses, copied after the table upload
   for (int32_t id : uniq) {
     p->stats.lookups++;
     const int32_t sl = p->slot_of[id];
@@ -190,9 +218,13 @@ moe_status moe_expert_pool_load(moe_pool* p, const int32_t* topk_idx, int32_t T,
       p->fail_at = -1;
     } else {
       if (p->fail_at > 0) p->fail_at--;
-      e = cudaMemcpyAsync(p->dev_pool + (int64_t)victim * p->stride, p->host_blobs + (int64_t)id * p->stride,
-                          (size_t)p->stride, cudaMemcpyHostToDevice, p->side);
-      failed = (e != cudaSuccess);
+      if (p->overlap) {
+        loads.push_back({id, victim});  // copied after the table upload, below
+      } else {
+        e = cudaMemcpyAsync(p->dev_pool + (int64_t)victim * p->stride, p->host_blobs + (int64_t)id * p->stride,
+                            (size_t)p->stride, cudaMemcpyHostToDevice, p->side);
+        failed = (e != cudaSuccess);
+      }
     }
     if (failed) {
       // slot stays empty; the expert stays non-resident
@@ -208,11 +240,38 @@ moe_status moe_expert_pool_load(moe_pool* p, const int32_t* topk_idx, int32_t T,
   }
   for (int32_t u : uniq) p->needed[u] = 0;
   for (int i = 0; i < E; ++i) p->h_table[i] = p->slot_of[i];
+  // Overlap mode: the table goes up first with this step's misses marked pending, and the
+  // caller's stream waits for that upload only.  Each miss's blob copy is then followed on
+  // the side stream by a 4-byte copy of its slot over the pending entry; the fused decode
+  // kernel waits for that entry before it streams the expert.
+  for (const Load& ld : loads) {
+    p->h_table[ld.id] = kSlotPending;
+    p->h_final[ld.id] = ld.slot;
+  }
   e = cudaMemcpyAsync(p->dev_slot_table, p->h_table, sizeof(int32_t) * E, cudaMemcpyHostToDevice, p->side);
   if (e == cudaSuccess) e = cudaEventRecord(p->ready, p->side);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s, p->ready, 0);
   if (e != cudaSuccess) return cuda_fail(e, "slot table upload");
   p->ready_recorded = true;
+  for (const Load& ld : loads) {
+    e = cudaMemcpyAsync(p->dev_pool + (int64_t)ld.slot * p->stride, p->host_blobs + (int64_t)ld.id * p->stride,
+                        (size_t)p->stride, cudaMemcpyHostToDevice, p->side);
+    if (e != cudaSuccess) {
+      // the entry must still be settled, or the kernel would wait for it: not resident
+      result = cuda_fail(e, "blob copy");
+      p->h_final[ld.id] = -1;
+      p->slot_of[ld.id] = -1;
+      p->expert_in[ld.slot] = -1;
+      p->stats.h2d_bytes -= p->stride;
+    }
+    const WriteValue32Fn wv = write_value32_fn();
+    if (!wv || wv(p->side, (CUdeviceptr)(p->dev_slot_table + ld.id), (cuuint32_t)p->h_final[ld.id], 0) !=
+                   CUDA_SUCCESS) {
+      e = cudaMemcpyAsync(p->dev_slot_table + ld.id, p->h_final + ld.id, sizeof(int32_t), cudaMemcpyHostToDevice,
+                          p->side);
+      if (e != cudaSuccess) return cuda_fail(e, "slot table entry");
+    }
+  }
   p->step_no++;
   if (result == MOE_OK) p->stats.steps++;
   return result;
@@ -239,6 +298,14 @@ moe_status moe_pool_set_policy(moe_pool* p, int32_t policy) {
   return MOE_OK;
 }
 
+moe_status moe_pool_set_overlap(moe_pool* p, int32_t on) {
+  if (!p) return set_error(MOE_ERR_INVALID, "pool is NULL");
+  if (on && !fused_shape_supported(p->shape.hidden, p->shape.inter, p->shape.bits, p->shape.n_experts))
+    return set_error(MOE_ERR_UNSUPPORTED, "overlap mode needs a shape of the fused decode kernel");
+  p->overlap = on != 0;
+  return MOE_OK;
+}
+
 moe_status moe_pool_inject_copy_failure(moe_pool* p, int64_t nth) {
   if (!p) return set_error(MOE_ERR_INVALID, "pool is NULL");
   p->fail_at = nth < 0 ? -1 : nth;
@@ -254,6 +321,7 @@ void moe_pool_destroy(moe_pool* p) {
   if (p->ready) cudaEventDestroy(p->ready);
   if (p->h_ids) cudaFreeHost(p->h_ids);
   if (p->h_table) cudaFreeHost(p->h_table);
+  if (p->h_final) cudaFreeHost(p->h_final);
   delete p;
 }
 

@@ -160,3 +160,47 @@ def test_pool_injected_copy_failure_leaves_consistent_state():
         assert torch.equal(P.dev[1].cpu(), P.host[9])
     finally:
         P.close()
+
+
+@pytest.mark.parametrize("wname,steps,T", [("pool_int4", 24, 1), ("pool_int8", 12, 1), ("pool_int4", 8, 8)])
+def test_pool_overlap_mode_bit_identical(wname, steps, T):
+    """Overlap mode: the forward is enqueued right after the load, while the misses are still
+    being copied; the fused kernel waits per expert for its pending slot-table entry.  Same
+    slot decisions as the oracle, the table settles to the host mirror, no device error, and
+    the output equals the all-resident forward bit for bit."""
+    w = synth.WORKLOADS[wname]
+    P = Pool(w, w.n_slots)
+    sim = oracle.SlotCache(w.n_experts, w.n_slots)
+    try:
+        abi.moe_pool_set_overlap(P.h, True)
+        for s in range(steps):
+            x = synth.activations(w, 100 + s, tokens=T, device=DEV)
+            idx, p = _route(P, x)
+            abi.moe_expert_pool_load(P.h, idx, T)
+            sim.step(idx.cpu().numpy().reshape(-1).tolist())
+            out_pool, _, _, ws = forward(w, P.L, x, residual=x, pool=P.dev, slot_table=P.table,
+                                         n_slots=P.n_slots, topk=(idx, p))
+            assert abi.moe_ws_check(ws) == 0
+            slot_of, expert_in = abi.moe_pool_slot_table(P.h, w.n_experts, w.n_slots)
+            assert slot_of == sim.slot_of.tolist()
+            assert expert_in == sim.expert_in.tolist()
+            assert P.table.cpu().tolist() == slot_of  # every pending entry settled
+            out_res, *_ = forward(w, P.L, x, residual=x, topk=(idx, p))
+            assert torch.equal(out_pool, out_res)
+        st = abi.moe_pool_stats(P.h)
+        assert (st["lookups"], st["hits"], st["misses"]) == (sim.lookups, sim.hits, sim.misses)
+        assert st["h2d_bytes"] == sim.misses * P.stride
+    finally:
+        P.close()
+
+
+def test_pool_overlap_mode_needs_fused_shape():
+    w = synth.WORKLOADS["tiny"].with_(hidden=384, inter=64, shared_inter=64)  # no fused kernel
+    P = Pool(w, 8)
+    try:
+        with pytest.raises(abi.MoeError) as ei:
+            abi.moe_pool_set_overlap(P.h, True)
+        assert ei.value.status == -5  # MOE_ERR_UNSUPPORTED
+        abi.moe_pool_set_overlap(P.h, False)
+    finally:
+        P.close()
