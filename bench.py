@@ -45,7 +45,10 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per layer-token of the kernel the
 # bench times, from the ncu capture summarised in profiles/k_fused_decode_decode80b_2layer_full.md
 # (2-layer case, scaled by layers).  Must be re-captured whenever the kernel changes.
-NCU_TRAFFIC_PER_LAYER = {("k_fused_decode", "decode80b", 1): 21_743_360}
+# Empty: the kernel gained the wait for pending slot-table entries (pool overlap mode) after
+# the last capture (profiles/k_fused_decode_decode80b_2layer_full.md: 21,743,360 B per layer);
+# the figure comes back with the next capture of the current kernel.
+NCU_TRAFFIC_PER_LAYER = {}
 # DRAM traffic per launch of the prefill gate/up GEMM on the prefill workload (full-size capture,
 # profiles/k_gemm_gateup_prefill_full.md).  Must be re-captured whenever the kernel changes.
 NCU_TRAFFIC_PREFILL_GATEUP = {("prefill", 4096): 830_150_912}
