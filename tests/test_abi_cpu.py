@@ -106,3 +106,13 @@ def test_pool_create_rejects_bad_args():
     assert abi.lib().moe_pool_create(ctypes.byref(s), 0, 16, 256, 16, ctypes.byref(h)) == -1
     assert abi.lib().moe_pool_create(ctypes.byref(s), 4, None, 256, 16, ctypes.byref(h)) == -1
     abi.moe_pool_destroy(None)
+
+
+def test_pool_calls_reject_a_null_pool():
+    """Every pool call checks its handle before touching anything (no device needed)."""
+    L = abi.lib()
+    assert L.moe_pool_set_policy(None, 0) == -1
+    assert L.moe_pool_set_overlap(None, 1) == -1
+    assert L.moe_pool_inject_copy_failure(None, 0) == -1
+    assert L.moe_expert_pool_load(None, None, 1, None) == -1
+    assert "NULL" in L.moe_last_error().decode()
