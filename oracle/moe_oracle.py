@@ -61,17 +61,31 @@ def bf16_to_f64(bits) -> np.ndarray:
 
 
 def f64_to_bf16_bits(v) -> np.ndarray:
-    """Round float64 to bf16 (via float32, round-half-even) -> uint16 patterns.
+    """Round float64 values to the nearest bf16 (ties to even), once -> uint16 patterns.
 
-    Used only to form the layer input of the next stacked layer in tests.
+    A bf16 number has 8 significant bits and float32's exponent range: normal numbers
+    m * 2^(e-8) with 128 <= m < 256, subnormal ones n * 2^-133 with n < 128.  The float64
+    value is rounded directly onto that grid (not through float32, which would round twice
+    and can move a value that lies just off a bf16 midpoint onto it).  Values at or beyond
+    the midpoint between the largest bf16 (2^128 - 2^120) and 2^128 become infinity; NaN
+    becomes the quiet NaN 0x7FC0.  Used to form the next stacked layer's input in tests and
+    the CPU baseline.
     """
-    f = np.asarray(v, dtype=np.float64).astype(np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    r = ((u + 0x7FFF + lsb) >> 16) & 0xFFFF
-    nan = np.isnan(f)
-    r = np.where(nan, 0x7FC0, r)
-    return r.astype(np.uint16)
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    neg = np.signbit(np.asarray(v, dtype=np.float64))
+    out = np.empty(a.shape, dtype=np.float64)
+    with np.errstate(over="ignore", invalid="ignore"):
+        m, e = np.frexp(a)                          # a = m * 2^e, 0.5 <= m < 1
+        normal = a >= 2.0 ** -126
+        # normal range: 8 significant bits, m * 2^8 in [128, 256), rounded half to even
+        out[normal] = np.ldexp(np.round(np.ldexp(m[normal], 8)), e[normal] - 8)
+        # subnormal range: multiples of 2^-133
+        out[~normal] = np.ldexp(np.round(np.ldexp(a[~normal], 133)), -133)
+        f32 = out.astype(np.float32)                # exact: a bf16 value, or inf past the top
+    u = (f32.view(np.uint32) >> 16).astype(np.uint32)
+    u = np.where(neg, u | 0x8000, u)
+    u = np.where(np.isnan(a), 0x7FC0, u)
+    return u.astype(np.uint16)
 
 
 # ----------------------------------------------------------------------------
@@ -216,7 +230,8 @@ def expert_hidden(weights, x: np.ndarray) -> np.ndarray:
     """The SwiGLU intermediate h = silu(Wg x) * (Wu x) (for checking the gate/up stage alone)."""
     wg, wu, _ = weights
     xx = np.atleast_2d(x)
-    return silu(xx @ wg.T) * (xx @ wu.T)
+    h = silu(xx @ wg.T) * (xx @ wu.T)
+    return h if np.ndim(x) == 2 else h[0]
 
 
 def layer_forward(x_bits, wr_bits, bias, top_k: int, expert_blob: Callable[[int], np.ndarray],
@@ -246,6 +261,39 @@ def layer_forward(x_bits, wr_bits, bias, top_k: int, expert_blob: Callable[[int]
     for t in range(T):
         for j in range(idx.shape[1]):
             out[t] += p[t, j] * expert_forward(weights_of(int(idx[t, j])), x[t])
+    ws = read_expert(shared_blob, hidden, shared_inter, bits)
+    gate = sigmoid(x @ bf16_to_f64(wsg_bits))
+    out += gate[:, None] * expert_forward(ws, x)
+    if residual_bits is not None:
+        out += bf16_to_f64(residual_bits)
+    return dict(out=out, idx=idx, p=p, logits=logits, gate=gate)
+
+
+def layer_forward_by_expert(x_bits, wr_bits, bias, top_k: int, expert_blob: Callable[[int], np.ndarray],
+                            shared_blob, wsg_bits, hidden: int, inter: int, shared_inter: int, bits: int,
+                            residual_bits=None, idx: Optional[np.ndarray] = None,
+                            p: Optional[np.ndarray] = None):
+    """The same layer as layer_forward, with the loops turned round for many tokens.
+
+    Each selected expert is decoded once and applied to all the tokens routed to it
+    (y = expert_forward(W_e, x[tokens of e])), then dropped, so a call over thousands of
+    tokens holds one expert's weights at a time.  Per token the arithmetic is that of
+    layer_forward: out[t] = sum_j p[t, j] y_{idx[t, j]}(x_t) + sigmoid(w_sg . x_t) y_s(x_t)
+    (+ residual), each term an fp64 matrix product; only the order in which the terms of
+    different tokens are formed changes.  Returns the same dict as layer_forward.
+    """
+    x = bf16_to_f64(x_bits)
+    T = x.shape[0]
+    logits = None
+    if idx is None:
+        logits = router_logits(x_bits, wr_bits, bias)
+        idx, p = route(logits, top_k)
+    out = np.zeros((T, hidden), dtype=np.float64)
+    for e in np.unique(idx):
+        tok, slot = np.nonzero(idx == e)
+        y = expert_forward(read_expert(expert_blob(int(e)), hidden, inter, bits), x[tok])
+        for n in range(tok.size):
+            out[tok[n]] += p[tok[n], slot[n]] * y[n]
     ws = read_expert(shared_blob, hidden, shared_inter, bits)
     gate = sigmoid(x @ bf16_to_f64(wsg_bits))
     out += gate[:, None] * expert_forward(ws, x)

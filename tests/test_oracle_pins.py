@@ -40,14 +40,37 @@ def test_bf16_patterns_hand():
         assert oracle.bf16_to_f64(np.array([int(c["bits_hex"], 16)]))[0] == c["value"]
 
 
-def test_bf16_rounding_half_even():
-    # 1 + 2^-8 is half-way between bf16 neighbours 1 and 1+2^-7 -> even (1.0)
-    assert oracle.f64_to_bf16_bits(np.array([1.0 + 2.0**-8]))[0] == 0x3F80
-    # 1 + 3*2^-8 is half-way between 1+2^-7 (odd) and 1+2^-6 (even) -> 1+2^-6
-    assert oracle.f64_to_bf16_bits(np.array([1.0 + 3 * 2.0**-8]))[0] == 0x3F82
-    v = np.random.default_rng(0).standard_normal(1000)
-    ref = torch.tensor(v, dtype=torch.float64).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
-    assert np.array_equal(oracle.f64_to_bf16_bits(v), ref)
+def test_bf16_rounding_hand_cases():
+    # hand-worked single-step roundings, including values where rounding through float32
+    # first would land on a bf16 midpoint and round the other way
+    for c in _gold("bf16_rounding.json")["cases"]:
+        got = int(oracle.f64_to_bf16_bits(np.array([c["value"]]))[0])
+        assert got == int(c["bits_hex"], 16), (c["expr"], hex(got))
+        if "double_rounding_gives" in c:
+            assert got != int(c["double_rounding_gives"], 16)
+    assert int(oracle.f64_to_bf16_bits(np.array([np.nan]))[0]) == 0x7FC0
+
+
+def test_bf16_rounding_float32_inputs_match_library():
+    # on inputs that are float32 values one rounding is all there is, so a library's
+    # float32 -> bf16 conversion must agree bit for bit
+    v = np.random.default_rng(0).standard_normal(1000).astype(np.float32)
+    v = np.concatenate([v, v * 1e-39, v * 1e30])
+    ref = torch.tensor(v).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    assert np.array_equal(oracle.f64_to_bf16_bits(v.astype(np.float64)), ref)
+
+
+def test_bf16_rounding_is_nearest():
+    # brute force: the chosen pattern is the nearest finite bf16, and on exact ties the even one
+    rng = np.random.default_rng(1)
+    v = rng.standard_normal(2000) * np.exp2(rng.integers(-20, 20, 2000))
+    got = oracle.f64_to_bf16_bits(v)
+    for x, b in zip(v, got):
+        cand = [int(b) - 1, int(b), int(b) + 1]
+        d = [abs(oracle.bf16_to_f64(np.array([c]))[0] - x) for c in cand]
+        assert d[1] <= d[0] and d[1] <= d[2]
+        if d[1] == d[0] or d[1] == d[2]:
+            assert int(b) % 2 == 0
 
 
 @pytest.mark.parametrize("case", ["int4", "int4_edges", "int8"])
@@ -225,12 +248,20 @@ def test_expert_selection_matrices_closed_form(bits):
     pd = rng.integers(0, I, H)
     blob = _pack(_onehot_parts(H, I, bits, pg, pu, pd), H, I, bits)[0]
     x = rng.standard_normal(H)
-    y = oracle.expert_forward(oracle.read_expert(blob, H, I, bits), x)
+    wts = oracle.read_expert(blob, H, I, bits)
+    y = oracle.expert_forward(wts, x)
     a = x[pg]
     u = x[pu]
     h = [a[r] / (1.0 + math.exp(-a[r])) * u[r] for r in range(I)]
     ref = np.array([h[pd[j]] for j in range(H)])
     assert np.allclose(y, ref, rtol=1e-14, atol=1e-15)
+    # the gate/up stage alone: h by index gathers (a gate/up swap breaks the silu side)
+    assert np.allclose(oracle.expert_hidden(wts, x), h, rtol=1e-14, atol=1e-15)
+    x2 = rng.standard_normal((3, H))
+    h2 = oracle.expert_hidden(wts, x2)
+    for t in range(3):
+        a2, u2 = x2[t][pg], x2[t][pu]
+        assert np.allclose(h2[t], a2 / (1.0 + np.exp(-a2)) * u2, rtol=1e-14, atol=1e-15)
 
 
 def test_expert_zero_scale_is_bias_broadcast():
@@ -297,6 +328,29 @@ def test_layer_sparse_equals_dense_masked_bruteforce(seed, E, k, bias):
                                               residual_bits=L["res"])
     assert np.allclose(r["out"], dense, rtol=1e-12, atol=1e-13)
     assert np.allclose(r["p"].sum(1), 1.0, atol=1e-15)
+
+
+@pytest.mark.parametrize("seed,E,k,bias,T", [(11, 16, 2, True, 7), (12, 9, 9, False, 3), (13, 5, 1, False, 12)])
+def test_layer_by_expert_equals_per_token_and_dense(seed, E, k, bias, T):
+    L = _tiny_layer(seed, E, k, bias=bias, T=T)
+    r = _sparse(L)
+    g = oracle.layer_forward_by_expert(L["x"], L["wr"], L["b"], k, lambda e: L["blobs"][e], L["shared"],
+                                       L["wsg"], L["H"], L["I"], L["Is"], L["bits"], residual_bits=L["res"])
+    assert np.array_equal(g["idx"], r["idx"])
+    assert np.allclose(g["out"], r["out"], rtol=1e-13, atol=1e-14)
+    dense = oracle.layer_forward_dense_masked(L["x"], L["wr"], L["b"], k, list(L["blobs"]), L["shared"],
+                                              L["wsg"], L["H"], L["I"], L["Is"], L["bits"],
+                                              residual_bits=L["res"])
+    assert np.allclose(g["out"], dense, rtol=1e-12, atol=1e-13)
+    # given routing: a zeroed weight drops exactly that expert's term
+    p0 = r["p"].copy()
+    p0[0, 0] = 0.0
+    g0 = oracle.layer_forward_by_expert(L["x"], None, None, k, lambda e: L["blobs"][e], L["shared"], L["wsg"],
+                                        L["H"], L["I"], L["Is"], L["bits"], residual_bits=L["res"],
+                                        idx=r["idx"], p=p0)
+    y = oracle.expert_forward(oracle.read_expert(L["blobs"][r["idx"][0, 0]], L["H"], L["I"], L["bits"]),
+                              oracle.bf16_to_f64(L["x"][0]))
+    assert np.allclose(g["out"][0] - g0["out"][0], r["p"][0, 0] * y, rtol=1e-12, atol=1e-13)
 
 
 def test_layer_single_expert_zero_gate_closed_form():
