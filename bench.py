@@ -42,15 +42,14 @@ import synth  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per layer-token of the kernel the
-# bench times, from the ncu capture summarised in profiles/k_fused_decode_decode80b_2layer_full.md
-# (2-layer case, scaled by layers).  Must be re-captured whenever the kernel changes.
-# Empty: the kernel gained the wait for pending slot-table entries (pool overlap mode) after
-# the last capture (profiles/k_fused_decode_decode80b_2layer_full.md: 21,743,360 B per layer);
-# the figure comes back with the next capture of the current kernel.
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per layer of the fused decode
+# kernel, from an ncu capture of a 2-layer stack of the same workload (the full stack is too
+# large to capture; every layer reads its own blobs, so traffic scales with the layers).  Keyed
+# by (kernel, workload, tokens); an entry is dropped whenever the kernel changes and comes back
+# with the next capture.
 NCU_TRAFFIC_PER_LAYER = {}
-# DRAM traffic per launch of the prefill gate/up GEMM on the prefill workload (full-size capture,
-# profiles/k_gemm_gateup_prefill_full.md).  Must be re-captured whenever the kernel changes.
+# DRAM traffic per launch of the prefill gate/up GEMM on the prefill workload (full-size,
+# one-pass capture).  Dropped whenever the kernel changes.
 NCU_TRAFFIC_PREFILL_GATEUP = {("prefill", 4096): 830_150_912}
 
 
@@ -369,6 +368,26 @@ def cpu_baseline_decode(w, T, device, stack, budget_s=12.0):
                       f"{per_layer * 1e3:.0f} ms/layer), scaled to the {w.layers}-layer step"}
 
 
+def workload_config(args, w, T, n_gpus):
+    """The `config` object of a result line: the workload alone, identical in both arms."""
+    cfg = {"workload": w.name, "hidden": w.hidden, "n_experts": w.n_experts, "top_k": w.top_k,
+           "inter": w.inter, "shared_inter": w.shared_inter, "bits": w.bits, "group": 64,
+           "router": w.router, "parallelism": f"replicas{n_gpus}"}
+    if w.name.startswith("pool"):
+        cfg.update({"tokens_per_step": 1, "layers": 1, "n_slots": w.n_slots, "slot_fraction": w.n_slots / w.n_experts,
+                    "steps_total": max(1024, args.steps + args.warmup),
+                    "policy": {"lfu_recency": "LFU + recency", "lru": "LRU", "lfu": "LFU"}[args.policy],
+                    "miss_path": "pinned host -> cudaMemcpyAsync on a side stream", "overlap": bool(args.overlap),
+                    "l2": "one layer; misses come over PCIe, hits from the slot pool"})
+    elif w.name == "prefill":
+        cfg.update({"tokens_per_call": T, "layers": 1,
+                    "l2": "inputs exceed L2 (906 MB of expert blobs per call)"})
+    else:
+        cfg.update({"tokens_per_step": T, "layers": w.layers,
+                    "l2": "inputs exceed L2 (>1 GB distinct blobs per step)"})
+    return cfg
+
+
 def decode_line(args, w, T, r, n_gpus, peaks, peak_kind, cpu_base):
     K = args.steps
     tok = T * K * n_gpus
@@ -384,15 +403,12 @@ def decode_line(args, w, T, r, n_gpus, peaks, peak_kind, cpu_base):
         "ms_per_step": round(r["ms"] / K, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": f"int{w.bits} weights, bf16 activations, fp32 accumulate",
         "data": "synthetic (seeded; weights ~N(0,0.02) quantised, x ~N(0,1))",
-        "config": {"workload": w.name, "hidden": w.hidden, "n_experts": w.n_experts, "top_k": w.top_k,
-                   "inter": w.inter, "shared_inter": w.shared_inter, "bits": w.bits, "group": 64,
-                   "tokens_per_step": T, "layers": w.layers, "router": w.router,
-                   "parallelism": f"replicas{n_gpus}", "l2": "inputs exceed L2 (>1 GB distinct blobs per step)",
-                   "launch": "one persistent kernel per step" + (" in a CUDA graph" if r["graph"] else "")},
+        "config": workload_config(args, w, T, n_gpus),
+        "launch": "one persistent kernel per step" + (" in a CUDA graph" if r["graph"] else ""),
         "hbm_step": {"bytes_per_step": r["step_bytes"], "achieved_gbs": round(r["step_bytes"] / step_s / 1e9, 1),
                      "frac_of_measured": round(r["step_bytes"] / step_s / 1e9 / hbm, 4),
                      "mean_distinct_experts_per_layer": round(float(np.mean(r["uniq"])), 2)},
-        "roofline": {"bound": "hbm", "kernel": "k_fused_decode (whole 48-layer step, one launch)",
+        "roofline": {"bound": "hbm", "kernel": f"k_fused_decode (whole {w.layers}-layer step, one launch)",
                      "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
                      "traffic": (NCU_TRAFFIC_PER_LAYER.get(("k_fused_decode", w.name, T), 0) * w.layers) or None,
                      "launch_us": round(k_us, 3), "bytes_per_launch": int(k_bytes),
@@ -532,11 +548,8 @@ def prefill_line(args, w, T, r, n_gpus, peaks, peak_kind, cpu_base):
         "ms_per_step": round(r["ms"] / K, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": f"int{w.bits} weights dequantised to bf16, bf16 x bf16 -> fp32 (tcgen05)",
         "data": "synthetic (seeded; weights ~N(0,0.02) quantised, x ~N(0,1))",
-        "config": {"workload": w.name, "hidden": w.hidden, "n_experts": w.n_experts, "top_k": w.top_k,
-                   "inter": w.inter, "shared_inter": w.shared_inter, "bits": w.bits, "group": 64,
-                   "tokens_per_call": T, "layers": 1, "parallelism": f"replicas{n_gpus}",
-                   "l2": "inputs exceed L2 (906 MB of expert blobs per call)",
-                   "tokens_per_expert_mean_min_max": r["tokens_per_expert"]},
+        "config": workload_config(args, w, T, n_gpus),
+        "tokens_per_expert_mean_min_max": r["tokens_per_expert"],
         "tensor_step": {"flops_per_call": total_f, "achieved_tflops": round(total_f / step_s / 1e12, 1),
                         "frac_of_measured": round(total_f / step_s / 1e12 / peak, 4)},
         "roofline": {"bound": "tensor", "kernel": "k_gemm<GATEUP> (gate/up grouped GEMM + SwiGLU)",
@@ -626,27 +639,45 @@ def run_pool(args, w, device, rank, total_steps=1024):
     cnt = cnt[cnt > 0]
     rk = np.arange(1, len(cnt) + 1)
     zipf_s = float(-np.polyfit(np.log(rk), np.log(cnt), 1)[0]) if len(cnt) > 2 else None
+    L.shared_host = L.shared.cpu().numpy()
     return dict(ms=ms, clocks=clocks, flags=flags, K=K, n_total=n_total, stats=st1,
                 hit_rate_all=st1["hits"] / max(1, st1["lookups"]), hit_rate_timed=hits / max(1, look),
-                h2d_timed=st1["h2d_bytes"] - st0["h2d_bytes"], zipf_s=zipf_s, stride=stride)
+                h2d_timed=st1["h2d_bytes"] - st0["h2d_bytes"], zipf_s=zipf_s, stride=stride,
+                layer=L, host_blobs=host_blobs, xs=xs[:64])
 
 
-def pool_line(args, w, r, n_gpus):
+def cpu_baseline_pool(w, r, budget_s=10.0):
+    """The fp64 oracle as it stands on host cores: one token per step through the layer (every
+    expert readable from host memory, no pool), as many steps as fit in ~budget_s."""
+    import oracle
+    L = r["layer"]
+    wr, wsg = _bits(L.w_router), _bits(L.w_sg)
+    b = None if L.router_bias is None else L.router_bias.cpu().numpy()
+    shared = L.shared_host
+    t_total, n = 0.0, 0
+    while t_total < budget_s and n < 200:
+        xb = _bits(r["xs"][n % r["xs"].shape[0]])
+        t0 = time.perf_counter()
+        oracle.layer_forward(xb, wr, b, w.top_k, lambda e: r["host_blobs"][e].numpy(), shared, wsg, w.hidden,
+                             w.inter, w.shared_inter, w.bits, residual_bits=xb)
+        t_total += time.perf_counter() - t0
+        n += 1
+    return {"value": round(n / t_total, 4), "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{n} decode steps (one token through the layer, fp64 numpy oracle, "
+                      f"{1e3 * t_total / n:.0f} ms/step), all experts in host memory"}
+
+
+def pool_line(args, w, r, n_gpus, cpu_base=None):
     K = r["K"]
     value = n_gpus * K / (r["ms"] / 1e3)
-    return {
+    line = {
         "metric": "routed-MoE layer tokens/s with a bounded slot pool; expert-cache hit rate",
         "value": round(value, 1), "unit": "tokens/s", "n_gpus": n_gpus, "steps": K, "warmup": args.warmup,
         "ms_per_step": round(r["ms"] / K, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": f"int{w.bits} weights, bf16 activations, fp32 accumulate",
         "data": "synthetic (seeded; Zipf(1.0) router bias)",
-        "config": {"workload": w.name, "hidden": w.hidden, "n_experts": w.n_experts, "top_k": w.top_k,
-                   "bits": w.bits, "n_slots": w.n_slots, "slot_fraction": w.n_slots / w.n_experts,
-                   "steps_total": r["n_total"], "tokens_per_step": 1,
-                   "policy": {"lfu_recency": "LFU + recency", "lru": "LRU", "lfu": "LFU"}[args.policy],
-                   "miss_path": "pinned host -> cudaMemcpyAsync on a side stream",
-                   "overlap": bool(args.overlap),
-                   "timing": "events around the timed steps; each step waits on the host for the ids"},
+        "config": workload_config(args, w, 1, n_gpus),
+        "timing": "events around the timed steps; each step waits on the host for the ids",
         "pool": {"hit_rate_all_steps": round(r["hit_rate_all"], 4), "hit_rate_timed": round(r["hit_rate_timed"], 4),
                  "stats": r["stats"], "h2d_bytes_timed": r["h2d_timed"],
                  "h2d_gbs_timed": round(r["h2d_timed"] / (r["ms"] / 1e3) / 1e9, 2),
@@ -657,19 +688,26 @@ def pool_line(args, w, r, n_gpus):
         "gpu_launches": 6 * K,
         "device_error_flags": r["flags"],
     }
+    if cpu_base is not None:
+        line["cpu_baseline"] = cpu_base
+    return line
 
 
 # --------------------------------------------------------------------------------------
 # reference arm: the fp64 oracle on host cores
 # --------------------------------------------------------------------------------------
 def run_reference(args, w, T):
+    """The reference arm: the fp64 oracle as it stands, timed on the host cores.  Each step is
+    a bounded sample of the workload: decode -- the step's T token(s) through one layer
+    (cycling over the first four layers), tokens/s scaled to the whole stack; prefill -- 32
+    seeded tokens of the call through the layer; pool -- one decode token through the layer.
+    ms_per_step is the time the timed steps actually took."""
     import oracle
-    rank, _, ws = dist_env()
+    rank, _, n_ranks = dist_env()
     if rank != 0:
         return None
     dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
     K, W = args.steps, args.warmup
-    # inputs: the same generator as our arm; only the sampled layer is materialised
     layers = {}
 
     def layer(l):
@@ -682,11 +720,18 @@ def run_reference(args, w, T):
     def bits(t):
         return t.contiguous().view(torch.int16).numpy().view(np.uint16)
 
+    prefill = w.name == "prefill"
+    n_tok = 32 if prefill else (1 if w.name.startswith("pool") else T)
     times = []
     for s in range(W + K):
-        l = s % min(w.layers, 4)
+        l = 0 if (prefill or w.name.startswith("pool")) else s % min(w.layers, 4)
         d = layer(l)
-        x = synth.activations(w, rank_step_seed(0, s), tokens=T, device=dev).cpu()
+        if prefill:
+            x = synth.activations(w, rank_step_seed(0, s % 3), tokens=T, device=dev)
+            sel = np.sort(np.random.default_rng(s).choice(T, n_tok, replace=False))
+            x = x[torch.from_numpy(sel).to(dev)].cpu()
+        else:
+            x = synth.activations(w, rank_step_seed(0, s), tokens=n_tok, device=dev).cpu()
         logits = oracle.router_logits(bits(x), bits(d["wr"]), d["b"])
         idx, _ = oracle.route(logits, w.top_k)
         blobs = {int(e): d["pool"][int(e)].cpu().numpy() for e in set(idx.reshape(-1).tolist())}
@@ -696,16 +741,27 @@ def run_reference(args, w, T):
         dt = time.perf_counter() - t0
         if s >= W:
             times.append(dt)
-    per_layer = statistics.mean(times)
-    value = T / (per_layer * w.layers)
-    sample = (f"each step: {T} token(s) through one layer (cycling layers 0-3) with the fp64 numpy oracle; "
-              f"tokens/s scaled to the {w.layers}-layer stack")
-    return {"impl": "reference", "metric": "routed-MoE layer tokens/s; achieved HBM GB/s (decode)",
+    per_step = statistics.mean(times)
+    if prefill:
+        value = n_tok / per_step
+        sample = (f"each step: {n_tok} seeded tokens of the {T}-token call through the layer (fp64 numpy oracle, "
+                  f"{per_step * 1e3:.0f} ms), scaled to tokens/s")
+        metric = "routed-MoE layer tokens/s; tensor % (prefill)"
+    elif w.name.startswith("pool"):
+        value = 1.0 / per_step
+        sample = (f"each step: one token through the layer (fp64 numpy oracle, {per_step * 1e3:.0f} ms), "
+                  f"every expert in host memory")
+        metric = "routed-MoE layer tokens/s with a bounded slot pool; expert-cache hit rate"
+    else:
+        value = T / (per_step * w.layers)
+        sample = (f"each step: {T} token(s) through one layer (cycling layers 0-3) with the fp64 numpy oracle "
+                  f"({per_step * 1e3:.0f} ms measured per step); tokens/s scaled to the {w.layers}-layer stack")
+        metric = "routed-MoE layer tokens/s; achieved HBM GB/s (decode)"
+    return {"impl": "reference", "metric": metric,
             "value": round(value, 4), "unit": "tokens/s", "n_gpus": 1, "steps": K, "warmup": W,
-            "ms_per_step": round(per_layer * w.layers * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": round(per_step * 1e3, 2), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-            "config": {"workload": w.name, "hidden": w.hidden, "n_experts": w.n_experts, "top_k": w.top_k,
-                       "tokens_per_step": T, "layers": w.layers, "bits": w.bits},
+            "config": workload_config(args, w, T, n_ranks),
             "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -763,7 +819,9 @@ def main(argv=None):
         line = prefill_line(args, w, T, r, ws, peaks, peak_kind, cpu_base)
     elif w.name.startswith("pool"):
         r = run_pool(args, w, device, rank)
-        line = pool_line(args, w, r, ws)
+        if want_cpu:
+            cpu_base = cpu_baseline_pool(w, r)
+        line = pool_line(args, w, r, ws, cpu_base)
     else:
         r = run_decode(args, w, T, device, rank, ws)
         if want_cpu:

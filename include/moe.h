@@ -113,9 +113,13 @@ MOE_API moe_status moe_workspace_size(const moe_shape* shape, int32_t T, size_t*
  *   topk_idx    (dev) int32 [T, k] out: expert ids, logit descending, ties lower id first
  *   topk_w      (dev) fp32  [T, k] out: softmax over the k selected logits
  *   ws          (dev) workspace of ws_bytes >= moe_workspace_size(shape, T)
- * Logits are accumulated in fp64 from exact bf16*bf16 products, so the selection is the
- * exact-arithmetic selection except for logits that tie to within fp64 rounding.
- * T: 1..8 on the decode path.
+ * Any T >= 1.  Up to 8 tokens (and, in groups of 8, shapes the many-token router does not
+ * cover): logits accumulated in fp64 from exact bf16*bf16 products.  More than 8 tokens with
+ * hidden % 128 == 0, hidden <= 4096 and E <= 512: the router of the many-token layer
+ * forward -- fp32 logits on the tensor cores, and every expert whose fp32 logit lies within
+ * the fp32 error bound of the k-th is recomputed exactly before the selection and the
+ * softmax.  Either way the selection is the exact-arithmetic selection except for logits
+ * that tie to within fp64 rounding.  ws must hold moe_workspace_size(shape, T) bytes.
  */
 MOE_API moe_status moe_router_topk(const moe_shape* shape, const void* x, int32_t T, const void* w_router,
                            const float* router_bias, int32_t* topk_idx, float* topk_w, void* ws,
@@ -210,6 +214,8 @@ MOE_API moe_status moe_stack_forward(const moe_shape* shape, int32_t T, const mo
  *     threads) race on the array and must not be issued.
  *   - Device-detected errors (bad slot or expert id) are skipped as in moe_layer_forward,
  *     but cannot be read back: the control block is cleared by the next call.
+ *   - A device reset (cudaDeviceReset) gives the device a new context; the next call notices
+ *     the change and looks the address up again (make that call outside stream capture too).
  *   - The control-block clear may already be enqueued when a later argument check fails;
  *     it touches only the library's own array.
  */
@@ -242,6 +248,30 @@ MOE_API moe_status moe_group_pairs(const moe_shape* shape, int32_t T, const int3
  */
 MOE_API moe_status moe_ws_check(void* ws, void* stream, uint32_t* flags);
 
+/*
+ * moe_ws_set_slot_wait -- how long the fused decode kernel waits for a slot-table entry that
+ * is still pending (a pool in overlap mode marks each miss pending until its blob copy has
+ * landed) before it treats the copy as failed: the expert is then skipped like an expert
+ * with a bad slot, and MOE_DEVERR_TIMEOUT | MOE_DEVERR_BAD_SLOT are set.
+ *   ws            (dev) workspace; the setting lives in its control block
+ *   microseconds  the bound; 0 restores the default of 2 seconds
+ * Enqueued on `stream` (one tiny kernel).  The setting stays with the workspace until changed
+ * (moe_layer_forward_static clears its own control block every call, so it always uses the
+ * default).  Failure detection by bounded waits: a copy that never lands ends in an error
+ * bit, never in a hung kernel.
+ */
+MOE_API moe_status moe_ws_set_slot_wait(void* ws, uint32_t microseconds, void* stream);
+
+/*
+ * moe_ws_router_logits -- inspection hook: *logits (host) receives the device address, inside
+ * ws, of the fp32 router logits [T, E+1] that the many-token router (moe_router_topk or
+ * moe_layer_forward with T > 8) last left there: row t holds token t's logits without router
+ * bias in columns 0..E-1 (column E is not written).  These are the tensor-core values before
+ * the exact recheck; the selection never rests on them alone.  T > 8.
+ */
+MOE_API moe_status moe_ws_router_logits(const moe_shape* shape, int32_t T, void* ws, size_t ws_bytes,
+                                        float** logits);
+
 /* ------------------------------------------------------------------------------------ */
 /* Bounded slot pool with LFU + recency eviction («Paquets Swiftlet…» paragraph 5;       */
 /* «Swiftlet: 在 Mac 和 iPhone 上執行…», 記憶體管理與權重串流).  Misses are copied from   */
@@ -270,7 +300,9 @@ MOE_API moe_status moe_pool_create(const moe_shape* shape, int32_t n_slots, cons
                            uint8_t* dev_pool, int32_t* dev_slot_table, moe_pool** out);
 
 /*
- * moe_expert_pool_load -- make every expert named in topk_idx (dev int32 [T, k]) resident.
+ * moe_expert_pool_load -- make every expert named in topk_idx (dev int32 [T, k], T >= 1)
+ * resident.  A step with more than 8 tokens grows the pool's pinned id read-back buffer once
+ * (one pinned host allocation).
  * SYNCHRONISES `stream` (the ids are needed on the host): copies the ids back, looks them
  * up (distinct ids in first-appearance order; hits refresh use count and last use), loads
  * each miss into the lowest empty slot, else evicts the slot with the smallest

@@ -66,6 +66,8 @@ _SIGS = {
                                          _SZ, _P]),
     "moe_group_pairs": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, _P, _P, _P, _P, _SZ, _P]),
     "moe_ws_check": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
+    "moe_ws_set_slot_wait": (ctypes.c_int, [_P, ctypes.c_uint32, _P]),
+    "moe_ws_router_logits": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, _P, _SZ, ctypes.POINTER(_P)]),
     "moe_pool_create": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, _P, _P, _P, ctypes.POINTER(_P)]),
     "moe_expert_pool_load": (ctypes.c_int, [_P, _P, _I32, _P]),
     "moe_pool_stats": (ctypes.c_int, [_P, ctypes.POINTER(moe_pool_stats_t)]),
@@ -203,6 +205,21 @@ def moe_ws_check(ws, stream=None, raise_on_error: bool = False) -> int:
     if st not in (MOE_OK, -7) or (raise_on_error and st != MOE_OK):
         _check(st)
     return int(flags.value)
+
+
+def moe_ws_set_slot_wait(ws, microseconds: int, stream=None):
+    """Bound (us; 0 = the 2 s default) of the decode kernel's waits for pending slot entries."""
+    _check(lib().moe_ws_set_slot_wait(_ptr(ws), int(microseconds), _stream(stream)))
+
+
+def moe_ws_router_logits(shape, T: int, ws) -> torch.Tensor:
+    """The many-token router's fp32 logits [T, E+1] inside ws, as a view (column E unused)."""
+    addr = _P()
+    _check(lib().moe_ws_router_logits(ctypes.byref(shape), T, _ptr(ws), ws.numel() * ws.element_size(),
+                                      ctypes.byref(addr)))
+    off = addr.value - ws.data_ptr()
+    n = T * (shape.n_experts + 1)
+    return ws[off:off + 4 * n].view(torch.float32).view(T, shape.n_experts + 1)
 
 
 def moe_pool_create(shape, n_slots, host_blobs, dev_pool, dev_slot_table) -> int:

@@ -89,6 +89,11 @@ moe_status moe_workspace_size(const moe_shape* shape, int32_t T, size_t* bytes) 
   return MOE_OK;
 }
 
+// Shapes whose many-token routing runs on the tensor cores (router GEMM + certified top-k).
+static bool route_shape_many(const moe_shape* s) {
+  return s->hidden % 128 == 0 && s->hidden <= 4096 && s->n_experts <= 512;
+}
+
 static moe_status fill_decode_args(const moe_shape* shape, int32_t T, void* ws, size_t ws_bytes, DecodeArgs* a) {
   memset(a, 0, sizeof *a);
   if (T < 1 || T > kMaxDecodeT)
@@ -129,20 +134,71 @@ moe_status moe_router_topk(const moe_shape* shape, const void* x, int32_t T, con
   if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) ||
       (router_bias && !aligned(router_bias, 4)))
     return set_error(MOE_ERR_INVALID, "x and w_router must be 16-byte aligned");
-  DecodeArgs a;
-  if ((st = fill_decode_args(shape, T, ws, ws_bytes, &a)) != MOE_OK) return st;
-  a.x = static_cast<const uint16_t*>(x);
-  a.wr = static_cast<const uint16_t*>(w_router);
-  a.rbias = router_bias;
-  // The shared-gate row is not needed here; point it at the first router row (its logit
-  // lands in the workspace and is ignored).
-  a.wsg = a.wr;
-  a.topk_idx = topk_idx;
-  a.topk_w = topk_w;
-  prof_mark(0, false, static_cast<cudaStream_t>(stream));
-  cudaError_t e = launch_router_decode(a, false, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "router launch");
-  prof_mark(0, true, static_cast<cudaStream_t>(stream));
+  if (T < 1) return set_error(MOE_ERR_INVALID, "T must be >= 1 (got %d)", T);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T > kMaxDecodeT && route_shape_many(shape)) {
+    // many tokens: tensor-core logits with the certified exact recheck (the routing step of
+    // the many-token layer forward)
+    const int E = shape->n_experts, k = shape->top_k, H = shape->hidden;
+    if (!ws || !aligned(ws, kAlign)) return set_error(MOE_ERR_INVALID, "ws must be non-NULL and 256-byte aligned");
+    const PrefillLayout W = make_prefill_layout(T, E, k, H, shape->inter);
+    if (ws_bytes < W.total) return set_error(MOE_ERR_INVALID, "ws_bytes %zu < required %zu", ws_bytes, W.total);
+    char* b = static_cast<char*>(ws);
+    PrefillArgs p{};
+    p.T = T;
+    p.E = E;
+    p.k = k;
+    p.H = H;
+    p.I = shape->inter;
+    p.x = static_cast<const uint16_t*>(x);
+    p.wr = static_cast<const uint16_t*>(w_router);
+    p.wsg = p.wr;  // the shared-gate logit is not needed here: its row is the first router row
+    p.rbias = router_bias;
+    p.route = true;
+    p.ctrl = reinterpret_cast<Ctrl*>(b + W.ctrl);
+    p.xnorm = reinterpret_cast<double*>(b + W.xnorm);
+    p.wnorm = reinterpret_cast<double*>(b + W.wnorm);
+    p.logits = reinterpret_cast<float*>(b + W.logits);
+    p.topk_idx = topk_idx;
+    p.topk_w = topk_w;
+    p.gate = reinterpret_cast<float*>(b + W.gate);
+    p.units_rt = reinterpret_cast<GemmUnit*>(b + W.units_rt);
+    p.n_units = reinterpret_cast<int*>(b + W.n_units);
+    GemmArgs& g = p.g;
+    g.H = H;
+    g.I = shape->inter;
+    g.E = E;
+    g.k = k;
+    g.T = T;
+    g.x = p.x;
+    g.wr = p.wr;
+    g.wsg = p.wsg;
+    g.logits = p.logits;
+    g.ctrl = p.ctrl;
+    prof_mark(0, false, s);
+    cudaError_t e = launch_prefill_route(p, s);
+    if (e != cudaSuccess) return cuda_fail(e, "router launch");
+    prof_mark(0, true, s);
+    return MOE_OK;
+  }
+  // up to 8 tokens at a time on the decode router (fp64 sums of exact products)
+  prof_mark(0, false, s);
+  for (int32_t t0 = 0; t0 < T; t0 += kMaxDecodeT) {
+    const int32_t Tc = T - t0 < kMaxDecodeT ? T - t0 : kMaxDecodeT;
+    DecodeArgs a;
+    if ((st = fill_decode_args(shape, Tc, ws, ws_bytes, &a)) != MOE_OK) return st;
+    a.x = static_cast<const uint16_t*>(x) + (size_t)t0 * shape->hidden;
+    a.wr = static_cast<const uint16_t*>(w_router);
+    a.rbias = router_bias;
+    // The shared-gate row is not needed here; point it at the first router row (its logit
+    // lands in the workspace and is ignored).
+    a.wsg = a.wr;
+    a.topk_idx = topk_idx + (size_t)t0 * shape->top_k;
+    a.topk_w = topk_w + (size_t)t0 * shape->top_k;
+    cudaError_t e = launch_router_decode(a, false, s);
+    if (e != cudaSuccess) return cuda_fail(e, "router launch");
+  }
+  prof_mark(0, true, s);
   return MOE_OK;
 }
 
@@ -449,6 +505,30 @@ moe_status moe_profile_events(void* const* events, int32_t n) {
   if (events && n < 0) return set_error(MOE_ERR_INVALID, "n must be >= 0");
   g_prof_events = events;
   g_prof_n = events ? n : 0;
+  return MOE_OK;
+}
+
+namespace {
+__global__ void k_set_u32(uint32_t* p, uint32_t v) { *p = v; }
+}  // namespace
+
+moe_status moe_ws_set_slot_wait(void* ws, uint32_t microseconds, void* stream) {
+  if (!ws || !aligned(ws, kAlign)) return set_error(MOE_ERR_INVALID, "ws must be non-NULL and 256-byte aligned");
+  Ctrl* c = static_cast<Ctrl*>(ws);
+  k_set_u32<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(&c->slot_wait_us, microseconds);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "slot wait setting");
+  return MOE_OK;
+}
+
+moe_status moe_ws_router_logits(const moe_shape* shape, int32_t T, void* ws, size_t ws_bytes, float** logits) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!ws || !logits) return set_error(MOE_ERR_INVALID, "ws and logits must be non-NULL");
+  if (T <= kMaxDecodeT) return set_error(MOE_ERR_INVALID, "T must be > %d (the many-token layout)", kMaxDecodeT);
+  const PrefillLayout W = make_prefill_layout(T, shape->n_experts, shape->top_k, shape->hidden, shape->inter);
+  if (ws_bytes < W.total) return set_error(MOE_ERR_INVALID, "ws_bytes %zu < required %zu", ws_bytes, W.total);
+  *logits = reinterpret_cast<float*>(static_cast<char*>(ws) + W.logits);
   return MOE_OK;
 }
 

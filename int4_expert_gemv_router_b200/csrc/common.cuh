@@ -62,7 +62,9 @@ struct Ctrl {
   int32_t n_valid;  // number of (token, k) pairs with a valid expert id
   uint32_t bar_count;  // fused decode kernel: grid-barrier arrivals (back to 0 at exit)
   uint32_t bar_gen;    // fused decode kernel: CTAs that have exited (back to 0 at exit)
-  uint32_t pad[58];
+  uint32_t slot_wait_us;  // bound of the fused decode kernel's waits for pending slot-table
+                          // entries, microseconds (0: kWaitNs); a setting, not a counter
+  uint32_t pad[57];
 };
 static_assert(sizeof(Ctrl) == 256, "ctrl block is 256 bytes");
 
@@ -194,7 +196,7 @@ struct FusedArgs {
 // Prefill path (prefill.cu)
 // ---------------------------------------------------------------------------------------
 constexpr int kModeRouter = 0, kModeGateUp = 1, kModeDown = 2;
-constexpr int kPrefillN = 128;  // tokens (MMA N) per GEMM work unit
+constexpr int kPrefillN = 128;  // tokens (the MMA's M) per GEMM work unit
 constexpr int kGroupChunk = 512;  // (token, k) pairs per CTA of the grouping kernels
 
 // One tcgen05 GEMM work unit: expert e (-1: shared expert, -2: router), row tile mt, first
@@ -319,6 +321,7 @@ bool prefill_shape_supported(int H, int I, int bits, int E);
 // Profiling hook of moe_profile_events (api.cu): event pair i around kernel group i.
 void prof_mark(int i, bool end, cudaStream_t s);
 cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s);
+cudaError_t launch_prefill_route(const PrefillArgs& p, cudaStream_t s);
 cudaError_t launch_group(const PrefillArgs& p, cudaStream_t s);
 
 // Kernel launchers (decode.cu).  Return cudaError_t of the launch.

@@ -238,6 +238,9 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
   constexpr int HS = (RPWd == 2 && V4 % 2 == 0) ? 2 : 1, VH = V4 / HS;
 
   const int T = a.T, E = a.E, k = a.k, G = gridDim.x;
+  // bound of the waits for pending slot-table entries (a blob copy that has not landed by
+  // then is treated as failed: the expert is skipped and flagged)
+  const unsigned long long slot_wait_ns = a.ctrl->slot_wait_us ? 1000ull * a.ctrl->slot_wait_us : kWaitNs;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int NS = a.n_stages, SB = a.stage_bytes;
   const int RG = (SB / ROWG_BYTES) / gG * gG;  // gate/up rows per stage
@@ -288,7 +291,12 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
     // The slot of distinct expert u of layer Lc.  An entry that was pending when phase X read
     // the table (the blob was still being copied) is polled until the copy stream has written
     // the slot; the result goes back to the plan, where the compute warps read it after the
-    // stage's full barrier.  Whole warp; bounded (-1 and MOE_DEVERR_TIMEOUT after kWaitNs).
+    // stage's full barrier.  Whole warp; bounded (-1 and MOE_DEVERR_TIMEOUT after slot_wait_ns).
+    // The entry is written by the copy stream (a stream memory operation after the blob's
+    // copy), so it is read with system-scope acquire loads; the blob itself is then read by
+    // cp.async.bulk, which goes through the async proxy: every lane orders its later bulk
+    // copies after the acquire with a proxy fence (the warp barrier carries lane 0's acquire
+    // to the other lanes first).
     const auto slot_of_unit = [&](const FusedLayer& L, int u) {
       int v = P_SLOT[u];
       if (v != kSlotPending) return v;
@@ -297,9 +305,9 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
         const unsigned long long t0 = now_ns();
         uint32_t ns = 64;
         for (;;) {
-          v = ld_acquire_s32(entry);
+          v = ld_acquire_sys_s32(entry);
           if (v != kSlotPending) break;
-          if (now_ns() - t0 > kWaitNs) {
+          if (now_ns() - t0 > slot_wait_ns) {
             atomicOr(&a.ctrl->err, kErrTimeout);
             v = -1;
             break;
@@ -311,6 +319,8 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
         if (v < 0) atomicOr(&a.ctrl->err, kErrBadSlot);
         P_SLOT[u] = v;
       }
+      __syncwarp();
+      fence_proxy_async_global();
       return __shfl_sync(0xffffffffu, v, 0);
     };
     for (int l = 0; l < a.n_layers && ok; ++l) {

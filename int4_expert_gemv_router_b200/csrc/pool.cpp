@@ -70,7 +70,8 @@ struct moe_pool {
   cudaStream_t side = nullptr;
   cudaEvent_t ready = nullptr;     // slot table + blobs of the last step are on the device
   bool ready_recorded = false;
-  int32_t* h_ids = nullptr;        // pinned [kMaxDecodeT * kMaxTopK]
+  int32_t* h_ids = nullptr;        // pinned [h_ids_cap]: the step's ids read back
+  int32_t h_ids_cap = 0;
   int32_t* h_table = nullptr;      // pinned [E]
   int32_t* h_final = nullptr;      // pinned [E]: the slot an overlap-mode miss resolves to
 };
@@ -117,6 +118,7 @@ moe_status moe_pool_create(const moe_shape* shape, int32_t n_slots, const uint8_
     moe_pool_destroy(p);
     return cuda_fail(e, "pool create");
   }
+  p->h_ids_cap = kMaxDecodeT * kMaxTopK;
   for (int i = 0; i < E; ++i) p->h_table[i] = -1;
   e = cudaMemcpyAsync(dev_slot_table, p->h_table, sizeof(int32_t) * E, cudaMemcpyHostToDevice, p->side);
   if (e == cudaSuccess) e = cudaEventRecord(p->ready, p->side);
@@ -133,9 +135,19 @@ moe_status moe_pool_create(const moe_shape* shape, int32_t n_slots, const uint8_
 moe_status moe_expert_pool_load(moe_pool* p, const int32_t* topk_idx, int32_t T, void* stream) {
   if (!p || !topk_idx) return set_error(MOE_ERR_INVALID, "pool and topk_idx must be non-NULL");
   const int k = p->shape.top_k, E = p->shape.n_experts;
-  if (T < 1 || T > kMaxDecodeT) return set_error(MOE_ERR_INVALID, "T must be in [1, %d]", kMaxDecodeT);
+  if (T < 1) return set_error(MOE_ERR_INVALID, "T must be >= 1 (got %d)", T);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int n = T * k;
+  if (n > p->h_ids_cap) {
+    // a larger step than any before: grow the pinned read-back buffer (decode-sized steps
+    // never reach this; the first many-token step pays one pinned allocation)
+    int32_t* grown = nullptr;
+    cudaError_t ea = cudaHostAlloc((void**)&grown, sizeof(int32_t) * (size_t)n, cudaHostAllocDefault);
+    if (ea != cudaSuccess) return cuda_fail(ea, "pinned id buffer");
+    cudaFreeHost(p->h_ids);
+    p->h_ids = grown;
+    p->h_ids_cap = n;
+  }
   // The ids are needed on the host.  Synchronising the caller stream also guarantees that
   // every earlier forward on it has finished reading the slots this step may overwrite.
   cudaError_t e = cudaMemcpyAsync(p->h_ids, topk_idx, sizeof(int32_t) * n, cudaMemcpyDeviceToHost, s);
@@ -253,7 +265,8 @@ moe_status moe_expert_pool_load(moe_pool* p, const int32_t* topk_idx, int32_t T,
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s, p->ready, 0);
   if (e != cudaSuccess) return cuda_fail(e, "slot table upload");
   p->ready_recorded = true;
-  for (const Load& ld : loads) {
+  for (size_t li = 0; li < loads.size(); ++li) {
+    const Load& ld = loads[li];
     e = cudaMemcpyAsync(p->dev_pool + (int64_t)ld.slot * p->stride, p->host_blobs + (int64_t)ld.id * p->stride,
                         (size_t)p->stride, cudaMemcpyHostToDevice, p->side);
     if (e != cudaSuccess) {
@@ -269,7 +282,23 @@ moe_status moe_expert_pool_load(moe_pool* p, const int32_t* topk_idx, int32_t T,
                    CUDA_SUCCESS) {
       e = cudaMemcpyAsync(p->dev_slot_table + ld.id, p->h_final + ld.id, sizeof(int32_t), cudaMemcpyHostToDevice,
                           p->side);
-      if (e != cudaSuccess) return cuda_fail(e, "slot table entry");
+      if (e != cudaSuccess) {
+        // This entry and those of the loads not yet issued stay pending on the device.  Undo
+        // them on the host, so that no later step counts them as hits on slots that hold
+        // other weights; the next load uploads the whole table again from the host mirror.
+        // The forward of this step must not run (its kernel would wait for the entries).
+        for (size_t lj = li; lj < loads.size(); ++lj) {
+          const Load& lr = loads[lj];
+          if (p->slot_of[lr.id] == lr.slot) {
+            p->slot_of[lr.id] = -1;
+            p->expert_in[lr.slot] = -1;
+            p->stats.h2d_bytes -= p->stride;
+          }
+          p->h_final[lr.id] = -1;
+        }
+        p->step_no++;
+        return cuda_fail(e, "slot table entry");
+      }
     }
   }
   p->step_no++;

@@ -1254,36 +1254,50 @@ cudaError_t launch_group(const PrefillArgs& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
+// Norms, fp32 router logits on the tensor cores and the certified top-k of p.T tokens
+// (p.route must be set): the routing step of the many-token path, also used alone by
+// moe_router_topk.
+static cudaError_t launch_route(const PrefillArgs& p, int n_sm, cudaStream_t s) {
+  const int T = p.T, E = p.E, H = p.H;
+  cudaError_t e;
+  const int rows = T + E + 1;
+  k_norms<<<(rows * 32 + 255) / 256, 256, 0, s>>>(p.x, T, H, p.wr, p.wsg, E, p.xnorm, p.wnorm);
+  const int mt_n = (E + 127) / 128, nt = (T + 127) / 128;
+  k_router_units<<<(mt_n * nt + 255) / 256, 256, 0, s>>>(p.units_rt, p.n_units + 2, T, E);
+  GemmArgs g = p.g;
+  g.units = p.units_rt;
+  g.n_units = p.n_units + 2;
+  g.n_rows = 128;
+  g.sc_tma = 0;
+  if ((e = map_bf16(&g.map_w, p.wr, E, H, H, 128)) != cudaSuccess) return e;
+  if ((e = map_bf16(&g.map_tok, p.x, T, H, H, kTRows)) != cudaSuccess) return e;
+  // the router GEMM reads bf16 rows only; the code width does not enter it
+  if ((e = launch_gemm<4, kModeRouter>(g, n_sm, s)) != cudaSuccess) return e;
+  k_route<<<(T + 7) / 8, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+static int sm_count() {
   int dev = 0, n_sm = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-  const int T = p.T, E = p.E, H = p.H;
+  return n_sm;
+}
+
+cudaError_t launch_prefill_route(const PrefillArgs& p, cudaStream_t s) { return launch_route(p, sm_count(), s); }
+
+cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
+  const int n_sm = sm_count();
+  const int T = p.T, H = p.H;
   cudaError_t e;
   // accumulator of the down products
   if ((e = cudaMemsetAsync(p.acc, 0, sizeof(float) * (size_t)T * H, s)) != cudaSuccess) return e;
   // norms, router logits, certified top-k
   prof_mark(0, false, s);
-  {
-    const int rows = T + E + 1;
-    if (p.route) {
-      k_norms<<<(rows * 32 + 255) / 256, 256, 0, s>>>(p.x, T, H, p.wr, p.wsg, E, p.xnorm, p.wnorm);
-      const int mt_n = (E + 127) / 128, nt = (T + 127) / 128;
-      k_router_units<<<(mt_n * nt + 255) / 256, 256, 0, s>>>(p.units_rt, p.n_units + 2, T, E);
-      GemmArgs g = p.g;
-      g.units = p.units_rt;
-      g.n_units = p.n_units + 2;
-      g.n_rows = 128;
-      g.sc_tma = 0;
-      if ((e = map_bf16(&g.map_w, p.wr, E, H, H, 128)) != cudaSuccess) return e;
-      if ((e = map_bf16(&g.map_tok, p.x, T, H, H, kTRows)) != cudaSuccess) return e;
-      if ((e = (bits == 4 ? launch_gemm<4, kModeRouter>(g, n_sm, s) : launch_gemm<8, kModeRouter>(g, n_sm, s))) !=
-          cudaSuccess)
-        return e;
-      k_route<<<(T + 7) / 8, 256, 0, s>>>(p);
-    } else {
-      k_gate<<<(T + 7) / 8, 256, 0, s>>>(p);
-    }
+  if (p.route) {
+    if ((e = launch_route(p, n_sm, s)) != cudaSuccess) return e;
+  } else {
+    k_gate<<<(T + 7) / 8, 256, 0, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   prof_mark(0, true, s);

@@ -33,19 +33,45 @@ __device__ __align__(256) unsigned char g_moe_static_scratch[kMoeStaticScratchBy
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};  // the context the cached address belongs to
 
-// Device address of the scratch on the current device, looked up once per device.
+// cuCtxGetCurrent through the runtime's driver entry point (the library does not link the
+// driver library); null if the driver does not offer it.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (CtxGetCurrentFn) nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  return fn;
+}
+
+// Device address of the scratch on the current device.  It is looked up once per device and
+// context: after a device reset (cudaDeviceReset) the device gets a new primary context, the
+// cached address no longer names the array, and the next call looks it up again.
 moe_status scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return set_error(MOE_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
+  const CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  const auto current_ctx = [&] {
+    CUcontext c = nullptr;
+    if (!get_ctx || get_ctx(&c) != CUDA_SUCCESS) c = nullptr;
+    return c;
+  };
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
+  if (!g_scratch_addr[dev] || g_scratch_ctx[dev] != current_ctx()) {
+    // the lookup also makes the device's primary context current (creating it if needed)
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_moe_static_scratch);
     if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress of the static scratch");
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = current_ctx();
   }
   *out = g_scratch_addr[dev];
   return MOE_OK;

@@ -9,7 +9,7 @@ import torch
 
 import oracle
 import synth
-from helpers import forward, ws_for
+from helpers import assert_close, forward, oracle_forward, ws_for
 from int4_expert_gemv_router_b200 import abi, build
 
 pytestmark = pytest.mark.gpu
@@ -202,5 +202,39 @@ def test_pool_overlap_mode_needs_fused_shape():
             abi.moe_pool_set_overlap(P.h, True)
         assert ei.value.status == -5  # MOE_ERR_UNSUPPORTED
         abi.moe_pool_set_overlap(P.h, False)
+    finally:
+        P.close()
+
+
+def test_pool_many_token_step():
+    """A many-token step through the pool: moe_router_topk and moe_expert_pool_load on 40
+    tokens (more than the decode path's 8), then the many-token layer forward reading the
+    experts through the slot table.  Slot decisions equal the oracle's, and the output matches
+    both the all-resident forward and the oracle within tolerance (the many-token path sums
+    its down products with atomics, so bits may differ in the last place)."""
+    w = synth.WORKLOADS["tiny"].with_(n_experts=16, top_k=2, seed=34)
+    n_slots = 12
+    P = Pool(w, n_slots)
+    sim = oracle.SlotCache(w.n_experts, n_slots)
+    try:
+        T = 40
+        for s in range(3):
+            x = synth.activations(w, 200 + s, tokens=T, device=DEV)
+            # a router bias that keeps the step within the pool's 12 slots
+            P.L.router_bias = torch.zeros(w.n_experts, dtype=torch.float32, device=DEV)
+            P.L.router_bias[(s * 5 + torch.arange(6)) % w.n_experts] = 40.0
+            idx, p = _route(P, x)
+            abi.moe_expert_pool_load(P.h, idx, T)
+            sim.step(idx.cpu().numpy().reshape(-1).tolist())
+            slot_of, expert_in = abi.moe_pool_slot_table(P.h, w.n_experts, n_slots)
+            assert slot_of == sim.slot_of.tolist() and expert_in == sim.expert_in.tolist()
+            out_pool, _, _, ws = forward(w, P.L, x, residual=x, pool=P.dev, slot_table=P.table, n_slots=n_slots,
+                                         topk=(idx, p))
+            assert abi.moe_ws_check(ws) == 0
+            out_res, *_ = forward(w, P.L, x, residual=x, topk=(idx, p))
+            a, b = out_pool.float(), out_res.float()
+            assert (a - b).abs().max().item() <= 1e-2 * b.abs().max().item() + 1e-3
+            ref = oracle_forward(w, P.L, x, residual=x, idx=idx.cpu().numpy(), p=p.cpu().numpy().astype(np.float64))
+            assert_close(out_pool, ref["out"])
     finally:
         P.close()

@@ -42,7 +42,10 @@ def test_static_scratch_matches_workspace_path_twice(wname, T):
         ref_out, ref_idx, ref_p, _ = forward(w, L, x, residual=x)
         out, idx, p = _static(w, L, x, x)
         assert torch.equal(idx, ref_idx)
-        assert torch.allclose(p, ref_p, rtol=1e-6, atol=0)
+        # the decode path is deterministic: the same kernel on the same inputs gives the same
+        # bits whichever scratch it uses
+        assert torch.equal(p, ref_p)
+        assert torch.equal(out, ref_out)
         r, o = ref_out.float(), out.float()
         assert (r - o).abs().max().item() <= REL * r.abs().max().item() + ABS
 
