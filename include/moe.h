@@ -194,6 +194,41 @@ MOE_API moe_status moe_stack_forward(const moe_shape* shape, int32_t T, const mo
                                      int32_t n_layers, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * moe_layer_forward_partial -- one rank's share of an expert-parallel layer (the routed
+ * experts of a layer sharded over GPUs; the Swiftlet pages run one device and describe no
+ * sharding, so this follows the plain reading of splitting the layer's experts, «Paquets
+ * Swiftlet 80B Qwen dans Mac…», paragraph 5: 10 of 512 experts per token).
+ * Arguments as moe_layer_forward, except:
+ *   slot_table     (dev) int32 [E]: this rank's slots; -3 marks an expert that another rank
+ *                  holds: its pairs are left out of this rank's sum (no error bit)
+ *   include_shared 1: the shared expert's term is part of this rank's sum (one rank only)
+ *   partial_out    (dev) fp32 [T, H] out: sum over this rank's selected experts of
+ *                  p * y_e (+ sigmoid gate * y_shared if include_shared), no residual, not rounded
+ * Every rank routes the same tokens and gets the same top-k (topk_idx_out), so the ranks'
+ * partials add up to the layer; sum them (e.g. an NCCL all-reduce) and finish with
+ * moe_combine_partials.  T: 1..8 on shapes with a fused decode kernel, else
+ * MOE_ERR_UNSUPPORTED.
+ */
+MOE_API moe_status moe_layer_forward_partial(const moe_shape* shape, const void* x, int32_t T,
+                                             const void* w_router, const float* router_bias,
+                                             const int32_t* topk_idx_in, const float* topk_w_in,
+                                             const uint8_t* pool, const int32_t* slot_table,
+                                             int64_t n_slots, const uint8_t* shared_blob,
+                                             const void* w_shared_gate, int32_t include_shared,
+                                             float* partial_out, int32_t* topk_idx_out, float* topk_w_out,
+                                             void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_combine_partials -- out = bf16_rne(partials[0] + ... + partials[n_parts-1] + residual),
+ * summed in index order: the end of an expert-parallel layer.
+ *   partials (host) array of n_parts (1..16) device pointers, each fp32 [T, H] (one pointer
+ *            after an all-reduce has summed the ranks' partials in place)
+ *   residual (dev) bf16 [T, H] or NULL;  out (dev) bf16 [T, H]
+ */
+MOE_API moe_status moe_combine_partials(const float* const* partials, int32_t n_parts, int32_t T,
+                                        int32_t hidden, const void* residual, void* out, void* stream);
+
+/*
  * moe_layer_forward_static -- moe_layer_forward for callers that cannot allocate device
  * memory.  The Swiftlet pages have no counterpart of this call.
  *

@@ -62,6 +62,9 @@ _SIGS = {
                                          _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_layer_forward_static": (ctypes.c_int, [ctypes.POINTER(moe_shape), _P, _I32, _P, _P, _P, _P, _P, _P,
                                                 _I64, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_layer_forward_partial": (ctypes.c_int, [ctypes.POINTER(moe_shape), _P, _I32, _P, _P, _P, _P, _P, _P, _I64,
+                                                 _P, _P, _I32, _P, _P, _P, _P, _SZ, _P]),
+    "moe_combine_partials": (ctypes.c_int, [_P, _I32, _I32, _I32, _P, _P, _P]),
     "moe_stack_forward": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, ctypes.POINTER(moe_layer_desc), _I32, _P,
                                          _SZ, _P]),
     "moe_group_pairs": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, _P, _P, _P, _P, _SZ, _P]),
@@ -167,6 +170,23 @@ def moe_layer_forward(shape, x, T, w_router, router_bias, topk_idx_in, topk_w_in
                                    _ptr(shared_blob), _ptr(w_shared_gate), _ptr(residual), _ptr(out),
                                    _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(ws),
                                    ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_layer_forward_partial(shape, x, T, w_router, router_bias, topk_idx_in, topk_w_in, pool, slot_table, n_slots,
+                              shared_blob, w_shared_gate, include_shared, partial_out, topk_idx_out, topk_w_out, ws,
+                              stream=None):
+    """One expert-parallel rank's fp32 share of the layer (slot_table -3: held by another rank)."""
+    _check(lib().moe_layer_forward_partial(ctypes.byref(shape), _ptr(x), T, _ptr(w_router), _ptr(router_bias),
+                                           _ptr(topk_idx_in), _ptr(topk_w_in), _ptr(pool), _ptr(slot_table), n_slots,
+                                           _ptr(shared_blob), _ptr(w_shared_gate), int(include_shared),
+                                           _ptr(partial_out), _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(ws),
+                                           ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_combine_partials(partials, T, hidden, residual, out, stream=None):
+    """out = bf16(sum of the fp32 partials in order + residual)."""
+    arr = (ctypes.c_void_p * len(partials))(*[_ptr(t) for t in partials])
+    _check(lib().moe_combine_partials(arr, len(partials), T, hidden, _ptr(residual), _ptr(out), _stream(stream)))
 
 
 def layer_desc(x=None, w_router=None, router_bias=None, topk_idx_in=None, topk_w_in=None, pool=None,

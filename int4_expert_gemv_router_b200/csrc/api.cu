@@ -203,7 +203,8 @@ moe_status moe_router_topk(const moe_shape* shape, const void* x, int32_t T, con
 }
 
 static moe_status run_fused_stack(const moe_shape* shape, int32_t T, const moe_layer_desc* L, int32_t n,
-                                  const DecodeArgs& a, cudaStream_t s) {
+                                  const DecodeArgs& a, cudaStream_t s, float* out_partial = nullptr,
+                                  int with_shared = 1) {
   static FusedArgs f;  // large (kMaxFusedLayers descriptors); filled per call under g_fused_mu
   static std::mutex g_fused_mu;
   std::lock_guard<std::mutex> lock(g_fused_mu);
@@ -236,6 +237,8 @@ static moe_status run_fused_stack(const moe_shape* shape, int32_t T, const moe_l
     d.topk_w_out = L[l].topk_w_out;
     d.topk_idx_in = L[l].topk_idx_in;
     d.topk_w_in = L[l].topk_w_in;
+    d.out_partial = out_partial;  // set only for single-layer partial calls
+    d.with_shared = with_shared;
   }
   bool ok = true;
   prof_mark(0, false, s);
@@ -437,6 +440,66 @@ moe_status moe_layer_forward(const moe_shape* shape, const void* x, int32_t T, c
   e = launch_down_decode(a, shape->bits, s, &ok);
   if (e != cudaSuccess) return cuda_fail(e, "down launch");
   prof_mark(2, true, s);
+  return MOE_OK;
+}
+
+moe_status moe_layer_forward_partial(const moe_shape* shape, const void* x, int32_t T, const void* w_router,
+                                     const float* router_bias, const int32_t* topk_idx_in, const float* topk_w_in,
+                                     const uint8_t* pool, const int32_t* slot_table, int64_t n_slots,
+                                     const uint8_t* shared_blob, const void* w_shared_gate, int32_t include_shared,
+                                     float* partial_out, int32_t* topk_idx_out, float* topk_w_out, void* ws,
+                                     size_t ws_bytes, void* stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->shared_inter != shape->inter)
+    return set_error(MOE_ERR_UNSUPPORTED, "this build needs shared_inter == inter");
+  if (T < 1 || T > kMaxDecodeT)
+    return set_error(MOE_ERR_UNSUPPORTED, "the partial forward takes 1..%d tokens (got %d)", kMaxDecodeT, T);
+  if (!fused_shape_supported(shape->hidden, shape->inter, shape->bits, shape->n_experts))
+    return set_error(MOE_ERR_UNSUPPORTED, "no fused decode kernel for hidden=%d inter=%d bits=%d E=%d",
+                     shape->hidden, shape->inter, shape->bits, shape->n_experts);
+  if (!partial_out || !aligned(partial_out, 16)) return set_error(MOE_ERR_INVALID, "partial_out must be non-NULL and 16-byte aligned");
+  if (include_shared != 0 && include_shared != 1) return set_error(MOE_ERR_INVALID, "include_shared must be 0 or 1");
+  moe_layer_desc d{};
+  d.x = x;
+  d.w_router = w_router;
+  d.router_bias = router_bias;
+  d.topk_idx_in = topk_idx_in;
+  d.topk_w_in = topk_w_in;
+  d.pool = pool;
+  d.slot_table = slot_table;
+  d.n_slots = n_slots;
+  d.shared_blob = shared_blob;
+  d.w_shared_gate = w_shared_gate;
+  d.residual = nullptr;
+  d.out = partial_out;  // checked for alignment only; the kernel writes partial_out
+  d.topk_idx_out = topk_idx_out;
+  d.topk_w_out = topk_w_out;
+  if ((st = check_layer(shape, &d, true)) != MOE_OK) return st;
+  DecodeArgs a;
+  if ((st = fill_decode_args(shape, T, ws, ws_bytes, &a)) != MOE_OK) return st;
+  return run_fused_stack(shape, T, &d, 1, a, static_cast<cudaStream_t>(stream), partial_out, include_shared);
+}
+
+moe_status moe_combine_partials(const float* const* partials, int32_t n_parts, int32_t T, int32_t hidden,
+                                const void* residual, void* out, void* stream) {
+  if (!partials || !out) return set_error(MOE_ERR_INVALID, "partials and out must be non-NULL");
+  if (n_parts < 1 || n_parts > kMaxPartials)
+    return set_error(MOE_ERR_INVALID, "n_parts must be in [1, %d] (got %d)", kMaxPartials, n_parts);
+  if (T < 1 || hidden < 1) return set_error(MOE_ERR_INVALID, "T and hidden must be >= 1");
+  PartialArgs p{};
+  for (int i = 0; i < n_parts; ++i) {
+    if (!partials[i] || !aligned(partials[i], 16)) return set_error(MOE_ERR_INVALID, "partial %d is NULL or misaligned", i);
+    p.part[i] = partials[i];
+  }
+  if (!aligned(out, 16) || (residual && !aligned(residual, 16)))
+    return set_error(MOE_ERR_INVALID, "out and residual must be 16-byte aligned");
+  p.n = n_parts;
+  p.count = (size_t)T * hidden;
+  p.residual = static_cast<const uint16_t*>(residual);
+  p.out = static_cast<uint16_t*>(out);
+  cudaError_t e = launch_combine_partials(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   return MOE_OK;
 }
 

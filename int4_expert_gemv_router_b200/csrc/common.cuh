@@ -17,6 +17,9 @@ constexpr int kMaxExperts = 1024;
 // Slot-table entry of an expert whose blob is still being copied into its slot (a pool in
 // overlap mode); the copy stream overwrites it with the slot once the blob has landed.
 constexpr int32_t kSlotPending = -2;
+// Slot-table entry of an expert that another rank holds (expert parallelism): the pair is
+// left out of this rank's partial sum without an error.
+constexpr int32_t kSlotRemote = -3;
 
 // Device error-word bits (mirrors MOE_DEVERR_* in include/moe.h).
 constexpr uint32_t kErrBadExpert = 0x1u;
@@ -177,6 +180,8 @@ struct FusedLayer {
   float* topk_w_out;
   const int32_t* topk_idx_in;
   const float* topk_w_in;
+  float* out_partial;  // fp32 [T, H]: if set, the layer's partial sum goes here (no residual, no rounding)
+  int with_shared;     // 1: the shared expert is part of this layer's sum
 };
 constexpr int kMaxFusedLayers = 64;
 
@@ -323,6 +328,17 @@ void prof_mark(int i, bool end, cudaStream_t s);
 cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s);
 cudaError_t launch_prefill_route(const PrefillArgs& p, cudaStream_t s);
 cudaError_t launch_group(const PrefillArgs& p, cudaStream_t s);
+
+// Sum of the expert-parallel ranks' fp32 partial outputs (fixed order) + residual -> bf16.
+constexpr int kMaxPartials = 16;
+struct PartialArgs {
+  const float* part[kMaxPartials];
+  int n;
+  size_t count;               // T * H elements
+  const uint16_t* residual;   // bf16 or null
+  uint16_t* out;              // bf16
+};
+cudaError_t launch_combine_partials(const PartialArgs& p, cudaStream_t s);
 
 // Kernel launchers (decode.cu).  Return cudaError_t of the launch.
 cudaError_t launch_router_decode(const DecodeArgs& a, bool build_plan, cudaStream_t s);

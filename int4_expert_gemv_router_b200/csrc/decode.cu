@@ -550,4 +550,46 @@ cudaError_t launch_down_decode(const DecodeArgs& a, int bits, cudaStream_t s, bo
   return cudaSuccess;
 }
 
+// out = bf16(sum of the partials in index order + residual): the combine of an
+// expert-parallel layer after the partials have been summed across ranks (or, on one GPU,
+// several ranks' partials summed here).
+__global__ void k_combine_partials(const PartialArgs p) {
+  const size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (i >= p.count) return;
+  if (i + 4 <= p.count) {
+    float4 v = __ldg(reinterpret_cast<const float4*>(p.part[0] + i));
+    for (int r = 1; r < p.n; ++r) {
+      const float4 w = __ldg(reinterpret_cast<const float4*>(p.part[r] + i));
+      v.x += w.x;
+      v.y += w.y;
+      v.z += w.z;
+      v.w += w.w;
+    }
+    if (p.residual) {
+      const uint2 rr = __ldg(reinterpret_cast<const uint2*>(p.residual + i));
+      v.x += bf_lo(rr.x);
+      v.y += bf_hi(rr.x);
+      v.z += bf_lo(rr.y);
+      v.w += bf_hi(rr.y);
+    }
+    uint2 o;
+    o.x = (uint32_t)f2bf(v.x) | ((uint32_t)f2bf(v.y) << 16);
+    o.y = (uint32_t)f2bf(v.z) | ((uint32_t)f2bf(v.w) << 16);
+    *reinterpret_cast<uint2*>(p.out + i) = o;
+  } else {
+    for (size_t j = i; j < p.count; ++j) {
+      float v = p.part[0][j];
+      for (int r = 1; r < p.n; ++r) v += p.part[r][j];
+      if (p.residual) v += bf1(p.residual[j]);
+      p.out[j] = f2bf(v);
+    }
+  }
+}
+
+cudaError_t launch_combine_partials(const PartialArgs& p, cudaStream_t s) {
+  const size_t n4 = (p.count + 3) / 4;
+  k_combine_partials<<<(unsigned)((n4 + 255) / 256), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
 }  // namespace moe

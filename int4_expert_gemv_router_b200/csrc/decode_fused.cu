@@ -398,8 +398,9 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
         for (int u = 0; u < act_n; ++u) slot_of_unit(Lc, u);  // every pending slot settled
         __syncwarp();
         const int per_stage = SB / (nJ * ROWD_BYTES);
-        for (int u = 0; u <= act_n && ok;) {
-          const int cnt = min(per_stage, act_n + 1 - u);
+        const int n_units_d = act_n + (Lc.with_shared ? 1 : 0);  // the shared expert last
+        for (int u = 0; u < n_units_d && ok;) {
+          const int cnt = min(per_stage, n_units_d - u);
           const int s = q % NS;
           if (!mbar_wait(&empty_bar[s], ((q / NS) & 1) ^ 1)) {
             ok = false;
@@ -477,7 +478,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
     // ---- phase R: router rows, shared-gate row, shared gate/up rows ----
     {
       const int n_router = (routed ? E : 0) + 1;
-      const int n_items = n_router + I / RPWg;
+      const int n_items = n_router + (Lc.with_shared ? I / RPWg : 0);
       for (int it = blockIdx.x + G * cw; it < n_items; it += NW) {  // item i: CTA i % G
         if (it < n_router) {
           const bool gate_row = (it == n_router - 1);
@@ -599,7 +600,9 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
           if (T == 1) {
             // one token: the k ids are distinct, so this warp groups them itself (ranks by
             // shuffles) and the CTA skips the general grouping below
-            const int key = lane < k ? (id >= 0 ? id : E) : 0x7fffffff;
+            // an expert held by another rank (expert parallelism) is left out like an
+            // invalid id, without a flag: its term is that rank's
+            const int key = lane < k ? ((id >= 0 && S_SLOT[id] != kSlotRemote) ? id : E) : 0x7fffffff;
             int rank = 0, before = 0;
             for (int j = 0; j < k; ++j) {
               const int kj = __shfl_sync(0xffffffffu, key, j);
@@ -644,7 +647,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
         const int e = P_IDS[i];
         const bool valid = e >= 0 && e < E;
         if (!valid && blockIdx.x == 0) atomicOr(&a.ctrl->err, kErrBadExpert);
-        key[i] = valid ? e : E;
+        key[i] = (valid && S_SLOT[e] != kSlotRemote) ? e : E;
       }
       bar_cons();
       for (int i = tid; i < TK; i += kConsThreads) {
@@ -769,8 +772,9 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
       const int per_stage = SB / (nJ * ROWD_BYTES);
       const int sub = lane % NCLd, rsub = lane / NCLd;
       float* red = reinterpret_cast<float*>(smem + a.sm.red) + (size_t)cw * a.jmax * (NCLd + 1);
-      for (int u0 = 0; u0 <= act_n;) {
-        const int cnt = min(per_stage, act_n + 1 - u0);
+      const int n_units_d = act_n + (Lc.with_shared ? 1 : 0);  // the shared expert last
+      for (int u0 = 0; u0 < n_units_d;) {
+        const int cnt = min(per_stage, n_units_d - u0);
         const int s = q % NS;
         if (!mbar_wait(&full_bar[s], (q / NS) & 1)) {
           ok = false;
@@ -881,9 +885,15 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
             const int p = P_POS[t * k + kk];
             if (p >= 0) v += partial[(size_t)p * a.jmax + jl];
           }
-          v += partial[(size_t)(n_valid + t) * a.jmax + jl];
-          if (Lc.residual) v += (i == tid) ? res_v : bf1(__ldcg(Lc.residual + (size_t)t * H + j0 + jl));
-          Lc.out[(size_t)t * H + j0 + jl] = f2bf(v);
+          if (Lc.with_shared) v += partial[(size_t)(n_valid + t) * a.jmax + jl];
+          if (Lc.out_partial) {
+            // expert parallelism: this rank's fp32 share of the sum; the ranks' shares are
+            // added by an all-reduce and rounded once, with the residual, by the combine
+            Lc.out_partial[(size_t)t * H + j0 + jl] = v;
+          } else {
+            if (Lc.residual) v += (i == tid) ? res_v : bf1(__ldcg(Lc.residual + (size_t)t * H + j0 + jl));
+            Lc.out[(size_t)t * H + j0 + jl] = f2bf(v);
+          }
         }
       }
     }
