@@ -414,6 +414,133 @@ def run_decode_ep(args, w, T, device, rank, world):
     }
 
 
+# ======================================================================================
+# Gated DeltaNet decode step (the linear-attention layers' recurrence)
+# ======================================================================================
+def run_gdn(args, name, device, rank):
+    """One step = one token of B sequences through the recurrence of every linear-attention
+    layer (36 launches, one per layer, in a CUDA graph; each layer has its own resident fp32
+    state and its own seeded q/k/v/gates).  Per-launch durations come from an eager pass with
+    events around each launch."""
+    from int4_expert_gemv_router_b200 import abi, build
+    build.build()
+    c = synth.GDN_WORKLOADS[name]
+    Hk, Hv, dk, dv, nL, B = c["n_k_heads"], c["n_v_heads"], c["d_k"], c["d_v"], c["layers"], c["batch"]
+    K, W = args.steps, args.warmup
+    shape = abi.moe_gdn_shape(Hk, Hv, dk, dv)
+    states = [synth.gdn_state(Hv, dk, dv, B, c["seed"] + 1000 * rank + l, device) for l in range(nL)]
+    ins = [synth.gdn_inputs(Hk, Hv, dk, dv, B, 1, c["seed"] + 1000 * rank + 100 + l, device) for l in range(nL)]
+    ins = [tuple(t[0].contiguous() for t in x) for x in ins]
+    outs = [torch.empty(B, Hv, dv, dtype=torch.bfloat16, device=device) for _ in range(nL)]
+    stream = torch.cuda.Stream(device)
+
+    def layer_calls():
+        for l in range(nL):
+            q, k, v, g, beta = ins[l]
+            abi.moe_gdn_decode_step(shape, B, states[l], q, k, v, g, beta, outs[l])
+
+    with torch.cuda.stream(stream):
+        layer_calls()
+    stream.synchronize()
+    g_ = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_, stream=stream):
+        layer_calls()
+    with torch.cuda.stream(stream):
+        for _ in range(W):
+            g_.replay()
+    stream.synchronize()
+    barrier(device)
+    clk = ClockSampler(device.index)
+    clk.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(K):
+            g_.replay()
+        e1.record(stream)
+    e1.synchronize()
+    clocks = clk.stop()
+    ms = reduce_max(e0.elapsed_time(e1), device)
+    # per-launch duration on the launching stream (a GPU sleep first, so the launches queue up)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nL)]
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(20_000_000)
+        for l in range(nL):
+            q, k, v, g, beta = ins[l]
+            evs[l][0].record(stream)
+            abi.moe_gdn_decode_step(shape, B, states[l], q, k, v, g, beta, outs[l])
+            evs[l][1].record(stream)
+    stream.synchronize()
+    launch_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in evs)
+    # end to end: the step's inputs from pinned host memory and its outputs back, every step
+    host_in = [tuple(t.cpu().pin_memory() for t in x) for x in ins]
+    host_out = torch.empty(nL, B, Hv, dv, dtype=torch.bfloat16).pin_memory()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for _ in range(K):
+            for l in range(nL):
+                for dst, src in zip(ins[l], host_in[l]):
+                    dst.copy_(src, non_blocking=True)
+            g_.replay()
+            for l in range(nL):
+                host_out[l].copy_(outs[l], non_blocking=True)
+        f1.record(stream)
+    f1.synchronize()
+    e2e_ms = reduce_max(f0.elapsed_time(f1), device)
+    in_bytes = sum(t.numel() * t.element_size() for t in ins[0])
+    return dict(c=c, ms=ms, clocks=clocks, launch_us=launch_us, e2e_ms=e2e_ms, in_bytes=in_bytes * nL,
+                out_bytes=nL * B * Hv * dv * 2, state=states[0], ins=ins[0])
+
+
+def cpu_baseline_gdn(r, budget_s=10.0):
+    """The fp64 oracle as it stands: one sequence's step through layers until ~budget_s, scaled."""
+    import oracle
+    c = r["c"]
+    q, k, v, g, beta = (t[0].float().double().cpu().numpy() for t in r["ins"])
+    S = r["state"][0].double().cpu().numpy()
+    t_total, n = 0.0, 0
+    while t_total < budget_s and n < 10 * c["layers"]:
+        t0 = time.perf_counter()
+        oracle.gdn_step(S, q, k, v, g, beta)
+        t_total += time.perf_counter() - t0
+        n += 1
+    per_layer = t_total / n
+    return {"value": round(1.0 / (per_layer * c["layers"]), 3), "unit": "tokens/s", "cores": cpu_threads(),
+            "kind": "oracle", "sample": f"{n} single-sequence layer steps (fp64 numpy oracle, {per_layer * 1e3:.1f} ms "
+                                        f"each), scaled to a {c['layers']}-layer token"}
+
+
+def gdn_line(args, name, r, n_gpus, peaks, peak_kind, cpu_base):
+    c = r["c"]
+    K = args.steps
+    B, nL = c["batch"], c["layers"]
+    per_launch = 2 * 4 * B * c["n_v_heads"] * c["d_v"] * c["d_k"] + 2 * B * (2 * c["n_k_heads"] * c["d_k"] +
+                                                                             2 * c["n_v_heads"] * c["d_v"]) + 8 * B * c["n_v_heads"]
+    hbm = peaks["hbm_gbs"]
+    achieved = per_launch / (r["launch_us"] * 1e-6) / 1e9
+    line = {
+        "metric": "Gated DeltaNet decode-step tokens/s; achieved HBM GB/s",
+        "value": round(n_gpus * B * K / (r["ms"] / 1e3), 1), "unit": "tokens/s", "n_gpus": n_gpus, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(r["ms"] / K, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp32 state, bf16 q/k/v/out", "data": "synthetic (seeded)",
+        "config": {"workload": name, "n_k_heads": c["n_k_heads"], "n_v_heads": c["n_v_heads"], "d_k": c["d_k"],
+                   "d_v": c["d_v"], "layers": nL, "sequences": B, "parallelism": f"replicas{n_gpus}",
+                   "l2": f"{nL * B * c['n_v_heads'] * c['d_v'] * c['d_k'] * 4 / 1e6:.0f} MB of state per step"},
+        "roofline": {"bound": "hbm", "kernel": "k_gdn_step (one layer)", "achieved": round(achieved, 1), "peak": hbm,
+                     "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
+                     "launch_us": round(r["launch_us"], 3), "bytes_per_launch": per_launch,
+                     "peak_kind": f"{peak_kind} hbm_gbs (burst copy)"},
+        "clocks": r["clocks"],
+        "e2e": {"value": round(n_gpus * B * K / (r["e2e_ms"] / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": r["in_bytes"], "d2h_bytes_per_step": r["out_bytes"]},
+        "gpu_launches": nL * K,
+    }
+    if cpu_base is not None:
+        line["cpu_baseline"] = cpu_base
+    return line
+
+
 def _bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
 
@@ -855,7 +982,7 @@ def parse(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode80b",
-                    choices=["decode80b", "decode35b", "prefill", "pool_int4", "pool_int8"])
+                    choices=["decode80b", "decode35b", "prefill", "pool_int4", "pool_int8", "gdn80b", "gdn80b_b8"])
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--policy", choices=["lfu_recency", "lru", "lfu"], default="lfu_recency",
@@ -871,10 +998,35 @@ def parse(argv=None):
     return ap.parse_args(argv)
 
 
+def main_gdn(args):
+    rank, local, n_ranks = dist_env()
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the MoE layer workloads"}))
+        return 0
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist("nccl")
+    peaks, peak_kind = load_peaks()
+    r = run_gdn(args, args.workload, device, rank)
+    cpu_base = cpu_baseline_gdn(r) if (rank == 0 and n_ranks == 1 and not args.no_cpu_baseline) else None
+    line = gdn_line(args, args.workload, r, n_ranks, peaks, peak_kind, cpu_base)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     args = parse(argv)
     if args.warmup < 3:
         args.warmup = 3
+    if args.workload.startswith("gdn"):
+        return main_gdn(args)
     w = synth.WORKLOADS[args.workload]
     if args.layers:
         w = w.with_(layers=args.layers)

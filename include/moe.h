@@ -308,6 +308,35 @@ MOE_API moe_status moe_ws_router_logits(const moe_shape* shape, int32_t T, void*
                                         float** logits);
 
 /* ------------------------------------------------------------------------------------ */
+/* Gated DeltaNet decode step: the linear-attention layers that make up three quarters of */
+/* the hybrid model's layers, each with a fixed-size recurrent state («Paquets Swiftlet 80B */
+/* Qwen dans Mac…», paragraph 6; «Swiftlet: 在 Mac 和 iPhone 上執行…», 技術譜系與正確性). */
+/* ------------------------------------------------------------------------------------ */
+typedef struct {
+  int32_t n_k_heads;  /* H_k: query/key heads                                              */
+  int32_t n_v_heads;  /* H_v: value heads (a multiple of H_k; value head h reads key head   */
+                      /*      h / (H_v / H_k))                                               */
+  int32_t d_k;        /* key/query head width: 64, 128 or 256                                */
+  int32_t d_v;        /* value head width                                                    */
+} moe_gdn_shape;
+
+/*
+ * moe_gdn_decode_step -- one token of B sequences through the gated delta rule, per value
+ * head (the pages print no formula; this is the rule that names the layer):
+ *   k^ = k / ||k||,  q^ = q / (||q|| sqrt(d_k)),  alpha = exp(g)
+ *   S' = alpha S + beta (v - alpha S k^) k^T   (= alpha S (I - beta k^ k^T) + beta v k^T)
+ *   out = S' q^
+ *   state (dev) fp32 [B, H_v, d_v, d_k], read and overwritten with S'
+ *   q, k  (dev) bf16 [B, H_k, d_k];  v (dev) bf16 [B, H_v, d_v]
+ *   g     (dev) fp32 [B, H_v] log decay (<= 0 for a decay);  beta (dev) fp32 [B, H_v]
+ *   out   (dev) bf16 [B, H_v, d_v] (round to nearest even of the fp32 value)
+ * The q/k/v projections, the gate activations and the output gate are the caller's.
+ */
+MOE_API moe_status moe_gdn_decode_step(const moe_gdn_shape* shape, int32_t B, float* state, const void* q,
+                                       const void* k, const void* v, const float* g, const float* beta,
+                                       void* out, void* stream);
+
+/* ------------------------------------------------------------------------------------ */
 /* Bounded slot pool with LFU + recency eviction («Paquets Swiftlet…» paragraph 5;       */
 /* «Swiftlet: 在 Mac 和 iPhone 上執行…», 記憶體管理與權重串流).  Misses are copied from   */
 /* pinned host blobs with cudaMemcpyAsync on the pool's own side stream.                 */

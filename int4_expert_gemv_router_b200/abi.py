@@ -52,6 +52,11 @@ class moe_layer_desc(ctypes.Structure):
                 ("topk_idx_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p)]
 
 
+class moe_gdn_shape(ctypes.Structure):
+    _fields_ = [("n_k_heads", ctypes.c_int32), ("n_v_heads", ctypes.c_int32), ("d_k", ctypes.c_int32),
+                ("d_v", ctypes.c_int32)]
+
+
 _P = ctypes.c_void_p
 _I32, _I64, _SZ = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
 _SIGS = {
@@ -71,6 +76,7 @@ _SIGS = {
     "moe_ws_check": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "moe_ws_set_slot_wait": (ctypes.c_int, [_P, ctypes.c_uint32, _P]),
     "moe_ws_router_logits": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, _P, _SZ, ctypes.POINTER(_P)]),
+    "moe_gdn_decode_step": (ctypes.c_int, [ctypes.POINTER(moe_gdn_shape), _I32, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_pool_create": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, _P, _P, _P, ctypes.POINTER(_P)]),
     "moe_expert_pool_load": (ctypes.c_int, [_P, _P, _I32, _P]),
     "moe_pool_stats": (ctypes.c_int, [_P, ctypes.POINTER(moe_pool_stats_t)]),
@@ -240,6 +246,12 @@ def moe_ws_router_logits(shape, T: int, ws) -> torch.Tensor:
     off = addr.value - ws.data_ptr()
     n = T * (shape.n_experts + 1)
     return ws[off:off + 4 * n].view(torch.float32).view(T, shape.n_experts + 1)
+
+
+def moe_gdn_decode_step(shape, B, state, q, k, v, g, beta, out, stream=None):
+    """One gated-delta-rule decode step of B sequences; state (fp32) is updated in place."""
+    _check(lib().moe_gdn_decode_step(ctypes.byref(shape), B, _ptr(state), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                     _ptr(beta), _ptr(out), _stream(stream)))
 
 
 def moe_pool_create(shape, n_slots, host_blobs, dev_pool, dev_slot_table) -> int:

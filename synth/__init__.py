@@ -298,3 +298,34 @@ def make_layer(w: Workload, layer: int, device, pool_out: Optional[torch.Tensor]
 def bf16_bits(t: torch.Tensor) -> torch.Tensor:
     """bf16 tensor -> int16 view -> the same bits as uint16 numpy-friendly int32."""
     return t.contiguous().view(torch.int16).to(torch.int32) & 0xFFFF
+
+
+# ----------------------------------------------------------------------------
+# Gated DeltaNet decode-step inputs
+# ----------------------------------------------------------------------------
+# Linear-attention shape of the 80B-like model: 16 query/key heads, 32 value heads, head
+# width 128 (the pages give no dimensions; this is the published layout of the model family
+# they run), hidden 2048, 36 of its 48 layers (three quarters).
+GDN_WORKLOADS = {
+    "gdn80b": dict(n_k_heads=16, n_v_heads=32, d_k=128, d_v=128, layers=36, batch=1, seed=7),
+    "gdn80b_b8": dict(n_k_heads=16, n_v_heads=32, d_k=128, d_v=128, layers=36, batch=8, seed=8),
+}
+
+
+def gdn_inputs(Hk: int, Hv: int, dk: int, dv: int, B: int, T: int, seed: int, device="cpu"):
+    """T tokens of decode-step inputs for B sequences: q, k bf16 [T, B, Hk, dk] and v bf16
+    [T, B, Hv, dv] ~ N(0, 1); log decay g fp32 [T, B, Hv] uniform in [-0.3, 0) (alpha = e^g
+    in (0.74, 1]); write strength beta fp32 [T, B, Hv] = sigmoid(N(0, 1))."""
+    g_ = _gen(device, seed, 505)
+    q = torch.empty(T, B, Hk, dk, device=device).normal_(generator=g_).to(torch.bfloat16)
+    k = torch.empty(T, B, Hk, dk, device=device).normal_(generator=g_).to(torch.bfloat16)
+    v = torch.empty(T, B, Hv, dv, device=device).normal_(generator=g_).to(torch.bfloat16)
+    g = -0.3 * torch.rand(T, B, Hv, device=device, generator=g_)
+    beta = torch.sigmoid(torch.empty(T, B, Hv, device=device).normal_(generator=g_))
+    return q, k, v, g.float(), beta.float()
+
+
+def gdn_state(Hv: int, dk: int, dv: int, B: int, seed: int, device="cpu", std: float = 0.1):
+    """A seeded fp32 starting state [B, Hv, dv, dk] ~ N(0, std)."""
+    g_ = _gen(device, seed, 606)
+    return torch.empty(B, Hv, dv, dk, device=device).normal_(0.0, std, generator=g_)
