@@ -584,7 +584,11 @@ def workload_config(args, w, T, n_gpus):
         cfg.update({"tokens_per_step": 1, "layers": 1, "n_slots": w.n_slots, "slot_fraction": w.n_slots / w.n_experts,
                     "steps_total": max(1024, args.steps + args.warmup),
                     "policy": {"lfu_recency": "LFU + recency", "lru": "LRU", "lfu": "LFU"}[args.policy],
-                    "miss_path": "pinned host -> cudaMemcpyAsync on a side stream", "overlap": bool(args.overlap),
+                    "miss_path": {"host": "pinned host -> cudaMemcpyAsync on a side stream",
+                                  "file": "pread from a file -> pinned staging -> cudaMemcpyAsync",
+                                  "file_direct": "O_DIRECT pread from a file -> pinned staging -> cudaMemcpyAsync"}[
+                                      getattr(args, "store", "host")],
+                    "overlap": bool(args.overlap),
                     "l2": "one layer; misses come over PCIe, hits from the slot pool"})
     elif w.name == "prefill":
         cfg.update({"tokens_per_call": T, "layers": 1,
@@ -797,7 +801,16 @@ def run_pool(args, w, device, rank, total_steps=1024):
     shape = abi.shape_of(w)
     dev_pool = torch.zeros(w.n_slots, stride, dtype=torch.uint8, device=device)
     table = torch.empty(w.n_experts, dtype=torch.int32, device=device)
-    pool = abi.moe_pool_create(shape, w.n_slots, host_blobs, dev_pool, table)
+    store_path = None
+    if args.store == "host":
+        pool = abi.moe_pool_create(shape, w.n_slots, host_blobs, dev_pool, table)
+    else:
+        # the storage tier: the blobs in a file, misses read with one pread each
+        fd, store_path = tempfile.mkstemp(suffix=".blobs", dir=os.environ.get("MOE_STORE_DIR"))
+        os.close(fd)
+        host_blobs.numpy().tofile(store_path)
+        pool = abi.moe_pool_create_file(shape, w.n_slots, store_path, dev_pool, table,
+                                        direct=(args.store == "file_direct"))
     abi.moe_pool_set_policy(pool, args.policy)
     abi.moe_pool_set_overlap(pool, args.overlap)
     T = 1
@@ -839,6 +852,8 @@ def run_pool(args, w, device, rank, total_steps=1024):
     st1 = abi.moe_pool_stats(pool)
     flags = abi.moe_ws_check(ws, stream)
     abi.moe_pool_destroy(pool)
+    if store_path:
+        os.unlink(store_path)
     hits = st1["hits"] - st0["hits"]
     look = st1["lookups"] - st0["lookups"]
     # Zipf exponent fitted to the measured popularity (log count vs log rank)
@@ -988,6 +1003,8 @@ def parse(argv=None):
     ap.add_argument("--policy", choices=["lfu_recency", "lru", "lfu"], default="lfu_recency",
                     help="pool workloads: eviction policy (the pages' LFU + recency by default)")
     ap.add_argument("--slots", type=int, default=None, help="pool workloads: number of slots (default 128)")
+    ap.add_argument("--store", choices=["host", "file", "file_direct"], default="host",
+                    help="pool workloads: where misses come from (pinned host memory, or a file read with pread)")
     ap.add_argument("--overlap", action="store_true",
                     help="pool workloads: the forward starts while the step's misses are still being copied")
     ap.add_argument("--parallel", choices=["replicas", "ep"], default="replicas",

@@ -70,7 +70,8 @@ typedef enum {
   MOE_ERR_NOT_RESIDENT = -4, /* reserved: an expert the call needs has no slot */
   MOE_ERR_UNSUPPORTED = -5,  /* valid request with no kernel in this build */
   MOE_ERR_TIMEOUT = -6,      /* a bounded device-side wait gave up */
-  MOE_ERR_DEVICE = -7        /* the device set an error bit (moe_ws_check) */
+  MOE_ERR_DEVICE = -7,       /* the device set an error bit (moe_ws_check) */
+  MOE_ERR_IO = -8            /* the pool's backing file could not be opened or read */
 } moe_status;
 
 /* Device error-word bits (moe_ws_check). */
@@ -362,6 +363,27 @@ typedef struct {
  */
 MOE_API moe_status moe_pool_create(const moe_shape* shape, int32_t n_slots, const uint8_t* host_blobs,
                            uint8_t* dev_pool, int32_t* dev_slot_table, moe_pool** out);
+
+/*
+ * moe_pool_create_file -- a pool whose misses are read from a file instead of host memory:
+ * the storage tier of the pages, where a missed expert is one read of its fixed-stride blob
+ * from the SSD, without mmap and without filling the page cache («Paquets Swiftlet…»,
+ * paragraph 5; «Swiftlet: 在 Mac 和 iPhone 上執行…», 記憶體管理與權重串流).
+ *   path   (host) a file holding E blobs back to back: expert e at byte e * stride
+ *   flags  MOE_POOL_FILE_DIRECT: open with O_DIRECT (reads bypass the page cache; used when
+ *          the stride is a multiple of 4096 and the file system accepts it, else buffered
+ *          reads whose pages are released after each read)
+ *   dev_pool, dev_slot_table, out: as for moe_pool_create.
+ * Every moe_expert_pool_load then reads its misses with one pread per blob, up to 8 at once
+ * on as many threads, into the pool's 8 pinned staging buffers, and copies each to its slot
+ * on the side stream (in overlap mode each miss's slot-table entry is settled after its
+ * copy, as for host blobs).  A blob that cannot be read leaves its slot empty and the load
+ * returns MOE_ERR_IO; the table stays consistent.  MOE_ERR_IO also if the file cannot be
+ * opened or is too short.  The file descriptor and buffers are released by moe_pool_destroy.
+ */
+#define MOE_POOL_FILE_DIRECT 0x1
+MOE_API moe_status moe_pool_create_file(const moe_shape* shape, int32_t n_slots, const char* path, int32_t flags,
+                                        uint8_t* dev_pool, int32_t* dev_slot_table, moe_pool** out);
 
 /*
  * moe_expert_pool_load -- make every expert named in topk_idx (dev int32 [T, k], T >= 1)

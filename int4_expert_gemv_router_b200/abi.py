@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe.so")
 MOE_OK = 0
 STATUS = {0: "MOE_OK", -1: "MOE_ERR_INVALID", -2: "MOE_ERR_CUDA", -3: "MOE_ERR_CAPACITY",
           -4: "MOE_ERR_NOT_RESIDENT", -5: "MOE_ERR_UNSUPPORTED", -6: "MOE_ERR_TIMEOUT",
-          -7: "MOE_ERR_DEVICE"}
+          -7: "MOE_ERR_DEVICE", -8: "MOE_ERR_IO"}
 DEVERR_BAD_EXPERT, DEVERR_BAD_SLOT, DEVERR_NONFINITE, DEVERR_TIMEOUT = 1, 2, 4, 8
 
 
@@ -78,6 +78,8 @@ _SIGS = {
     "moe_ws_router_logits": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, _P, _SZ, ctypes.POINTER(_P)]),
     "moe_gdn_decode_step": (ctypes.c_int, [ctypes.POINTER(moe_gdn_shape), _I32, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_pool_create": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, _P, _P, _P, ctypes.POINTER(_P)]),
+    "moe_pool_create_file": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, ctypes.c_char_p, _I32, _P, _P,
+                                            ctypes.POINTER(_P)]),
     "moe_expert_pool_load": (ctypes.c_int, [_P, _P, _I32, _P]),
     "moe_pool_stats": (ctypes.c_int, [_P, ctypes.POINTER(moe_pool_stats_t)]),
     "moe_pool_slot_table": (ctypes.c_int, [_P, _P, _P]),
@@ -258,6 +260,17 @@ def moe_pool_create(shape, n_slots, host_blobs, dev_pool, dev_slot_table) -> int
     h = _P()
     _check(lib().moe_pool_create(ctypes.byref(shape), n_slots, _ptr(host_blobs), _ptr(dev_pool),
                                  _ptr(dev_slot_table), ctypes.byref(h)))
+    return h.value
+
+
+POOL_FILE_DIRECT = 1
+
+
+def moe_pool_create_file(shape, n_slots, path: str, dev_pool, dev_slot_table, direct: bool = False) -> int:
+    """A pool whose misses are read from a file of fixed-stride blobs (see moe.h)."""
+    h = _P()
+    _check(lib().moe_pool_create_file(ctypes.byref(shape), n_slots, os.fsencode(path), POOL_FILE_DIRECT if direct else 0,
+                                      _ptr(dev_pool), _ptr(dev_slot_table), ctypes.byref(h)))
     return h.value
 
 

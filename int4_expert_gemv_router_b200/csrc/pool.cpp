@@ -20,8 +20,14 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <fcntl.h>
+#include <sys/stat.h>
+#include <unistd.h>
+
+#include <cerrno>
 #include <cstring>
 #include <new>
+#include <thread>
 #include <vector>
 
 namespace moe {
@@ -74,7 +80,97 @@ struct moe_pool {
   int32_t h_ids_cap = 0;
   int32_t* h_table = nullptr;      // pinned [E]
   int32_t* h_final = nullptr;      // pinned [E]: the slot an overlap-mode miss resolves to
+  // storage tier (moe_pool_create_file): misses are read from a file of fixed-stride blobs
+  int fd = -1;
+  bool direct = false;             // opened with O_DIRECT (no page cache)
+  std::vector<uint8_t*> stage;     // pinned staging buffers, one blob each
+  std::vector<cudaEvent_t> stage_ev;  // the copy out of each staging buffer has finished
+  std::vector<bool> stage_busy;
 };
+
+namespace {
+constexpr int kStageBufs = 8;  // blobs read from the file at once (one thread each)
+
+struct Load {
+  int32_t id, slot;
+};
+
+// Reads blob `id` (stride bytes at id * stride) into `dst`; false on an error or a short read.
+bool read_blob(const moe_pool* p, int32_t id, uint8_t* dst) {
+  int64_t done = 0;
+  const int64_t off = (int64_t)id * p->stride;
+  while (done < p->stride) {
+    const ssize_t r = pread(p->fd, dst + done, (size_t)(p->stride - done), off + done);
+    if (r < 0 && errno == EINTR) continue;
+    if (r <= 0) return false;
+    done += r;
+  }
+  // the blob is in the staging buffer now: do not let it take page-cache room from others
+  if (!p->direct) posix_fadvise(p->fd, off, p->stride, POSIX_FADV_DONTNEED);
+  return true;
+}
+
+// Overlap mode: the side stream writes the final slot of a miss over its pending entry once
+// the blob copy before it has finished.
+cudaError_t settle_entry(moe_pool* p, int32_t id) {
+  const WriteValue32Fn wv = write_value32_fn();
+  if (wv && wv(p->side, (CUdeviceptr)(p->dev_slot_table + id), (cuuint32_t)p->h_final[id], 0) == CUDA_SUCCESS)
+    return cudaSuccess;
+  return cudaMemcpyAsync(p->dev_slot_table + id, p->h_final + id, sizeof(int32_t), cudaMemcpyHostToDevice, p->side);
+}
+
+// The misses of a file-backed pool: in waves of kStageBufs, every blob of the wave is read
+// by its own thread into a staging buffer (after the previous copy out of that buffer has
+// finished), then copied to its slot on the side stream.  A blob that cannot be read leaves
+// its slot empty (host state rolled back; ok[i] = 0).  With `settle` each miss's pending
+// slot-table entry is written after its copy (or -1 for a failed read).  Returns the first
+// CUDA error of a copy; reads do not raise one.
+cudaError_t file_loads(moe_pool* p, const std::vector<Load>& loads, std::vector<char>& ok, bool settle) {
+  ok.assign(loads.size(), 1);
+  for (size_t w0 = 0; w0 < loads.size(); w0 += kStageBufs) {
+    const size_t w1 = std::min(loads.size(), w0 + (size_t)kStageBufs);
+    for (size_t i = w0; i < w1; ++i) {
+      const int b = (int)(i - w0);
+      if (p->stage_busy[b]) {
+        cudaError_t e = cudaEventSynchronize(p->stage_ev[b]);
+        if (e != cudaSuccess) return e;
+        p->stage_busy[b] = false;
+      }
+    }
+    std::vector<std::thread> readers;
+    readers.reserve(w1 - w0);
+    for (size_t i = w0; i < w1; ++i)
+      readers.emplace_back([p, &loads, &ok, i, w0] { ok[i] = read_blob(p, loads[i].id, p->stage[i - w0]) ? 1 : 0; });
+    for (auto& t : readers) t.join();
+    for (size_t i = w0; i < w1; ++i) {
+      const Load& ld = loads[i];
+      const int b = (int)(i - w0);
+      if (ok[i]) {
+        cudaError_t e = cudaMemcpyAsync(p->dev_pool + (int64_t)ld.slot * p->stride, p->stage[b], (size_t)p->stride,
+                                        cudaMemcpyHostToDevice, p->side);
+        if (e == cudaSuccess) e = cudaEventRecord(p->stage_ev[b], p->side);
+        if (e != cudaSuccess) return e;
+        p->stage_busy[b] = true;
+      } else {
+        p->slot_of[ld.id] = -1;
+        p->expert_in[ld.slot] = -1;
+        p->stats.h2d_bytes -= p->stride;
+        p->h_final[ld.id] = -1;
+      }
+      if (settle) {
+        cudaError_t e = settle_entry(p, ld.id);
+        if (e != cudaSuccess) return e;
+      }
+    }
+  }
+  return cudaSuccess;
+}
+}  // namespace
+
+namespace {
+moe_status pool_init(moe_pool* p, const moe_shape* shape, int32_t n_slots, const uint8_t* host_blobs,
+                     uint8_t* dev_pool, int32_t* dev_slot_table);
+}  // namespace
 
 extern "C" {
 
@@ -96,6 +192,19 @@ moe_status moe_pool_create(const moe_shape* shape, int32_t n_slots, const uint8_
   }
   moe_pool* p = new (std::nothrow) moe_pool();
   if (!p) return set_error(MOE_ERR_INVALID, "out of host memory");
+  st = pool_init(p, shape, n_slots, host_blobs, dev_pool, dev_slot_table);
+  if (st != MOE_OK) return st;
+  *out = p;
+  return MOE_OK;
+}
+
+}  // extern "C"
+
+namespace {
+// The bookkeeping, side stream, events and pinned buffers every pool has; on failure the
+// pool is destroyed.
+moe_status pool_init(moe_pool* p, const moe_shape* shape, int32_t n_slots, const uint8_t* host_blobs,
+                     uint8_t* dev_pool, int32_t* dev_slot_table) {
   p->shape = *shape;
   p->n_slots = n_slots;
   p->stride = make_blob_layout(shape->hidden, shape->inter, shape->bits).stride;
@@ -128,6 +237,60 @@ moe_status moe_pool_create(const moe_shape* shape, int32_t n_slots, const uint8_
     return cuda_fail(e, "pool slot table init");
   }
   p->ready_recorded = true;
+  return MOE_OK;
+}
+}  // namespace
+
+extern "C" {
+
+moe_status moe_pool_create_file(const moe_shape* shape, int32_t n_slots, const char* path, int32_t flags,
+                                uint8_t* dev_pool, int32_t* dev_slot_table, moe_pool** out) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!out) return set_error(MOE_ERR_INVALID, "out is NULL");
+  *out = nullptr;
+  if (!path) return set_error(MOE_ERR_INVALID, "path is NULL");
+  if (flags & ~MOE_POOL_FILE_DIRECT) return set_error(MOE_ERR_INVALID, "unknown flags 0x%x", flags);
+  if (n_slots < 1) return set_error(MOE_ERR_INVALID, "n_slots must be >= 1");
+  if (!dev_pool || !dev_slot_table) return set_error(MOE_ERR_INVALID, "dev_pool and dev_slot_table must be non-NULL");
+  if ((uintptr_t)dev_pool & 255) return set_error(MOE_ERR_INVALID, "dev_pool must be 256-byte aligned");
+  const int64_t stride = make_blob_layout(shape->hidden, shape->inter, shape->bits).stride;
+  // O_DIRECT needs block-aligned offsets and lengths: blob offsets are multiples of the stride
+  bool direct = (flags & MOE_POOL_FILE_DIRECT) && stride % 4096 == 0;
+  int fd = open(path, O_RDONLY | O_CLOEXEC | (direct ? O_DIRECT : 0));
+  if (fd < 0 && direct) {  // a file system without O_DIRECT: buffered reads, page cache released
+    direct = false;
+    fd = open(path, O_RDONLY | O_CLOEXEC);
+  }
+  if (fd < 0) return set_error(MOE_ERR_IO, "cannot open %s: %s", path, strerror(errno));
+  struct stat sb {};
+  if (fstat(fd, &sb) != 0 || (int64_t)sb.st_size < stride * shape->n_experts) {
+    close(fd);
+    return set_error(MOE_ERR_IO, "%s holds %lld bytes, fewer than %d blobs of %lld", path, (long long)sb.st_size,
+                     shape->n_experts, (long long)stride);
+  }
+  // the pool itself, without a host copy of the blobs
+  moe_pool* p = new (std::nothrow) moe_pool();
+  if (!p) {
+    close(fd);
+    return set_error(MOE_ERR_INVALID, "out of host memory");
+  }
+  p->fd = fd;
+  p->direct = direct;
+  const moe_status s2 = pool_init(p, shape, n_slots, nullptr, dev_pool, dev_slot_table);
+  if (s2 != MOE_OK) return s2;  // pool_init released p (and closed fd)
+  cudaError_t e = cudaSuccess;
+  p->stage.assign(kStageBufs, nullptr);
+  p->stage_ev.assign(kStageBufs, nullptr);
+  p->stage_busy.assign(kStageBufs, false);
+  for (int b = 0; b < kStageBufs && e == cudaSuccess; ++b) {
+    e = cudaHostAlloc((void**)&p->stage[b], (size_t)stride, cudaHostAllocDefault);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->stage_ev[b], cudaEventDisableTiming);
+  }
+  if (e != cudaSuccess) {
+    moe_pool_destroy(p);
+    return cuda_fail(e, "staging buffers");
+  }
   *out = p;
   return MOE_OK;
 }
@@ -178,9 +341,6 @@ moe_status moe_expert_pool_load(moe_pool* p, const int32_t* topk_idx, int32_t T,
   }
   const int64_t now = p->step_no;
   moe_status result = MOE_OK;
-  struct Load {
-    int32_t id, slot;
-  };
   std::vector<Load> loads;  // overlap mode: the misses, copied after the table upload
   for (int32_t id : uniq) {
     p->stats.lookups++;
@@ -230,8 +390,8 @@ moe_status moe_expert_pool_load(moe_pool* p, const int32_t* topk_idx, int32_t T,
       p->fail_at = -1;
     } else {
       if (p->fail_at > 0) p->fail_at--;
-      if (p->overlap) {
-        loads.push_back({id, victim});  // copied after the table upload, below
+      if (p->overlap || p->fd >= 0) {
+        loads.push_back({id, victim});  // copied below (overlap: after the table upload)
       } else {
         e = cudaMemcpyAsync(p->dev_pool + (int64_t)victim * p->stride, p->host_blobs + (int64_t)id * p->stride,
                             (size_t)p->stride, cudaMemcpyHostToDevice, p->side);
@@ -251,7 +411,27 @@ moe_status moe_expert_pool_load(moe_pool* p, const int32_t* topk_idx, int32_t T,
     p->stats.h2d_bytes += p->stride;
   }
   for (int32_t u : uniq) p->needed[u] = 0;
+  if (p->fd >= 0 && !p->overlap) {
+    // storage tier: the misses' blobs are read from the file (in waves of kStageBufs
+    // parallel preads into pinned staging buffers) and copied to their slots; a failed read
+    // leaves its slot empty before the table goes up
+    std::vector<char> ok;
+    e = file_loads(p, loads, ok, false);
+    if (e != cudaSuccess) return cuda_fail(e, "blob copy from staging");
+    for (size_t i = 0; i < loads.size(); ++i)
+      if (!ok[i]) result = set_error(MOE_ERR_IO, "reading expert %d from the backing file failed", loads[i].id);
+  }
   for (int i = 0; i < E; ++i) p->h_table[i] = p->slot_of[i];
+  if (!p->overlap) {
+    e = cudaMemcpyAsync(p->dev_slot_table, p->h_table, sizeof(int32_t) * E, cudaMemcpyHostToDevice, p->side);
+    if (e == cudaSuccess) e = cudaEventRecord(p->ready, p->side);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, p->ready, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "slot table upload");
+    p->ready_recorded = true;
+    p->step_no++;
+    if (result == MOE_OK) p->stats.steps++;
+    return result;
+  }
   // Overlap mode: the table goes up first with this step's misses marked pending, and the
   // caller's stream waits for that upload only.  Each miss's blob copy is then followed on
   // the side stream by a 4-byte copy of its slot over the pending entry; the fused decode
@@ -265,6 +445,14 @@ moe_status moe_expert_pool_load(moe_pool* p, const int32_t* topk_idx, int32_t T,
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s, p->ready, 0);
   if (e != cudaSuccess) return cuda_fail(e, "slot table upload");
   p->ready_recorded = true;
+  if (p->fd >= 0) {
+    std::vector<char> ok;
+    e = file_loads(p, loads, ok, true);
+    if (e != cudaSuccess) return cuda_fail(e, "blob copy from staging");
+    for (size_t i = 0; i < loads.size(); ++i)
+      if (!ok[i]) result = set_error(MOE_ERR_IO, "reading expert %d from the backing file failed", loads[i].id);
+    loads.clear();
+  }
   for (size_t li = 0; li < loads.size(); ++li) {
     const Load& ld = loads[li];
     e = cudaMemcpyAsync(p->dev_pool + (int64_t)ld.slot * p->stride, p->host_blobs + (int64_t)ld.id * p->stride,
@@ -351,6 +539,11 @@ void moe_pool_destroy(moe_pool* p) {
   if (p->h_ids) cudaFreeHost(p->h_ids);
   if (p->h_table) cudaFreeHost(p->h_table);
   if (p->h_final) cudaFreeHost(p->h_final);
+  for (size_t i = 0; i < p->stage_ev.size(); ++i)
+    if (p->stage_ev[i]) cudaEventDestroy(p->stage_ev[i]);
+  for (size_t i = 0; i < p->stage.size(); ++i)
+    if (p->stage[i]) cudaFreeHost(p->stage[i]);
+  if (p->fd >= 0) close(p->fd);
   delete p;
 }
 

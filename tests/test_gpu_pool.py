@@ -3,6 +3,8 @@ oracle's LFU + recency simulation step by step (and its LRU / pure LFU variants 
 eviction ablation), missed blobs land byte-for-byte, the
 pool-mode forward is bit-identical to the all-resident forward, and failures leave the
 pool consistent."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -238,3 +240,81 @@ def test_pool_many_token_step():
             assert_close(out_pool, ref["out"])
     finally:
         P.close()
+
+
+@pytest.mark.parametrize("wname,direct,overlap,T", [("pool_int4", True, False, 1), ("pool_int4", False, True, 1),
+                                                    ("pool_int8", True, True, 8)])
+def test_file_backed_pool(tmp_path, wname, direct, overlap, T):
+    """The storage tier: misses read from a file of fixed-stride blobs (one pread per blob,
+    O_DIRECT where the file system allows it) instead of pinned host memory.  Slot decisions
+    equal the oracle's, slot bytes equal the file's, and the forward through the slots is
+    bit-identical to the all-resident forward."""
+    w = synth.WORKLOADS[wname]
+    L = synth.make_layer(w, 0, DEV)
+    path = str(tmp_path / "experts.blobs")
+    L.pool.cpu().numpy().tofile(path)
+    host = torch.from_numpy(np.fromfile(path, dtype=np.uint8).reshape(w.n_experts, -1))
+    shape = abi.shape_of(w)
+    dev = torch.zeros(w.n_slots, L.pool.shape[1], dtype=torch.uint8, device=DEV)
+    table = torch.empty(w.n_experts, dtype=torch.int32, device=DEV)
+    h = abi.moe_pool_create_file(shape, w.n_slots, path, dev, table, direct=direct)
+    sim = oracle.SlotCache(w.n_experts, w.n_slots)
+    try:
+        if overlap:
+            abi.moe_pool_set_overlap(h, True)
+        for s in range(12):
+            x = synth.activations(w, 300 + s, tokens=T, device=DEV)
+            ws = ws_for(shape, T)
+            idx = torch.empty(T, w.top_k, dtype=torch.int32, device=DEV)
+            p = torch.empty(T, w.top_k, dtype=torch.float32, device=DEV)
+            abi.moe_router_topk(shape, x, T, L.w_router, L.router_bias, idx, p, ws)
+            abi.moe_expert_pool_load(h, idx, T)
+            sim.step(idx.cpu().numpy().reshape(-1).tolist())
+            out_pool, _, _, ws2 = forward(w, L, x, residual=x, pool=dev, slot_table=table, n_slots=w.n_slots,
+                                          topk=(idx, p))
+            assert abi.moe_ws_check(ws2) == 0
+            slot_of, expert_in = abi.moe_pool_slot_table(h, w.n_experts, w.n_slots)
+            assert slot_of == sim.slot_of.tolist() and expert_in == sim.expert_in.tolist()
+            assert table.cpu().tolist() == slot_of
+            for e in set(idx.cpu().numpy().reshape(-1).tolist()):
+                assert torch.equal(dev[slot_of[e]].cpu(), host[e])
+            out_res, *_ = forward(w, L, x, residual=x, topk=(idx, p))
+            assert torch.equal(out_pool, out_res)
+        st = abi.moe_pool_stats(h)
+        assert (st["lookups"], st["hits"], st["misses"]) == (sim.lookups, sim.hits, sim.misses)
+        assert st["h2d_bytes"] == sim.misses * L.pool.shape[1]
+    finally:
+        abi.moe_pool_destroy(h)
+
+
+def test_file_backed_pool_read_errors(tmp_path):
+    """A file too short for E blobs is refused at creation; a blob that cannot be read later
+    (the file shrank) fails its load with MOE_ERR_IO and leaves its slot empty."""
+    w = synth.WORKLOADS["tiny"].with_(n_experts=16, top_k=2, seed=35)
+    L = synth.make_layer(w, 0, DEV)
+    shape = abi.shape_of(w)
+    stride = L.pool.shape[1]
+    dev = torch.zeros(4, stride, dtype=torch.uint8, device=DEV)
+    table = torch.empty(w.n_experts, dtype=torch.int32, device=DEV)
+    short = str(tmp_path / "short.blobs")
+    L.pool[:8].cpu().numpy().tofile(short)
+    with pytest.raises(abi.MoeError) as ei:
+        abi.moe_pool_create_file(shape, 4, short, dev, table)
+    assert ei.value.status == -8
+    path = str(tmp_path / "full.blobs")
+    L.pool.cpu().numpy().tofile(path)
+    h = abi.moe_pool_create_file(shape, 4, path, dev, table)
+    try:
+        abi.moe_expert_pool_load(h, torch.tensor([[1, 2]], dtype=torch.int32, device=DEV), 1)
+        os.truncate(path, 10 * stride)  # experts 10.. can no longer be read
+        with pytest.raises(abi.MoeError) as ei:
+            abi.moe_expert_pool_load(h, torch.tensor([[3, 12]], dtype=torch.int32, device=DEV), 1)
+        assert ei.value.status == -8
+        slot_of, expert_in = abi.moe_pool_slot_table(h, 16, 4)
+        assert slot_of[12] == -1 and slot_of[3] >= 0 and slot_of[1] >= 0 and slot_of[2] >= 0
+        assert 12 not in expert_in
+        torch.cuda.synchronize()
+        assert table.cpu().tolist() == slot_of
+        assert torch.equal(dev[slot_of[3]].cpu(), L.pool[3].cpu())
+    finally:
+        abi.moe_pool_destroy(h)
