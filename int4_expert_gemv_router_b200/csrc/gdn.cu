@@ -15,8 +15,8 @@
 // is independent given k^ and q^ (u_i, the row update and o_i use row i only), so a warp
 // owns whole rows: each lane holds d_k / 32 consecutive elements of a row in registers
 // (one 16-byte load for d_k = 128), two warp sums give u_i and o_i, and the row is written
-// back once.  A CTA covers 16 rows of one (sequence, value head): it normalises that head's
-// k and q once, in shared memory.  The step reads and writes the state once: HBM bound,
+// back once.  A CTA covers 16 or 32 rows of one (sequence, value head) (2 or 4 per warp, all
+// loaded at once): it normalises that head's k and q once, in shared memory.  The step reads and writes the state once: HBM bound,
 // 2 * 4 * d_k * d_v bytes per (sequence, value head).
 #include "../../include/moe.h"
 #include "common.cuh"
@@ -37,8 +37,7 @@ struct GdnArgs {
 
 namespace {
 
-constexpr int kGdnWarps = 8, kGdnRowsPerWarp = 2;
-constexpr int kGdnRows = kGdnWarps * kGdnRowsPerWarp;  // rows of S per CTA
+constexpr int kGdnWarps = 8;
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -46,8 +45,11 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-template <int DK>
+// RPW rows per warp: 2 when the launch has few rows in all (every SM gets a CTA), 4 when it
+// has many (more bytes in flight per SM).
+template <int DK, int RPW>
 __global__ void __launch_bounds__(kGdnWarps * 32) k_gdn_step(const GdnArgs a) {
+  constexpr int kGdnRowsPerWarp = RPW, kGdnRows = kGdnWarps * RPW;  // rows of S per CTA
   constexpr int EPL = DK / 32;  // elements of a row per lane
   static_assert(EPL == 2 || EPL == 4 || EPL == 8, "d_k of 64, 128 or 256");
   __shared__ float s_kq[2][DK];
@@ -139,15 +141,28 @@ __global__ void __launch_bounds__(kGdnWarps * 32) k_gdn_step(const GdnArgs a) {
 
 }  // namespace
 
-cudaError_t launch_gdn_step(const GdnArgs& a, cudaStream_t s) {
-  const int blocks = a.B * a.Hv * ((a.dv + kGdnRows - 1) / kGdnRows);
+// Rows of S per CTA for a launch: 16, or 32 once the launch has at least 4 CTAs of 32 rows
+// per SM.
+int gdn_rows_per_cta(const GdnArgs& a) {
+  const long long rows = (long long)a.B * a.Hv * a.dv;
+  return rows >= 4LL * 148 * 32 ? 32 : 16;
+}
+
+template <int RPW>
+static cudaError_t launch_gdn_rpw(const GdnArgs& a, cudaStream_t s) {
+  const int rows_cta = kGdnWarps * RPW;
+  const int blocks = a.B * a.Hv * ((a.dv + rows_cta - 1) / rows_cta);
   switch (a.dk) {
-    case 64: k_gdn_step<64><<<blocks, kGdnWarps * 32, 0, s>>>(a); break;
-    case 128: k_gdn_step<128><<<blocks, kGdnWarps * 32, 0, s>>>(a); break;
-    case 256: k_gdn_step<256><<<blocks, kGdnWarps * 32, 0, s>>>(a); break;
+    case 64: k_gdn_step<64, RPW><<<blocks, kGdnWarps * 32, 0, s>>>(a); break;
+    case 128: k_gdn_step<128, RPW><<<blocks, kGdnWarps * 32, 0, s>>>(a); break;
+    case 256: k_gdn_step<256, RPW><<<blocks, kGdnWarps * 32, 0, s>>>(a); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
+}
+
+cudaError_t launch_gdn_step(const GdnArgs& a, cudaStream_t s) {
+  return gdn_rows_per_cta(a) == 32 ? launch_gdn_rpw<4>(a, s) : launch_gdn_rpw<2>(a, s);
 }
 
 moe_status set_error(moe_status s, const char* fmt, ...);
@@ -171,7 +186,7 @@ extern "C" moe_status moe_gdn_decode_step(const moe_gdn_shape* shape, int32_t B,
   if (((uintptr_t)state & 15) || ((uintptr_t)q & 15) || ((uintptr_t)k & 15) || ((uintptr_t)v & 1) ||
       ((uintptr_t)out & 1) || ((uintptr_t)g & 3) || ((uintptr_t)beta & 3))
     return set_error(MOE_ERR_INVALID, "state, q and k must be 16-byte aligned");
-  const long long blocks = (long long)B * Hv * ((dv + kGdnRows - 1) / kGdnRows);
+  const long long blocks = (long long)B * Hv * ((dv + 15) / 16);
   if (blocks > 0x7fffffffLL) return set_error(MOE_ERR_INVALID, "B * n_v_heads * d_v too large");
   GdnArgs a{B, Hk, Hv, dk, dv, state, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
             static_cast<const uint16_t*>(v), g, beta, static_cast<uint16_t*>(out)};
