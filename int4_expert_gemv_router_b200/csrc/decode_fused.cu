@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
 
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&full_bar[s], 32);  // one cp.async arrival per lane of the streaming warp
+      mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], kCons);
     }
     mbar_init(&plan_bar, 1);
@@ -364,26 +364,25 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
           break;
         }
         {
-          // the stage's gate codes, up codes and four scale/bias sections, in 16-byte
-          // cp.async copies spread over the 32 lanes; each lane then arrives on the stage's
-          // full barrier once its copies have landed
+          // lane 0 announces the bytes, then lanes 0..5 issue the stage's six copies at once
+          // (gate codes, up codes, then the four scale/bias sections)
           uint8_t* st = ring + (size_t)s * SB;
           const int slot = slot_of_unit(Lc, u);
-          if (slot >= 0) {
-            const uint8_t* b = Lc.pool + (int64_t)slot * a.L.stride;
-            const int cb = n * ROWBg / 16, sb = n * SRg / 16;  // 16-byte pieces per section
-            const uint8_t* gsrc = b + a.L.off[0] + (int64_t)r0 * ROWBg;
-            const uint8_t* usrc = b + a.L.off[1] + (int64_t)r0 * ROWBg;
-            for (int i = lane; i < cb; i += 32) {
-              cp_async16(st + 16 * i, gsrc + 16 * i);
-              cp_async16(st + n * ROWBg + 16 * i, usrc + 16 * i);
-            }
-            for (int i = lane; i < 4 * sb; i += 32) {
-              const int sec = i / sb, j = i - sec * sb;
-              cp_async16(st + 2 * n * ROWBg + sec * n * SRg + 16 * j, b + a.L.off[3 + sec] + (int64_t)r0 * SRg + 16 * j);
-            }
+          if (lane == 0) {
+            if (slot < 0)
+              mbar_arrive(&full_bar[s]);
+            else
+              mbar_expect_tx(&full_bar[s], (uint32_t)(n * ROWG_BYTES));
           }
-          cp_async_arrive(&full_bar[s]);
+          __syncwarp();
+          if (slot >= 0 && lane < 6) {
+            const uint8_t* b = Lc.pool + (int64_t)slot * a.L.stride;
+            if (lane < 2)
+              bulk_g2s(st + lane * n * ROWBg, b + a.L.off[lane] + (int64_t)r0 * ROWBg, n * ROWBg, &full_bar[s]);
+            else
+              bulk_g2s(st + 2 * n * ROWBg + (lane - 2) * n * SRg, b + a.L.off[lane + 1] + (int64_t)r0 * SRg,
+                       n * SRg, &full_bar[s]);
+          }
         }
         __syncwarp();
         ++q;
@@ -408,11 +407,20 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
             break;
           }
           uint8_t* st = ring + (size_t)s * SB;
-          // per expert its down rows j0..j1 (codes), then their scales and biases, in 16-byte
-          // cp.async copies spread over the lanes
-          const int pcode = nJ * ROWBd / 16, psc = nJ * SRd / 16, per_e = pcode + 2 * psc;
-          for (int ci = lane; ci < per_e * cnt; ci += 32) {
-            const int z = ci / per_e, i = ci - z * per_e, uu = u + z;
+          if (lane == 0) {
+            uint32_t bytes = 0;
+            for (int z = 0; z < cnt; ++z) {
+              const int uu = u + z;
+              const int slot = (uu < act_n) ? P_SLOT[uu] : 0;
+              if (uu < act_n && slot < 0) continue;
+              bytes += nJ * ROWD_BYTES;
+            }
+            mbar_expect_tx(&full_bar[s], bytes);
+          }
+          __syncwarp();
+          // three copies per expert (down codes, scales, biases), spread over the lanes
+          for (int ci = lane; ci < 3 * cnt; ci += 32) {
+            const int z = ci / 3, part = ci - 3 * z, uu = u + z;
             const uint8_t* b;
             if (uu < act_n) {
               const int slot = P_SLOT[uu];
@@ -422,14 +430,12 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
               b = Lc.shared;
             }
             uint8_t* d = st + (size_t)z * nJ * ROWD_BYTES;
-            if (i < pcode) {
-              cp_async16(d + 16 * i, b + a.L.off[2] + (int64_t)j0 * ROWBd + 16 * i);
-            } else {
-              const int sec = (i - pcode) / psc, j = (i - pcode) - sec * psc;  // 0: scales, 1: biases
-              cp_async16(d + nJ * ROWBd + sec * nJ * SRd + 16 * j, b + a.L.off[7 + sec] + (int64_t)j0 * SRd + 16 * j);
-            }
+            if (part == 0)
+              bulk_g2s(d, b + a.L.off[2] + (int64_t)j0 * ROWBd, nJ * ROWBd, &full_bar[s]);
+            else
+              bulk_g2s(d + nJ * ROWBd + (part - 1) * nJ * SRd, b + a.L.off[6 + part] + (int64_t)j0 * SRd, nJ * SRd,
+                       &full_bar[s]);
           }
-          cp_async_arrive(&full_bar[s]);
           __syncwarp();
           ++q;
           u += cnt;
@@ -441,7 +447,6 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
       s_abort = 1;
     }
     // let every issued copy land before the CTA may exit
-    cp_async_wait_all();
     if (lane == 0) {
       const uint32_t first = q > (uint32_t)NS ? q - NS : 0;
       for (uint32_t qq = first; qq < q; ++qq) mbar_wait(&full_bar[qq % NS], (qq / NS) & 1);

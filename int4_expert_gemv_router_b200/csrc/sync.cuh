@@ -81,6 +81,17 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* b) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(b)) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Per-thread L2 prefetch of the 128-byte line holding p (a hint: no register result, no
+// completion; unlike cp.async.bulk.prefetch it does not occupy the SM's bulk-copy engine).
+__device__ __forceinline__ void prefetch_line_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+// Lines [p, p + bytes) into L2, spread over the lanes of a warp.
+__device__ __forceinline__ void prefetch_range_l2(const void* p, uint32_t bytes, int lane) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(p) & ~uintptr_t(127);
+  const uintptr_t a1 = reinterpret_cast<uintptr_t>(p) + bytes;
+  for (uintptr_t a = a0 + (uintptr_t)lane * 128; a < a1; a += 32 * 128) prefetch_line_l2(reinterpret_cast<const void*>(a));
+}
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
