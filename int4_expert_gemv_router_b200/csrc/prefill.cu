@@ -65,7 +65,6 @@ constexpr int kGemmThreads = (kEWarp0 + kEWarps) * 32;  // 736
 constexpr int kSBO = (kKC / 8) * 128;     // 1024: 8-row group stride of a no-swizzle K-major tile
 constexpr int kTmemCols = 2 * kNMax;      // two accumulators of up to 256 columns
 constexpr int kTRows = 32;                // rows per token-tile load
-constexpr int kTokPrefetch = 4;           // token tiles are prefetched into L2 this many stages ahead
 constexpr int kStageMax = 6;
 constexpr int kChunk = 8;                 // groups per scale chunk
 constexpr int kChunkBytes = kNMax * 2 * kChunk * 2;  // 8 KB: scales + biases of 8 groups, 256 rows
@@ -159,11 +158,6 @@ __device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int
           dst),
       "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar))
       : "memory");
-}
-// L2 prefetch of a 2-D box (no shared-memory destination, no completion to wait for).
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, int c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(c0), "r"(c1)
-               : "memory");
 }
 __device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, uint64_t* bar) {
   asm volatile(
@@ -452,13 +446,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
       const int nrt = (U.n + kTRows - 1) / kTRows;
       const uint32_t bytes = (uint32_t)nrt * kTRows * 128u;
       bool stop = false;
-      // the unit's first stages go to L2 at once; then each stage's load is preceded by the
-      // prefetch of the stage kTokPrefetch ahead, so that the load, which can only be issued
-      // once its ring slot is free, finds its rows in L2
-      if (lane < nrt)
-        for (int kp = 0; kp < kTokPrefetch && kp < nK; ++kp) tma_prefetch_2d(mt, kp * kKC, U.p0 + lane * kTRows);
       for (int kc = 0; kc < nK; ++kc, r.next()) {
-        if (lane < nrt && kc + kTokPrefetch < nK) tma_prefetch_2d(mt, (kc + kTokPrefetch) * kKC, U.p0 + lane * kTRows);
         if (!warp_wait(&empty[r.s], r.ph ^ 1, a.ctrl, lane)) {
           stop = true;
           break;
