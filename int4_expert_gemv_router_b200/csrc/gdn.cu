@@ -15,8 +15,8 @@
 // is independent given k^ and q^ (u_i, the row update and o_i use row i only), so a warp
 // owns whole rows: each lane holds d_k / 32 consecutive elements of a row in registers
 // (one 16-byte load for d_k = 128), two warp sums give u_i and o_i, and the row is written
-// back once.  A CTA covers 16 or 32 rows of one (sequence, value head) (2 or 4 per warp, all
-// loaded at once): it normalises that head's k and q once, in shared memory.  The step reads and writes the state once: HBM bound,
+// back once.  A CTA covers 16, 32 or 64 rows of one (sequence, value head) (2, 4 or 8 per warp,
+// all loaded at once): it normalises that head's k and q once, in shared memory.  The step reads and writes the state once: HBM bound,
 // 2 * 4 * d_k * d_v bytes per (sequence, value head).
 #include "../../include/moe.h"
 #include "common.cuh"
@@ -45,8 +45,8 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// RPW rows per warp: 2 when the launch has few rows in all (every SM gets a CTA), 4 when it
-// has many (more bytes in flight per SM).
+// RPW rows per warp (2, 4 or 8), all loaded at once: the fewest that still fit the launch in
+// one round of resident CTAs, so that every SM has as many bytes in flight as its rows give.
 template <int DK, int RPW>
 __global__ void __launch_bounds__(kGdnWarps * 32) k_gdn_step(const GdnArgs a) {
   constexpr int kGdnRowsPerWarp = RPW, kGdnRows = kGdnWarps * RPW;  // rows of S per CTA
@@ -141,11 +141,16 @@ __global__ void __launch_bounds__(kGdnWarps * 32) k_gdn_step(const GdnArgs a) {
 
 }  // namespace
 
-// Rows of S per CTA for a launch: 16, or 32 once the launch has at least 4 CTAs of 32 rows
-// per SM.
-int gdn_rows_per_cta(const GdnArgs& a) {
-  const long long rows = (long long)a.B * a.Hv * a.dv;
-  return rows >= 4LL * 148 * 32 ? 32 : 16;
+// Rows per warp for a launch: the smallest of 2, 4, 8 whose CTAs (8 warps each) number at
+// most four per SM, so that they are all resident at once (8 only while a row takes at most
+// four registers per lane).
+static int gdn_rows_per_warp(const GdnArgs& a, int n_sm) {
+  const int max_rpw = a.dk <= 128 ? 8 : 4;
+  for (int rpw = 2; rpw < max_rpw; rpw *= 2) {
+    const long long ctas = (long long)a.B * a.Hv * ((a.dv + kGdnWarps * rpw - 1) / (kGdnWarps * rpw));
+    if (ctas <= 4LL * n_sm) return rpw;
+  }
+  return max_rpw;
 }
 
 template <int RPW>
@@ -162,7 +167,18 @@ static cudaError_t launch_gdn_rpw(const GdnArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_gdn_step(const GdnArgs& a, cudaStream_t s) {
-  return gdn_rows_per_cta(a) == 32 ? launch_gdn_rpw<4>(a, s) : launch_gdn_rpw<2>(a, s);
+  static int n_sm = 0;
+  if (!n_sm) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    if (n_sm < 1) n_sm = 1;
+  }
+  switch (gdn_rows_per_warp(a, n_sm)) {
+    case 2: return launch_gdn_rpw<2>(a, s);
+    case 4: return launch_gdn_rpw<4>(a, s);
+    default: return launch_gdn_rpw<8>(a, s);
+  }
 }
 
 moe_status set_error(moe_status s, const char* fmt, ...);

@@ -48,9 +48,9 @@ def _run(Hk, Hv, dk, dv, B, T, seed, start_random):
 
 @pytest.mark.parametrize("Hk,Hv,dk,dv,B,T,start_random", [
     (16, 32, 128, 128, 1, 6, False),   # the 80B-like linear-attention shape, from a zero state
-    (16, 32, 128, 128, 3, 4, True),    # three sequences, from a random state
-    (16, 32, 128, 128, 8, 2, True),    # eight sequences: 32 rows per CTA (4 per warp)
-    (4, 8, 256, 200, 12, 2, True),     # 32 rows per CTA with d_k 256 and a ragged d_v
+    (16, 32, 128, 128, 3, 4, True),    # three sequences, from a random state: 4 rows per warp
+    (16, 32, 128, 128, 8, 2, True),    # eight sequences: 8 rows per warp
+    (4, 8, 256, 200, 12, 2, True),     # 4 rows per warp with d_k 256 and a ragged d_v
     (2, 2, 64, 40, 2, 5, True),        # d_k 64 (two elements per lane), ragged d_v
     (1, 4, 256, 24, 1, 3, True),       # d_k 256, four value heads on one key head
 ])
