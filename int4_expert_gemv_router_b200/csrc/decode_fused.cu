@@ -773,6 +773,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
       const int sub = lane % NCLd, rsub = lane / NCLd;
       float* red = reinterpret_cast<float*>(smem + a.sm.red) + (size_t)cw * a.jmax * (NCLd + 1);
       const int n_units_d = act_n + (Lc.with_shared ? 1 : 0);  // the shared expert last
+      int it0 = 0;  // work items of the earlier stages
       for (int u0 = 0; u0 < n_units_d;) {
         const int cnt = min(per_stage, n_units_d - u0);
         const int s = q % NS;
@@ -782,17 +783,23 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
           break;
         }
         const uint8_t* st = ring + (size_t)s * SB;
-        // expert slices are dealt to warps round-robin over the layer
-        for (int z = (cw - u0 % kCons + kCons) % kCons; z < cnt; z += kCons) {
+        // work items: (expert of the stage, one of its token pairs), in stage order and dealt
+        // to warps round-robin over the layer, so that an expert with many pairs (the shared
+        // one has T) is spread over several warps
+        const auto n_pairs = [&](int u) { return u == act_n ? T : P_BEGIN[u + 1] - P_BEGIN[u]; };
+        int n_items = 0;
+        for (int z = 0; z < cnt; ++z) n_items += n_pairs(u0 + z);
+        for (int i = (cw - it0 % kCons + kCons) % kCons; i < n_items; i += kCons) {
+          int z = 0, rem = i;
+          while (rem >= n_pairs(u0 + z)) rem -= n_pairs(u0 + z++);
           const int u = u0 + z;
           const bool shared = (u == act_n);
           const uint8_t* dq = st + (size_t)z * nJ * ROWD_BYTES;
           const uint8_t* ds = dq + nJ * ROWBd;
           const uint8_t* db = ds + nJ * SRd;
           const bool have = shared || P_SLOT[u] >= 0;
-          const int pb = shared ? n_valid : P_BEGIN[u];
-          const int pe = shared ? n_valid + T : P_BEGIN[u + 1];
-          for (int p = pb; p < pe; ++p) {
+          const int p = (shared ? n_valid : P_BEGIN[u]) + rem;
+          {
             int t;
             float w;
             const float* hsrc;
@@ -870,6 +877,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
             __syncwarp();
           }
         }
+        it0 += n_items;
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_bar[s]);
         ++q;
