@@ -128,13 +128,15 @@ struct DecodeArgs {
 // host to size the launch and by the kernel to find its arrays.
 struct FusedSmem {
   uint32_t xs4, xsum, partial, ids, pw, order, pos_of, act_e, act_slot, act_begin, gate, scratch, slot, topk, red,
-      total;
+      rbuf, rpart, total;
 };
 // Per-token top-k scratch of the fused kernel: 32 lane maxima (double + id), 64 candidates
 // (double + id), a counter and the threshold lane.
 constexpr int kTopkScratchBytes = 32 * 8 + 32 * 4 + 64 * 8 + 64 * 4 + 16;
+// rr_max, rs_max: router rows and shared-expert rows one CTA stages for phase R.
 __host__ __device__ inline FusedSmem fused_smem_layout(int T, int H, int I, int E, int bits, int k, int jmax,
-                                                       int n_stages, int stage_bytes, int n_cons) {
+                                                       int n_stages, int stage_bytes, int n_cons, int rr_max,
+                                                       int rs_max) {
   FusedSmem m{};
   size_t off = (size_t)n_stages * stage_bytes;
   auto carve = [&](size_t bytes) {
@@ -156,10 +158,13 @@ __host__ __device__ inline FusedSmem fused_smem_layout(int T, int H, int I, int 
   m.act_slot = carve((size_t)TK * 4);
   m.act_begin = carve((size_t)(TK + 1) * 4);
   m.gate = carve((size_t)T * 4);
-  m.scratch = carve((size_t)2 * TK * 4);
+  m.scratch = carve((size_t)5 * TK * 4);
   m.slot = carve((size_t)E * 4);
   m.topk = carve((size_t)T * kTopkScratchBytes);
   m.red = carve((size_t)n_cons * jmax * (NCLd + 1) * 4);
+  const size_t rowg = 2 * (size_t)H * bits / 8 + 4 * (size_t)(H / kGroup) * 2;
+  m.rbuf = carve((size_t)rr_max * H * 2 + (size_t)rs_max * rowg);
+  m.rpart = carve((size_t)rr_max * 4 * T * 8);
   m.total = (uint32_t)((off + 127) / 128 * 128);
   return m;
 }
@@ -188,7 +193,8 @@ constexpr int kMaxFusedLayers = 64;
 struct FusedArgs {
   int H, I, E, k, T, n_layers, bits;
   int n_stages, stage_bytes, jmax;
-  FusedSmem sm;  // shared-memory carve (host-computed)
+  int rr_max, rs_max;  // most router rows / shared-expert rows a CTA stages for phase R
+  FusedSmem sm;        // shared-memory carve (host-computed)
   BlobLayout L;
   Ctrl* ctrl;
   double* logits;

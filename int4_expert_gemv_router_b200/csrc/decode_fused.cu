@@ -222,6 +222,23 @@ __device__ __forceinline__ int gate_block_rows(int rows, int G, int RG, int gG) 
   return max(gG, (br + gG - 1) / gG * gG);
 }
 
+// Phase-R rows of CTA c (of G) in layer L: router rows [rr0, rr1) of the n_router = E + 1
+// (the last one is the shared-gate row; only that one when the layer's routing is given) and
+// shared-expert rows [sr0, sr1), each a contiguous range so that it is staged in a few copies.
+struct RRange {
+  int rr0, rr1, sr0, sr1, n_router;
+};
+__device__ __forceinline__ RRange r_ranges(const FusedLayer& L, int E, int I, int gG, int c, int G) {
+  RRange r;
+  r.n_router = (L.topk_idx_in ? 0 : E) + 1;
+  r.rr0 = (int)((long long)c * r.n_router / G);
+  r.rr1 = (int)((long long)(c + 1) * r.n_router / G);
+  const int ngr = L.with_shared ? I / gG : 0;
+  r.sr0 = (int)((long long)c * ngr / G) * gG;
+  r.sr1 = (int)((long long)(c + 1) * ngr / G) * gG;
+  return r;
+}
+
 template <int BITS, int H, int I, int TM>
 __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_constant__ FusedArgs a) {
   // ---- constants ----
@@ -247,9 +264,12 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
 
   // ---- shared memory ----
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(8) uint64_t full_bar[kMaxStages], empty_bar[kMaxStages], plan_bar;
+  __shared__ __align__(8) uint64_t full_bar[kMaxStages], empty_bar[kMaxStages], plan_bar, rbar;
   __shared__ int s_act_n, s_n_valid, s_abort;
   uint8_t* ring = smem;
+  uint8_t* rbuf = smem + a.sm.rbuf;                             // this CTA's phase-R rows
+  uint8_t* rbuf_s = rbuf + (size_t)a.rr_max * H * 2;            // ... the shared-expert part
+  double* rpart = reinterpret_cast<double*>(smem + a.sm.rpart);  // router-row quarter sums
   float4* xs4 = reinterpret_cast<float4*>(smem + a.sm.xs4);
   float* xsum = reinterpret_cast<float*>(smem + a.sm.xsum);
   float* partial = reinterpret_cast<float*>(smem + a.sm.partial);  // [(T*k + T) * jmax]
@@ -271,6 +291,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
       mbar_init(&empty_bar[s], kCons);
     }
     mbar_init(&plan_bar, 1);
+    mbar_init(&rbar, 1);
     s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -323,26 +344,43 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
       fence_proxy_async_global();
       return __shfl_sync(0xffffffffu, v, 0);
     };
+    // This CTA's phase-R rows of layer ln (its router rows, the shared-gate row if it holds
+    // it, its shared-expert rows with their scales) copied into rbuf: at most eight bulk
+    // copies, tracked on rbar.  pf: only an L2 prefetch of the same bytes.
+    const auto issue_r = [&](int ln, bool pf) {
+      const FusedLayer& Ln = a.layer[ln];
+      const RRange R = r_ranges(Ln, E, I, gG, blockIdx.x, G);
+      const int n_wr = max(0, min(R.rr1, R.n_router - 1) - R.rr0);  // rows of the router matrix
+      const bool has_gate = R.rr1 == R.n_router && R.rr1 > R.rr0;
+      const int ns = R.sr1 - R.sr0;
+      if (!pf && lane == 0)
+        mbar_expect_tx(&rbar, (uint32_t)((n_wr + (has_gate ? 1 : 0)) * H * 2 + ns * ROWG_BYTES));
+      __syncwarp();
+      if (lane == 0 && n_wr > 0) {
+        if (pf) prefetch_l2(Ln.wr + (size_t)R.rr0 * H, n_wr * H * 2);
+        else bulk_g2s(rbuf, Ln.wr + (size_t)R.rr0 * H, n_wr * H * 2, &rbar);
+      }
+      if (lane == 1 && has_gate) {
+        if (pf) prefetch_l2(Ln.wsg, H * 2);
+        else bulk_g2s(rbuf + (size_t)(R.n_router - 1 - R.rr0) * H * 2, Ln.wsg, H * 2, &rbar);
+      }
+      if (ns > 0 && lane >= 2 && lane < 8) {
+        const int sec = lane - 2;
+        const uint8_t* src = sec < 2 ? Ln.shared + a.L.off[sec] + (int64_t)R.sr0 * ROWBg
+                                     : Ln.shared + a.L.off[1 + sec] + (int64_t)R.sr0 * SRg;
+        const int bytes = sec < 2 ? ns * ROWBg : ns * SRg;
+        if (pf) prefetch_l2(src, bytes);
+        else bulk_g2s(rbuf_s + (sec < 2 ? sec * ns * ROWBg : 2 * ns * ROWBg + (sec - 2) * ns * SRg), src, bytes, &rbar);
+      }
+      __syncwarp();
+    };
+    int n_r_issued = 0;  // rbar phases announced
+    issue_r(0, false);
+    ++n_r_issued;
     for (int l = 0; l < a.n_layers && ok; ++l) {
       const FusedLayer& Lc = a.layer[l];
-      // L2 prefetch of the next layer's routing-independent rows this CTA's warps will read
-      // (phase-R item i belongs to CTA i % G), one lane per item
-      if (l + 1 < a.n_layers) {
-        const FusedLayer& Ln = a.layer[l + 1];
-        const int n_router = (Ln.topk_idx_in ? 0 : E) + 1;
-        const int n_items = n_router + I / RPWg;
-        for (int it = blockIdx.x + G * lane; it < n_items; it += G * 32) {
-          if (it < n_router) {
-            const bool gate_row = (it == n_router - 1);
-            const uint16_t* row = gate_row ? Ln.wsg : Ln.wr + (size_t)it * H;
-            prefetch_l2(row, H * 2);
-          } else {
-            const int r = (it - n_router) * RPWg;
-            prefetch_l2(Ln.shared + a.L.off[0] + (int64_t)r * ROWBg, RPWg * ROWBg);
-            prefetch_l2(Ln.shared + a.L.off[1] + (int64_t)r * ROWBg, RPWg * ROWBg);
-          }
-        }
-      }
+      // L2 prefetch of the next layer's phase-R rows (copied to shared memory later in this layer)
+      if (l + 1 < a.n_layers) issue_r(l + 1, true);
       // wait for this layer's plan
       if (!mbar_wait(&plan_bar, l & 1)) {
         ok = false;
@@ -441,6 +479,11 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
           u += cnt;
         }
       }
+      // the next layer's phase-R rows: this CTA finished reading rbuf before the plan
+      if (ok && l + 1 < a.n_layers) {
+        issue_r(l + 1, false);
+        ++n_r_issued;
+      }
     }
     if (!ok && lane == 0) {
       atomicOr(&a.ctrl->err, kErrTimeout);
@@ -448,6 +491,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
     }
     // let every issued copy land before the CTA may exit
     if (lane == 0) {
+      mbar_wait(&rbar, (uint32_t)(n_r_issued - 1) & 1);
       const uint32_t first = q > (uint32_t)NS ? q - NS : 0;
       for (uint32_t qq = first; qq < q; ++qq) mbar_wait(&full_bar[qq % NS], (qq / NS) & 1);
     }
@@ -475,24 +519,39 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
     for (int e = tid; e < E; e += kConsThreads) S_SLOT[e] = __ldg(Lc.slot_table + e);
     bar_cons();
 
-    // ---- phase R: router rows, shared-gate row, shared gate/up rows ----
+    // ---- phase R: router rows, shared-gate row, shared gate/up rows (staged in rbuf) ----
     {
-      const int n_router = (routed ? E : 0) + 1;
-      const int n_items = n_router + (Lc.with_shared ? I / RPWg : 0);
-      for (int it = blockIdx.x + G * cw; it < n_items; it += NW) {  // item i: CTA i % G
-        if (it < n_router) {
-          const bool gate_row = (it == n_router - 1);
-          const int e = gate_row ? E : it;
-          const uint16_t* row = gate_row ? Lc.wsg : Lc.wr + (size_t)e * H;
+      const RRange R = r_ranges(Lc, E, I, gG, blockIdx.x, G);
+      const int nrr = R.rr1 - R.rr0, ns = R.sr1 - R.sr0, nsi = ns / RPWg;
+      // with several tokens a router row is split into nq column ranges on nq warps (their
+      // fp64 sums added in a fixed order below), as far as the CTA's 15 warps go
+      constexpr int NQ = (TM > 1 && (H / 8 / 4) % 32 == 0) ? 4 : 1;
+      const int nq = (NQ == 4 && nrr * 4 + nsi <= kCons) ? 4 : (NQ == 4 && nrr * 2 + nsi <= kCons) ? 2 : 1;
+      const int n_it = nrr * nq + nsi;
+      if (cw < n_it && !mbar_wait(&rbar, l & 1)) {
+        atomicOr(&a.ctrl->err, kErrTimeout);
+        s_abort = 1;
+      }
+      for (int z = cw; z < n_it && !s_abort; z += kCons) {
+        if (z < nrr * nq) {
+          const int lr = z / nq, qq = z - lr * nq;
+          const bool gate_row = (R.rr0 + lr == R.n_router - 1);
+          const int e = gate_row ? E : R.rr0 + lr;
+          const uint16_t* row = reinterpret_cast<const uint16_t*>(rbuf + (size_t)lr * H * 2);
+          const int cq = H / 8 / nq;
           double acc[TM];
 #pragma unroll
           for (int t = 0; t < TM; ++t) acc[t] = 0.0;
 #pragma unroll 4
-          for (int c8 = lane; c8 < H / 8; c8 += 32) {
-            const uint4 w = ld_stream(row + c8 * 8);
-            const float wv[8] = {bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y),
-                                 bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w)};
+          for (int c8 = qq * cq + lane; c8 < (qq + 1) * cq; c8 += 32) {
+            const uint4 w = *reinterpret_cast<const uint4*>(row + c8 * 8);
             const int c = c8 / (CC / 8), v0 = (c8 % (CC / 8)) * 2;
+            // the weights times the inverse staging scales (powers of two: exact), so that
+            // each product with a staged activation is the exact w * x
+            const float wv[8] = {bf_lo(w.x) * stage_unscale<BITS>(v0 * 4 + 0), bf_hi(w.x) * stage_unscale<BITS>(v0 * 4 + 1),
+                                 bf_lo(w.y) * stage_unscale<BITS>(v0 * 4 + 2), bf_hi(w.y) * stage_unscale<BITS>(v0 * 4 + 3),
+                                 bf_lo(w.z) * stage_unscale<BITS>(v0 * 4 + 4), bf_hi(w.z) * stage_unscale<BITS>(v0 * 4 + 5),
+                                 bf_lo(w.w) * stage_unscale<BITS>(v0 * 4 + 6), bf_hi(w.w) * stage_unscale<BITS>(v0 * 4 + 7)};
 #pragma unroll
             for (int t = 0; t < TM; ++t) {
               if (t < T) {
@@ -501,11 +560,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
                 const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
                 double s = 0.0;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  // undo the staging scale (a power of two): the product stays exact
-                  const float xr = xv[i] * stage_unscale<BITS>(v0 * 4 + i);
-                  s += (double)(wv[i] * xr);
-                }
+                for (int i = 0; i < 8; ++i) s += (double)(wv[i] * xv[i]);
                 acc[t] += s;
               }
             }
@@ -517,36 +572,76 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
 #pragma unroll
               for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
               if (lane == 0) {
-                if (!gate_row && Lc.rbias) v += (double)Lc.rbias[e];
-                a.logits[(size_t)t * (E + 1) + e] = v;
+                if (nq > 1) {
+                  rpart[((size_t)lr * nq + qq) * T + t] = v;
+                } else {
+                  if (!gate_row && Lc.rbias) v += (double)Lc.rbias[e];
+                  a.logits[(size_t)t * (E + 1) + e] = v;
+                }
               }
             }
           }
         } else {
           // shared expert gate/up row(s): chunk by chunk, every token against each chunk
-          const int r = (it - n_router) * RPWg + lane / NCLg;
+          const int rl = (z - nrr * nq) * RPWg + lane / NCLg;  // row within this CTA's range
           const int sub = lane % NCLg;
-          const uint8_t* b = Lc.shared;
+          const uint8_t* gq = rbuf_s + (size_t)rl * ROWBg;
+          const uint8_t* uq = rbuf_s + (size_t)ns * ROWBg + rl * ROWBg;
+          const uint8_t* sc = rbuf_s + 2 * (size_t)ns * ROWBg + rl * SRg;
           float ag[TM], au[TM];
 #pragma unroll
           for (int t = 0; t < TM; ++t) ag[t] = au[t] = 0.f;
 #pragma unroll 1
           for (int m = 0; m < CPLg; ++m) {
             const int c = sub + NCLg * m, g = c * CC / kGroup;
-            const uint4 qg = ld_stream(b + a.L.off[0] + (int64_t)r * ROWBg + c * 16);
-            const uint4 qu = ld_stream(b + a.L.off[1] + (int64_t)r * ROWBg + c * 16);
-            const float sg = bf1(ld_u16(b + a.L.off[3] + (int64_t)r * SRg + g * 2));
-            const float bg = bf1(ld_u16(b + a.L.off[4] + (int64_t)r * SRg + g * 2));
-            const float su = bf1(ld_u16(b + a.L.off[5] + (int64_t)r * SRg + g * 2));
-            const float bu = bf1(ld_u16(b + a.L.off[6] + (int64_t)r * SRg + g * 2));
+            const uint4 qg = *reinterpret_cast<const uint4*>(gq + c * 16);
+            const uint4 qu = *reinterpret_cast<const uint4*>(uq + c * 16);
+            const float sg = bf1(*reinterpret_cast<const uint16_t*>(sc + g * 2));
+            const float bg = bf1(*reinterpret_cast<const uint16_t*>(sc + ns * SRg + g * 2));
+            const float su = bf1(*reinterpret_cast<const uint16_t*>(sc + 2 * ns * SRg + g * 2));
+            const float bu = bf1(*reinterpret_cast<const uint16_t*>(sc + 3 * ns * SRg + g * 2));
+            if constexpr (TM == 1) {
+              float dg, du;
+              dot_chunk2<BITS>(qg, qu, xs4 + c, NCg, dg, du);
+              const float xc = xsum[c];
+              ag[0] = fmaf(sg, dg, fmaf(bg, xc, ag[0]));
+              au[0] = fmaf(su, du, fmaf(bu, xc, au[0]));
+            } else {
+              // several tokens: each code pair becomes floats once and meets every token
+              float2 gacc[TM], uacc[TM];
 #pragma unroll
-            for (int t = 0; t < TM; ++t) {
-              if (t < T) {
-                float dg, du;
-                dot_chunk2<BITS>(qg, qu, xs4 + (size_t)t * V4 * NCg + c, NCg, dg, du);
-                const float xc = xsum[t * NCg + c];
-                ag[t] = fmaf(sg, dg, fmaf(bg, xc, ag[t]));
-                au[t] = fmaf(su, du, fmaf(bu, xc, au[t]));
+              for (int t = 0; t < TM; ++t) gacc[t] = uacc[t] = make_float2(0.f, 0.f);
+#pragma unroll
+              for (int wi = 0; wi < 4; ++wi) {
+                float2 cg[4], cu[4];
+                codes_of_word<BITS>(word_of(qg, wi), cg);
+                codes_of_word<BITS>(word_of(qu, wi), cu);
+#pragma unroll
+                for (int t = 0; t < TM; ++t) {
+                  if (t < T) {
+                    const float4* xt = xs4 + (size_t)t * V4 * NCg + c;
+                    if constexpr (BITS == 4) {
+                      const float4 xa = xt[(2 * wi) * NCg], xb = xt[(2 * wi + 1) * NCg];
+                      const float2 x01 = make_float2(xa.x, xa.y), x23 = make_float2(xa.z, xa.w);
+                      const float2 x45 = make_float2(xb.x, xb.y), x67 = make_float2(xb.z, xb.w);
+                      gacc[t] = ffma2(cg[3], x67, ffma2(cg[2], x45, ffma2(cg[1], x23, ffma2(cg[0], x01, gacc[t]))));
+                      uacc[t] = ffma2(cu[3], x67, ffma2(cu[2], x45, ffma2(cu[1], x23, ffma2(cu[0], x01, uacc[t]))));
+                    } else {
+                      const float4 xa = xt[wi * NCg];
+                      const float2 x01 = make_float2(xa.x, xa.y), x23 = make_float2(xa.z, xa.w);
+                      gacc[t] = ffma2(cg[1], x23, ffma2(cg[0], x01, gacc[t]));
+                      uacc[t] = ffma2(cu[1], x23, ffma2(cu[0], x01, uacc[t]));
+                    }
+                  }
+                }
+              }
+#pragma unroll
+              for (int t = 0; t < TM; ++t) {
+                if (t < T) {
+                  const float xc = xsum[t * NCg + c];
+                  ag[t] = fmaf(sg, gacc[t].x + gacc[t].y, fmaf(bg, xc, ag[t]));
+                  au[t] = fmaf(su, uacc[t].x + uacc[t].y, fmaf(bu, xc, au[t]));
+                }
               }
             }
           }
@@ -559,9 +654,22 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
                 g2 += __shfl_xor_sync(0xffffffffu, g2, o);
                 u2 += __shfl_xor_sync(0xffffffffu, u2, o);
               }
-              if (sub == 0) a.hs[(size_t)t * I + r] = g2 / (1.0f + expf(-g2)) * u2;
+              if (sub == 0) a.hs[(size_t)t * I + R.sr0 + rl] = g2 / (1.0f + expf(-g2)) * u2;
             }
           }
+        }
+      }
+      if (nq > 1) {
+        // the router rows' column-range sums, added in range order
+        bar_cons();
+        for (int i = tid; i < nrr * T; i += kConsThreads) {
+          const int lr = i / T, t = i - lr * T;
+          double v = 0.0;
+          for (int qq = 0; qq < nq; ++qq) v += rpart[((size_t)lr * nq + qq) * T + t];
+          const bool gate_row = (R.rr0 + lr == R.n_router - 1);
+          const int e = gate_row ? E : R.rr0 + lr;
+          if (!gate_row && Lc.rbias) v += (double)Lc.rbias[e];
+          a.logits[(size_t)t * (E + 1) + e] = v;
         }
       }
     }
@@ -639,40 +747,64 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
         if (cw == (T + t) % kCons && lane == 0) P_GATE[t] = (float)(1.0 / (1.0 + exp(-__ldcg(a.logits + (size_t)t * (E + 1) + E))));
     }
     bar_cons();
-    // grouping: pairs sorted by (expert, pair number); invalid ids left out
+    // grouping: pairs sorted by (expert, pair number); invalid ids left out.  The pairwise
+    // comparisons are spread over all compute threads (pair i against a block of pairs j),
+    // their counts added with integer atomics, so the result does not depend on the order.
     if (ok && !(T == 1 && routed)) {
-      int* key = P_SCRATCH;
-      int* first = P_SCRATCH + TK;
+      int* key = P_SCRATCH;            // [TK] expert of pair i (E: left out)
+      int* rnk = P_SCRATCH + TK;       // [TK] rank of pair i in (expert, pair) order
+      int* dup = P_SCRATCH + 2 * TK;   // [TK] an earlier pair has the same expert
+      int* first = P_SCRATCH + 3 * TK; // [TK] pair i is its expert's first
+      int* actc = P_SCRATCH + 4 * TK;  // [TK] distinct experts below pair i's
+      __shared__ int s_an, s_nv;
       for (int i = tid; i < TK; i += kConsThreads) {
         const int e = P_IDS[i];
         const bool valid = e >= 0 && e < E;
         if (!valid && blockIdx.x == 0) atomicOr(&a.ctrl->err, kErrBadExpert);
         key[i] = (valid && S_SLOT[e] != kSlotRemote) ? e : E;
+        rnk[i] = 0;
+        dup[i] = 0;
+        actc[i] = 0;
+      }
+      if (tid == 0) s_an = s_nv = 0;
+      const int nb = kConsThreads / TK > 0 ? kConsThreads / TK : 1, jb = (TK + nb - 1) / nb;
+      bar_cons();
+      for (int w = tid; w < TK * nb; w += kConsThreads) {
+        const int i = w % TK, j0b = (w / TK) * jb, ki = key[i];
+        int r = 0, d = 0;
+        for (int j = j0b; j < min(TK, j0b + jb); ++j) {
+          const int kj = key[j];
+          r += (kj < ki) || (kj == ki && j < i);
+          d |= (kj == ki && j < i);
+        }
+        if (r) atomicAdd(&rnk[i], r);
+        if (d) atomicOr(&dup[i], 1);
       }
       bar_cons();
       for (int i = tid; i < TK; i += kConsThreads) {
+        const int ki = key[i], r = rnk[i];
+        const bool f = !dup[i] && ki < E;
+        P_ORDER[r] = i;
+        P_POS[i] = (ki < E) ? r : -1;
+        first[i] = f ? 1 : 0;
+        if (ki < E) atomicAdd(&s_nv, 1);
+        if (f) atomicAdd(&s_an, 1);
+      }
+      bar_cons();
+      for (int w = tid; w < TK * nb; w += kConsThreads) {
+        const int i = w % TK, j0b = (w / TK) * jb;
+        if (!first[i]) continue;
         const int ki = key[i];
-        int rank = 0, fst = 1;
-        for (int j = 0; j < TK; ++j) {
-          const int kj = key[j];
-          rank += (kj < ki) || (kj == ki && j < i);
-          if (kj == ki && j < i) fst = 0;
-        }
-        P_ORDER[rank] = i;
-        P_POS[i] = (ki < E) ? rank : -1;
-        first[i] = (fst && ki < E) ? 1 : 0;
+        int c = 0;
+        for (int j = j0b; j < min(TK, j0b + jb); ++j) c += (first[j] && key[j] < ki);
+        if (c) atomicAdd(&actc[i], c);
       }
       bar_cons();
       for (int i = tid; i < TK; i += kConsThreads) {
         if (first[i]) {
-          const int ki = key[i];
-          int act = 0, before = 0;
-          for (int j = 0; j < TK; ++j) {
-            act += (first[j] && key[j] < ki);
-            before += (key[j] < ki);
-          }
+          const int ki = key[i], act = actc[i];
           P_ACTE[act] = ki;
-          P_BEGIN[act] = before;
+          P_BEGIN[act] = rnk[i];  // the first pair of an expert: its rank counts the pairs below
           const int slot = S_SLOT[ki];
           const bool sok = (slot >= 0 && slot < Lc.n_slots) || slot == kSlotPending;
           if (!sok) atomicOr(&a.ctrl->err, kErrBadSlot);
@@ -680,14 +812,9 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
         }
       }
       if (tid == 0) {
-        int an = 0, nv = 0;
-        for (int i = 0; i < TK; ++i) {
-          an += first[i];
-          nv += key[i] < E;
-        }
-        s_act_n = an;
-        s_n_valid = nv;
-        P_BEGIN[an] = nv;
+        s_act_n = s_an;
+        s_n_valid = s_nv;
+        P_BEGIN[s_an] = s_nv;
       }
     }
     bar_cons();
@@ -922,7 +1049,8 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
 }  // namespace
 
 static size_t fused_smem_bytes(const FusedArgs& a, int stages) {
-  return fused_smem_layout(a.T, a.H, a.I, a.E, a.bits, a.k, a.jmax, stages, a.stage_bytes, kCons).total;
+  return fused_smem_layout(a.T, a.H, a.I, a.E, a.bits, a.k, a.jmax, stages, a.stage_bytes, kCons, a.rr_max,
+                           a.rs_max).total;
 }
 
 template <int BITS, int H, int I, int TM>
@@ -943,11 +1071,23 @@ static cudaError_t run_fused(FusedArgs a, cudaStream_t s) {
   constexpr int gD = clcm(16 / cgcd(16, SRd), RPWd);
   const int nGran = H / gD;
   a.jmax = ((nGran + n_sm - 1) / n_sm) * gD;
-  a.stage_bytes = 32768;
-  int stages = kMaxStages;
-  while (stages > 2 && fused_smem_bytes(a, stages) > (size_t)max_smem) --stages;
+  // phase-R rows a CTA stages: its share of the E + 1 router rows and of the shared expert's
+  // rows (in granules of gG rows)
+  constexpr int NCg = H / CC, NCLg = NCg < 32 ? NCg : 32, RPWg = 32 / NCLg, SRg = (H / kGroup) * 2;
+  constexpr int gG = clcm(16 / cgcd(16, SRg), RPWg);
+  a.rr_max = (a.E + 1 + n_sm - 1) / n_sm;
+  a.rs_max = ((I / gG + n_sm - 1) / n_sm) * gG;
+  // ring stages of 32 KB, or 24 KB where that keeps four of them
+  int stages = 2;
+  for (int sb : {32768, 24576}) {
+    a.stage_bytes = sb;
+    stages = kMaxStages;
+    while (stages > 2 && fused_smem_bytes(a, stages) > (size_t)max_smem) --stages;
+    if (stages >= 4) break;
+  }
   a.n_stages = stages;
-  a.sm = fused_smem_layout(a.T, a.H, a.I, a.E, a.bits, a.k, a.jmax, stages, a.stage_bytes, kCons);
+  a.sm = fused_smem_layout(a.T, a.H, a.I, a.E, a.bits, a.k, a.jmax, stages, a.stage_bytes, kCons, a.rr_max,
+                           a.rs_max);
   const size_t smem = a.sm.total;
   if (smem > (size_t)max_smem) return cudaErrorInvalidConfiguration;
   // one stage must hold one gate/up row and one expert's down slice

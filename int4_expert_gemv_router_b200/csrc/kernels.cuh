@@ -109,6 +109,23 @@ __device__ __forceinline__ float dot_chunk(const uint4& q, const float4* x4, int
   return (a0.x + a0.y) + (a1.x + a1.y);
 }
 
+// The codes of one 32-bit word of a chunk as float pairs, in the pairing the dot products
+// above use: int4 (c0, c1), (c2, c3), (c4, c5), (c6, c7); int8 (c0, c1), (c2, c3) in out[0..1].
+template <int BITS>
+__device__ __forceinline__ void codes_of_word(uint32_t w, float2 out[4]) {
+  if constexpr (BITS == 4) {
+    const uint32_t wh = w >> 12;
+    out[0] = codes2(w & 0xFu, w & 0xF0u);
+    out[1] = codes2(w & 0xF00u, w & 0xF000u);
+    out[2] = codes2(w & 0xF0000u, wh & 0xF00u);
+    out[3] = codes2(wh & 0xF000u, wh & 0xF0000u);
+  } else {
+    const uint32_t wh = w >> 16;
+    out[0] = codes2(w & 0xFFu, w & 0xFF00u);
+    out[1] = codes2(wh & 0xFFu, wh & 0xFF00u);
+  }
+}
+
 // Two code rows (gate and up) sharing the same activations.
 template <int BITS>
 __device__ __forceinline__ void dot_chunk2(const uint4& qa, const uint4& qb, const float4* x4, int ns,
