@@ -431,13 +431,36 @@ def run_gdn(args, name, device, rank):
     states = [synth.gdn_state(Hv, dk, dv, B, c["seed"] + 1000 * rank + l, device) for l in range(nL)]
     ins = [synth.gdn_inputs(Hk, Hv, dk, dv, B, 1, c["seed"] + 1000 * rank + 100 + l, device) for l in range(nL)]
     ins = [tuple(t[0].contiguous() for t in x) for x in ins]
-    outs = [torch.empty(B, Hv, dv, dtype=torch.bfloat16, device=device) for _ in range(nL)]
+    # every layer's q, k, v, g, beta as views of one flat byte buffer (two of them, for the
+    # end-to-end pipeline), and every layer's output as a slice of one [layers, B, Hv, dv] tensor
+    sizes = [t.numel() * t.element_size() for t in ins[0]]
+    per_layer = sum((n + 15) // 16 * 16 for n in sizes)
+    flat = [torch.empty(nL * per_layer, dtype=torch.uint8, device=device) for _ in range(2)]
+
+    def views(buf):
+        res = []
+        for l in range(nL):
+            off, vs = l * per_layer, []
+            for t, n in zip(ins[l], sizes):
+                vs.append(buf[off:off + n].view(t.dtype).view(t.shape))
+                off += (n + 15) // 16 * 16
+            res.append(tuple(vs))
+        return res
+
+    ins_b = [views(flat[0]), views(flat[1])]
+    for b in range(2):
+        for l in range(nL):
+            for dst, src in zip(ins_b[b][l], ins[l]):
+                dst.copy_(src)
+    ins = ins_b[0]
+    outs_b = [torch.empty(nL, B, Hv, dv, dtype=torch.bfloat16, device=device) for _ in range(2)]
+    outs = outs_b[0]
     stream = torch.cuda.Stream(device)
 
-    def layer_calls():
+    def layer_calls(b=0):
         for l in range(nL):
-            q, k, v, g, beta = ins[l]
-            abi.moe_gdn_decode_step(shape, B, states[l], q, k, v, g, beta, outs[l])
+            q, k, v, g, beta = ins_b[b][l]
+            abi.moe_gdn_decode_step(shape, B, states[l], q, k, v, g, beta, outs_b[b][l])
 
     with torch.cuda.stream(stream):
         layer_calls()
@@ -472,23 +495,19 @@ def run_gdn(args, name, device, rank):
             evs[l][1].record(stream)
     stream.synchronize()
     launch_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in evs)
-    # end to end: the step's inputs from pinned host memory and its outputs back, every step
-    host_in = [tuple(t.cpu().pin_memory() for t in x) for x in ins]
-    host_out = torch.empty(nL, B, Hv, dv, dtype=torch.bfloat16).pin_memory()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        f0.record(stream)
-        for _ in range(K):
-            for l in range(nL):
-                for dst, src in zip(ins[l], host_in[l]):
-                    dst.copy_(src, non_blocking=True)
-            g_.replay()
-            for l in range(nL):
-                host_out[l].copy_(outs[l], non_blocking=True)
-        f1.record(stream)
-    f1.synchronize()
-    e2e_ms = reduce_max(f0.elapsed_time(f1), device)
-    in_bytes = sum(t.numel() * t.element_size() for t in ins[0])
+    # end to end: every step's inputs of all layers come up from pinned host memory in one copy
+    # and all outputs go back in one, pipelined over two buffer sets (one graph per set)
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=stream):
+        layer_calls(1)
+    graphs = [g_, g2]
+    host_in = flat[0].cpu().pin_memory()
+    host_out = [torch.empty(nL, B, Hv, dv, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    barrier(device)
+    e2e_ms = pipelined_e2e(device, stream, K, lambda i, b: flat[b].copy_(host_in, non_blocking=True),
+                           lambda i, b: graphs[b].replay(),
+                           lambda i, b: host_out[b].copy_(outs_b[b], non_blocking=True))
+    in_bytes = per_layer  # the flat upload, padding included
     return dict(c=c, ms=ms, clocks=clocks, launch_us=launch_us, e2e_ms=e2e_ms, in_bytes=in_bytes * nL,
                 out_bytes=nL * B * Hv * dv * 2, state=states[0], ins=ins[0])
 
@@ -567,7 +586,9 @@ def gdn_line(args, name, r, n_gpus, peaks, peak_kind, cpu_base):
                      "bytes_per_launch": per_launch, "peak_kind": f"{peak_kind} hbm_gbs (burst copy)"},
         "clocks": r["clocks"],
         "e2e": {"value": round(n_gpus * B * K / (r["e2e_ms"] / 1e3), 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": r["in_bytes"], "d2h_bytes_per_step": r["out_bytes"]},
+                "h2d_bytes_per_step": r["in_bytes"], "d2h_bytes_per_step": r["out_bytes"],
+                "copies": "one upload and one download per step (all layers), two buffer sets, on copy "
+                          "streams overlapping the neighbouring steps"},
         "gpu_launches": nL * K,
     }
     if cpu_base is not None:
@@ -681,6 +702,45 @@ def prefill_flops(w, T):
     return router, gateup, down
 
 
+def pipelined_e2e(device, stream, K, upload, compute, download):
+    """Device time of K steps end to end, with two buffers each way: upload(i, b) copies step
+    i's inputs from pinned host memory into device buffer b (b = i % 2), compute(i, b) runs the
+    step on buffer b and download(i, b) copies its result back to pinned host memory.  Uploads
+    run on one copy stream and downloads on another, so that step i + 1's upload and step
+    i - 1's download overlap step i's compute; events keep a buffer from being overwritten
+    before the step that reads it is done.  The timed region runs from before the first upload
+    to after the last download."""
+    up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    in_free, out_free = [f0, f0], [f0, f0]
+    for i in range(K):
+        b = i % 2
+        up.wait_event(in_free[b])
+        with torch.cuda.stream(up):
+            upload(i, b)
+        ready = torch.cuda.Event()
+        ready.record(up)
+        stream.wait_event(ready)
+        stream.wait_event(out_free[b])
+        with torch.cuda.stream(stream):
+            compute(i, b)
+        done = torch.cuda.Event()
+        done.record(stream)
+        in_free[b] = done
+        down.wait_event(done)
+        with torch.cuda.stream(down):
+            download(i, b)
+        read = torch.cuda.Event()
+        read.record(down)
+        out_free[b] = read
+    stream.wait_event(out_free[0])
+    stream.wait_event(out_free[1])
+    f1.record(stream)
+    f1.synchronize()
+    return reduce_max(f0.elapsed_time(f1), device)
+
+
 def run_prefill(args, w, T, device, rank):
     from int4_expert_gemv_router_b200 import abi, build
     build.build()
@@ -739,20 +799,21 @@ def run_prefill(args, w, T, device, rank):
         for g in range(5):
             kern[g].append(event_ms(evs[2 * g], evs[2 * g + 1]))
     kern_us = [1e3 * statistics.mean(v) for v in kern]
-    # end to end: pinned host x in, out back, every step
+    # end to end: every step's x comes up from pinned host memory and its output goes back,
+    # as a serving loop runs it: two device buffers each way, step i + 1's upload and step
+    # i - 1's download on two copy streams while step i computes
     x_host = [x.cpu().pin_memory() for x in xs]
-    out_host = torch.empty(T, w.hidden, dtype=torch.bfloat16).pin_memory()
+    out_host = [torch.empty(T, w.hidden, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    xb = [xbuf, torch.empty_like(xbuf)]
+    ob = [out, torch.empty_like(out)]
+
+    def call_on(b):
+        abi.moe_layer_forward(shape, xb[b], T, L.w_router, L.router_bias, None, None, L.pool, slots, w.n_experts,
+                              L.shared, L.w_sg, xb[b], ob[b], idx, p, ws)
+
     barrier(device)
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        f0.record(stream)
-        for i in range(K):
-            xbuf.copy_(x_host[i % n_in], non_blocking=True)
-            call()
-            out_host.copy_(out, non_blocking=True)
-        f1.record(stream)
-    f1.synchronize()
-    e2e_ms = reduce_max(f0.elapsed_time(f1), device)
+    e2e_ms = pipelined_e2e(device, stream, K, lambda i, b: xb[b].copy_(x_host[i % n_in], non_blocking=True),
+                           lambda i, b: call_on(b), lambda i, b: out_host[b].copy_(ob[b], non_blocking=True))
     counts = np.bincount(idx.cpu().numpy().reshape(-1), minlength=w.n_experts)
     return dict(ms=ms, clocks=clocks, flags=flags, kern_us=kern_us, e2e_ms=e2e_ms, layer=L, x=xs[0],
                 tokens_per_expert=(float(counts.mean()), int(counts.min()), int(counts.max())))
@@ -807,7 +868,9 @@ def prefill_line(args, w, T, r, n_gpus, peaks, peak_kind, cpu_base):
                        "finalize": round(r["kern_us"][4], 2)},
         "clocks": r["clocks"],
         "e2e": {"value": round(n_gpus * T * K / (r["e2e_ms"] / 1e3), 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": T * w.hidden * 2, "d2h_bytes_per_step": T * w.hidden * 2},
+                "h2d_bytes_per_step": T * w.hidden * 2, "d2h_bytes_per_step": T * w.hidden * 2,
+                "copies": "two buffers each way, uploads and downloads on copy streams overlapping the "
+                          "neighbouring steps"},
         "gpu_launches": 8 * K,
         "device_error_flags": r["flags"],
     }
