@@ -458,9 +458,11 @@ def run_gdn(args, name, device, rank):
     stream = torch.cuda.Stream(device)
 
     def layer_calls(b=0):
+        # each layer's step reads its own state early, while the previous layer finishes
+        # (consecutive layers never share a state)
         for l in range(nL):
             q, k, v, g, beta = ins_b[b][l]
-            abi.moe_gdn_decode_step(shape, B, states[l], q, k, v, g, beta, outs_b[b][l])
+            abi.moe_gdn_decode_step(shape, B, states[l], q, k, v, g, beta, outs_b[b][l], flags=abi.MOE_GDN_EARLY_STATE)
 
     with torch.cuda.stream(stream):
         layer_calls()

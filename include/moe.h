@@ -337,6 +337,20 @@ MOE_API moe_status moe_gdn_decode_step(const moe_gdn_shape* shape, int32_t B, fl
                                        const void* k, const void* v, const float* g, const float* beta,
                                        void* out, void* stream);
 
+/*
+ * moe_gdn_decode_step_ex -- moe_gdn_decode_step with flags (0: the same call).
+ *   MOE_GDN_EARLY_STATE: the step is launched as a programmatic dependent of the kernel
+ *   before it on the stream and reads its state rows before that kernel has finished; it
+ *   waits for that kernel only before reading q, k, v, g and beta and before writing
+ *   anything.  The caller guarantees that the preceding kernel on the stream does not write
+ *   this call's state (true of consecutive layers, each with its own state).  Everything
+ *   else, ownership and errors as moe_gdn_decode_step.
+ */
+#define MOE_GDN_EARLY_STATE 1
+MOE_API moe_status moe_gdn_decode_step_ex(const moe_gdn_shape* shape, int32_t B, float* state, const void* q,
+                                          const void* k, const void* v, const float* g, const float* beta,
+                                          void* out, int32_t flags, void* stream);
+
 /* ------------------------------------------------------------------------------------ */
 /* Bounded slot pool with LFU + recency eviction («Paquets Swiftlet…» paragraph 5;       */
 /* «Swiftlet: 在 Mac 和 iPhone 上執行…», 記憶體管理與權重串流).  Misses are copied from   */

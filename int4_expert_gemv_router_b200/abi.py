@@ -77,6 +77,8 @@ _SIGS = {
     "moe_ws_set_slot_wait": (ctypes.c_int, [_P, ctypes.c_uint32, _P]),
     "moe_ws_router_logits": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, _P, _SZ, ctypes.POINTER(_P)]),
     "moe_gdn_decode_step": (ctypes.c_int, [ctypes.POINTER(moe_gdn_shape), _I32, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_gdn_decode_step_ex": (ctypes.c_int, [ctypes.POINTER(moe_gdn_shape), _I32, _P, _P, _P, _P, _P, _P, _P, _I32,
+                                              _P]),
     "moe_pool_create": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, _P, _P, _P, ctypes.POINTER(_P)]),
     "moe_pool_create_file": (ctypes.c_int, [ctypes.POINTER(moe_shape), _I32, ctypes.c_char_p, _I32, _P, _P,
                                             ctypes.POINTER(_P)]),
@@ -250,10 +252,19 @@ def moe_ws_router_logits(shape, T: int, ws) -> torch.Tensor:
     return ws[off:off + 4 * n].view(torch.float32).view(T, shape.n_experts + 1)
 
 
-def moe_gdn_decode_step(shape, B, state, q, k, v, g, beta, out, stream=None):
-    """One gated-delta-rule decode step of B sequences; state (fp32) is updated in place."""
-    _check(lib().moe_gdn_decode_step(ctypes.byref(shape), B, _ptr(state), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
-                                     _ptr(beta), _ptr(out), _stream(stream)))
+MOE_GDN_EARLY_STATE = 1
+
+
+def moe_gdn_decode_step(shape, B, state, q, k, v, g, beta, out, stream=None, flags=0):
+    """One gated-delta-rule decode step of B sequences; state (fp32) is updated in place.
+    flags=MOE_GDN_EARLY_STATE: the state rows may be read before the preceding kernel on the
+    stream has finished (that kernel must not write this state)."""
+    if flags:
+        _check(lib().moe_gdn_decode_step_ex(ctypes.byref(shape), B, _ptr(state), _ptr(q), _ptr(k), _ptr(v),
+                                            _ptr(g), _ptr(beta), _ptr(out), flags, _stream(stream)))
+    else:
+        _check(lib().moe_gdn_decode_step(ctypes.byref(shape), B, _ptr(state), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                         _ptr(beta), _ptr(out), _stream(stream)))
 
 
 def moe_pool_create(shape, n_slots, host_blobs, dev_pool, dev_slot_table) -> int:

@@ -60,6 +60,8 @@ __global__ void __launch_bounds__(kGdnWarps * 32) k_gdn_step(const GdnArgs a) {
   const int kh = h / (a.Hv / a.Hk);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* Sh = a.S + (size_t)bh * a.dv * DK;
+  // the next kernel on the stream may start launching (it waits for this one where it must)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // the rows this warp owns, loaded first so that their latency overlaps the normalisation
   float row[kGdnRowsPerWarp][EPL];
@@ -85,6 +87,11 @@ __global__ void __launch_bounds__(kGdnWarps * 32) k_gdn_step(const GdnArgs a) {
       }
     }
   }
+  // Launched as a programmatic dependent (MOE_GDN_EARLY_STATE), the state rows above were read
+  // while the kernel before may still run (the caller guarantees it does not write them);
+  // from here on every read and write waits for it to have finished.  Without that launch
+  // attribute the wait returns at once.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // k and q of this head's key head: warp 0 normalises k, warp 1 q (fp32 sums of squares)
   if (warp < 2) {
     const uint16_t* src = (warp == 0 ? a.k : a.q) + ((size_t)b * a.Hk + kh) * DK;
@@ -154,19 +161,29 @@ static int gdn_rows_per_warp(const GdnArgs& a, int n_sm) {
 }
 
 template <int RPW>
-static cudaError_t launch_gdn_rpw(const GdnArgs& a, cudaStream_t s) {
+static cudaError_t launch_gdn_rpw(const GdnArgs& a, cudaStream_t s, bool early_state) {
   const int rows_cta = kGdnWarps * RPW;
   const int blocks = a.B * a.Hv * ((a.dv + rows_cta - 1) / rows_cta);
+  void (*fn)(GdnArgs) = nullptr;
   switch (a.dk) {
-    case 64: k_gdn_step<64, RPW><<<blocks, kGdnWarps * 32, 0, s>>>(a); break;
-    case 128: k_gdn_step<128, RPW><<<blocks, kGdnWarps * 32, 0, s>>>(a); break;
-    case 256: k_gdn_step<256, RPW><<<blocks, kGdnWarps * 32, 0, s>>>(a); break;
+    case 64: fn = k_gdn_step<64, RPW>; break;
+    case 128: fn = k_gdn_step<128, RPW>; break;
+    case 256: fn = k_gdn_step<256, RPW>; break;
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(kGdnWarps * 32);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = early_state ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, fn, a);
 }
 
-cudaError_t launch_gdn_step(const GdnArgs& a, cudaStream_t s) {
+cudaError_t launch_gdn_step(const GdnArgs& a, cudaStream_t s, bool early_state) {
   static int n_sm = 0;
   if (!n_sm) {
     int dev = 0;
@@ -175,9 +192,9 @@ cudaError_t launch_gdn_step(const GdnArgs& a, cudaStream_t s) {
     if (n_sm < 1) n_sm = 1;
   }
   switch (gdn_rows_per_warp(a, n_sm)) {
-    case 2: return launch_gdn_rpw<2>(a, s);
-    case 4: return launch_gdn_rpw<4>(a, s);
-    default: return launch_gdn_rpw<8>(a, s);
+    case 2: return launch_gdn_rpw<2>(a, s, early_state);
+    case 4: return launch_gdn_rpw<4>(a, s, early_state);
+    default: return launch_gdn_rpw<8>(a, s, early_state);
   }
 }
 
@@ -188,9 +205,10 @@ moe_status cuda_fail(cudaError_t e, const char* what);
 
 using namespace moe;
 
-extern "C" moe_status moe_gdn_decode_step(const moe_gdn_shape* shape, int32_t B, float* state, const void* q,
-                                          const void* k, const void* v, const float* g, const float* beta, void* out,
-                                          void* stream) {
+extern "C" moe_status moe_gdn_decode_step_ex(const moe_gdn_shape* shape, int32_t B, float* state, const void* q,
+                                             const void* k, const void* v, const float* g, const float* beta,
+                                             void* out, int32_t flags, void* stream) {
+  if (flags & ~MOE_GDN_EARLY_STATE) return set_error(MOE_ERR_INVALID, "unknown flags 0x%x", flags);
   if (!shape) return set_error(MOE_ERR_INVALID, "shape is NULL");
   const int Hk = shape->n_k_heads, Hv = shape->n_v_heads, dk = shape->d_k, dv = shape->d_v;
   if (Hk < 1 || Hv < 1 || Hv % Hk) return set_error(MOE_ERR_INVALID, "n_v_heads must be a positive multiple of n_k_heads");
@@ -206,7 +224,13 @@ extern "C" moe_status moe_gdn_decode_step(const moe_gdn_shape* shape, int32_t B,
   if (blocks > 0x7fffffffLL) return set_error(MOE_ERR_INVALID, "B * n_v_heads * d_v too large");
   GdnArgs a{B, Hk, Hv, dk, dv, state, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
             static_cast<const uint16_t*>(v), g, beta, static_cast<uint16_t*>(out)};
-  cudaError_t e = launch_gdn_step(a, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_gdn_step(a, static_cast<cudaStream_t>(stream), (flags & MOE_GDN_EARLY_STATE) != 0);
   if (e != cudaSuccess) return cuda_fail(e, "gated delta step launch");
   return MOE_OK;
+}
+
+extern "C" moe_status moe_gdn_decode_step(const moe_gdn_shape* shape, int32_t B, float* state, const void* q,
+                                          const void* k, const void* v, const float* g, const float* beta, void* out,
+                                          void* stream) {
+  return moe_gdn_decode_step_ex(shape, B, state, q, k, v, g, beta, out, 0, stream);
 }

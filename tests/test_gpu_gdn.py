@@ -83,3 +83,72 @@ def test_gdn_rejects_bad_shapes():
     with pytest.raises(abi.MoeError) as ei:
         abi.moe_gdn_decode_step(abi.moe_gdn_shape(2, 2, 96, 128), 1, t, t, t, t, t, t, t)
     assert ei.value.status == -5
+
+
+@pytest.mark.parametrize("B,graph", [(1, False), (1, True), (8, True)])
+def test_gdn_early_state_chain_matches_plain(B, graph):
+    """A chain of layers (each its own state) run for two steps with MOE_GDN_EARLY_STATE —
+    each step launched as a programmatic dependent of the one before, reading its state rows
+    early — gives bit for bit the outputs and states of the same chain launched plainly, and
+    the first layer matches the oracle."""
+    Hk, Hv, dk, dv, nL, steps = 16, 32, 128, 128, 4, 2
+    shape = abi.moe_gdn_shape(Hk, Hv, dk, dv)
+    ins = [synth.gdn_inputs(Hk, Hv, dk, dv, B, steps, 300 + l, DEV) for l in range(nL)]
+    S0 = [synth.gdn_state(Hv, dk, dv, B, 400 + l, DEV) for l in range(nL)]
+
+    def chain(flags):
+        S = [s.clone() for s in S0]
+        outs = torch.empty(steps, nL, B, Hv, dv, dtype=torch.bfloat16, device=DEV)
+        stream = torch.cuda.Stream()
+
+        def one_step(t):
+            for l in range(nL):
+                q, k, v, g, beta = (x[t].contiguous() for x in ins[l])
+                abi.moe_gdn_decode_step(shape, B, S[l], q, k, v, g, beta, outs[t, l], stream=stream, flags=flags)
+
+        with torch.cuda.stream(stream):
+            if graph:
+                # the inputs are made contiguous once, outside the captured calls
+                flat = [[tuple(x[t].contiguous() for x in ins[l]) for l in range(nL)] for t in range(steps)]
+                graphs = []
+                for t in range(steps):
+                    gr = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(gr, stream=stream):
+                        for l in range(nL):
+                            abi.moe_gdn_decode_step(shape, B, S[l], *flat[t][l], outs[t, l], stream=stream,
+                                                    flags=flags)
+                    graphs.append(gr)
+                # capture ran nothing: reset the states the captures did not touch, then replay
+                for l in range(nL):
+                    S[l].copy_(S0[l])
+                for gr in graphs:
+                    gr.replay()
+            else:
+                for t in range(steps):
+                    one_step(t)
+        stream.synchronize()
+        return outs, S
+
+    o0, s0 = chain(0)
+    o1, s1 = chain(abi.MOE_GDN_EARLY_STATE)
+    assert torch.equal(o0, o1)
+    for a_, b_ in zip(s0, s1):
+        assert torch.equal(a_, b_)
+    f = lambda t: t.float().double().cpu().numpy()  # noqa: E731
+    Sb = S0[0][0].double().cpu().numpy()
+    q, k, v, g, beta = ins[0]
+    for t in range(steps):
+        Sb, o_ref = oracle.gdn_step(Sb, f(q[t, 0]), f(k[t, 0]), f(v[t, 0]), f(g[t, 0]), f(beta[t, 0]))
+        err = np.abs(f(o1[t, 0, 0]) - o_ref).max()
+        assert err <= 1e-2 * np.abs(o_ref).max() + 1e-3, (t, err)
+
+
+def test_gdn_rejects_unknown_flags():
+    shape = abi.moe_gdn_shape(2, 2, 64, 16)
+    S = torch.zeros(1, 2, 16, 64, device=DEV)
+    q = torch.zeros(1, 2, 64, dtype=torch.bfloat16, device=DEV)
+    v = torch.zeros(1, 2, 16, dtype=torch.bfloat16, device=DEV)
+    g = torch.zeros(1, 2, device=DEV)
+    out = torch.empty(1, 2, 16, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(abi.MoeError):
+        abi.moe_gdn_decode_step(shape, 1, S, q, q, v, g, g, out, flags=6)
