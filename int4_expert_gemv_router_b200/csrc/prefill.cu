@@ -347,14 +347,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
   const int K = (MODE == kModeDown) ? a.I : a.H;
   const int nK = K / kKC;
   const int NR = a.n_rows;  // weight rows per unit (the MMA's N): 128 or 256
-  const int n_units = *a.n_units;
+  pdl_launch_dependents();
   const GemmSmem P = gemm_smem<BITS, MODE>();
   const uint32_t wbytes = MODE == kModeRouter ? (uint32_t)(kTok * kKC * 2) : (uint32_t)kWBytes;  // per stage
   // stage tiles start on 1024-byte boundaries (128-byte swizzle atoms)
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (smem_base - smem_u32(smem_raw));
   const uint32_t w_area = smem_base + P.w;
-  const int my_units = n_units > (int)blockIdx.x ? (n_units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (tid == 0) {
     for (int s = 0; s < P.n_st; ++s) {
@@ -386,6 +385,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
+  // the setup above overlaps the kernel before; the work units and every input are its output
+  pdl_wait();
+  const int n_units = *a.n_units;
+  const int my_units = n_units > (int)blockIdx.x ? (n_units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (warp == 0) {
     // ------------------------------ MMA issuer ------------------------------
@@ -742,6 +745,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
 // ---------------------------------------------------------------------------------------
 __global__ void k_norms(const uint16_t* x, int T, int H, const uint16_t* wr, const uint16_t* wsg, int E,
                         double* xnorm, double* wnorm) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int rows = T + E + 1;
   if (warp >= rows) return;
@@ -790,6 +795,8 @@ __device__ __forceinline__ double warp_dot_exact(const uint16_t* a, const uint16
 constexpr int kRouteCand = 96;
 
 __global__ void __launch_bounds__(256) k_gate(PrefillArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + wl;
   if (t >= a.T) return;
@@ -798,6 +805,8 @@ __global__ void __launch_bounds__(256) k_gate(PrefillArgs a) {
 }
 
 __global__ void __launch_bounds__(256) k_route(PrefillArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ double s_cv[8][kRouteCand];
   __shared__ int s_ce[8][kRouteCand];
   __shared__ int s_cnt[8];
@@ -948,6 +957,8 @@ static_assert(kGroupChunk % kGroupThreads == 0, "chunk must split into whole war
 static_assert(kMaxExperts <= 4 * kGroupThreads, "block scan takes 4 experts per thread");
 
 __global__ void __launch_bounds__(kGroupThreads) k_ghist(PrefillArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ int hsm[];  // [E]
   const int E = a.E, n = a.T * a.k;
   for (int e = threadIdx.x; e < E; e += kGroupThreads) hsm[e] = 0;
@@ -968,6 +979,8 @@ __global__ void __launch_bounds__(kGroupThreads) k_ghist(PrefillArgs a) {
 }
 
 __global__ void __launch_bounds__(1024) k_gcol(PrefillArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int e = blockIdx.x * 32 + (threadIdx.x >> 5);
   if (e >= a.E) return;
@@ -1039,6 +1052,8 @@ __device__ void block_scan4(int E, F val, int* out, int* wsum) {
 }
 
 __global__ void __launch_bounds__(kGroupThreads) k_gplace(PrefillArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ int wc[];  // [8][E]: per-warp counts, then per-warp running slots
   __shared__ int s_off[kMaxExperts + 1];
   __shared__ int s_wsum[kGroupThreads / 32 + 1];
@@ -1122,6 +1137,8 @@ __global__ void __launch_bounds__(kGroupThreads) k_gplace(PrefillArgs a) {
 // xg[p] = x[order[p] / k] for every grouped pair position p < offsets[E]: the routed gate/up
 // GEMM then reads each expert's tokens as consecutive rows.  One warp per row.
 __global__ void __launch_bounds__(256) k_permute(PrefillArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
   // warps [0, T*k): xg row p (valid pairs only); with perm, warps [T*k, T*k + T): xp row t
   const int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int n_pairs = a.T * a.k;
@@ -1144,11 +1161,15 @@ __global__ void __launch_bounds__(256) k_permute(PrefillArgs a) {
 }
 
 __global__ void k_finalize(const float* acc, const uint16_t* residual, uint16_t* out, size_t n) {
+  pdl_launch_dependents();
+  pdl_wait();
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = f2bf(acc[i] + (residual ? bf1(residual[i]) : 0.f));
 }
 
 __global__ void k_router_units(GemmUnit* units, int* n_units, int T, int E) {
+  pdl_launch_dependents();
+  pdl_wait();
   // E rows in tiles of 128 x tokens in tiles of 128 (the shared-expert gate logit is
   // computed exactly by k_route)
   const int mt_n = (E + 127) / 128;
@@ -1161,6 +1182,24 @@ __global__ void k_router_units(GemmUnit* units, int* n_units, int T, int E) {
   if (i == 0) *n_units = mt_n * nt;
 }
 
+// Launches a kernel as a programmatic dependent of the kernel before it on the stream: it may
+// start while that kernel finishes and waits for it (pdl_wait) before reading its results.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*fn)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fn, std::forward<Args>(args)...);
+}
+
 template <int BITS, int MODE>
 cudaError_t launch_gemm(const GemmArgs& g, int n_sm, cudaStream_t s) {
   const GemmSmem P = gemm_smem<BITS, MODE>();
@@ -1168,8 +1207,7 @@ cudaError_t launch_gemm(const GemmArgs& g, int n_sm, cudaStream_t s) {
   auto fn = k_gemm<BITS, MODE>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.total);
   if (e != cudaSuccess) return e;
-  fn<<<n_sm, kGemmThreads, P.total, s>>>(g);
-  return cudaGetLastError();
+  return launch_pdl(fn, dim3(n_sm), dim3(kGemmThreads), P.total, s, g);
 }
 
 // ---- TMA descriptors (host) ----
@@ -1247,11 +1285,11 @@ bool prefill_shape_supported(int H, int I, int bits, int E) {
 
 cudaError_t launch_group(const PrefillArgs& p, cudaStream_t s) {
   const int n_chunks = (p.T * p.k + kGroupChunk - 1) / kGroupChunk;
-  k_ghist<<<n_chunks, kGroupThreads, sizeof(int) * p.E, s>>>(p);
-  k_gcol<<<(p.E + 31) / 32, 1024, 0, s>>>(p);
+  cudaError_t e = launch_pdl(k_ghist, dim3(n_chunks), dim3(kGroupThreads), sizeof(int) * p.E, s, p);
+  if (e == cudaSuccess) e = launch_pdl(k_gcol, dim3((p.E + 31) / 32), dim3(1024), 0, s, p);
   const size_t smem = sizeof(int) * (size_t)(kGroupThreads / 32) * p.E;
-  k_gplace<<<n_chunks, kGroupThreads, smem, s>>>(p);
-  return cudaGetLastError();
+  if (e == cudaSuccess) e = launch_pdl(k_gplace, dim3(n_chunks), dim3(kGroupThreads), smem, s, p);
+  return e;
 }
 
 // Norms, fp32 router logits on the tensor cores and the certified top-k of p.T tokens
@@ -1261,9 +1299,13 @@ static cudaError_t launch_route(const PrefillArgs& p, int n_sm, cudaStream_t s) 
   const int T = p.T, E = p.E, H = p.H;
   cudaError_t e;
   const int rows = T + E + 1;
-  k_norms<<<(rows * 32 + 255) / 256, 256, 0, s>>>(p.x, T, H, p.wr, p.wsg, E, p.xnorm, p.wnorm);
+  if ((e = launch_pdl(k_norms, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, p.x, T, H, p.wr, p.wsg, E,
+                      p.xnorm, p.wnorm)) != cudaSuccess)
+    return e;
   const int mt_n = (E + 127) / 128, nt = (T + 127) / 128;
-  k_router_units<<<(mt_n * nt + 255) / 256, 256, 0, s>>>(p.units_rt, p.n_units + 2, T, E);
+  if ((e = launch_pdl(k_router_units, dim3((mt_n * nt + 255) / 256), dim3(256), 0, s, p.units_rt, p.n_units + 2, T,
+                      E)) != cudaSuccess)
+    return e;
   GemmArgs g = p.g;
   g.units = p.units_rt;
   g.n_units = p.n_units + 2;
@@ -1273,8 +1315,7 @@ static cudaError_t launch_route(const PrefillArgs& p, int n_sm, cudaStream_t s) 
   if ((e = map_bf16(&g.map_tok, p.x, T, H, H, kTRows)) != cudaSuccess) return e;
   // the router GEMM reads bf16 rows only; the code width does not enter it
   if ((e = launch_gemm<4, kModeRouter>(g, n_sm, s)) != cudaSuccess) return e;
-  k_route<<<(T + 7) / 8, 256, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(k_route, dim3((T + 7) / 8), dim3(256), 0, s, p);
 }
 
 static int sm_count() {
@@ -1297,14 +1338,15 @@ cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
   if (p.route) {
     if ((e = launch_route(p, n_sm, s)) != cudaSuccess) return e;
   } else {
-    k_gate<<<(T + 7) / 8, 256, 0, s>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(k_gate, dim3((T + 7) / 8), dim3(256), 0, s, p)) != cudaSuccess) return e;
   }
   prof_mark(0, true, s);
   // grouping and work units
   prof_mark(1, false, s);
   if ((e = launch_group(p, s)) != cudaSuccess) return e;
-  k_permute<<<(unsigned)((((size_t)T * p.k + (p.perm ? T : 0)) * 32 + 255) / 256), 256, 0, s>>>(p);
+  if ((e = launch_pdl(k_permute, dim3((unsigned)((((size_t)T * p.k + (p.perm ? T : 0)) * 32 + 255) / 256)), dim3(256),
+                      0, s, p)) != cudaSuccess)
+    return e;
   prof_mark(1, true, s);
   // gate/up + SwiGLU, then down + scatter
   {
@@ -1349,9 +1391,11 @@ cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
   }
   const size_t n = (size_t)T * H;
   prof_mark(4, false, s);
-  k_finalize<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p.acc, p.residual, p.out, n);
+  if ((e = launch_pdl(k_finalize, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, p.acc, p.residual, p.out, n)) !=
+      cudaSuccess)
+    return e;
   prof_mark(4, true, s);
-  return cudaGetLastError();
+  return cudaSuccess;
 }
 
 }  // namespace moe

@@ -81,6 +81,12 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* b) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(b)) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Programmatic dependent launch: the kernel after this one on the stream may start launching
+// now (it waits for this one's completion where it must) ...
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// ... and this kernel waits, before its first read of what earlier work wrote, until the kernel
+// before it has finished and its writes are visible (at once when not launched as a dependent).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // Per-thread L2 prefetch of the 128-byte line holding p (a hint: no register result, no
 // completion; unlike cp.async.bulk.prefetch it does not occupy the SM's bulk-copy engine).
 __device__ __forceinline__ void prefetch_line_l2(const void* p) {
