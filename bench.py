@@ -50,7 +50,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC_PER_LAYER = {("k_fused_decode", "decode80b", 1): 21_760_000}
 # DRAM traffic per launch of the prefill gate/up GEMM on the prefill workload (full-size,
 # one-pass capture).  Dropped whenever the kernel changes.
-NCU_TRAFFIC_PREFILL_GATEUP = {("prefill", 4096): 830_150_912}
+NCU_TRAFFIC_PREFILL_GATEUP = {("prefill", 4096): 829_744_640}
 
 
 # --------------------------------------------------------------------------------------
@@ -334,11 +334,12 @@ def run_decode(args, w, T, device, rank, ws_n):
     return res
 
 
-def run_decode_ep(args, w, T, device, rank, world):
-    """Expert-parallel decode stack: rank r holds the experts e % world == r of every layer
-    (its pool shard), router and shared expert replicated; per layer the partial kernel, one
-    NCCL sum all-reduce of the [T, H] fp32 partials, and the combine kernel.  All ranks work
-    on the same token stream, so the job's tokens per step are T (strong scaling)."""
+def run_ep(args, w, T, device, rank, world):
+    """Expert-parallel layer stack: rank r holds the experts e % world == r of every layer
+    (its pool shard), router and shared expert replicated; per layer the partial forward (the
+    fused decode kernel for T <= 8, the prefill path above that), one NCCL sum all-reduce of
+    the [T, H] fp32 partials, and the combine kernel.  All ranks work on the same tokens, so
+    the job's tokens per step are T (strong scaling)."""
     from int4_expert_gemv_router_b200 import abi, build, ep
     build.build()
     K, W = args.steps, args.warmup
@@ -399,17 +400,20 @@ def run_decode_ep(args, w, T, device, rank, world):
     e2e_ms = reduce_max(f0.elapsed_time(f1), device)
     value = T * K / (ms / 1e3)
     return {
-        "metric": "routed-MoE layer tokens/s; achieved HBM GB/s (decode)",
+        "metric": ("routed-MoE layer tokens/s; tensor % (prefill)" if w.name == "prefill"
+                   else "routed-MoE layer tokens/s; achieved HBM GB/s (decode)"),
         "value": round(value, 2), "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(ms / K, 4), "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
         "dtype": f"int{w.bits} weights, bf16 activations, fp32 accumulate",
         "data": "synthetic (seeded; weights ~N(0,0.02) quantised, x ~N(0,1))",
         "config": dict(workload_config(args, w, T, world), parallelism=f"ep{world}"),
-        "launch": "per layer: partial kernel, NCCL all-reduce of the fp32 partial, combine kernel",
+        "launch": ("per call: the prefill path over this rank's experts (fp32 partial), NCCL all-reduce, "
+                   "combine kernel" if w.name == "prefill" else
+                   "per layer: partial kernel, NCCL all-reduce of the fp32 partial, combine kernel"),
         "clocks": clocks,
         "e2e": {"value": round(T * K / (e2e_ms / 1e3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * w.hidden * 2, "d2h_bytes_per_step": T * w.hidden * 2},
-        "gpu_launches": 2 * nL * K,
+        "gpu_launches": (12 if w.name == "prefill" else 2) * nL * K,
         "device_error_flags": flags,
     }
 
@@ -1107,8 +1111,9 @@ def parse(argv=None):
     ap.add_argument("--overlap", action="store_true",
                     help="pool workloads: the forward starts while the step's misses are still being copied")
     ap.add_argument("--parallel", choices=["replicas", "ep"], default="replicas",
-                    help="decode workloads with --gpus N: N independent replicas (default, weak scaling) or "
-                         "expert parallelism (each rank holds 1/N of every layer's experts, strong scaling)")
+                    help="decode and prefill workloads with --gpus N: N independent replicas (default, weak "
+                         "scaling) or expert parallelism (each rank holds 1/N of every layer's experts, strong "
+                         "scaling)")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the stack depth (profiling of a small case only; not a bench value)")
     return ap.parse_args(argv)
@@ -1163,7 +1168,9 @@ def main(argv=None):
     peaks, peak_kind = load_peaks()
     cpu_base = None
     want_cpu = rank == 0 and ws == 1 and not args.no_cpu_baseline
-    if w.name == "prefill":
+    if args.parallel == "ep" and not w.name.startswith("pool"):
+        line = run_ep(args, w, T, device, rank, ws)
+    elif w.name == "prefill":
         r = run_prefill(args, w, T, device, rank)
         if want_cpu:
             cpu_base = cpu_baseline_prefill(w, T, r)
@@ -1173,8 +1180,6 @@ def main(argv=None):
         if want_cpu:
             cpu_base = cpu_baseline_pool(w, r)
         line = pool_line(args, w, r, ws, cpu_base)
-    elif args.parallel == "ep":
-        line = run_decode_ep(args, w, T, device, rank, ws)
     else:
         r = run_decode(args, w, T, device, rank, ws)
         if want_cpu:

@@ -207,8 +207,10 @@ MOE_API moe_status moe_stack_forward(const moe_shape* shape, int32_t T, const mo
  *                  p * y_e (+ sigmoid gate * y_shared if include_shared), no residual, not rounded
  * Every rank routes the same tokens and gets the same top-k (topk_idx_out), so the ranks'
  * partials add up to the layer; sum them (e.g. an NCCL all-reduce) and finish with
- * moe_combine_partials.  T: 1..8 on shapes with a fused decode kernel, else
- * MOE_ERR_UNSUPPORTED.
+ * moe_combine_partials.  T <= 8: the fused decode kernel (shapes as moe_stack_forward);
+ * T > 8: the prefill path, grouping only this rank's pairs and summing their down products
+ * (and the shared expert's) into partial_out in fp32 (shapes as the prefill path:
+ * hidden % 128 == 0, E <= 512).  Other shapes: MOE_ERR_UNSUPPORTED.
  */
 MOE_API moe_status moe_layer_forward_partial(const moe_shape* shape, const void* x, int32_t T,
                                              const void* w_router, const float* router_bias,

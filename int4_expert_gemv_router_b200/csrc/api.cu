@@ -274,7 +274,7 @@ static moe_status prefill_forward(const moe_shape* shape, const void* x, int32_t
                                   const uint8_t* pool, const int32_t* slot_table, int64_t n_slots,
                                   const uint8_t* shared_blob, const void* w_shared_gate, const void* residual,
                                   void* out, int32_t* topk_idx_out, float* topk_w_out, void* ws, size_t ws_bytes,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, float* partial_out = nullptr, int include_shared = 1) {
   if (!prefill_shape_supported(shape->hidden, shape->inter, shape->bits, shape->n_experts))
     return set_error(MOE_ERR_UNSUPPORTED,
                      "no prefill kernel for hidden=%d inter=%d bits=%d E=%d (hidden %% 128 == 0, E <= 512)",
@@ -295,7 +295,11 @@ static moe_status prefill_forward(const moe_shape* shape, const void* x, int32_t
   p.wsg = static_cast<const uint16_t*>(w_shared_gate);
   p.rbias = router_bias;
   p.residual = static_cast<const uint16_t*>(residual);
-  p.out = static_cast<uint16_t*>(out);
+  // a partial forward (expert parallelism): the down products of this rank's experts (and the
+  // shared expert's if included) are summed in fp32 straight into partial_out; no residual,
+  // no rounding, no finalize
+  p.out = partial_out ? nullptr : static_cast<uint16_t*>(out);
+  p.no_shared = include_shared ? 0 : 1;
   p.route = (topk_idx_in == nullptr);
   p.ctrl = reinterpret_cast<Ctrl*>(b + W.ctrl);
   p.xnorm = reinterpret_cast<double*>(b + W.xnorm);
@@ -320,7 +324,7 @@ static moe_status prefill_forward(const moe_shape* shape, const void* x, int32_t
   p.units_gu = reinterpret_cast<GemmUnit*>(b + W.units_gu);
   p.units_dn = reinterpret_cast<GemmUnit*>(b + W.units_dn);
   p.n_units = reinterpret_cast<int*>(b + W.n_units);
-  p.acc = reinterpret_cast<float*>(b + W.acc);
+  p.acc = partial_out ? partial_out : reinterpret_cast<float*>(b + W.acc);
   p.h = reinterpret_cast<uint16_t*>(b + W.h);
   p.hs = reinterpret_cast<uint16_t*>(b + W.hs);
   p.xg = reinterpret_cast<uint16_t*>(b + W.xg);
@@ -453,13 +457,33 @@ moe_status moe_layer_forward_partial(const moe_shape* shape, const void* x, int3
   if (st != MOE_OK) return st;
   if (shape->shared_inter != shape->inter)
     return set_error(MOE_ERR_UNSUPPORTED, "this build needs shared_inter == inter");
-  if (T < 1 || T > kMaxDecodeT)
-    return set_error(MOE_ERR_UNSUPPORTED, "the partial forward takes 1..%d tokens (got %d)", kMaxDecodeT, T);
-  if (!fused_shape_supported(shape->hidden, shape->inter, shape->bits, shape->n_experts))
+  if (T < 1) return set_error(MOE_ERR_INVALID, "T must be >= 1 (got %d)", T);
+  if (T <= kMaxDecodeT && !fused_shape_supported(shape->hidden, shape->inter, shape->bits, shape->n_experts))
     return set_error(MOE_ERR_UNSUPPORTED, "no fused decode kernel for hidden=%d inter=%d bits=%d E=%d",
                      shape->hidden, shape->inter, shape->bits, shape->n_experts);
   if (!partial_out || !aligned(partial_out, 16)) return set_error(MOE_ERR_INVALID, "partial_out must be non-NULL and 16-byte aligned");
   if (include_shared != 0 && include_shared != 1) return set_error(MOE_ERR_INVALID, "include_shared must be 0 or 1");
+  if (T > kMaxDecodeT) {
+    // many tokens: the prefill path over this rank's experts, summed into partial_out
+    moe_layer_desc d{};
+    d.x = x;
+    d.w_router = w_router;
+    d.router_bias = router_bias;
+    d.topk_idx_in = topk_idx_in;
+    d.topk_w_in = topk_w_in;
+    d.pool = pool;
+    d.slot_table = slot_table;
+    d.n_slots = n_slots;
+    d.shared_blob = shared_blob;
+    d.w_shared_gate = w_shared_gate;
+    d.out = partial_out;
+    d.topk_idx_out = topk_idx_out;
+    d.topk_w_out = topk_w_out;
+    if ((st = check_layer(shape, &d, true)) != MOE_OK) return st;
+    return prefill_forward(shape, x, T, w_router, router_bias, topk_idx_in, topk_w_in, pool, slot_table, n_slots,
+                           shared_blob, w_shared_gate, nullptr, nullptr, topk_idx_out, topk_w_out, ws, ws_bytes,
+                           static_cast<cudaStream_t>(stream), partial_out, include_shared);
+  }
   moe_layer_desc d{};
   d.x = x;
   d.w_router = w_router;

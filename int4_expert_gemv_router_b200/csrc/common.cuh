@@ -284,6 +284,7 @@ struct PrefillArgs {
   uint16_t* xg;         // bf16 [T*k, H]: x rows in grouped pair order
   uint16_t* xp;         // bf16 [T, H]: x for the shared expert's gate/up (k-octet order, int4)
   int perm;             // int4: operands of the expert GEMMs in k-octet order (see prefill.cu)
+  int no_shared;        // 1: the shared expert's work units are left out (a partial forward)
   Ctrl* ctrl;
   GemmArgs g;           // shared GEMM arguments (units filled per launch)
 };

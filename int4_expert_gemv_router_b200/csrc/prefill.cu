@@ -956,6 +956,12 @@ constexpr int kGroupThreads = 256;  // 8 warps; each takes kGroupChunk / 8 conse
 static_assert(kGroupChunk % kGroupThreads == 0, "chunk must split into whole warp rounds");
 static_assert(kMaxExperts <= 4 * kGroupThreads, "block scan takes 4 experts per thread");
 
+// An expert whose slot-table entry marks it as held by another rank (expert parallelism):
+// its pairs are left out of the grouping here, without an error; that rank computes them.
+__device__ __forceinline__ bool remote_expert(const PrefillArgs& a, int e) {
+  return a.g.slot_table && __ldg(a.g.slot_table + e) == kSlotRemote;
+}
+
 __global__ void __launch_bounds__(kGroupThreads) k_ghist(PrefillArgs a) {
   pdl_launch_dependents();
   pdl_wait();
@@ -970,7 +976,7 @@ __global__ void __launch_bounds__(kGroupThreads) k_ghist(PrefillArgs a) {
     if (p < n) {
       const int e = __ldg(a.topk_idx + p);
       if (e < 0 || e >= E) atomicOr(&a.ctrl->err, kErrBadExpert);
-      else atomicAdd(&hsm[e], 1);
+      else if (!remote_expert(a, e)) atomicAdd(&hsm[e], 1);
     }
   }
   __syncthreads();
@@ -1069,7 +1075,7 @@ __global__ void __launch_bounds__(kGroupThreads) k_gplace(PrefillArgs a) {
   for (int r = 0; r < kRounds; ++r) {
     const int p = pw + r * 32 + lane;
     const int e = p < n ? __ldg(a.topk_idx + p) : -1;
-    ev[r] = (e >= 0 && e < E) ? e : -1;
+    ev[r] = (e >= 0 && e < E && !remote_expert(a, e)) ? e : -1;
   }
 #pragma unroll
   for (int r = 0; r < kRounds; ++r) {
@@ -1119,7 +1125,7 @@ __global__ void __launch_bounds__(kGroupThreads) k_gplace(PrefillArgs a) {
   }
   if (blockIdx.x != 0) return;
   const int tiles_r = tile_base[E];
-  const int st_n = (a.T + kTok - 1) / kTok;
+  const int st_n = a.no_shared ? 0 : (a.T + kTok - 1) / kTok;  // the shared expert's token tiles
   for (int i = threadIdx.x; i < st_n * mt_gu; i += kGroupThreads) {
     const int st = i / mt_gu, mt = i - st * mt_gu, t0 = st * kTok;
     a.units_gu[(tiles_r + st) * mt_gu + mt] = GemmUnit{-1, mt, t0, min(kTok, a.T - t0)};
@@ -1391,8 +1397,9 @@ cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
   }
   const size_t n = (size_t)T * H;
   prof_mark(4, false, s);
-  if ((e = launch_pdl(k_finalize, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, p.acc, p.residual, p.out, n)) !=
-      cudaSuccess)
+  // a partial forward leaves its fp32 sum in acc (the caller's buffer): no finalize
+  if (p.out && (e = launch_pdl(k_finalize, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, p.acc, p.residual,
+                               p.out, n)) != cudaSuccess)
     return e;
   prof_mark(4, true, s);
   return cudaSuccess;

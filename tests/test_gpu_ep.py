@@ -9,8 +9,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
-from helpers import assert_close, assert_routing, forward, oracle_forward, ws_for
+from helpers import assert_close, assert_routing, forward, host_bits, oracle_forward, ws_for
 from int4_expert_gemv_router_b200 import abi, build, ep
 
 pytestmark = pytest.mark.gpu
@@ -89,9 +90,44 @@ def test_combine_partials_order_and_tail():
 
 
 def test_partial_rejects_unsupported():
-    w = synth.WORKLOADS["tiny"]
+    """A shape neither path takes (hidden 192: no fused decode instantiation, and the
+    prefill GEMMs need hidden % 128 == 0), with one token and with many."""
+    w = synth.WORKLOADS["tiny"].with_(hidden=192)
     shape = abi.shape_of(w)
-    t = torch.zeros(64, dtype=torch.uint8, device=DEV)
-    with pytest.raises(abi.MoeError) as ei:
-        abi.moe_layer_forward_partial(shape, t, 9, t, None, None, None, t, t, 1, t, t, 1, t, None, None, t)
-    assert ei.value.status == -5
+    t = torch.zeros(1 << 16, dtype=torch.uint8, device=DEV)
+    for T in (1, 9):
+        with pytest.raises(abi.MoeError) as ei:
+            abi.moe_layer_forward_partial(shape, t, T, t, None, None, None, t, t, 1, t, t, 1, t, None, None, t)
+        assert ei.value.status == -5
+
+
+@pytest.mark.parametrize("wname,world,T", [("tiny", 2, 40), ("decode80b", 2, 64), ("decode80b", 4, 300)])
+def test_prefill_ranks_sum_to_the_layer(wname, world, T):
+    """More than 8 tokens take the prefill path: each rank groups only the pairs of its own
+    experts (the others' slot entries are -3) and runs the grouped GEMMs over them, the
+    shared expert on rank 0; the fp32 partials summed by the combine give the layer."""
+    w = synth.WORKLOADS[wname].with_(layers=1)
+    L = synth.make_layer(w, 0, DEV)
+    x = synth.activations(w, 63, tokens=T, device=DEV)
+    parts, ids = [], []
+    for r in range(world):
+        part, idx, p = _rank_partial(w, L, x, r, world)
+        assert torch.isfinite(part).all()
+        parts.append(part)
+        ids.append((idx, p))
+    for idx, p in ids[1:]:
+        assert torch.equal(idx, ids[0][0]) and torch.equal(p, ids[0][1])
+    out = torch.empty(T, w.hidden, dtype=torch.bfloat16, device=DEV)
+    abi.moe_combine_partials(parts, T, w.hidden, x, out)
+    torch.cuda.synchronize()
+    # the oracle with each selected expert decoded once for all its tokens
+    xb, wrb = host_bits(x), host_bits(L.w_router)
+    bias = None if L.router_bias is None else L.router_bias.cpu().numpy()
+    logits = oracle.router_logits(xb, wrb, bias)
+    ref_idx, ref_p = oracle.route(logits, w.top_k)
+    assert_routing(ids[0][0], ref_idx, logits)
+    pool = L.pool.cpu().numpy()
+    ref = oracle.layer_forward_by_expert(xb, wrb, bias, w.top_k, lambda e: pool[e], L.shared.cpu().numpy(),
+                                         host_bits(L.w_sg), w.hidden, w.inter, w.shared_inter, w.bits,
+                                         residual_bits=xb, idx=ref_idx, p=ref_p)
+    assert_close(out, ref["out"])
