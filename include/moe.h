@@ -36,7 +36,7 @@
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and
  *     is asynchronous, except where a call says it synchronises.
  *   - Arguments are validated before anything is enqueued; a bad argument returns
- *     MOE_ERR_INVALID (or MOE_ERR_UNSUPPORTED for a valid shape this build has no
+ *     MOE_ERR_INVALID (or MOE_ERR_UNSUPPORTED for a valid shape this library has no
  *     kernel for) and enqueues nothing.  Nothing aborts or throws across this ABI.
  *     moe_last_error() gives a message for the calling thread's last failure.
  *   - Errors detected on the device (an expert id outside [0, E), a slot outside
@@ -68,7 +68,7 @@ typedef enum {
   MOE_ERR_CUDA = -2,         /* a CUDA runtime call failed; see moe_last_error() */
   MOE_ERR_CAPACITY = -3,     /* a pool step needs more distinct experts than slots */
   MOE_ERR_NOT_RESIDENT = -4, /* reserved: an expert the call needs has no slot */
-  MOE_ERR_UNSUPPORTED = -5,  /* valid request with no kernel in this build */
+  MOE_ERR_UNSUPPORTED = -5,  /* valid request with no kernel in this library */
   MOE_ERR_TIMEOUT = -6,      /* a bounded device-side wait gave up */
   MOE_ERR_DEVICE = -7,       /* the device set an error bit (moe_ws_check) */
   MOE_ERR_IO = -8            /* the pool's backing file could not be opened or read */
@@ -83,7 +83,7 @@ typedef enum {
 typedef struct {
   int32_t hidden;       /* H: model width (multiple of 64)                                 */
   int32_t inter;        /* I: routed-expert intermediate width (multiple of 64)            */
-  int32_t shared_inter; /* I_s: shared-expert intermediate width (this build: I_s == I)    */
+  int32_t shared_inter; /* I_s: shared-expert intermediate width (this library: I_s == I)  */
   int32_t n_experts;    /* E: routed experts per layer (1..1024)                           */
   int32_t top_k;        /* k: experts per token (1..min(E, 32))                            */
   int32_t bits;         /* 4 or 8                                                          */

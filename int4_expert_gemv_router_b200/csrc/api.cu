@@ -365,7 +365,7 @@ moe_status moe_layer_forward(const moe_shape* shape, const void* x, int32_t T, c
   moe_status st = check_shape(shape);
   if (st != MOE_OK) return st;
   if (shape->shared_inter != shape->inter)
-    return set_error(MOE_ERR_UNSUPPORTED, "this build needs shared_inter == inter (%d vs %d)", shape->shared_inter,
+    return set_error(MOE_ERR_UNSUPPORTED, "this library needs shared_inter == inter (%d vs %d)", shape->shared_inter,
                      shape->inter);
   if (!decode_shape_supported(shape->hidden, shape->inter, shape->bits))
     return set_error(MOE_ERR_UNSUPPORTED,
@@ -456,7 +456,7 @@ moe_status moe_layer_forward_partial(const moe_shape* shape, const void* x, int3
   moe_status st = check_shape(shape);
   if (st != MOE_OK) return st;
   if (shape->shared_inter != shape->inter)
-    return set_error(MOE_ERR_UNSUPPORTED, "this build needs shared_inter == inter");
+    return set_error(MOE_ERR_UNSUPPORTED, "this library needs shared_inter == inter");
   if (T < 1) return set_error(MOE_ERR_INVALID, "T must be >= 1 (got %d)", T);
   if (T <= kMaxDecodeT && !fused_shape_supported(shape->hidden, shape->inter, shape->bits, shape->n_experts))
     return set_error(MOE_ERR_UNSUPPORTED, "no fused decode kernel for hidden=%d inter=%d bits=%d E=%d",
@@ -535,7 +535,7 @@ moe_status moe_stack_forward(const moe_shape* shape, int32_t T, const moe_layer_
   if (n_layers < 1 || n_layers > kMaxFusedLayers)
     return set_error(MOE_ERR_INVALID, "n_layers must be in [1, %d] (got %d)", kMaxFusedLayers, n_layers);
   if (shape->shared_inter != shape->inter)
-    return set_error(MOE_ERR_UNSUPPORTED, "this build needs shared_inter == inter");
+    return set_error(MOE_ERR_UNSUPPORTED, "this library needs shared_inter == inter");
   if (!decode_shape_supported(shape->hidden, shape->inter, shape->bits))
     return set_error(MOE_ERR_UNSUPPORTED, "no decode kernel for hidden=%d inter=%d bits=%d", shape->hidden,
                      shape->inter, shape->bits);
