@@ -561,6 +561,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     const int sec = MODE == kModeGateUp && m >= NR / 2 ? 2 : 0;
     const int crow = MODE == kModeGateUp ? m % (NR / 2) : m;
     const uint32_t c_s = (uint32_t)((sec * sec_rows + crow) * kChunk), c_b = c_s + (uint32_t)(sec_rows * kChunk);
+    // Raw-code reads go chunk by chunk (16 bytes) in an order rotated per lane, so that the
+    // eight lanes of each quarter-warp read eight different bank groups (rows are 32 or 64
+    // bytes apart: in plain order two or four of them would hit the same banks).
+    constexpr int kRawChunks = kRowB / 16;
+    const int rot = BITS == 4 ? (m >> 2) & 1 : (m >> 1) & 3;
+    uint4 sv4 = make_uint4(0, 0, 0, 0), bv4 = make_uint4(0, 0, 0, 0);  // this row's chunk scales
     Ring ra(P.n_st), rr(P.n_raw);
     int g = 0;  // stage of the CTA's stream
     for (int j = 0; j < my_units && !warp_aborted(&s_abort); ++j) {
@@ -592,55 +598,86 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
           stop = true;
           break;
         }
-        uint32_t w[kRowB / 4];  // this thread's 64 codes
+        uint32_t w[kRowB / 4];  // this thread's 64 codes, raw chunk (o + rot) % kRawChunks at w[4o..]
         uint32_t sbits = 0, bbits = 0;
         if (active) {
           const uint8_t* rp = smem + P.raw + rr.s * kRawB + raw_off;
 #pragma unroll
-          for (int o = 0; o < kRowB / 16; ++o) {
-            const uint4 v = *reinterpret_cast<const uint4*>(rp + o * 16);
+          for (int o = 0; o < kRawChunks; ++o) {
+            const uint4 v = *reinterpret_cast<const uint4*>(rp + ((o + rot) & (kRawChunks - 1)) * 16);
             w[4 * o + 0] = v.x;
             w[4 * o + 1] = v.y;
             w[4 * o + 2] = v.z;
             w[4 * o + 3] = v.w;
           }
           if (a.sc_tma) {
-            // chunk g / 8 sits in slot (g / 8) & 1, on that slot's ((g / 8) >> 1)-th fill
-            if (!mbar_wait_backoff(&chunk_full[(g / kChunk) & 1], ((g / kChunk) >> 1) & 1)) {
-              atomicOr(&a.ctrl->err, kErrTimeout);
-              s_abort = 1;
+            // The rows of a chunk hold 8 groups (16 bytes): the group takes all 8 scales and
+            // biases of its row at its first stage of the chunk (kc % 8 == grp; nK is a
+            // multiple of 8 here, so kc and g have the same parity) and keeps them in
+            // registers.  Chunk g / 8 sits in slot (g / 8) & 1, on that slot's
+            // ((g / 8) >> 1)-th fill; the loader refills the slot (with chunk g / 8 + 2) only
+            // after the release of raw stage 8 (g / 8 + 2) - n_raw > g, which comes after the
+            // conversion of that stage and therefore after this read.
+            if ((kc % kChunk) == grp) {
+              if (!mbar_wait_backoff(&chunk_full[(g / kChunk) & 1], ((g / kChunk) >> 1) & 1)) {
+                atomicOr(&a.ctrl->err, kErrTimeout);
+                s_abort = 1;
+              }
+              const uint16_t* ch = reinterpret_cast<const uint16_t*>(smem + P.sc + ((g / kChunk) & 1) * kChunkBytes);
+              sv4 = *reinterpret_cast<const uint4*>(ch + c_s);
+              bv4 = *reinterpret_cast<const uint4*>(ch + c_b);
             }
-            const uint16_t* ch = reinterpret_cast<const uint16_t*>(smem + P.sc + ((g / kChunk) & 1) * kChunkBytes);
-            sbits = ch[c_s + kc % kChunk];
-            bbits = ch[c_b + kc % kChunk];
+            // group kc % 8 sits in word (kc % 8) / 2, half kc % 2 (= grp)
+            const int q = (kc % kChunk) >> 1;
+            const uint32_t sw = q == 0 ? sv4.x : q == 1 ? sv4.y : q == 2 ? sv4.z : sv4.w;
+            const uint32_t bw = q == 0 ? bv4.x : q == 1 ? bv4.y : q == 2 ? bv4.z : bv4.w;
+            sbits = (sw >> (16 * grp)) & 0xFFFFu;
+            bbits = (bw >> (16 * grp)) & 0xFFFFu;
           } else if (gs) {
             sbits = __ldg(gs + kc);
             bbits = __ldg(gb + kc);
           }
         }
-        __syncwarp();  // every lane holds its codes and scales: the raw slot can be refilled
-        if (lane == 0) mbar_arrive(&raw_empty[rr.s]);
         if (!warp_wait(&empty[ra.s], ra.ph ^ 1, a.ctrl, lane)) {
           stop = true;
           break;
         }
         if (active) {
-          uint8_t* w_tile = smem + P.w + ra.s * kWBytes;
+          // raw chunk c holds k-octets 4c .. 4c+3 (int4: one word each) or 2c, 2c+1 (int8: two
+          // words each); k-octet j goes to core_off(m, j) = core_off(m, 0) + 128 j
+          uint8_t* row_tile = smem + P.w + ra.s * kWBytes + core_off(m, 0);
           if (BITS == 4) {
             const uint32_t s2 = sbits | (sbits << 16), b2 = bbits | (bbits << 16);
 #pragma unroll
-            for (int o = 0; o < 8; ++o)  // 8 k-octets of 8 values = the stage's 64 columns
-              *reinterpret_cast<uint4*>(w_tile + core_off(m, o)) = dq8_int4_bf(w[o], s2, b2);
+            for (int o = 0; o < kRawChunks; ++o) {
+              uint8_t* dst = row_tile + ((o + rot) & (kRawChunks - 1)) * 512;
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<uint4*>(dst + i * 128) = dq8_int4_bf(w[4 * o + i], s2, b2);
+            }
           } else {
             const float sv = __uint_as_float(sbits << 16), bv = __uint_as_float(bbits << 16);
 #pragma unroll
-            for (int o = 0; o < 8; ++o)
-              *reinterpret_cast<uint4*>(w_tile + core_off(m, o)) = dq8_int8(w[2 * o], w[2 * o + 1], sv, bv);
+            for (int o = 0; o < kRawChunks; ++o) {
+              uint8_t* dst = row_tile + ((o + rot) & (kRawChunks - 1)) * 256;
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+                *reinterpret_cast<uint4*>(dst + j * 128) = dq8_int8(w[4 * o + 2 * j], w[4 * o + 2 * j + 1], sv, bv);
+            }
           }
         }
         proxy_fence();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&full[ra.s]);
+        // The raw slot is released only here, once its codes have been used in the
+        // conversion: with the release placed right after the loads into registers, the down
+        // GEMM gave wrong outputs on the full prefill workload (the loader's next copy into
+        // the slot reached codes that were still to be converted).  The scale chunk's slot is
+        // refilled only after a later raw stage's release, so every read of a chunk also
+        // precedes its refill by a whole conversion.
+        if (lane == 0) {
+          mbar_arrive(&full[ra.s]);
+          mbar_arrive(&raw_empty[rr.s]);
+        }
       }
       if (stop) {
         s_abort = 1;
