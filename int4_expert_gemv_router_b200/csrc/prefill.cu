@@ -115,6 +115,11 @@ __host__ __device__ inline GemmSmem gemm_smem() {
     p.n_st = 3;
     const int nr = (int)((rest - 3u * ((uint32_t)kTBytes + wb)) / (uint32_t)Raw<BITS>::kBytes);
     p.n_raw = nr > kRawMax ? kRawMax : nr;
+    // A group waiting for raw stage s has converted s - 2 (the MMA has consumed s - 5), so the
+    // slot's previous fill s - n_raw is known to have landed, and the parity wait cannot
+    // mistake it for the fill it waits for, when n_raw >= 5 or n_raw is even (then s - n_raw
+    // is one of the group's own earlier stages).  int8 leaves room for 3: use 2.
+    if (p.n_raw < 5 && (p.n_raw & 1)) --p.n_raw;
   }
   p.w = (uint32_t)p.n_st * kTBytes;
   p.raw = p.w + (uint32_t)p.n_st * wb;
@@ -417,8 +422,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             s_abort = 1;
             break;
           }
-          // dequantised tiles were written through the generic proxy (st.shared)
-          if (MODE != kModeRouter) proxy_fence();
+          // the dequantised tiles were written through the generic proxy (st.shared); each
+          // writing thread fenced them to the async proxy before its arrival
           tc_fence_after();
           const uint64_t da = da0 + (uint64_t)(r.s * (kTBytes >> 4));
           const uint64_t db = db0 + (uint64_t)(r.s * (wbytes >> 4));
