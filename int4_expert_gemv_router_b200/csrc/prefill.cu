@@ -21,7 +21,7 @@
 //                  memory) x the expert's rows of xg, SwiGLU in the epilogue -> h
 //   k_gemm DOWN    per unit: down rows x the expert's h, weighted scatter-add into an fp32
 //                  accumulator (the shared expert is one more "expert" over all tokens)
-//   k_finalize     out = bf16(acc + residual)
+//   k_finalize     out = bf16(acc + residual) (8 elements per thread for aligned buffers)
 //
 // GEMM kernel (the unit's tokens are the MMA's M = 128 TMEM lanes, its weight rows the N <= 256
 // columns; one kind::f16 MMA per 16-deep k-step):
@@ -1214,6 +1214,23 @@ __global__ void k_finalize(const float* acc, const uint16_t* residual, uint16_t*
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = f2bf(acc[i] + (residual ? bf1(residual[i]) : 0.f));
 }
+// The same, 8 elements per thread (two 16-byte loads of acc, one of the residual, one 16-byte
+// store), grid-stride; for 16-byte aligned buffers.  acc is read for the last time: streaming
+// loads.
+__global__ void __launch_bounds__(256) k_finalize8(const float4* acc, const uint4* residual, uint4* out, size_t n8) {
+  pdl_launch_dependents();
+  pdl_wait();
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
+    const float4 a0 = __ldcs(acc + 2 * i), a1 = __ldcs(acc + 2 * i + 1);
+    const uint4 r = residual ? __ldcs(residual + i) : make_uint4(0, 0, 0, 0);
+    uint4 o;
+    o.x = (uint32_t)f2bf(a0.x + bf_lo(r.x)) | ((uint32_t)f2bf(a0.y + bf_hi(r.x)) << 16);
+    o.y = (uint32_t)f2bf(a0.z + bf_lo(r.y)) | ((uint32_t)f2bf(a0.w + bf_hi(r.y)) << 16);
+    o.z = (uint32_t)f2bf(a1.x + bf_lo(r.z)) | ((uint32_t)f2bf(a1.y + bf_hi(r.z)) << 16);
+    o.w = (uint32_t)f2bf(a1.z + bf_lo(r.w)) | ((uint32_t)f2bf(a1.w + bf_hi(r.w)) << 16);
+    out[i] = o;
+  }
+}
 
 __global__ void k_router_units(GemmUnit* units, int* n_units, int T, int E) {
   pdl_launch_dependents();
@@ -1440,9 +1457,19 @@ cudaError_t launch_prefill(const PrefillArgs& p, int bits, cudaStream_t s) {
   const size_t n = (size_t)T * H;
   prof_mark(4, false, s);
   // a partial forward leaves its fp32 sum in acc (the caller's buffer): no finalize
-  if (p.out && (e = launch_pdl(k_finalize, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, p.acc, p.residual,
-                               p.out, n)) != cudaSuccess)
-    return e;
+  if (p.out) {
+    const bool vec = n % 8 == 0 && (reinterpret_cast<uintptr_t>(p.acc) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(p.residual) & 15) == 0 && (reinterpret_cast<uintptr_t>(p.out) & 15) == 0;
+    if (vec) {
+      const size_t n8 = n / 8;
+      const unsigned blocks = (unsigned)std::min<size_t>((n8 + 255) / 256, (size_t)n_sm * 8);
+      e = launch_pdl(k_finalize8, dim3(blocks), dim3(256), 0, s, reinterpret_cast<const float4*>(p.acc),
+                     reinterpret_cast<const uint4*>(p.residual), reinterpret_cast<uint4*>(p.out), n8);
+    } else {
+      e = launch_pdl(k_finalize, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, p.acc, p.residual, p.out, n);
+    }
+    if (e != cudaSuccess) return e;
+  }
   prof_mark(4, true, s);
   return cudaSuccess;
 }
