@@ -849,8 +849,10 @@ __global__ void __launch_bounds__(256) k_gate(PrefillArgs a) {
 __global__ void __launch_bounds__(256) k_route(PrefillArgs a) {
   pdl_launch_dependents();
   pdl_wait();
-  __shared__ double s_cv[8][kRouteCand];
+  __shared__ double s_cl[8][kRouteCand];  // candidates' fp32 logits (with bias): the order key
+  __shared__ double s_cu[8][kRouteCand];  // and their certified upper bounds
   __shared__ int s_ce[8][kRouteCand];
+  __shared__ int s_ord[8][kRouteCand];
   __shared__ int s_cnt[8];
   const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + wl;
@@ -901,51 +903,56 @@ __global__ void __launch_bounds__(256) k_route(PrefillArgs a) {
     overflow = true;  // recompute everything exactly (rare: many near-equal logits)
     n = E;
   }
-  // exact values of the candidates (fp64 sums of exact products, fixed order)
-  if (!overflow) {
-    for (int i = 0; i < n; ++i) {
-      const int e = s_ce[wl][i];
-      const double v = warp_dot_exact(xt, a.wr + (size_t)e * H, H) + (a.rbias ? (double)a.rbias[e] : 0.0);
-      if (lane == 0) s_cv[wl][i] = v;
-    }
-  }
-  __syncwarp();
-  // select the k best exact keys (value desc, id asc) by k rounds over the candidates
+  // Exact values (fp64 sums of exact products, fixed order) in decreasing order of the fp32
+  // logit, lanes 0..k-1 keeping the best k so far (value desc, id asc).  A candidate whose
+  // certified upper bound is below the k-th kept exact value is skipped: its exact value is
+  // below every value of the final top k, so the selection is the one over all candidates.
   double sv = -INFINITY;
   int se = 0x7fffffff;
   if (!overflow) {
-    uint32_t taken[(kRouteCand + 31) / 32] = {0, 0, 0};
-    for (int r = 0; r < k; ++r) {
-      double bv = -INFINITY;
-      int be = 0x7fffffff, bi = -1;
-      for (int i = lane; i < n; i += 32) {
-        if ((taken[i >> 5] >> (i & 31)) & 1u) continue;
-        const double v = s_cv[wl][i];
-        const int e = s_ce[wl][i];
-        if (v > bv || (v == bv && e < be) || bi < 0) {
-          if (v == v) {
-            bv = v;
-            be = e;
-            bi = i;
-          }
-        }
+    for (int i = lane; i < n; i += 32) {
+      const int e = s_ce[wl][i];
+      const double l = (double)lt[e] + (a.rbias ? (double)a.rbias[e] : 0.0);
+      s_cl[wl][i] = (l == l) ? l : INFINITY;  // a NaN logit first (its exact value decides)
+      s_cu[wl][i] = l + cb * a.wnorm[e];      // NaN for a NaN logit: never skipped
+    }
+    __syncwarp();
+    for (int i = lane; i < n; i += 32) {
+      const double ki = s_cl[wl][i];
+      int rank = 0;
+      for (int j = 0; j < n; ++j) {
+        const double kj = s_cl[wl][j];
+        rank += (kj > ki || (kj == ki && j < i)) ? 1 : 0;
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (oi >= 0 && (bi < 0 || ov > bv || (ov == bv && oe < be))) {
-          bv = ov;
-          be = oe;
-          bi = oi;
-        }
+      s_ord[wl][rank] = i;
+    }
+    __syncwarp();
+    int cnt = 0;  // kept so far (<= k)
+    for (int r = 0; r < n; ++r) {
+      const int i = s_ord[wl][r];
+      const int e = s_ce[wl][i];
+      const double vk = __shfl_sync(0xffffffffu, sv, k - 1);
+      if (cnt == k && s_cu[wl][i] < vk) continue;
+      const double v = warp_dot_exact(xt, a.wr + (size_t)e * H, H) + (a.rbias ? (double)a.rbias[e] : 0.0);
+      if (!(v == v)) continue;  // a NaN is never selected
+      const bool before = lane < cnt && (sv > v || (sv == v && se < e));
+      const int pos = __popc(__ballot_sync(0xffffffffu, before));
+      if (pos >= k) continue;
+      const double pv = __shfl_up_sync(0xffffffffu, sv, 1);
+      const int pe = __shfl_up_sync(0xffffffffu, se, 1);
+      if (lane > pos) {
+        sv = pv;
+        se = pe;
       }
-      if (bi >= 0) taken[bi >> 5] |= 1u << (bi & 31);
-      if (lane == r) {
-        sv = bv;
-        se = bi >= 0 ? be : 0x7fffffff;
+      if (lane == pos) {
+        sv = v;
+        se = e;
       }
+      cnt = cnt < k ? cnt + 1 : k;
+    }
+    if (lane >= cnt) {
+      sv = -INFINITY;
+      se = 0x7fffffff;
     }
   } else {
     // exact value of every expert, k rounds of warp arg-max
