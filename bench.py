@@ -50,7 +50,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC_PER_LAYER = {("k_fused_decode", "decode80b", 1): 21_760_000}
 # DRAM traffic per launch of the prefill gate/up GEMM on the prefill workload (full-size,
 # one-pass capture).  Dropped whenever the kernel changes.
-NCU_TRAFFIC_PREFILL_GATEUP = {("prefill", 4096): 829_711_616}
+NCU_TRAFFIC_PREFILL_GATEUP = {("prefill", 4096): 829_933_568}
 
 
 # --------------------------------------------------------------------------------------
