@@ -5,6 +5,8 @@
   the decode top-k past its 64-candidate fast path and the many-token router past its
   96-candidate certified path into their exact fallbacks;
 * an exact two-way tie at the k-th place: the lower id is selected;
+* logits that differ by less than the fp32 router's rounding (half an ulp): the exact order
+  decides, through both routers;
 * the int8 layer at the full 80B-like width (hidden 2048, 512 experts, top-10), whose fused
   decode kernel no smaller case instantiates;
 * the router alone on many tokens (4096 on the prefill shape, and a shape the tensor-core
@@ -111,6 +113,36 @@ def test_router_topk_many_tokens_prefill_shape():
     logits = oracle.router_logits(host_bits(x), host_bits(wr), None if bias is None else bias.cpu().numpy())
     ref_idx, ref_p = oracle.route(logits, w.top_k)
     assert_routing(idx, ref_idx, logits)
+    assert np.allclose(p.cpu().numpy(), ref_p, rtol=2e-6, atol=1e-7)
+
+
+@pytest.mark.parametrize("T", [4, 16])
+def test_router_orders_logits_fp32_cannot_tell_apart(T):
+    """Every expert has the same router row except coordinate 0, where expert e has
+    (e + 1) * 2^-10, and every token has x_0 = 2^-18: the logits (0.05 to 0.55 here) differ
+    only by (e + 1) * 2^-28, below the resolution of an fp32 sum (a sequential fp32 sum gives
+    3 to 17 distinct values for the 64 experts), while the exact sums order them.  The router
+    must select the k highest ids in decreasing order (T = 4: the fused decode router;
+    T = 16: the many-token certified router, whose candidates are then every expert)."""
+    w = TINY.with_(n_experts=64, top_k=4, seed=79)
+    wr, _, _ = synth.router_weights(w, 0, DEV)
+    base = wr[0].clone()
+    wr = base.repeat(w.n_experts, 1)
+    wr[:, 0] = ((torch.arange(w.n_experts, dtype=torch.float32) + 1) * 2.0 ** -10).to(torch.bfloat16).to(DEV)
+    x = synth.activations(w, 79, tokens=T, device=DEV)
+    x[:, 0] = 2.0 ** -18
+    shape = abi.shape_of(w)
+    ws = ws_for(shape, T)
+    idx = torch.full((T, w.top_k), -7, dtype=torch.int32, device=DEV)
+    p = torch.full((T, w.top_k), -7.0, dtype=torch.float32, device=DEV)
+    abi.moe_router_topk(shape, x, T, wr, None, idx, p, ws)
+    torch.cuda.synchronize()
+    assert abi.moe_ws_check(ws) == 0
+    logits = oracle.router_logits(host_bits(x), host_bits(wr), None)
+    ref_idx, ref_p = oracle.route(logits, w.top_k)
+    want = np.tile(np.arange(w.n_experts - 1, w.n_experts - 1 - w.top_k, -1, dtype=np.int32), (T, 1))
+    assert np.array_equal(ref_idx, want)  # the construction does what it says
+    assert np.array_equal(idx.cpu().numpy(), want)
     assert np.allclose(p.cpu().numpy(), ref_p, rtol=2e-6, atol=1e-7)
 
 
