@@ -793,11 +793,22 @@ __global__ void k_norms(const uint16_t* x, int T, int H, const uint16_t* wr, con
   const int rows = T + E + 1;
   if (warp >= rows) return;
   const uint16_t* row = warp < T ? x + (size_t)warp * H : (warp < T + E ? wr + (size_t)(warp - T) * H : wsg);
-  double s = 0.0;
-  for (int i = lane; i < H; i += 32) {
-    const double v = (double)bf1(row[i]);
-    s += v * v;
+  // 16-byte loads (rows are 16-byte aligned: the router GEMM reads x and w_r by TMA, the exact
+  // dot products read w_sg 16 bytes at a time), eight partial sums per lane; the bound needs
+  // the norm only to fp64 accuracy, not in a fixed order
+  const uint4* r4 = reinterpret_cast<const uint4*>(row);
+  double sp[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+  for (int i = lane; i < H / 8; i += 32) {
+    const uint4 v = __ldg(r4 + i);
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const double lo = (double)bf_lo(w4[j]), hi = (double)bf_hi(w4[j]);
+      sp[2 * j] = fma(lo, lo, sp[2 * j]);
+      sp[2 * j + 1] = fma(hi, hi, sp[2 * j + 1]);
+    }
   }
+  double s = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (lane == 0) {
