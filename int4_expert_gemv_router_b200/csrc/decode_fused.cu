@@ -747,74 +747,61 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
         if (cw == (T + t) % kCons && lane == 0) P_GATE[t] = (float)(1.0 / (1.0 + exp(-__ldcg(a.logits + (size_t)t * (E + 1) + E))));
     }
     bar_cons();
-    // grouping: pairs sorted by (expert, pair number); invalid ids left out.  The pairwise
-    // comparisons are spread over all compute threads (pair i against a block of pairs j),
-    // their counts added with integer atomics, so the result does not depend on the order.
-    if (ok && !(T == 1 && routed)) {
+    // grouping: pairs sorted by (expert, pair number); invalid ids and experts held by another
+    // rank left out (sorted last).  One warp ranks the T*k pairs by counting (each lane its
+    // pairs against all keys, read as shared-memory broadcasts), then numbers the distinct
+    // experts the same way: no CTA barrier inside, and the result does not depend on timing.
+    if (ok && !(T == 1 && routed) && cw == 0) {
       int* key = P_SCRATCH;            // [TK] expert of pair i (E: left out)
       int* rnk = P_SCRATCH + TK;       // [TK] rank of pair i in (expert, pair) order
-      int* dup = P_SCRATCH + 2 * TK;   // [TK] an earlier pair has the same expert
       int* first = P_SCRATCH + 3 * TK; // [TK] pair i is its expert's first
-      int* actc = P_SCRATCH + 4 * TK;  // [TK] distinct experts below pair i's
-      __shared__ int s_an, s_nv;
-      for (int i = tid; i < TK; i += kConsThreads) {
+      for (int i = lane; i < TK; i += 32) {
         const int e = P_IDS[i];
         const bool valid = e >= 0 && e < E;
         if (!valid && blockIdx.x == 0) atomicOr(&a.ctrl->err, kErrBadExpert);
         key[i] = (valid && S_SLOT[e] != kSlotRemote) ? e : E;
-        rnk[i] = 0;
-        dup[i] = 0;
-        actc[i] = 0;
       }
-      if (tid == 0) s_an = s_nv = 0;
-      const int nb = kConsThreads / TK > 0 ? kConsThreads / TK : 1, jb = (TK + nb - 1) / nb;
-      bar_cons();
-      for (int w = tid; w < TK * nb; w += kConsThreads) {
-        const int i = w % TK, j0b = (w / TK) * jb, ki = key[i];
-        int r = 0, d = 0;
-        for (int j = j0b; j < min(TK, j0b + jb); ++j) {
+      __syncwarp();
+      int nv = 0, an = 0;
+      for (int i = lane; i < TK; i += 32) {
+        const int ki = key[i];
+        int r = 0;
+        bool d = false;
+        for (int j = 0; j < TK; ++j) {
           const int kj = key[j];
           r += (kj < ki) || (kj == ki && j < i);
-          d |= (kj == ki && j < i);
+          d = d || (kj == ki && j < i);
         }
-        if (r) atomicAdd(&rnk[i], r);
-        if (d) atomicOr(&dup[i], 1);
-      }
-      bar_cons();
-      for (int i = tid; i < TK; i += kConsThreads) {
-        const int ki = key[i], r = rnk[i];
-        const bool f = !dup[i] && ki < E;
+        const bool f = !d && ki < E;
+        rnk[i] = r;
         P_ORDER[r] = i;
         P_POS[i] = (ki < E) ? r : -1;
         first[i] = f ? 1 : 0;
-        if (ki < E) atomicAdd(&s_nv, 1);
-        if (f) atomicAdd(&s_an, 1);
+        nv += ki < E;
+        an += f;
       }
-      bar_cons();
-      for (int w = tid; w < TK * nb; w += kConsThreads) {
-        const int i = w % TK, j0b = (w / TK) * jb;
+      __syncwarp();
+      for (int i = lane; i < TK; i += 32) {
         if (!first[i]) continue;
         const int ki = key[i];
-        int c = 0;
-        for (int j = j0b; j < min(TK, j0b + jb); ++j) c += (first[j] && key[j] < ki);
-        if (c) atomicAdd(&actc[i], c);
+        int act = 0;  // distinct experts below this one
+        for (int j = 0; j < TK; ++j) act += (first[j] && key[j] < ki);
+        P_ACTE[act] = ki;
+        P_BEGIN[act] = rnk[i];  // the first pair of an expert: its rank counts the pairs below
+        const int slot = S_SLOT[ki];
+        const bool sok = (slot >= 0 && slot < Lc.n_slots) || slot == kSlotPending;
+        if (!sok) atomicOr(&a.ctrl->err, kErrBadSlot);
+        P_SLOT[act] = sok ? slot : -1;
       }
-      bar_cons();
-      for (int i = tid; i < TK; i += kConsThreads) {
-        if (first[i]) {
-          const int ki = key[i], act = actc[i];
-          P_ACTE[act] = ki;
-          P_BEGIN[act] = rnk[i];  // the first pair of an expert: its rank counts the pairs below
-          const int slot = S_SLOT[ki];
-          const bool sok = (slot >= 0 && slot < Lc.n_slots) || slot == kSlotPending;
-          if (!sok) atomicOr(&a.ctrl->err, kErrBadSlot);
-          P_SLOT[act] = sok ? slot : -1;
-        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        nv += __shfl_xor_sync(0xffffffffu, nv, o);
+        an += __shfl_xor_sync(0xffffffffu, an, o);
       }
-      if (tid == 0) {
-        s_act_n = s_an;
-        s_n_valid = s_nv;
-        P_BEGIN[s_an] = s_nv;
+      if (lane == 0) {
+        s_act_n = an;
+        s_n_valid = nv;
+        P_BEGIN[an] = nv;
       }
     }
     bar_cons();
