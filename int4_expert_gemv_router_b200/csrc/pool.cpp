@@ -124,16 +124,32 @@ cudaError_t settle_entry(moe_pool* p, int32_t id) {
 // finished), then copied to its slot on the side stream.  A blob that cannot be read leaves
 // its slot empty (host state rolled back; ok[i] = 0).  With `settle` each miss's pending
 // slot-table entry is written after its copy (or -1 for a failed read).  Returns the first
-// CUDA error of a copy; reads do not raise one.
+// CUDA error of a copy (the loads from that one on rolled back); reads do not raise one.
 cudaError_t file_loads(moe_pool* p, const std::vector<Load>& loads, std::vector<char>& ok, bool settle) {
   ok.assign(loads.size(), 1);
+  // On a CUDA error at load i0, the loads from i0 on keep no host state: their slots are left
+  // empty and they stay non-resident, so that no later step counts them as hits on slots that
+  // hold other weights (the next load uploads the whole table from the host mirror).
+  const auto fail_from = [&](size_t i0, cudaError_t e) {
+    for (size_t j = i0; j < loads.size(); ++j) {
+      const Load& lr = loads[j];
+      if (p->slot_of[lr.id] == lr.slot) {
+        p->slot_of[lr.id] = -1;
+        p->expert_in[lr.slot] = -1;
+        p->stats.h2d_bytes -= p->stride;
+      }
+      p->h_final[lr.id] = -1;
+      ok[j] = 0;
+    }
+    return e;
+  };
   for (size_t w0 = 0; w0 < loads.size(); w0 += kStageBufs) {
     const size_t w1 = std::min(loads.size(), w0 + (size_t)kStageBufs);
     for (size_t i = w0; i < w1; ++i) {
       const int b = (int)(i - w0);
       if (p->stage_busy[b]) {
         cudaError_t e = cudaEventSynchronize(p->stage_ev[b]);
-        if (e != cudaSuccess) return e;
+        if (e != cudaSuccess) return fail_from(w0, e);
         p->stage_busy[b] = false;
       }
     }
@@ -149,7 +165,7 @@ cudaError_t file_loads(moe_pool* p, const std::vector<Load>& loads, std::vector<
         cudaError_t e = cudaMemcpyAsync(p->dev_pool + (int64_t)ld.slot * p->stride, p->stage[b], (size_t)p->stride,
                                         cudaMemcpyHostToDevice, p->side);
         if (e == cudaSuccess) e = cudaEventRecord(p->stage_ev[b], p->side);
-        if (e != cudaSuccess) return e;
+        if (e != cudaSuccess) return fail_from(i, e);
         p->stage_busy[b] = true;
       } else {
         p->slot_of[ld.id] = -1;
@@ -159,7 +175,7 @@ cudaError_t file_loads(moe_pool* p, const std::vector<Load>& loads, std::vector<
       }
       if (settle) {
         cudaError_t e = settle_entry(p, ld.id);
-        if (e != cudaSuccess) return e;
+        if (e != cudaSuccess) return fail_from(i, e);
       }
     }
   }
