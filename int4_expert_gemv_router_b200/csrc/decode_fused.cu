@@ -899,13 +899,10 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
         const uint8_t* st = ring + (size_t)s * SB;
         // work items: (expert of the stage, one of its token pairs), in stage order and dealt
         // to warps round-robin over the layer, so that an expert with many pairs (the shared
-        // one has T) is spread over several warps
+        // one has T) is spread over several warps.  At one token every expert has one pair:
+        // the experts themselves are dealt (the same assignment, in a simpler loop).
         const auto n_pairs = [&](int u) { return u == act_n ? T : P_BEGIN[u + 1] - P_BEGIN[u]; };
-        int n_items = 0;
-        for (int z = 0; z < cnt; ++z) n_items += n_pairs(u0 + z);
-        for (int i = (cw - it0 % kCons + kCons) % kCons; i < n_items; i += kCons) {
-          int z = 0, rem = i;
-          while (rem >= n_pairs(u0 + z)) rem -= n_pairs(u0 + z++);
+        const auto do_item = [&](int z, int rem) {
           const int u = u0 + z;
           const bool shared = (u == act_n);
           const uint8_t* dq = st + (size_t)z * nJ * ROWD_BYTES;
@@ -989,6 +986,19 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
               partial[(size_t)p * a.jmax + jl] = w * sum;
             }
             __syncwarp();
+          }
+        };
+        int n_items = 0;
+        if constexpr (TM == 1) {
+          for (int z = (cw - u0 % kCons + kCons) % kCons; z < cnt; z += kCons)
+            for (int rem = 0; rem < n_pairs(u0 + z); ++rem) do_item(z, rem);
+          n_items = cnt;
+        } else {
+          for (int z = 0; z < cnt; ++z) n_items += n_pairs(u0 + z);
+          for (int i = (cw - it0 % kCons + kCons) % kCons; i < n_items; i += kCons) {
+            int z = 0, rem = i;
+            while (rem >= n_pairs(u0 + z)) rem -= n_pairs(u0 + z++);
+            do_item(z, rem);
           }
         }
         it0 += n_items;
