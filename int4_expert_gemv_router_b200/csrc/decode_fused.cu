@@ -374,13 +374,37 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
       }
       __syncwarp();
     };
+    // At one token phase R reads its rows from global memory (item i on CTA i % G; measured
+    // faster there than staging them), and this warp only prefetches the next layer's rows
+    // into L2; with several tokens the rows are staged in shared memory (issue_r).
     int n_r_issued = 0;  // rbar phases announced
-    issue_r(0, false);
-    ++n_r_issued;
+    if constexpr (TM > 1) {
+      issue_r(0, false);
+      ++n_r_issued;
+    }
     for (int l = 0; l < a.n_layers && ok; ++l) {
       const FusedLayer& Lc = a.layer[l];
-      // L2 prefetch of the next layer's phase-R rows (copied to shared memory later in this layer)
-      if (l + 1 < a.n_layers) issue_r(l + 1, true);
+      if constexpr (TM > 1) {
+        // L2 prefetch of the next layer's phase-R rows (copied to shared memory later in this layer)
+        if (l + 1 < a.n_layers) issue_r(l + 1, true);
+      } else if (l + 1 < a.n_layers) {
+        // L2 prefetch of the next layer's routing-independent rows this CTA's warps will read
+        // (phase-R item i belongs to CTA i % G), one lane per item
+        const FusedLayer& Ln = a.layer[l + 1];
+        const int n_router = (Ln.topk_idx_in ? 0 : E) + 1;
+        const int n_items = n_router + I / RPWg;
+        for (int it = blockIdx.x + G * lane; it < n_items; it += G * 32) {
+          if (it < n_router) {
+            const bool gate_row = (it == n_router - 1);
+            const uint16_t* row = gate_row ? Ln.wsg : Ln.wr + (size_t)it * H;
+            prefetch_l2(row, H * 2);
+          } else {
+            const int r = (it - n_router) * RPWg;
+            prefetch_l2(Ln.shared + a.L.off[0] + (int64_t)r * ROWBg, RPWg * ROWBg);
+            prefetch_l2(Ln.shared + a.L.off[1] + (int64_t)r * ROWBg, RPWg * ROWBg);
+          }
+        }
+      }
       // wait for this layer's plan
       if (!mbar_wait(&plan_bar, l & 1)) {
         ok = false;
@@ -480,7 +504,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
         }
       }
       // the next layer's phase-R rows: this CTA finished reading rbuf before the plan
-      if (ok && l + 1 < a.n_layers) {
+      if (TM > 1 && ok && l + 1 < a.n_layers) {
         issue_r(l + 1, false);
         ++n_r_issued;
       }
@@ -491,7 +515,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
     }
     // let every issued copy land before the CTA may exit
     if (lane == 0) {
-      mbar_wait(&rbar, (uint32_t)(n_r_issued - 1) & 1);
+      if (n_r_issued > 0) mbar_wait(&rbar, (uint32_t)(n_r_issued - 1) & 1);
       const uint32_t first = q > (uint32_t)NS ? q - NS : 0;
       for (uint32_t qq = first; qq < q; ++qq) mbar_wait(&full_bar[qq % NS], (qq / NS) & 1);
     }
@@ -502,7 +526,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
   // compute warps
   // =====================================================================================
   const int cw = warp;  // 0..14
-  const int NW = G * kCons;
+  const int NW = G * kCons;  // compute warps of the grid (one-token phase R)
   uint32_t q = 0;
   uint32_t nb = 0;  // grid barriers passed in this launch
   bool ok = true;
@@ -519,6 +543,70 @@ __global__ void __launch_bounds__(kFThreads, 1) k_fused_decode(const __grid_cons
     for (int e = tid; e < E; e += kConsThreads) S_SLOT[e] = __ldg(Lc.slot_table + e);
     bar_cons();
 
+    // ---- phase R, one token: router rows, shared-gate row, shared gate/up rows from global ----
+    if constexpr (TM == 1) {
+      const int n_router = (routed ? E : 0) + 1;
+      const int n_items = n_router + (Lc.with_shared ? I / RPWg : 0);
+      for (int it = blockIdx.x + G * cw; it < n_items; it += NW) {  // item i: CTA i % G
+        if (it < n_router) {
+          const bool gate_row = (it == n_router - 1);
+          const int e = gate_row ? E : it;
+          const uint16_t* row = gate_row ? Lc.wsg : Lc.wr + (size_t)e * H;
+          double acc = 0.0;
+#pragma unroll 4
+          for (int c8 = lane; c8 < H / 8; c8 += 32) {
+            const uint4 w = ld_stream(row + c8 * 8);
+            const float wv[8] = {bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y),
+                                 bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w)};
+            const int c = c8 / (CC / 8), v0 = (c8 % (CC / 8)) * 2;
+            const float4 xa = xs4[(size_t)v0 * NCg + c];
+            const float4 xb = xs4[(size_t)(v0 + 1) * NCg + c];
+            const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+            double sp = 0.0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              // undo the staging scale (a power of two): the product stays exact
+              const float xr = xv[i] * stage_unscale<BITS>(v0 * 4 + i);
+              sp += (double)(wv[i] * xr);
+            }
+            acc += sp;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          if (lane == 0) {
+            if (!gate_row && Lc.rbias) acc += (double)Lc.rbias[e];
+            a.logits[e] = acc;
+          }
+        } else {
+          // shared expert gate/up row(s)
+          const int r = (it - n_router) * RPWg + lane / NCLg;
+          const int sub = lane % NCLg;
+          const uint8_t* b = Lc.shared;
+          float ag = 0.f, au = 0.f;
+#pragma unroll 1
+          for (int m = 0; m < CPLg; ++m) {
+            const int c = sub + NCLg * m, g = c * CC / kGroup;
+            const uint4 qg = ld_stream(b + a.L.off[0] + (int64_t)r * ROWBg + c * 16);
+            const uint4 qu = ld_stream(b + a.L.off[1] + (int64_t)r * ROWBg + c * 16);
+            const float sg = bf1(ld_u16(b + a.L.off[3] + (int64_t)r * SRg + g * 2));
+            const float bg = bf1(ld_u16(b + a.L.off[4] + (int64_t)r * SRg + g * 2));
+            const float su = bf1(ld_u16(b + a.L.off[5] + (int64_t)r * SRg + g * 2));
+            const float bu = bf1(ld_u16(b + a.L.off[6] + (int64_t)r * SRg + g * 2));
+            float dg, du;
+            dot_chunk2<BITS>(qg, qu, xs4 + c, NCg, dg, du);
+            const float xc = xsum[c];
+            ag = fmaf(sg, dg, fmaf(bg, xc, ag));
+            au = fmaf(su, du, fmaf(bu, xc, au));
+          }
+#pragma unroll
+          for (int o = NCLg / 2; o > 0; o >>= 1) {
+            ag += __shfl_xor_sync(0xffffffffu, ag, o);
+            au += __shfl_xor_sync(0xffffffffu, au, o);
+          }
+          if (sub == 0) a.hs[r] = ag / (1.0f + expf(-ag)) * au;
+        }
+      }
+    } else
     // ---- phase R: router rows, shared-gate row, shared gate/up rows (staged in rbuf) ----
     {
       const RRange R = r_ranges(Lc, E, I, gG, blockIdx.x, G);
