@@ -47,7 +47,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # large to capture; every layer reads its own blobs, so traffic scales with the layers).  Keyed
 # by (kernel, workload, tokens); an entry is dropped whenever the kernel changes and comes back
 # with the next capture.
-NCU_TRAFFIC_PER_LAYER = {("k_fused_decode", "decode80b", 1): 21_631_360}
+NCU_TRAFFIC_PER_LAYER = {("k_fused_decode", "decode80b", 1): 21_664_640}
 # DRAM traffic per launch of the prefill gate/up GEMM on the prefill workload (full-size,
 # one-pass capture).  Dropped whenever the kernel changes.
 NCU_TRAFFIC_PREFILL_GATEUP = {("prefill", 4096): 829_933_568}
