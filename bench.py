@@ -2,8 +2,9 @@
 """Benchmark of the routed-MoE layer forward on B200 (one process per GPU).
 
     python bench.py [--gpus N] [--steps K] [--warmup W]
-                    [--workload decode80b|decode35b|prefill|pool_int4|pool_int8]
-                    [--tokens T] [--impl ours|reference] [--policy lfu_recency|lru|lfu] [--slots S] [--overlap]
+                    [--workload decode80b|decode35b|prefill|pool_int4|pool_int8|gdn80b|gdn80b_b8]
+                    [--tokens T] [--impl ours|reference] [--parallel replicas|ep] [--no-cpu-baseline]
+                    [--policy lfu_recency|lru|lfu] [--slots S] [--store host|file|file_direct] [--overlap]
 
 Default workload: the 80B-like decode stack -- hidden 2048, 512 experts, top-10,
 intermediate 512, shared expert 512, int4 group 64, one token per step through 48
@@ -16,8 +17,10 @@ residual chain x_l + moe_l(x_l) grows without bound under random weights).
 Timing: W untimed warm-up steps, then K steps timed with CUDA events on the launching
 stream, bracketed by a barrier and a device synchronize; the max over ranks is taken.
 Each step reads >1 GB of distinct expert blobs, larger than the 126 MB L2, so no flush is
-needed between steps.  With N > 1 every rank runs an independent replica (weak scaling;
-the path has no exchange step).  Rank 0 prints one JSON line.
+needed between steps.  With N > 1 every rank runs an independent replica by default (weak
+scaling; one token stream's layer has no exchange step); `--parallel ep` splits every layer's
+experts over the ranks instead (strong scaling, one NCCL all-reduce per layer).  Rank 0 prints
+one JSON line.
 """
 from __future__ import annotations
 
