@@ -914,12 +914,35 @@ __global__ void __launch_bounds__(256) k_route(PrefillArgs a) {
     overflow = true;  // recompute everything exactly (rare: many near-equal logits)
     n = E;
   }
-  // Exact values (fp64 sums of exact products, fixed order) in decreasing order of the fp32
-  // logit, lanes 0..k-1 keeping the best k so far (value desc, id asc).  A candidate whose
-  // certified upper bound is below the k-th kept exact value is skipped: its exact value is
-  // below every value of the final top k, so the selection is the one over all candidates.
+  // Exact values (fp64 sums of exact products, fixed order), lanes 0..k-1 keeping the best k
+  // so far (value desc, id asc).  A candidate whose certified upper bound is below the k-th
+  // kept exact value is skipped: its exact value is below every value of the final top k, so
+  // the selection is the one over all candidates.  Normally the candidates come in decreasing
+  // order of the fp32 logit; after an overflow every expert comes, in id order, under the
+  // same test (at most E exact dots, most of them skipped once k are kept).
   double sv = -INFINITY;
   int se = 0x7fffffff;
+  int cnt = 0;  // kept so far (<= k)
+  const auto consider = [&](int e, double upper) {
+    const double vk = __shfl_sync(0xffffffffu, sv, k - 1);
+    if (cnt == k && upper < vk) return;
+    const double v = warp_dot_exact(xt, a.wr + (size_t)e * H, H) + (a.rbias ? (double)a.rbias[e] : 0.0);
+    if (!(v == v)) return;  // a NaN is never selected
+    const bool before = lane < cnt && (sv > v || (sv == v && se < e));
+    const int pos = __popc(__ballot_sync(0xffffffffu, before));
+    if (pos >= k) return;
+    const double pv = __shfl_up_sync(0xffffffffu, sv, 1);
+    const int pe = __shfl_up_sync(0xffffffffu, se, 1);
+    if (lane > pos) {
+      sv = pv;
+      se = pe;
+    }
+    if (lane == pos) {
+      sv = v;
+      se = e;
+    }
+    cnt = cnt < k ? cnt + 1 : k;
+  };
   if (!overflow) {
     for (int i = lane; i < n; i += 32) {
       const int e = s_ce[wl][i];
@@ -938,53 +961,17 @@ __global__ void __launch_bounds__(256) k_route(PrefillArgs a) {
       s_ord[wl][rank] = i;
     }
     __syncwarp();
-    int cnt = 0;  // kept so far (<= k)
     for (int r = 0; r < n; ++r) {
       const int i = s_ord[wl][r];
-      const int e = s_ce[wl][i];
-      const double vk = __shfl_sync(0xffffffffu, sv, k - 1);
-      if (cnt == k && s_cu[wl][i] < vk) continue;
-      const double v = warp_dot_exact(xt, a.wr + (size_t)e * H, H) + (a.rbias ? (double)a.rbias[e] : 0.0);
-      if (!(v == v)) continue;  // a NaN is never selected
-      const bool before = lane < cnt && (sv > v || (sv == v && se < e));
-      const int pos = __popc(__ballot_sync(0xffffffffu, before));
-      if (pos >= k) continue;
-      const double pv = __shfl_up_sync(0xffffffffu, sv, 1);
-      const int pe = __shfl_up_sync(0xffffffffu, se, 1);
-      if (lane > pos) {
-        sv = pv;
-        se = pe;
-      }
-      if (lane == pos) {
-        sv = v;
-        se = e;
-      }
-      cnt = cnt < k ? cnt + 1 : k;
-    }
-    if (lane >= cnt) {
-      sv = -INFINITY;
-      se = 0x7fffffff;
+      consider(s_ce[wl][i], s_cu[wl][i]);
     }
   } else {
-    // exact value of every expert, k rounds of warp arg-max
-    uint32_t taken[kMaxExperts / 32] = {};
-    for (int r = 0; r < k; ++r) {
-      double bv = -INFINITY;
-      int be = 0x7fffffff;
-      for (int e = 0; e < E; ++e) {
-        if ((taken[e >> 5] >> (e & 31)) & 1u) continue;
-        const double v = warp_dot_exact(xt, a.wr + (size_t)e * H, H) + (a.rbias ? (double)a.rbias[e] : 0.0);
-        if (v == v && (be == 0x7fffffff || v > bv || (v == bv && e < be))) {
-          bv = v;
-          be = e;
-        }
-      }
-      if (be != 0x7fffffff) taken[be >> 5] |= 1u << (be & 31);
-      if (lane == r) {
-        sv = bv;
-        se = be;
-      }
-    }
+    for (int e = 0; e < E; ++e)
+      consider(e, (double)lt[e] + (a.rbias ? (double)a.rbias[e] : 0.0) + cb * a.wnorm[e]);
+  }
+  if (lane >= cnt) {
+    sv = -INFINITY;
+    se = 0x7fffffff;
   }
   const double v0 = __shfl_sync(0xffffffffu, sv, 0);
   const bool valid = lane < k && se != 0x7fffffff;

@@ -81,6 +81,34 @@ def test_exact_tie_at_kth_place_goes_to_lower_id(T):
     assert_close(out, ref["out"])
 
 
+def test_many_near_equal_candidates_take_the_exact_fallback():
+    """Token 0's best router row copied to 200 rows, each copy nudged by one bf16 ulp in a
+    column of its own: their logits differ by far less than the fp32 error bound, so token 0
+    has more than 96 candidates and the many-token router takes its fallback (every expert's
+    exact value, skipped by the certified bound once k are kept).  Ids must be the oracle's
+    fp64 selection."""
+    w, L = _layer_80b_shape(seed=73)
+    L.router_bias = None
+    T = 16
+    x = synth.activations(w, 7, tokens=T, device=DEV)
+    logits = oracle.router_logits(host_bits(x), host_bits(L.w_router), None)
+    best = int(np.argmax(logits[0]))
+    base = L.w_router[best].clone().view(torch.int16)
+    others = [e for e in range(w.n_experts) if e != best][:199]
+    for j, e in enumerate(others):
+        r = base.clone()
+        r[(37 * j) % w.hidden] += 1  # the next bf16 away from zero
+        L.w_router[e] = r.view(torch.bfloat16)
+    ref = oracle_forward(w, L, x, residual=x)
+    near = np.abs(ref["logits"][0, others + [best]] - ref["logits"][0, best])
+    assert near.max() < 1e-2 and np.unique(ref["logits"][0, others]).size > 150  # near-equal, mostly distinct
+    out, idx, p, ws = forward(w, L, x, residual=x)
+    assert abi.moe_ws_check(ws) == 0
+    assert_routing(idx, ref["idx"], ref["logits"])
+    assert np.allclose(p.cpu().numpy(), ref["p"], rtol=2e-6, atol=1e-7)
+    assert_close(out, ref["out"])
+
+
 @pytest.mark.parametrize("T", [1, 8])
 def test_int8_full_width_layer(T):
     """The int8 layer of the bounded-pool workload's shape (hidden 2048, inter 512, 512
